@@ -1,0 +1,238 @@
+"""Float64 CPU oracle for Heavily Compressed Attention (HCA).
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path imports, links or runs
+this module; only the test suite, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / reference leg of ``bench.py`` may call it.  It shares no
+code, table or helper with the CUDA path.
+
+What it restates (each function cites its passage):
+
+* "280B总参数、14B激活！百度开源文心5.5 Flash Base" (aitest123.com news),
+  section 二.1 "Latent-Gated Sparse Attention" -- cited below as [news 二.1]:
+  an HCA layer turns every 128 tokens into one cache entry, and attention
+  runs only over the compressed entries plus a window made of the most
+  recent, still uncompressed tokens.
+* "百度 ERNIE 5.5 Flash Base 完整解析" (communeify.com), section "六大核心架構
+  創新" item 1 "Hybrid MLA-DSA + HCA 與 VHA" -- cited below as [analysis 1]:
+  128 consecutive tokens become a single entry (128x compression); the layer
+  attends to all compressed history entries together with a short window of
+  recent raw tokens; head dimension 512.
+* Both pages, "Low-Rank Gated Attention" paragraph: the attention output is
+  multiplied by a learned gate.
+
+Readings taken where the pages are silent:
+
+* pooling rule = arithmetic mean over the valid tokens of the block;
+* window = the last W raw tokens, inclusive of the query itself, causal;
+* visible compressed entries = blocks that END before the window starts
+  (no overlap with the window; a gap of up to block-1 tokens is allowed);
+* the partially filled last block is compressed but never visible;
+* one softmax over the union of the two key sets, scale supplied (1/sqrt(512));
+* the gate is supplied already passed through the sigmoid; it multiplies O.
+
+Everything is float64 NumPy.  The per-position loop is the definition written
+out: for each query position, gather its visible keys, one softmax, one
+weighted sum.  All heads of a position are handled by one matmul (a library
+primitive); there is no tiling across positions.
+
+Parity status: exact values for random inputs are not printed by the pages
+("parity unpinned" in that narrow sense); every function below is pinned by
+the invariants, reductions to library routines and brute-force checks in
+``tests/test_oracle.py``.
+"""
+
+from __future__ import annotations
+
+from typing import Iterable, Optional, Tuple
+
+import numpy as np
+
+
+# ---------------------------------------------------------------------------
+# Visibility (integer, exact)
+# ---------------------------------------------------------------------------
+
+def window_bounds(t: int, window: int) -> Tuple[int, int]:
+    """Raw window of query position ``t``: tokens [lo, hi], inclusive.
+
+    [news 二.1] / [analysis 1]: the window holds the most
+    recent uncompressed tokens.  Reading: the last ``window`` tokens up to and
+    including ``t`` (causal), clipped at token 0.
+    """
+    return max(0, t - window + 1), t
+
+
+def visible_compressed_count(t: int, block: int, window: int) -> int:
+    """Number of compressed entries query position ``t`` may attend to.
+
+    Reading of the same passages: entry j (tokens [j*block, (j+1)*block)) is
+    visible iff the whole block ends before the raw window starts, i.e.
+    (j+1)*block <= t - window + 1.  Entries are a prefix 0..n-1.
+    """
+    return max(0, (t + 1 - window) // block)
+
+
+def compressed_entry_count(T: int, block: int) -> int:
+    """Entries a sequence of T tokens produces: one per started block.
+
+    [news 二.1]: every 128 tokens become one cache entry; the
+    partial last block also gets an entry (reading), hence ceil(T / block).
+    """
+    return -(-T // block)
+
+
+def mask_table(T: int, block: int, window: int) -> np.ndarray:
+    """int64 [T, 3] rows (n_c, win_lo, win_hi) for every query position."""
+    out = np.zeros((T, 3), dtype=np.int64)
+    for t in range(T):
+        lo, hi = window_bounds(t, window)
+        out[t] = (visible_compressed_count(t, block, window), lo, hi)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Compression (mean pooling of each block)
+# ---------------------------------------------------------------------------
+
+def compress_blocks(X: np.ndarray, block: int) -> np.ndarray:
+    """Mean-pool each run of ``block`` consecutive tokens into one entry.
+
+    X: [T, H, D] (any float dtype, promoted to float64).  Returns
+    [ceil(T/block), H, D] float64.  [news 二.1] / [analysis 1]
+    (128 tokens -> one entry); pooling = mean (reading), over the
+    tokens actually present in the block.
+    """
+    X = np.asarray(X, dtype=np.float64)
+    T = X.shape[0]
+    n = compressed_entry_count(T, block)
+    out = np.empty((n,) + X.shape[1:], dtype=np.float64)
+    for j in range(n):
+        seg = X[j * block: min((j + 1) * block, T)]
+        out[j] = seg.sum(axis=0) / seg.shape[0]
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Attention for one query position
+# ---------------------------------------------------------------------------
+
+def _softmax_weighted(scores: np.ndarray, values: np.ndarray):
+    """Row softmax of ``scores`` [H, n] and the weighted sum of ``values`` [n, D].
+
+    Returns (out [H, D], lse [H], weights [H, n]); the max is subtracted
+    before exponentiation.
+    """
+    m = scores.max(axis=1, keepdims=True)
+    e = np.exp(scores - m)
+    s = e.sum(axis=1, keepdims=True)
+    w = e / s
+    return w @ values, (m + np.log(s))[:, 0], w
+
+
+def attend_position(q: np.ndarray, Kc: np.ndarray, Vc: np.ndarray,
+                    K: np.ndarray, V: np.ndarray, t: int, block: int,
+                    window: int, scale: float, return_weights: bool = False):
+    """HCA output of all query heads at position ``t``.
+
+    q: [Hq, D]; Kc, Vc: [n_entries, Hkv, D]; K, V: [>= t+1, Hkv, D] raw tokens
+    indexed by absolute position.  Query head h reads KV head
+    h * Hkv // Hq.  The key set is the visible compressed entries followed by
+    the raw window; one softmax runs over both ([news 二.1],
+    [analysis 1]).  Returns (o [Hq, D], lse [Hq]) and optionally the
+    softmax weights [Hq, n_keys].
+    """
+    q = np.asarray(q, dtype=np.float64)
+    Hq, D = q.shape
+    Hkv = K.shape[1]
+    nc = visible_compressed_count(t, block, window)
+    lo, hi = window_bounds(t, window)
+    if nc > Kc.shape[0]:
+        raise ValueError("compressed cache holds fewer entries than visible")
+    o = np.empty((Hq, V.shape[2]), dtype=np.float64)
+    lse = np.empty((Hq,), dtype=np.float64)
+    weights = []
+    for g in range(Hkv):
+        heads = [h for h in range(Hq) if h * Hkv // Hq == g]
+        keys = np.concatenate([np.asarray(Kc[:nc, g], np.float64),
+                               np.asarray(K[lo:hi + 1, g], np.float64)], axis=0)
+        vals = np.concatenate([np.asarray(Vc[:nc, g], np.float64),
+                               np.asarray(V[lo:hi + 1, g], np.float64)], axis=0)
+        scores = (q[heads] @ keys.T) * scale
+        og, lg, wg = _softmax_weighted(scores, vals)
+        o[heads] = og
+        lse[heads] = lg
+        weights.append((heads, wg))
+    if return_weights:
+        w = np.empty((Hq, nc + hi - lo + 1), dtype=np.float64)
+        for heads, wg in weights:
+            w[heads] = wg
+        return o, lse, w
+    return o, lse
+
+
+# ---------------------------------------------------------------------------
+# Prefill and decode front ends
+# ---------------------------------------------------------------------------
+
+def hca_prefill(Q: np.ndarray, K: np.ndarray, V: np.ndarray, block: int,
+                window: int, scale: float, gate: Optional[np.ndarray] = None,
+                positions: Optional[Iterable[int]] = None):
+    """HCA attention of one sequence.
+
+    Q: [T, Hq, D]; K, V: [T, Hkv, D]; gate: [T, Hq, D] already sigmoided
+    (low-rank gated attention paragraph of [news 二.1] and [analysis 1]: the
+    output is multiplied by a gate) or None.  ``positions`` selects the
+    query positions to evaluate (default: all).  Returns (O [P, Hq, D],
+    LSE [P, Hq]) in float64 for the selected positions, in order.
+    """
+    Kc = compress_blocks(K, block)
+    Vc = compress_blocks(V, block)
+    T = Q.shape[0]
+    pos = list(range(T)) if positions is None else [int(p) for p in positions]
+    O = np.empty((len(pos), Q.shape[1], V.shape[2]), dtype=np.float64)
+    L = np.empty((len(pos), Q.shape[1]), dtype=np.float64)
+    for i, t in enumerate(pos):
+        o, lse = attend_position(Q[t], Kc, Vc, K, V, t, block, window, scale)
+        if gate is not None:
+            o = o * np.asarray(gate[t], dtype=np.float64)
+        O[i] = o
+        L[i] = lse
+    return O, L
+
+
+def hca_decode(q: np.ndarray, Kc: np.ndarray, Vc: np.ndarray,
+               ring_k: np.ndarray, ring_v: np.ndarray, ctx_len: int,
+               block: int, window: int, scale: float,
+               gate: Optional[np.ndarray] = None):
+    """One decode step: the new token is position t = ctx_len - 1.
+
+    q: [Hq, D]; Kc, Vc: [>= n_c, Hkv, D] cached entries; ring_k, ring_v:
+    [window, Hkv, D] where raw token u sits in slot u % window.  The key set
+    is exactly the prefill key set of position t ([news 二.1]).
+    Returns (o [Hq, D], lse [Hq]).
+    """
+    t = ctx_len - 1
+    lo, hi = window_bounds(t, window)
+    Hkv = ring_k.shape[1]
+    D = ring_k.shape[2]
+    # Lay the window tokens out at their absolute positions.
+    Kw = np.zeros((hi + 1, Hkv, D), dtype=np.float64)
+    Vw = np.zeros((hi + 1, Hkv, ring_v.shape[2]), dtype=np.float64)
+    for u in range(lo, hi + 1):
+        Kw[u] = ring_k[u % window]
+        Vw[u] = ring_v[u % window]
+    o, lse = attend_position(q, Kc, Vc, Kw, Vw, t, block, window, scale)
+    if gate is not None:
+        o = o * np.asarray(gate, dtype=np.float64)
+    return o, lse
+
+
+def visible_pairs(T: int, block: int, window: int) -> Tuple[int, int]:
+    """(compressed, raw) query-key pairs per head for a sequence of T tokens."""
+    c = 0
+    w = 0
+    for t in range(T):
+        c += visible_compressed_count(t, block, window)
+        lo, hi = window_bounds(t, window)
+        w += hi - lo + 1
+    return c, w

@@ -1,0 +1,329 @@
+"""Pins for the float64 oracle (CPU only).
+
+Each pin checks the oracle against something other than itself: a table
+worked out by hand, a set-based brute force, a closed form, or a reduction to
+a library routine (torch scaled_dot_product_attention in float64, numpy mean,
+scipy logsumexp).  ``test_planted_mistakes_are_caught`` plants plausible
+mistakes in the oracle and checks that every one of them fails some pin.
+"""
+
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+from scipy.special import logsumexp
+
+from oracle import hca_oracle as ORC
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ---------------------------------------------------------------------------
+# helpers that do not use the oracle
+# ---------------------------------------------------------------------------
+
+def _rand(shape, seed):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+def _sdpa(q, k, v, scale, mask=None, causal=False):
+    """torch SDPA in float64. q [L, H, D]; k, v [S, H, D]; mask [L, S] bool."""
+    tq = torch.from_numpy(np.ascontiguousarray(q.transpose(1, 0, 2)))[None]
+    tk = torch.from_numpy(np.ascontiguousarray(k.transpose(1, 0, 2)))[None]
+    tv = torch.from_numpy(np.ascontiguousarray(v.transpose(1, 0, 2)))[None]
+    m = None if mask is None else torch.from_numpy(mask)[None, None]
+    o = F.scaled_dot_product_attention(tq, tk, tv, attn_mask=m, is_causal=causal,
+                                       scale=scale)
+    return o[0].numpy().transpose(1, 0, 2)
+
+
+def _expand_kv(x, hq):
+    """[S, Hkv, D] -> [S, Hq, D]; query head h reads KV head h*Hkv//Hq."""
+    hkv = x.shape[1]
+    idx = [h * hkv // hq for h in range(hq)]
+    return x[:, idx]
+
+
+def _brute_visibility(T, B, W):
+    """Set-based visibility: (compressed set, window set) for every t."""
+    out = []
+    for t in range(T):
+        win = {u for u in range(T) if t - W + 1 <= u <= t}
+        comp = set()
+        for j in range((T + B - 1) // B):
+            toks = set(range(j * B, min((j + 1) * B, T)))
+            if len(toks) == B and max(toks) < t - W + 1:
+                comp.add(j)
+        out.append((comp, win))
+    return out
+
+
+# ---------------------------------------------------------------------------
+# pins, written as plain functions of the oracle module so that the planted
+# mistake test can run them against a patched copy
+# ---------------------------------------------------------------------------
+
+def pin_golden_mask(orc):
+    rows = []
+    with open(os.path.join(GOLDEN, "mask_T10_B4_W3.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            t, nc, lo, hi, _gap = line.split()
+            rows.append((int(t), int(nc), int(lo), int(hi)))
+    got = orc.mask_table(10, 4, 3)
+    for t, nc, lo, hi in rows:
+        assert tuple(got[t]) == (nc, lo, hi), (t, tuple(got[t]), (nc, lo, hi))
+    assert orc.compressed_entry_count(10, 4) == 3
+
+
+def pin_brute_visibility(orc):
+    for T, B, W in [(10, 4, 3), (37, 5, 7), (64, 8, 8), (50, 16, 3), (20, 1, 4),
+                    (30, 4, 40), (300, 128, 128)]:
+        brute = _brute_visibility(T, B, W)
+        for t in range(T):
+            comp, win = brute[t]
+            nc = orc.visible_compressed_count(t, B, W)
+            lo, hi = orc.window_bounds(t, W)
+            assert set(range(nc)) == comp, (T, B, W, t)
+            assert set(range(lo, hi + 1)) == win, (T, B, W, t)
+            # partition of [0, t]: compressed tokens, gap, window are disjoint
+            ctoks = set(range(nc * B))
+            assert not (ctoks & win)
+            gap = set(range(t + 1)) - ctoks - win
+            assert len(gap) < B or nc == 0 and len(gap) < B + W
+            if t + 1 >= W + B:
+                assert len(gap) < B
+
+
+def pin_entry_count(orc):
+    for T, B in [(1, 128), (127, 128), (128, 128), (129, 128), (1024, 128),
+                 (131072, 128), (10, 4), (7, 1)]:
+        X = np.zeros((T, 1, 1))
+        assert orc.compressed_entry_count(T, B) == math.ceil(T / B)
+        if T <= 2000:
+            assert orc.compress_blocks(X, B).shape[0] == math.ceil(T / B)
+
+
+def pin_compress_mean(orc):
+    X = _rand((512, 2, 16), 1)
+    got = orc.compress_blocks(X, 128)
+    ref = X.reshape(4, 128, 2, 16).mean(axis=1)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-13)
+    # partial last block: mean over the tokens present
+    Y = _rand((300, 1, 8), 2)
+    got = orc.compress_blocks(Y, 128)
+    np.testing.assert_allclose(got[2], np.mean(Y[256:300], axis=0), rtol=0,
+                               atol=1e-13)
+
+
+def pin_full_window_is_causal(orc):
+    # W >= T: no block is ever visible, every query sees tokens 0..t
+    for D in (8, 512):
+        T, hq = 40, 3
+        Q, K, V = _rand((T, hq, D), 3), _rand((T, 1, D), 4), _rand((T, 1, D), 5)
+        s = 1.0 / math.sqrt(D)
+        O, L = orc.hca_prefill(Q, K, V, block=4, window=T, scale=s)
+        ref = _sdpa(Q, _expand_kv(K, hq), _expand_kv(V, hq), s, causal=True)
+        np.testing.assert_allclose(O, ref, rtol=1e-10, atol=1e-12)
+        # log-sum-exp of the causal scores, by scipy
+        for t in (0, 7, T - 1):
+            sc = (Q[t] @ K[:t + 1, 0].T) * s
+            np.testing.assert_allclose(L[t], logsumexp(sc, axis=1), rtol=1e-12)
+
+
+def pin_block1_is_full(orc):
+    # block = 1: every compressed entry is one raw token, so the union is 0..t
+    for D, W in ((8, 3), (512, 5)):
+        T, hq = 33, 2
+        Q, K, V = _rand((T, hq, D), 6), _rand((T, 1, D), 7), _rand((T, 1, D), 8)
+        s = 1.0 / math.sqrt(D)
+        O, _ = orc.hca_prefill(Q, K, V, block=1, window=W, scale=s)
+        ref = _sdpa(Q, _expand_kv(K, hq), _expand_kv(V, hq), s, causal=True)
+        np.testing.assert_allclose(O, ref, rtol=1e-10, atol=1e-12)
+
+
+def pin_augmented_sdpa(orc):
+    # HCA == SDPA over [block means ; raw tokens] with a set-built mask
+    for (T, B, W, hq, hkv, D) in [(50, 4, 3, 4, 2, 16), (70, 8, 5, 3, 1, 8),
+                                  (300, 128, 128, 2, 1, 32)]:
+        Q = _rand((T, hq, D), 9)
+        K = _rand((T, hkv, D), 10)
+        V = _rand((T, hkv, D), 11)
+        nb = (T + B - 1) // B
+        means_k = np.stack([K[j * B:min((j + 1) * B, T)].mean(0) for j in range(nb)])
+        means_v = np.stack([V[j * B:min((j + 1) * B, T)].mean(0) for j in range(nb)])
+        Ka = np.concatenate([means_k, K])
+        Va = np.concatenate([means_v, V])
+        mask = np.zeros((T, nb + T), dtype=bool)
+        for t, (comp, win) in enumerate(_brute_visibility(T, B, W)):
+            for j in comp:
+                mask[t, j] = True
+            for u in win:
+                mask[t, nb + u] = True
+        s = 1.0 / math.sqrt(D)
+        ref = _sdpa(Q, _expand_kv(Ka, hq), _expand_kv(Va, hq), s, mask=mask)
+        O, _ = orc.hca_prefill(Q, K, V, block=B, window=W, scale=s)
+        np.testing.assert_allclose(O, ref, rtol=1e-10, atol=1e-12)
+
+
+def pin_constant_v(orc):
+    T, hq, D = 60, 2, 16
+    Q, K = _rand((T, hq, D), 12) * 3, _rand((T, 1, D), 13) * 3
+    c = _rand((1, 1, D), 14)
+    V = np.repeat(c, T, axis=0)
+    O, _ = orc.hca_prefill(Q, K, V, block=4, window=5, scale=0.25)
+    np.testing.assert_allclose(O, np.broadcast_to(c, O.shape), rtol=0, atol=1e-12)
+    G = 1.0 / (1.0 + np.exp(-_rand((T, hq, D), 15)))
+    Og, _ = orc.hca_prefill(Q, K, V, block=4, window=5, scale=0.25, gate=G)
+    np.testing.assert_allclose(Og, c * G, rtol=0, atol=1e-12)
+
+
+def pin_weights_sum_to_one(orc):
+    T, hq, D, B, W = 40, 3, 8, 4, 3
+    Q, K, V = _rand((T, hq, D), 16), _rand((T, 1, D), 17), _rand((T, 1, D), 18)
+    Kc, Vc = orc.compress_blocks(K, B), orc.compress_blocks(V, B)
+    for t in range(T):
+        o, lse, w = orc.attend_position(Q[t], Kc, Vc, K, V, t, B, W, 0.3,
+                                        return_weights=True)
+        np.testing.assert_allclose(w.sum(axis=1), 1.0, rtol=0, atol=1e-13)
+        nc = orc.visible_compressed_count(t, B, W)
+        lo, hi = orc.window_bounds(t, W)
+        assert w.shape[1] == nc + hi - lo + 1
+
+
+def pin_single_key(orc):
+    T, hq, D = 9, 4, 8
+    Q, K, V = _rand((T, hq, D), 19), _rand((T, 1, D), 20), _rand((T, 1, D), 21)
+    O, L = orc.hca_prefill(Q, K, V, block=4, window=3, scale=0.5, positions=[0])
+    np.testing.assert_allclose(O[0], np.broadcast_to(V[0, 0], (hq, D)), rtol=0,
+                               atol=1e-14)
+    np.testing.assert_allclose(L[0], 0.5 * (Q[0] @ K[0, 0]), rtol=1e-13)
+
+
+def pin_decode_matches_prefill_row(orc):
+    T, hq, D, B, W = 77, 4, 16, 8, 6
+    Q, K, V = _rand((T, hq, D), 22), _rand((T, 1, D), 23), _rand((T, 1, D), 24)
+    G = 1.0 / (1.0 + np.exp(-_rand((T, hq, D), 25)))
+    Kc, Vc = orc.compress_blocks(K, B), orc.compress_blocks(V, B)
+    O, L = orc.hca_prefill(Q, K, V, B, W, 0.2, gate=G)
+    for t in (0, 3, W - 1, W, 40, T - 1):
+        rk = np.zeros((W, 1, D))
+        rv = np.zeros((W, 1, D))
+        for u in range(max(0, t - W + 1), t + 1):
+            rk[u % W] = K[u]
+            rv[u % W] = V[u]
+        o, lse = orc.hca_decode(Q[t], Kc, Vc, rk, rv, t + 1, B, W, 0.2, gate=G[t])
+        np.testing.assert_allclose(o, O[t], rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(lse, L[t], rtol=1e-12)
+
+
+PINS = [pin_golden_mask, pin_brute_visibility, pin_entry_count, pin_compress_mean,
+        pin_full_window_is_causal, pin_block1_is_full, pin_augmented_sdpa,
+        pin_constant_v, pin_weights_sum_to_one, pin_single_key,
+        pin_decode_matches_prefill_row]
+
+
+@pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
+def test_oracle_pin(pin):
+    pin(ORC)
+
+
+# ---------------------------------------------------------------------------
+# planted mistakes: each must fail at least one pin
+# ---------------------------------------------------------------------------
+
+def _mut_nc_plus_one(t, block, window):
+    return max(0, (t + 2 - window) // block)
+
+
+def _mut_nc_overlap(t, block, window):
+    return max(0, (t + 1) // block)
+
+
+def _mut_window_wide(t, window):
+    return max(0, t - window), t
+
+
+def _mut_compress_sum(X, block):
+    X = np.asarray(X, dtype=np.float64)
+    n = -(-X.shape[0] // block)
+    return np.stack([X[j * block:(j + 1) * block].sum(0) for j in range(n)])
+
+
+def _mut_compress_first(X, block):
+    X = np.asarray(X, dtype=np.float64)
+    n = -(-X.shape[0] // block)
+    return np.stack([X[j * block] for j in range(n)])
+
+
+def _mut_compress_divide_by_block(X, block):
+    X = np.asarray(X, dtype=np.float64)
+    n = -(-X.shape[0] // block)
+    return np.stack([X[j * block:(j + 1) * block].sum(0) / block for j in range(n)])
+
+
+MUTANTS = {
+    "nc_plus_one": ("visible_compressed_count", _mut_nc_plus_one),
+    "nc_overlap": ("visible_compressed_count", _mut_nc_overlap),
+    "window_wide": ("window_bounds", _mut_window_wide),
+    "compress_sum": ("compress_blocks", _mut_compress_sum),
+    "compress_first": ("compress_blocks", _mut_compress_first),
+    "compress_div_block": ("compress_blocks", _mut_compress_divide_by_block),
+}
+
+
+def _mutant_attend(kind):
+    real = ORC.attend_position
+
+    def attend(q, Kc, Vc, K, V, t, block, window, scale, return_weights=False):
+        if kind == "no_scale":
+            scale = 1.0
+        if kind == "kv_head_mod":
+            # wrong GQA mapping: query head h reads KV head h % Hkv
+            Hq, Hkv = q.shape[0], K.shape[1]
+            perm = [h * Hkv // Hq for h in range(Hq)]
+            wrong = [h % Hkv for h in range(Hq)]
+            if perm != wrong:
+                order = np.argsort(np.array(wrong), kind="stable")
+                inv = np.argsort(order)
+                q = q[order]
+                res = real(q, Kc, Vc, K, V, t, block, window, scale, return_weights)
+                return tuple(r[inv] for r in res)
+        if kind == "transposed_values":
+            Kc, Vc, K, V = Kc, Kc, K, K
+        return real(q, Kc, Vc, K, V, t, block, window, scale, return_weights)
+    return attend
+
+
+def _mutant_prefill_no_gate():
+    real = ORC.hca_prefill
+
+    def prefill(Q, K, V, block, window, scale, gate=None, positions=None):
+        return real(Q, K, V, block, window, scale, None, positions)
+    return prefill
+
+
+ALL_MUTANTS = sorted(MUTANTS) + ["no_scale", "kv_head_mod", "transposed_values",
+                                 "no_gate"]
+
+
+@pytest.mark.parametrize("name", ALL_MUTANTS)
+def test_planted_mistakes_are_caught(name, monkeypatch):
+    if name in MUTANTS:
+        attr, fn = MUTANTS[name]
+        monkeypatch.setattr(ORC, attr, fn)
+    elif name == "no_gate":
+        monkeypatch.setattr(ORC, "hca_prefill", _mutant_prefill_no_gate())
+    else:
+        monkeypatch.setattr(ORC, "attend_position", _mutant_attend(name))
+    failed = []
+    for pin in PINS:
+        try:
+            pin(ORC)
+        except (AssertionError, ValueError, IndexError):
+            failed.append(pin.__name__)
+    assert failed, f"planted mistake {name!r} passed every pin"
