@@ -1,0 +1,195 @@
+// compress.cu -- block mean pooling into the paged compressed cache.
+//
+// [news 二.1] / [analysis 1] (see include/hca.h): every `block` consecutive tokens become
+// one cache entry; the pooling rule is the mean over the tokens present (reading).
+//
+// HBM-bound: each block of K (and V) is read once with 16-byte non-allocating loads and a
+// single row of the pool is written. One CTA handles one (block, sequence, tensor): its
+// threads split the row into 16-byte vectors and the block's tokens into `groups`
+// interleaved row sets; partial float32 sums meet in shared memory. Accumulation is
+// float32, the mean is an IEEE division by the token count, rounded once to the storage
+// type.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "hca_internal.h"
+#include "sm100.cuh"
+
+namespace hca {
+namespace {
+
+constexpr int kThreads = 256;
+
+template <typename T>
+struct Vec16;
+template <>
+struct Vec16<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ static void add(const uint4& v, float* acc) {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 f = __bfloat1622float2(h[i]);
+      acc[2 * i] += f.x;
+      acc[2 * i + 1] += f.y;
+    }
+  }
+  __device__ static uint4 pack(const float* x) {
+    uint4 v;
+    uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
+    return v;
+  }
+};
+template <>
+struct Vec16<float> {
+  static constexpr int N = 4;
+  __device__ static void add(const uint4& v, float* acc) {
+    acc[0] += __uint_as_float(v.x);
+    acc[1] += __uint_as_float(v.y);
+    acc[2] += __uint_as_float(v.z);
+    acc[3] += __uint_as_float(v.w);
+  }
+  __device__ static uint4 pack(const float* x) {
+    return make_uint4(__float_as_uint(x[0]), __float_as_uint(x[1]), __float_as_uint(x[2]),
+                      __float_as_uint(x[3]));
+  }
+};
+
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+struct CompressArgs {
+  const void* src[2];  // K, V: first token of block first_block of sequence 0
+  void* pool[2];       // kc_pool, vc_pool
+  const int32_t* page_table;
+  int32_t* n_entries;
+  int32_t* err_word;
+  int64_t batch_stride_rows;  // token rows between sequences
+  int32_t row_vecs;           // 16-byte vectors per token row (hkv * head_dim)
+  int32_t groups;             // row groups per CTA
+  int32_t seqlen, block, first_block, n_blocks;
+  int32_t page_entries, max_pages, num_pages;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) compress_kernel(CompressArgs a) {
+  using V16 = Vec16<T>;
+  constexpr int N = V16::N;
+  const int jrel = blockIdx.x;
+  const int b = blockIdx.y;
+  const int which = blockIdx.z;  // 0: K, 1: V
+  const int j = a.first_block + jrel;
+  const int tok0 = j * a.block;
+  const int count = min(a.block, a.seqlen - tok0);
+
+  extern __shared__ float red[];  // [groups][row_vecs*N] partial sums
+
+  const uint4* src = reinterpret_cast<const uint4*>(a.src[which]) +
+                     ((int64_t)b * a.batch_stride_rows + (int64_t)jrel * a.block) * a.row_vecs;
+  const int lanes = a.row_vecs < kThreads ? a.row_vecs : kThreads;
+  const int g = threadIdx.x / lanes;
+  const int v0 = threadIdx.x % lanes;
+  const bool active = g < a.groups;
+
+  for (int vbase = 0; vbase < a.row_vecs; vbase += lanes) {
+    const int v = vbase + v0;
+    float acc[N];
+#pragma unroll
+    for (int i = 0; i < N; ++i) acc[i] = 0.f;
+    if (active && v < a.row_vecs) {
+      int r = g;
+      // 4 independent 16-byte loads in flight per thread
+      for (; r + 3 * a.groups < count; r += 4 * a.groups) {
+        uint4 x0 = ld_stream(src + (int64_t)r * a.row_vecs + v);
+        uint4 x1 = ld_stream(src + (int64_t)(r + a.groups) * a.row_vecs + v);
+        uint4 x2 = ld_stream(src + (int64_t)(r + 2 * a.groups) * a.row_vecs + v);
+        uint4 x3 = ld_stream(src + (int64_t)(r + 3 * a.groups) * a.row_vecs + v);
+        V16::add(x0, acc);
+        V16::add(x1, acc);
+        V16::add(x2, acc);
+        V16::add(x3, acc);
+      }
+      for (; r < count; r += a.groups) V16::add(ld_stream(src + (int64_t)r * a.row_vecs + v), acc);
+      float* dst = red + ((int64_t)g * lanes + v0) * N;
+#pragma unroll
+      for (int i = 0; i < N; ++i) dst[i] = acc[i];
+    }
+    __syncthreads();
+    if (g == 0 && v < a.row_vecs) {
+      float sum[N];
+#pragma unroll
+      for (int i = 0; i < N; ++i) sum[i] = 0.f;
+      for (int gg = 0; gg < a.groups; ++gg) {
+        const float* p = red + ((int64_t)gg * lanes + v0) * N;
+#pragma unroll
+        for (int i = 0; i < N; ++i) sum[i] += p[i];
+      }
+      const float cnt = (float)count;
+#pragma unroll
+      for (int i = 0; i < N; ++i) sum[i] = __fdiv_rn(sum[i], cnt);
+      const int page = a.page_table[(int64_t)b * a.max_pages + j / a.page_entries];
+      if (page < 0 || page >= a.num_pages) {
+        if (a.err_word) atomicOr(a.err_word, kErrPageRange);
+      } else {
+        const int64_t row = (int64_t)page * a.page_entries + j % a.page_entries;
+        uint4* dst = reinterpret_cast<uint4*>(a.pool[which]) + row * a.row_vecs + v;
+        *dst = V16::pack(sum);
+      }
+    }
+    __syncthreads();
+  }
+  if (which == 0 && jrel == a.n_blocks - 1 && threadIdx.x == 0)
+    a.n_entries[b] = a.first_block + a.n_blocks;
+}
+
+}  // namespace
+
+cudaError_t launch_compress(const hca_desc& d, const void* K, const void* V,
+                            int64_t batch_stride_tokens, int32_t first_block,
+                            int32_t n_blocks, const hca_cache& c, cudaStream_t s) {
+  CompressArgs a;
+  a.src[0] = K;
+  a.src[1] = V;
+  a.pool[0] = c.kc_pool;
+  a.pool[1] = c.vc_pool;
+  a.page_table = c.page_table;
+  a.n_entries = c.n_entries;
+  a.err_word = c.err_word;
+  const int esize = d.dtype == HCA_BF16 ? 2 : 4;
+  a.row_vecs = (int32_t)((int64_t)d.hkv * d.head_dim * esize / 16);
+  a.batch_stride_rows = batch_stride_tokens;
+  a.seqlen = d.seqlen;
+  a.block = d.block;
+  a.first_block = first_block;
+  a.n_blocks = n_blocks;
+  a.page_entries = c.page_entries;
+  a.max_pages = c.max_pages;
+  a.num_pages = c.num_pages;
+  const int lanes = a.row_vecs < kThreads ? a.row_vecs : kThreads;
+  a.groups = kThreads / lanes;
+  if (a.groups > d.block) a.groups = d.block;
+  const int vec_elems = 16 / esize;
+  const size_t smem = (size_t)a.groups * lanes * vec_elems * sizeof(float);
+  dim3 grid(n_blocks, d.batch, 2);
+  if (d.dtype == HCA_BF16) {
+    if (smem > 48 * 1024)
+      cudaFuncSetAttribute(compress_kernel<__nv_bfloat16>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    compress_kernel<__nv_bfloat16><<<grid, kThreads, smem, s>>>(a);
+  } else {
+    if (smem > 48 * 1024)
+      cudaFuncSetAttribute(compress_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem);
+    compress_kernel<float><<<grid, kThreads, smem, s>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace hca

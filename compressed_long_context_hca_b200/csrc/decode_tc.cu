@@ -1,0 +1,553 @@
+// decode_tc.cu -- one HCA decode step on tcgen05 tensor cores, split over the key list,
+// followed by a merge of the split partials.
+//
+// Operation ([news 二.1] / [analysis 1] / [gate] in include/hca.h): the newest token of a
+// sequence (position t = ctx_len - 1) attends with one softmax to the compressed entries
+// j < n_c(t) and to the last `window` raw tokens, held in a ring of `window` slots.
+//
+// Design for sm_100a (HBM-bound: every key row is read once, ~63 flop per byte):
+//  * The hq <= 64 query heads of a sequence share its KV head, so they form the M = 64 rows
+//    of every UMMA. An M = 64 accumulator occupies TMEM lanes 0-15 of each 32-lane
+//    subpartition; a second one sits at lane offset 16. O (64 x 512 f32) takes lanes
+//    0-15 x 512 columns and the double-buffered scores (64 x 256 each) take lanes 16-31.
+//  * The key list (compressed tiles of up to 256 entries, then the ring tile) is cut into
+//    `nsplit` contiguous ranges; grid = (nsplit, sequences). Each CTA streams its K/V tiles
+//    through a 4-deep ring of 32 KB TMA chunks (256 rows x 64 elements, 128-byte swizzle),
+//    runs S = Q K^T (both operands in shared memory), a two-pass softmax per tile (max,
+//    then exp and the bf16 P written to shared memory in the UMMA K-major swizzled layout),
+//    and O += P V with V N-major.
+//  * Lazy rescaling as in prefill (reference moves when the max grows by more than 8 in
+//    log2 units). A rescale reads and writes whole 32-lane rows of TMEM, so it first waits
+//    until no UMMA is in flight.
+//  * Each CTA writes float32 partials (unnormalised O, reference m in log2 units, sum l) to
+//    the workspace; merge_kernel combines them per head, applies the gate and casts.
+//  * All mbarrier waits are bounded (HCA_ERR_TIMEOUT on give-up).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <string.h>
+
+#include "hca_internal.h"
+#include "sm100.cuh"
+#include "tmap.h"
+
+namespace hca {
+namespace {
+
+constexpr int kM = 64;                    // head rows
+constexpr int kD = 512;
+constexpr int kKC = 64;
+constexpr int kNCh = kD / kKC;            // 8
+constexpr int kTN = 256;                  // keys per compressed tile
+constexpr int kRingRows = 128;            // rows of the ring box (window <= 128)
+constexpr uint32_t kChunkBytes = kTN * kKC * 2;         // 32 KB
+constexpr uint32_t kHalfChunkBytes = 128 * kKC * 2;     // 16 KB
+constexpr uint32_t kQChunkBytes = kM * kKC * 2;         // 8 KB
+constexpr uint32_t kQBytes = kNCh * kQChunkBytes;       // 64 KB
+constexpr uint32_t kPChunkBytes = kM * kKC * 2;         // 8 KB (64 rows x 64 keys)
+constexpr uint32_t kPBytes = (kTN / kKC) * kPChunkBytes;  // 32 KB
+constexpr int kStages = 4;
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kLaneS = 16u << 16;   // lane offset of the score accumulator
+constexpr float kRescaleThreshold = 8.0f;
+
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffP = kQBytes;
+constexpr uint32_t kOffRing = kOffP + kPBytes;
+constexpr uint32_t kOffBar = kOffRing + kStages * kChunkBytes;
+constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
+
+enum { kCompressed = 0, kRing = 1 };
+
+struct Params {
+  CUtensorMap tmQ, tmKc, tmVc, tmRk, tmRv;
+  const int32_t* ctx_len;
+  const int32_t* page_table;
+  const int32_t* n_entries;
+  int32_t* err_word;
+  float* ws_ml;   // [nseq, nsplit, hq, 2]
+  float* ws_o;    // [nseq, nsplit, hq, 512]
+  int32_t nseq, hq, W, block, PE, max_pages, num_pages, nsplit;
+  float scale_log2;
+};
+
+struct Bars {
+  uint64_t q_full;
+  uint64_t ring_full[kStages], ring_empty[kStages];
+  uint64_t s_full[2], p_full;
+  uint64_t o_done, drain;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(Bars) <= 256, "barrier block too large");
+
+struct Seq {
+  int t, nc, nct, total, j0, j1;  // tiles [j0, j1) belong to this split
+};
+
+struct Tile {
+  int kind, key0, n;
+};
+
+__device__ __forceinline__ int round16(int x) { return (x + 15) & ~15; }
+
+__device__ __forceinline__ Seq make_seq(const Params& p, int b, int split) {
+  Seq s;
+  s.t = max(p.ctx_len[b] - 1, 0);
+  int x = s.t + 1 - p.W;
+  int nc = x < 0 ? 0 : x / p.block;
+  s.nc = min(nc, min(p.n_entries[b], p.max_pages * p.PE));
+  s.nct = (s.nc + kTN - 1) / kTN;
+  s.total = s.nct + 1;
+  const int tps = (s.total + p.nsplit - 1) / p.nsplit;
+  s.j0 = min(s.total, split * tps);
+  s.j1 = min(s.total, s.j0 + tps);
+  return s;
+}
+
+__device__ __forceinline__ Tile tile_of(const Params& p, const Seq& s, int j) {
+  Tile t;
+  if (j < s.nct) {
+    t.kind = kCompressed;
+    t.key0 = j * kTN;
+    t.n = min(kTN, round16(s.nc - j * kTN));
+  } else {
+    t.kind = kRing;
+    t.key0 = 0;
+    t.n = round16(p.W);
+  }
+  return t;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_constant__ Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sQ = smem + kOffQ;
+  uint8_t* sP = smem + kOffP;
+  uint8_t* sRing = smem + kOffRing;
+  Bars* bars = reinterpret_cast<Bars*>(smem + kOffBar);
+  volatile int* abort = &bars->abort;
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const int b = blockIdx.y;
+  const int split = blockIdx.x;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars->ring_full[s], 1);
+      mbar_init(&bars->ring_empty[s], 1);
+    }
+    mbar_init(&bars->s_full[0], 1);
+    mbar_init(&bars->s_full[1], 1);
+    mbar_init(&bars->p_full, 4);
+    mbar_init(&bars->o_done, 1);
+    mbar_init(&bars->drain, 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const Seq sq = make_seq(p, b, split);
+  const int ntiles = sq.j1 - sq.j0;
+
+  if (ntiles <= 0) {
+    // empty split: an all-zero partial that the merge skips
+    for (int h = threadIdx.x; h < p.hq; h += blockDim.x) {
+      float* ml = p.ws_ml + (((int64_t)b * p.nsplit + split) * p.hq + h) * 2;
+      ml[0] = -INFINITY;
+      ml[1] = 0.f;
+    }
+  } else if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (elect_one()) {
+      bool ok = true;
+      mbar_expect_tx(&bars->q_full, kQBytes);
+      for (int ch = 0; ch < kNCh; ++ch)
+        tma_load_2d(sQ + ch * kQChunkBytes, &p.tmQ, &bars->q_full, ch * kKC, b * p.hq);
+      uint32_t cnt = 0;
+      auto load_tile = [&](int j, bool is_v) -> bool {
+        const Tile t = tile_of(p, sq, j);
+        for (int ch = 0; ch < kNCh; ++ch) {
+          const uint32_t s = cnt % kStages;
+          const uint32_t round = cnt / kStages;
+          if (round > 0 && !mbar_wait(&bars->ring_empty[s], (round - 1) & 1, abort)) return false;
+          uint8_t* dst = sRing + s * kChunkBytes;
+          if (t.kind == kCompressed) {
+            const int halves = t.key0 + 128 < sq.nc ? 2 : 1;
+            mbar_expect_tx(&bars->ring_full[s], halves * kHalfChunkBytes);
+            for (int hh = 0; hh < halves; ++hh) {
+              const int e = t.key0 + hh * 128;
+              int page = p.page_table[(int64_t)b * p.max_pages + e / p.PE];
+              if (page < 0 || page >= p.num_pages) {
+                if (p.err_word) atomicOr(p.err_word, kErrPageRange);
+                page = 0;
+              }
+              tma_load_2d(dst + hh * kHalfChunkBytes, is_v ? &p.tmVc : &p.tmKc,
+                          &bars->ring_full[s], ch * kKC, page * p.PE + e % p.PE);
+            }
+          } else {
+            mbar_expect_tx(&bars->ring_full[s], kHalfChunkBytes);
+            tma_load_2d(dst, is_v ? &p.tmRv : &p.tmRk, &bars->ring_full[s], ch * kKC, b * p.W);
+          }
+          ++cnt;
+        }
+        return true;
+      };
+      for (int j = 0; j < ntiles && ok; ++j) {
+        ok = load_tile(sq.j0 + j, false);
+        if (ok && j >= 1) ok = load_tile(sq.j0 + j - 1, true);
+      }
+      if (ok) ok = load_tile(sq.j0 + ntiles - 1, true);
+      if (!ok) {
+        bars->abort = 1;
+        if (p.err_word) atomicOr(p.err_word, kErrTimeout);
+        volatile int no_abort = 0;
+        const uint32_t first = cnt > kStages ? cnt - kStages : 0;
+        for (uint32_t q = first; q < cnt; ++q)
+          mbar_wait(&bars->ring_full[q % kStages], (q / kStages) & 1, &no_abort, 100000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ UMMA issuer
+    if (elect_one()) {
+      bool ok = mbar_wait(&bars->q_full, 0, abort);
+      tc_fence_after();
+      uint32_t cnt = 0;
+      const uint32_t qbase = smem_u32(sQ);
+      const uint32_t pbase = smem_u32(sP);
+      const uint32_t rbase = smem_u32(sRing);
+      auto issue_s = [&](int j) -> bool {
+        const Tile t = tile_of(p, sq, sq.j0 + j);
+        const uint32_t sb = j & 1;
+        const uint32_t d_tmem = tmem + kLaneS + sb * kTN;
+        const uint32_t idesc = idesc_bf16_f32(kM, t.n, false);
+        for (int ch = 0; ch < kNCh; ++ch) {
+          const uint32_t s = cnt % kStages;
+          if (!mbar_wait(&bars->ring_full[s], (cnt / kStages) & 1, abort)) return false;
+          tc_fence_after();
+          const uint32_t kaddr = rbase + s * kChunkBytes;
+          const uint32_t qaddr = qbase + ch * kQChunkBytes;
+#pragma unroll
+          for (int kk = 0; kk < kKC / 16; ++kk)
+            umma_ss(d_tmem, sdesc_sw128(qaddr + kk * 32, 16, 1024),
+                    sdesc_sw128(kaddr + kk * 32, 16, 1024), idesc, (ch | kk) != 0);
+          umma_commit(&bars->ring_empty[s]);
+          ++cnt;
+        }
+        umma_commit(&bars->s_full[sb]);
+        return true;
+      };
+      auto issue_pv = [&](int j) -> bool {
+        const Tile t = tile_of(p, sq, sq.j0 + j);
+        if (!mbar_wait(&bars->p_full, j & 1, abort)) return false;
+        tc_fence_after();
+        const uint32_t idesc = idesc_bf16_f32(kM, kKC, true);
+        for (int ch = 0; ch < kNCh; ++ch) {
+          const uint32_t s = cnt % kStages;
+          if (!mbar_wait(&bars->ring_full[s], (cnt / kStages) & 1, abort)) return false;
+          tc_fence_after();
+          const uint32_t vaddr = rbase + s * kChunkBytes;
+          for (int kk = 0; kk < t.n / 16; ++kk) {
+            const uint32_t paddr = pbase + (kk >> 2) * kPChunkBytes + (kk & 3) * 32;
+            umma_ss(tmem + ch * kKC, sdesc_sw128(paddr, 16, 1024),
+                    sdesc_sw128(vaddr + kk * 2048, kChunkBytes, 1024), idesc, (j > 0 || kk > 0));
+          }
+          umma_commit(&bars->ring_empty[s]);
+          ++cnt;
+        }
+        umma_commit(&bars->o_done);
+        return true;
+      };
+      for (int j = 0; j < ntiles && ok; ++j) {
+        ok = issue_s(j);
+        if (ok && j >= 1) ok = issue_pv(j - 1);
+      }
+      if (ok) ok = issue_pv(ntiles - 1);
+      if (!ok) {
+        bars->abort = 1;
+        if (p.err_word) atomicOr(p.err_word, kErrTimeout);
+      }
+      volatile int no_abort = 0;
+      umma_commit(&bars->drain);
+      mbar_wait(&bars->drain, 0, &no_abort, 100000000ull);
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax + partials
+    const int quad = warp & 3;
+    const bool s_lane = lane >= 16;           // this thread holds a score row
+    const int hrow = quad * 16 + (lane & 15);  // head row of both the score and O lanes
+    const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+    const int t = sq.t;
+    const int W = p.W;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < ntiles && ok; ++j) {
+      const Tile tl = tile_of(p, sq, sq.j0 + j);
+      const uint32_t sb = j & 1;
+      if (!(ok = mbar_wait(&bars->s_full[sb], (j >> 1) & 1, abort))) break;
+      tc_fence_after();
+      const uint32_t s_addr = tmem + lane_addr + sb * kTN;  // lanes 16-31 hold the scores
+      auto valid = [&](int col) -> bool {
+        if (col >= tl.n) return false;
+        if (tl.kind == kCompressed) return tl.key0 + col < sq.nc;
+        return col < W && (t >= W - 1 || col <= t);
+      };
+      // pass 1: row max
+      float mt = -INFINITY;
+      for (int q = 0; q < kTN / 32; ++q) {
+        if (q * 32 >= tl.n) break;
+        uint32_t v[32];
+        tmem_ld32(s_addr + q * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          if (valid(q * 32 + e)) mt = fmaxf(mt, __uint_as_float(v[e]) * p.scale_log2);
+      }
+      const float mn = fmaxf(m, mt);
+      float ref = m, alpha = 1.f;
+      bool rescale = false;
+      if (m == -INFINITY) {
+        ref = mn;
+      } else if (mn > m + kRescaleThreshold) {
+        ref = mn;
+        alpha = fast_exp2(m - mn);
+        rescale = true;
+      }
+      if (!s_lane) rescale = false;
+      const float base = ref == -INFINITY ? 0.f : ref;
+      // P of the previous tile must have been consumed before P is overwritten
+      if (j > 0) {
+        if (!(ok = mbar_wait(&bars->o_done, (j - 1) & 1, abort))) break;
+        tc_fence_after();
+      }
+      if (__any_sync(0xffffffffu, rescale)) {
+        // no UMMA may write TMEM during the read-modify-write of whole lanes
+        if (j + 1 < ntiles && !(ok = mbar_wait(&bars->s_full[sb ^ 1], ((j + 1) >> 1) & 1, abort)))
+          break;
+        tc_fence_after();
+        const float a_o = __shfl_sync(0xffffffffu, alpha, (lane & 15) + 16);
+        const float a_me = s_lane ? 1.f : a_o;
+#pragma unroll 1
+        for (int q = 0; q < kD / 32; ++q) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_addr + q * 32, v);
+          tmem_wait_ld();
+          if (!s_lane) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * a_me);
+          }
+          tmem_st32(tmem + lane_addr + q * 32, v);
+        }
+        tmem_wait_st();
+      }
+      // pass 2: P = exp2(s - ref) -> bf16, K-major 128B-swizzled rows of sP
+      float psum = 0.f;
+      for (int q = 0; q < kTN / 32; ++q) {
+        if (q * 32 >= tl.n) break;
+        uint32_t v[32];
+        tmem_ld32(s_addr + q * 32, v);
+        tmem_wait_ld();
+        if (s_lane) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int c0 = q * 32 + 2 * e;
+            const float x0 = valid(c0) ? __uint_as_float(v[2 * e]) * p.scale_log2 : -INFINITY;
+            const float x1 =
+                valid(c0 + 1) ? __uint_as_float(v[2 * e + 1]) * p.scale_log2 : -INFINITY;
+            pk[e] = pack_bf16x2(fast_exp2(x0 - base), fast_exp2(x1 - base));
+            const float2 f2 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&pk[e]));
+            psum += f2.x + f2.y;
+          }
+          // keys q*32 .. q*32+31 -> chunk (q/2), 16-byte units u = (q&1)*4 + w
+          uint8_t* rowp = sP + (q >> 1) * kPChunkBytes + hrow * 128;
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const int u = (q & 1) * 4 + w;
+            const int us = u ^ (hrow & 7);
+            *reinterpret_cast<uint4*>(rowp + us * 16) =
+                make_uint4(pk[4 * w], pk[4 * w + 1], pk[4 * w + 2], pk[4 * w + 3]);
+          }
+        }
+      }
+      l = l * alpha + psum;
+      m = ref;
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->p_full);
+    }
+    if (ok) ok = mbar_wait(&bars->o_done, (ntiles - 1) & 1, abort);
+    if (ok) {
+      tc_fence_after();
+      const float m_o = __shfl_sync(0xffffffffu, m, (lane & 15) + 16);
+      const float l_o = __shfl_sync(0xffffffffu, l, (lane & 15) + 16);
+      const bool store = !s_lane && hrow < p.hq;
+      const int64_t slot = ((int64_t)b * p.nsplit + split) * p.hq + hrow;
+      float* op = p.ws_o + slot * kD;
+#pragma unroll 1
+      for (int q = 0; q < kD / 32; ++q) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_addr + q * 32, v);
+        tmem_wait_ld();
+        if (store) {
+          float4* o4 = reinterpret_cast<float4*>(op + q * 32);
+#pragma unroll
+          for (int w = 0; w < 8; ++w)
+            o4[w] = make_float4(__uint_as_float(v[4 * w]), __uint_as_float(v[4 * w + 1]),
+                                __uint_as_float(v[4 * w + 2]), __uint_as_float(v[4 * w + 3]));
+        }
+      }
+      if (store) {
+        p.ws_ml[slot * 2] = m_o;
+        p.ws_ml[slot * 2 + 1] = l_o;
+      }
+    } else {
+      bars->abort = 1;
+      if (p.err_word) atomicOr(p.err_word, kErrTimeout);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Combine the split partials of one sequence: per head, O = sum_s 2^(m_s - M) O_s /
+// sum_s 2^(m_s - M) l_s, then the gate and the cast to bf16; lse in natural log.
+__global__ void __launch_bounds__(256) merge_kernel(const float* ws_ml, const float* ws_o,
+                                                    int nsplit, int hq,
+                                                    const __nv_bfloat16* gate, int64_t gs0,
+                                                    int64_t gs2, __nv_bfloat16* O, float* lse) {
+  const int b = blockIdx.y;
+  const int h = blockIdx.x;
+  const int d = threadIdx.x * 2;
+  const float* ml = ws_ml + ((int64_t)b * nsplit * hq + h) * 2;
+  float M = -INFINITY;
+  for (int s = 0; s < nsplit; ++s) {
+    const float ms = ml[(int64_t)s * hq * 2];
+    const float ls = ml[(int64_t)s * hq * 2 + 1];
+    if (ls > 0.f) M = fmaxf(M, ms);
+  }
+  float L = 0.f, o0 = 0.f, o1 = 0.f;
+  for (int s = 0; s < nsplit; ++s) {
+    const float ms = ml[(int64_t)s * hq * 2];
+    const float ls = ml[(int64_t)s * hq * 2 + 1];
+    if (!(ls > 0.f)) continue;
+    const float w = exp2f(ms - M);
+    L += w * ls;
+    const float2 ov = *reinterpret_cast<const float2*>(
+        ws_o + (((int64_t)b * nsplit + s) * hq + h) * kD + d);
+    o0 += w * ov.x;
+    o1 += w * ov.y;
+  }
+  const float inv = 1.f / L;
+  o0 *= inv;
+  o1 *= inv;
+  if (gate) {
+    const float2 g = __bfloat1622float2(
+        *reinterpret_cast<const __nv_bfloat162*>(gate + (int64_t)b * gs0 + (int64_t)h * gs2 + d));
+    o0 *= g.x;
+    o1 *= g.y;
+  }
+  *reinterpret_cast<uint32_t*>(O + ((int64_t)b * hq + h) * kD + d) = pack_bf16x2(o0, o1);
+  if (lse && threadIdx.x == 0) lse[(int64_t)b * hq + h] = (M + __log2f(L)) * 0.69314718055994531f;
+}
+
+}  // namespace
+
+bool decode_tc_supported(const hca_desc& d, const hca_cache& c) {
+  if (d.dtype != HCA_BF16 || d.head_dim != kD || d.hkv != 1) return false;
+  if (d.hq < 1 || d.hq > kM) return false;
+  if (d.window < 1 || d.window > kRingRows || d.block < 1) return false;
+  if (c.page_entries % 128 != 0) return false;
+  if (d.gate) {
+    const uintptr_t ga = reinterpret_cast<uintptr_t>(d.gate);
+    if (ga % 4 || d.gate_strides[0] % 2 || d.gate_strides[2] % 2) return false;
+  }
+  return true;
+}
+
+int decode_num_splits(const hca_desc& d) {
+  const int64_t x = (int64_t)d.seqlen - d.window;
+  const int64_t nc = x < 0 ? 0 : x / d.block;
+  const int tiles = (int)((nc + kTN - 1) / kTN) + 1;
+  if (d.decode_splits > 0) return d.decode_splits < tiles ? d.decode_splits : tiles;
+  const int sms = device_sm_count();
+  int s = d.batch >= sms ? 1 : (2 * sms + d.batch / 2) / (d.batch > 0 ? d.batch : 1);
+  if (d.batch < sms && d.batch * 2 > sms) s = 2;
+  if (d.batch <= sms / 2) s = sms / (d.batch > 0 ? d.batch : 1);
+  if (s < 1) s = 1;
+  if (s > tiles) s = tiles;
+  return s;
+}
+
+size_t decode_tc_workspace_bytes(const hca_desc& d) {
+  const size_t ns = (size_t)decode_num_splits(d);
+  return (size_t)d.batch * ns * d.hq * (kD + 2) * sizeof(float);
+}
+
+cudaError_t launch_decode_tc(const hca_desc& d, const void* Q, const int32_t* ctx_len,
+                             const hca_cache& c, const void* ring_k, const void* ring_v,
+                             void* O, float* lse, void* ws, cudaStream_t s) {
+  Params p;
+  memset(&p, 0, sizeof(p));
+  const int nsplit = decode_num_splits(d);
+  cudaError_t e;
+  const uint64_t rowsC = (uint64_t)c.num_pages * c.page_entries;
+  if ((e = encode_bf16_rows(&p.tmQ, Q, (uint64_t)d.batch * d.hq, kD, kKC, kM)) != cudaSuccess)
+    return e;
+  if ((e = encode_bf16_rows(&p.tmKc, c.kc_pool, rowsC, kD, kKC, 128)) != cudaSuccess) return e;
+  if ((e = encode_bf16_rows(&p.tmVc, c.vc_pool, rowsC, kD, kKC, 128)) != cudaSuccess) return e;
+  const uint64_t rowsR = (uint64_t)d.batch * d.window;
+  if ((e = encode_bf16_rows(&p.tmRk, ring_k, rowsR, kD, kKC, kRingRows)) != cudaSuccess) return e;
+  if ((e = encode_bf16_rows(&p.tmRv, ring_v, rowsR, kD, kKC, kRingRows)) != cudaSuccess) return e;
+  p.ctx_len = ctx_len;
+  p.page_table = c.page_table;
+  p.n_entries = c.n_entries;
+  p.err_word = c.err_word;
+  p.ws_ml = static_cast<float*>(ws);
+  p.ws_o = p.ws_ml + (size_t)d.batch * nsplit * d.hq * 2;
+  p.nseq = d.batch;
+  p.hq = d.hq;
+  p.W = d.window;
+  p.block = d.block;
+  p.PE = c.page_entries;
+  p.max_pages = c.max_pages;
+  p.num_pages = c.num_pages;
+  p.nsplit = nsplit;
+  p.scale_log2 = d.scale * 1.4426950408889634f;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  dim3 grid(nsplit, d.batch);
+  decode_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  dim3 mgrid(d.hq, d.batch);
+  merge_kernel<<<mgrid, kD / 2, 0, s>>>(p.ws_ml, p.ws_o, nsplit, d.hq,
+                                        static_cast<const __nv_bfloat16*>(d.gate),
+                                        d.gate_strides[0], d.gate_strides[2],
+                                        static_cast<__nv_bfloat16*>(O), lse);
+  return cudaGetLastError();
+}
+
+}  // namespace hca

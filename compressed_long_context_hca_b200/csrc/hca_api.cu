@@ -1,0 +1,188 @@
+// hca_api.cu -- the exported C ABI of libhca (see include/hca.h for the contract).
+//
+// Host code only: argument validation, choice of kernel by dtype, launch on the caller's
+// stream. Nothing here allocates device memory or keeps state between calls (apart from
+// per-device caches of the SM count and of kernel attributes).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "hca_internal.h"
+#include "tmap.h"
+
+namespace hca {
+
+int device_sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    n = 148;
+  if (dev >= 0 && dev < 64) cache[dev] = n;
+  return n;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn) return fn;
+  void* ptr = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+          cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  return fn;
+}
+
+cudaError_t encode_bf16_rows(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                             uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  if (rows == 0) rows = 1;  // a map needs a non-empty extent; nothing reads past the data
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+}  // namespace hca
+
+using namespace hca;
+
+namespace {
+
+int32_t from_cuda(cudaError_t e) { return e == cudaSuccess ? HCA_OK : HCA_ECUDA; }
+
+int32_t check_desc(const hca_desc* d) {
+  if (!d) return HCA_EINVAL;
+  if (d->batch < 0 || d->seqlen < 0 || d->hq < 1 || d->hkv < 1 || d->head_dim < 1 ||
+      d->block < 1 || d->window < 1 || d->decode_splits < 0)
+    return HCA_EINVAL;
+  if (d->hq % d->hkv != 0) return HCA_EINVAL;
+  if (d->dtype != HCA_BF16 && d->dtype != HCA_F32) return HCA_EUNSUPPORTED;
+  if (!(d->scale == d->scale)) return HCA_EINVAL;  // NaN
+  return HCA_OK;
+}
+
+int32_t check_cache(const hca_cache* c) {
+  if (!c || !c->kc_pool || !c->vc_pool || !c->page_table || !c->n_entries) return HCA_EINVAL;
+  if (c->page_entries < 1 || c->max_pages < 1 || c->num_pages < 1) return HCA_EINVAL;
+  return HCA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+int32_t hca_abi_version(void) { return HCA_ABI_VERSION; }
+
+const char* hca_status_string(int32_t status) {
+  switch (status) {
+    case HCA_OK: return "HCA_OK";
+    case HCA_EINVAL: return "HCA_EINVAL: invalid argument";
+    case HCA_EUNSUPPORTED: return "HCA_EUNSUPPORTED: no kernel for this shape/dtype";
+    case HCA_ENOSPACE: return "HCA_ENOSPACE: cache or workspace too small";
+    case HCA_ECUDA: return "HCA_ECUDA: CUDA call failed";
+    default: return "HCA: unknown status";
+  }
+}
+
+int32_t hca_set_gate(hca_desc* d, const void* gate, const int64_t* strides) {
+  if (!d) return HCA_EINVAL;
+  if (gate && !strides) return HCA_EINVAL;
+  d->gate = gate;
+  for (int i = 0; i < 3; ++i) d->gate_strides[i] = gate ? strides[i] : 0;
+  return HCA_OK;
+}
+
+int32_t hca_compress(const hca_desc* d, const void* K, const void* V,
+                     int64_t batch_stride_tokens, int32_t first_block, int32_t n_blocks,
+                     const hca_cache* cache, hca_stream_t stream) {
+  int32_t st = check_desc(d);
+  if (st != HCA_OK) return st;
+  if ((st = check_cache(cache)) != HCA_OK) return st;
+  if (first_block < 0 || n_blocks < 0 || batch_stride_tokens < 0) return HCA_EINVAL;
+  if (n_blocks == 0 || d->batch == 0) return HCA_OK;
+  if (!K || !V) return HCA_EINVAL;
+  if ((int64_t)(first_block + n_blocks - 1) * d->block >= d->seqlen) return HCA_EINVAL;
+  if ((int64_t)first_block + n_blocks > (int64_t)cache->max_pages * cache->page_entries)
+    return HCA_ENOSPACE;
+  if (d->head_dim % 8 != 0) return HCA_EUNSUPPORTED;
+  const int esize = d->dtype == HCA_BF16 ? 2 : 4;
+  if (((int64_t)d->hkv * d->head_dim * esize) % 16 != 0) return HCA_EUNSUPPORTED;
+  if (!aligned16(K) || !aligned16(V) || !aligned16(cache->kc_pool) ||
+      !aligned16(cache->vc_pool))
+    return HCA_EINVAL;
+  return from_cuda(launch_compress(*d, K, V, batch_stride_tokens, first_block, n_blocks, *cache,
+                                   reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int32_t hca_attn_prefill(const hca_desc* d, const void* Q, const void* K, const void* V,
+                         const hca_cache* cache, void* O, float* lse, int32_t* dbg_mask,
+                         hca_stream_t stream) {
+  int32_t st = check_desc(d);
+  if (st != HCA_OK) return st;
+  if ((st = check_cache(cache)) != HCA_OK) return st;
+  if (d->batch == 0 || d->seqlen == 0) return HCA_OK;
+  if (!Q || !K || !V || !O) return HCA_EINVAL;
+  if (d->gate && (d->gate_strides[0] < 0 || d->gate_strides[1] < 0 || d->gate_strides[2] < 0))
+    return HCA_EINVAL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d->dtype == HCA_F32) {
+    if (d->head_dim % 32 != 0 || d->head_dim > 512) return HCA_EUNSUPPORTED;
+    return from_cuda(launch_prefill_simt(*d, Q, K, V, *cache, O, lse, dbg_mask, s));
+  }
+  if (!prefill_tc_supported(*d, *cache)) return HCA_EUNSUPPORTED;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) ||
+      !aligned16(cache->kc_pool) || !aligned16(cache->vc_pool))
+    return HCA_EINVAL;
+  return from_cuda(launch_prefill_tc(*d, Q, K, V, *cache, O, lse, dbg_mask, s));
+}
+
+size_t hca_decode_workspace_bytes(const hca_desc* d) {
+  if (check_desc(d) != HCA_OK) return 0;
+  if (d->dtype != HCA_BF16) return 0;
+  return decode_tc_workspace_bytes(*d);
+}
+
+int32_t hca_attn_decode(const hca_desc* d, const void* Q, const int32_t* ctx_len,
+                        const hca_cache* cache, const void* ring_k, const void* ring_v,
+                        void* O, float* lse, void* workspace, size_t workspace_bytes,
+                        hca_stream_t stream) {
+  int32_t st = check_desc(d);
+  if (st != HCA_OK) return st;
+  if ((st = check_cache(cache)) != HCA_OK) return st;
+  if (d->batch == 0) return HCA_OK;
+  if (!Q || !ctx_len || !ring_k || !ring_v || !O) return HCA_EINVAL;
+  if (d->seqlen < 1) return HCA_EINVAL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d->dtype == HCA_F32) {
+    if (d->head_dim % 32 != 0 || d->head_dim > 512) return HCA_EUNSUPPORTED;
+    return from_cuda(launch_decode_simt(*d, Q, ctx_len, *cache, ring_k, ring_v, O, lse, s));
+  }
+  if (!decode_tc_supported(*d, *cache)) return HCA_EUNSUPPORTED;
+  const size_t need = decode_tc_workspace_bytes(*d);
+  if (!workspace || workspace_bytes < need) return HCA_ENOSPACE;
+  if (!aligned16(Q) || !aligned16(ring_k) || !aligned16(ring_v) || !aligned16(O) ||
+      !aligned16(workspace) || !aligned16(cache->kc_pool) || !aligned16(cache->vc_pool))
+    return HCA_EINVAL;
+  return from_cuda(
+      launch_decode_tc(*d, Q, ctx_len, *cache, ring_k, ring_v, O, lse, workspace, s));
+}
+
+}  // extern "C"

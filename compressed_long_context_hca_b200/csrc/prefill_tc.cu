@@ -1,0 +1,602 @@
+// prefill_tc.cu -- HCA prefill attention on tcgen05 tensor cores (bf16 in, f32 accumulate).
+//
+// Operation ([news 二.1] / [analysis 1] / [gate] in include/hca.h): every query position t
+// attends with one softmax to the compressed entries j < n_c(t) (blocks that end before its
+// window) and to the raw tokens max(0, t-W+1) .. t, head_dim 512; the output is optionally
+// multiplied by a supplied gate.
+//
+// Design for sm_100a:
+//  * A tile is 128 rows = (128 / hq) consecutive positions x hq query heads. All rows share
+//    the single KV head, so one K/V tile in shared memory serves 128 rows.
+//  * head_dim 512 in float32 would fill all 512 TMEM columns for 128 rows, leaving no room
+//    for scores. Each CTA therefore owns one 256-wide half of the output: TMEM holds the
+//    output half (256 columns) and two 128-column score buffers. Both halves compute the
+//    full scores (the price of the split: 1.5x tensor work; a later design removes it).
+//  * Q (128 x 512 bf16, 128 KB) stays in shared memory for the tile; K and V stream through
+//    a ring of 16 KB TMA chunks (128 rows x 64 elements, 128-byte swizzle).
+//  * Warp roles: warp 0 issues TMA, warp 1 issues UMMA (single thread), warps 2-5 run the
+//    online softmax (one row per thread, TMEM lane = row) and the epilogue.
+//  * S = Q K^T runs as kind::f16 with both operands in shared memory; P is rounded to bf16
+//    and written back into the score columns of TMEM, and O += P V runs with A from TMEM
+//    and V (N-major) from shared memory.
+//  * The key list of a tile is: compressed tiles of up to 128 entries (the last one cut to
+//    a multiple of 16), an optional 16-row raw tile for the keys that only the first
+//    position of the tile still sees, then one 128-row raw tile ending at the last position.
+//  * Online softmax in base 2 with lazy rescaling: the running reference only moves when
+//    the row max grows by more than 8 (a factor of 256), so O is rarely touched.
+//  * Persistent grid, one CTA per SM, work items (tile, half) in decreasing-work order and
+//    handed out in a snake so that every CTA gets a similar share.
+//  * Every mbarrier wait is bounded; on time-out the CTA raises HCA_ERR_TIMEOUT (4) in the
+//    error word and unwinds, releasing its TMEM.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <string.h>
+
+#include "hca_internal.h"
+#include "sm100.cuh"
+#include "tmap.h"
+
+namespace hca {
+namespace {
+
+constexpr int kBM = 128;               // rows per tile
+constexpr int kD = 512;                // head_dim
+constexpr int kDH = 256;               // output half per CTA
+constexpr int kKC = 64;                // elements per 128-byte swizzle row
+constexpr int kNCh = kD / kKC;         // 8 chunks of Q / K
+constexpr int kNVCh = kDH / kKC;       // 4 chunks of V per half
+constexpr int kBN = 128;               // max keys per tile
+constexpr uint32_t kChunkBytes = kBN * kKC * 2;   // 16 KB
+constexpr uint32_t kChunk16Bytes = 16 * kKC * 2;  // 2 KB
+constexpr int kStages = 5;
+constexpr uint32_t kQBytes = kNCh * kBM * kKC * 2;  // 128 KB
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmS0 = 0, kTmO = 256;
+constexpr int kThreads = 192;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+enum TileKind { kCompressed = 0, kRaw16 = 1, kRaw128 = 2 };
+
+struct Params {
+  CUtensorMap tmQ, tmK, tmV, tmK16, tmV16, tmKc, tmVc;
+  __nv_bfloat16* O;
+  float* lse;
+  int32_t* dbg;
+  const __nv_bfloat16* gate;
+  int64_t gs0, gs1, gs2;
+  const int32_t* page_table;
+  const int32_t* n_entries;
+  int32_t* err_word;
+  int32_t batch, T, hq, P, W, block, PE, max_pages, num_pages;
+  int32_t n_rt;     // row tiles per sequence
+  int32_t n_items;  // 2 * batch * n_rt
+  float scale_log2;
+};
+
+struct Item {
+  int b, i, half;
+  int t0, tl;       // first / last valid position of the tile
+  int nc_last;      // compressed entries visible to the last position (clamped)
+  int nct;          // compressed tiles
+  int lo, hi;       // raw key range of the tile
+  int rawA_n;       // keys used from the 128-row raw tile
+  int strag;        // 1 if the 16-row raw tile exists
+  int ntiles;
+};
+
+struct Tile {
+  int kind;
+  int n;       // keys (MMA N), multiple of 16
+  int rowoff;  // first used row inside the loaded box
+  int key0;    // compressed: first entry; raw: token of the first used row
+};
+
+__device__ __forceinline__ int round16(int x) { return (x + 15) & ~15; }
+
+__device__ __forceinline__ int visible_count(int t, int block, int W) {
+  const int x = t + 1 - W;
+  return x < 0 ? 0 : x / block;
+}
+
+__device__ __forceinline__ Item make_item(const Params& p, int k) {
+  Item it;
+  it.half = k & 1;
+  const int rt = k >> 1;
+  it.b = rt % p.batch;
+  it.i = p.n_rt - 1 - rt / p.batch;  // heaviest tiles first
+  it.t0 = it.i * p.P;
+  it.tl = min(it.t0 + p.P - 1, p.T - 1);
+  // never trust the device count beyond what the page table can address
+  const int have = min(p.n_entries[it.b], p.max_pages * p.PE);
+  it.nc_last = min(visible_count(it.tl, p.block, p.W), have);
+  it.nct = (it.nc_last + kBN - 1) / kBN;
+  it.lo = max(0, it.t0 - p.W + 1);
+  it.hi = it.tl;
+  const int R = it.hi - it.lo + 1;
+  it.rawA_n = min(kBN, round16(min(R, kBN)));
+  it.strag = R > kBN ? 1 : 0;
+  it.ntiles = it.nct + it.strag + 1;
+  return it;
+}
+
+__device__ __forceinline__ Tile tile_of(const Item& it, int j) {
+  Tile t;
+  if (j < it.nct) {
+    t.kind = kCompressed;
+    t.key0 = j * kBN;
+    t.n = min(kBN, round16(it.nc_last - j * kBN));
+    t.rowoff = 0;
+  } else if (it.strag && j == it.nct) {
+    t.kind = kRaw16;
+    t.key0 = it.hi - 143;
+    t.n = 16;
+    t.rowoff = 0;
+  } else {
+    t.kind = kRaw128;
+    t.n = it.rawA_n;
+    t.rowoff = kBN - it.rawA_n;
+    t.key0 = it.hi - kBN + 1 + t.rowoff;
+  }
+  return t;
+}
+
+// Shared-memory carve-up (offsets from a 1024-byte aligned base).
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffRing = kQBytes;
+constexpr uint32_t kOffBar = kOffRing + kStages * kChunkBytes;
+constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // + barriers + alignment slack
+
+struct Bars {
+  uint64_t q_full, q_empty;
+  uint64_t ring_full[kStages], ring_empty[kStages];
+  uint64_t s_full[2], p_full[2];
+  uint64_t o_done, o_free, drain;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(Bars) <= 256, "barrier block too large");
+
+__device__ __forceinline__ void raise_timeout(const Params& p, Bars* bars) {
+  bars->abort = 1;
+  if (p.err_word) atomicOr(p.err_word, kErrTimeout);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_constant__ Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sQ = smem + kOffQ;
+  uint8_t* sRing = smem + kOffRing;
+  Bars* bars = reinterpret_cast<Bars*>(smem + kOffBar);
+  volatile int* abort = &bars->abort;
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->q_empty, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars->ring_full[s], 1);
+      mbar_init(&bars->ring_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars->s_full[s], 1);
+      mbar_init(&bars->p_full[s], 4);
+    }
+    mbar_init(&bars->o_done, 1);
+    mbar_init(&bars->o_free, 4);
+    mbar_init(&bars->drain, 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&p.tmQ);
+    tma_prefetch_desc(&p.tmK);
+    tma_prefetch_desc(&p.tmV);
+    tma_prefetch_desc(&p.tmK16);
+    tma_prefetch_desc(&p.tmV16);
+    tma_prefetch_desc(&p.tmKc);
+    tma_prefetch_desc(&p.tmVc);
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const int G = gridDim.x;
+  const int c = blockIdx.x;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (elect_one()) {
+      uint32_t cnt = 0;  // ring loads issued
+      int nitem = 0;
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int k = r * G + ((r & 1) ? (G - 1 - c) : c);
+        if (k >= p.n_items) break;
+        const Item it = make_item(p, k);
+        // Q tile
+        if (nitem > 0 && !(ok = mbar_wait(&bars->q_empty, (nitem - 1) & 1, abort))) break;
+        mbar_expect_tx(&bars->q_full, kQBytes);
+        const int qrow = (it.b * p.T + it.t0) * p.hq;
+        for (int ch = 0; ch < kNCh; ++ch)
+          tma_load_2d(sQ + ch * (kBM * kKC * 2), &p.tmQ, &bars->q_full, ch * kKC, qrow);
+        // ring, in the order the MMA warp consumes it: K0, K1, V0, K2, V1, ..., V(n-1)
+        auto load_tile = [&](int j, bool is_v) -> bool {
+          const Tile t = tile_of(it, j);
+          const int nch = is_v ? kNVCh : kNCh;
+          for (int ch = 0; ch < nch; ++ch) {
+            const uint32_t s = cnt % kStages;
+            const uint32_t round = cnt / kStages;
+            if (round > 0 && !mbar_wait(&bars->ring_empty[s], (round - 1) & 1, abort)) return false;
+            const int x = is_v ? it.half * kDH + ch * kKC : ch * kKC;
+            uint8_t* dst = sRing + s * kChunkBytes;
+            if (t.kind == kCompressed) {
+              int page = p.page_table[(int64_t)it.b * p.max_pages + t.key0 / p.PE];
+              if (page < 0 || page >= p.num_pages) {
+                if (p.err_word) atomicOr(p.err_word, kErrPageRange);
+                page = 0;
+              }
+              const int y = page * p.PE + (t.key0 % p.PE);
+              mbar_expect_tx(&bars->ring_full[s], kChunkBytes);
+              tma_load_2d(dst, is_v ? &p.tmVc : &p.tmKc, &bars->ring_full[s], x, y);
+            } else if (t.kind == kRaw16) {
+              mbar_expect_tx(&bars->ring_full[s], kChunk16Bytes);
+              tma_load_2d(dst, is_v ? &p.tmV16 : &p.tmK16, &bars->ring_full[s], x,
+                          it.b * p.T + t.key0);
+            } else {
+              mbar_expect_tx(&bars->ring_full[s], kChunkBytes);
+              tma_load_2d(dst, is_v ? &p.tmV : &p.tmK, &bars->ring_full[s], x,
+                          it.b * p.T + it.hi - kBN + 1);
+            }
+            ++cnt;
+          }
+          return true;
+        };
+        for (int j = 0; j < it.ntiles && ok; ++j) {
+          ok = load_tile(j, false);
+          if (ok && j >= 1) ok = load_tile(j - 1, true);
+        }
+        if (ok) ok = load_tile(it.ntiles - 1, true);
+        ++nitem;
+      }
+      if (!ok) {
+        raise_timeout(p, bars);
+        // let loads already in flight land before the CTA's shared memory goes away
+        volatile int no_abort = 0;
+        const uint32_t first = cnt > kStages ? cnt - kStages : 0;
+        for (uint32_t q = first; q < cnt; ++q)
+          mbar_wait(&bars->ring_full[q % kStages], (q / kStages) & 1, &no_abort, 100000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ UMMA issuer
+    if (elect_one()) {
+      uint32_t cnt = 0;   // ring chunks consumed
+      uint32_t g = 0;     // tiles processed (score buffer / phase counter)
+      int nitem = 0;
+      bool ok = true;
+      const uint32_t qbase = smem_u32(sQ);
+      const uint32_t rbase = smem_u32(sRing);
+      for (int r = 0; ok; ++r) {
+        const int k = r * G + ((r & 1) ? (G - 1 - c) : c);
+        if (k >= p.n_items) break;
+        const Item it = make_item(p, k);
+        if (!(ok = mbar_wait(&bars->q_full, nitem & 1, abort))) break;
+        tc_fence_after();
+
+        auto issue_s = [&](int j) -> bool {
+          const Tile t = tile_of(it, j);
+          const uint32_t sb = (g + j) & 1;
+          const uint32_t d_tmem = tmem + kTmS0 + sb * 128;
+          const uint32_t idesc = idesc_bf16_f32(kBM, t.n, false);
+          for (int ch = 0; ch < kNCh; ++ch) {
+            const uint32_t s = cnt % kStages;
+            if (!mbar_wait(&bars->ring_full[s], (cnt / kStages) & 1, abort)) return false;
+            tc_fence_after();
+            const uint32_t kaddr = rbase + s * kChunkBytes + t.rowoff * 128;
+            const uint32_t qaddr = qbase + ch * (kBM * kKC * 2);
+#pragma unroll
+            for (int kk = 0; kk < kKC / 16; ++kk) {
+              const uint64_t ad = sdesc_sw128(qaddr + kk * 32, 16, 1024);
+              const uint64_t bd = sdesc_sw128(kaddr + kk * 32, 16, 1024);
+              umma_ss(d_tmem, ad, bd, idesc, (ch | kk) != 0);
+            }
+            umma_commit(&bars->ring_empty[s]);
+            ++cnt;
+          }
+          umma_commit(&bars->s_full[sb]);
+          if (j == it.ntiles - 1) umma_commit(&bars->q_empty);
+          return true;
+        };
+        auto issue_pv = [&](int j) -> bool {
+          const Tile t = tile_of(it, j);
+          const uint32_t gg = g + j;
+          const uint32_t sb = gg & 1;
+          if (!mbar_wait(&bars->p_full[sb], (gg >> 1) & 1, abort)) return false;
+          if (j == 0 && nitem > 0 && !mbar_wait(&bars->o_free, (nitem - 1) & 1, abort))
+            return false;
+          tc_fence_after();
+          const uint32_t a_tmem = tmem + kTmS0 + sb * 128;
+          const uint32_t idesc = idesc_bf16_f32(kBM, kKC, true);
+          for (int ch = 0; ch < kNVCh; ++ch) {
+            const uint32_t s = cnt % kStages;
+            if (!mbar_wait(&bars->ring_full[s], (cnt / kStages) & 1, abort)) return false;
+            tc_fence_after();
+            const uint32_t vaddr = rbase + s * kChunkBytes + t.rowoff * 128;
+            for (int kk = 0; kk < t.n / 16; ++kk) {
+              // 16 keys = two 8-row swizzle atoms = 2 KB; N-major, one 64-wide block
+              const uint64_t bd = sdesc_sw128(vaddr + kk * 2048, kChunkBytes, 1024);
+              umma_ts(tmem + kTmO + ch * kKC, a_tmem + kk * 8, bd, idesc, (j > 0 || kk > 0));
+            }
+            umma_commit(&bars->ring_empty[s]);
+            ++cnt;
+          }
+          umma_commit(&bars->o_done);
+          return true;
+        };
+        for (int j = 0; j < it.ntiles && ok; ++j) {
+          ok = issue_s(j);
+          if (ok && j >= 1) ok = issue_pv(j - 1);
+        }
+        if (ok) ok = issue_pv(it.ntiles - 1);
+        g += it.ntiles;
+        ++nitem;
+      }
+      if (!ok) raise_timeout(p, bars);
+      // drain: every UMMA issued above has finished before TMEM is released
+      volatile int no_abort = 0;
+      umma_commit(&bars->drain);
+      mbar_wait(&bars->drain, 0, &no_abort, 100000000ull);
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax + epilogue
+    const int quad = warp & 3;               // TMEM lane quadrant of this warp
+    const int row = quad * 32 + lane;        // tile row == TMEM lane
+    const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+    uint32_t g = 0;
+    int nitem = 0;
+    bool ok = true;
+    for (int r = 0; ok; ++r) {
+      const int k = r * G + ((r & 1) ? (G - 1 - c) : c);
+      if (k >= p.n_items) break;
+      const Item it = make_item(p, k);
+      const int pos = it.t0 + row / p.hq;
+      const int h = row % p.hq;
+      const bool row_valid = pos < p.T;
+      const int t = min(pos, p.T - 1);
+      const int nc_row = min(visible_count(t, p.block, p.W), min(p.n_entries[it.b], p.max_pages * p.PE));
+      const int lo_row = max(0, t - p.W + 1);
+      float m = -INFINITY;  // reference of the stored P / O (log2 domain)
+      float l = 0.f;
+      for (int j = 0; j < it.ntiles; ++j) {
+        const Tile tl = tile_of(it, j);
+        const uint32_t gg = g + j;
+        const uint32_t sb = gg & 1;
+        if (!(ok = mbar_wait(&bars->s_full[sb], (gg >> 1) & 1, abort))) break;
+        tc_fence_after();
+        const uint32_t s_addr = tmem + lane_addr + kTmS0 + sb * 128;
+        auto valid = [&](int e) -> bool {
+          const int key = tl.key0 + e;
+          return e < tl.n &&
+                 (tl.kind == kCompressed ? (key < nc_row) : (key >= lo_row && key <= t));
+        };
+        // pass 1: row max of the masked, scaled scores
+        float mt = -INFINITY;
+#pragma unroll 1
+        for (int q = 0; q < kBN / 32; ++q) {
+          if (q * 32 >= tl.n) break;
+          uint32_t v[32];
+          tmem_ld32(s_addr + q * 32, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (valid(q * 32 + e)) mt = fmaxf(mt, __uint_as_float(v[e]) * p.scale_log2);
+        }
+        const float mn = fmaxf(m, mt);
+        float ref = m;
+        float alpha = 1.f;
+        bool rescale = false;
+        if (m == -INFINITY) {
+          ref = mn;
+        } else if (mn > m + kRescaleThreshold) {
+          ref = mn;
+          alpha = fast_exp2(m - mn);
+          rescale = true;
+        }
+        const float base = ref == -INFINITY ? 0.f : ref;
+        // pass 2: P = exp2(s - ref) in bf16, written over the score columns (A of P.V).
+        // Piece q reads score columns [32q, 32q+32) and writes P columns [16q, 16q+16),
+        // which were read in an earlier piece (or this one).
+        float psum = 0.f;
+#pragma unroll 1
+        for (int q = 0; q < kBN / 32; ++q) {
+          if (q * 32 >= tl.n) break;
+          uint32_t v[32];
+          tmem_ld32(s_addr + q * 32, v);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int c0 = q * 32 + 2 * e;
+            const float x0 = valid(c0) ? __uint_as_float(v[2 * e]) * p.scale_log2 : -INFINITY;
+            const float x1 =
+                valid(c0 + 1) ? __uint_as_float(v[2 * e + 1]) * p.scale_log2 : -INFINITY;
+            pk[e] = pack_bf16x2(fast_exp2(x0 - base), fast_exp2(x1 - base));
+            const float2 f2 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&pk[e]));
+            psum += f2.x + f2.y;
+          }
+          tmem_st16(s_addr + q * 16, pk);
+        }
+        l = l * alpha + psum;
+        m = ref;
+        // rescale O (all lanes of the warp take part in the TMEM round trip)
+        if (__any_sync(0xffffffffu, rescale) && j > 0) {
+          if (!(ok = mbar_wait(&bars->o_done, (gg - 1) & 1, abort))) break;
+          tc_fence_after();
+          const uint32_t o_addr = tmem + lane_addr + kTmO;
+#pragma unroll 1
+          for (int q = 0; q < kDH / 32; ++q) {
+            uint32_t v[32];
+            tmem_ld32(o_addr + q * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+            tmem_st32(o_addr + q * 32, v);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->p_full[sb]);
+      }
+      if (!ok) break;
+      // epilogue: O half / l (* gate) -> bf16
+      const uint32_t glast = g + it.ntiles - 1;
+      if (!(ok = mbar_wait(&bars->o_done, glast & 1, abort))) break;
+      tc_fence_after();
+      const float inv = 1.f / l;
+      const int64_t orow = ((int64_t)it.b * p.T + t) * p.hq + h;
+      __nv_bfloat16* op = p.O + orow * kD + it.half * kDH;
+      const __nv_bfloat16* gp =
+          p.gate ? p.gate + (int64_t)it.b * p.gs0 + (int64_t)t * p.gs1 + (int64_t)h * p.gs2 +
+                       it.half * kDH
+                 : nullptr;
+      const uint32_t o_addr = tmem + lane_addr + kTmO;
+#pragma unroll 1
+      for (int q = 0; q < kDH / 32; ++q) {
+        uint32_t v[32];
+        tmem_ld32(o_addr + q * 32, v);
+        tmem_wait_ld();
+        float o[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[e] = __uint_as_float(v[e]) * inv;
+        if (gp) {
+          const uint4* g4 = reinterpret_cast<const uint4*>(gp + q * 32);
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const uint4 gv = g4[w];
+            const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __bfloat1622float2(g2[e]);
+              o[w * 8 + 2 * e] *= f.x;
+              o[w * 8 + 2 * e + 1] *= f.y;
+            }
+          }
+        }
+        if (row_valid) {
+          uint4* o4 = reinterpret_cast<uint4*>(op + q * 32);
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            uint4 pk;
+            pk.x = pack_bf16x2(o[w * 8 + 0], o[w * 8 + 1]);
+            pk.y = pack_bf16x2(o[w * 8 + 2], o[w * 8 + 3]);
+            pk.z = pack_bf16x2(o[w * 8 + 4], o[w * 8 + 5]);
+            pk.w = pack_bf16x2(o[w * 8 + 6], o[w * 8 + 7]);
+            o4[w] = pk;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->o_free);
+      if (row_valid && it.half == 0) {
+        if (p.lse) p.lse[orow] = (m + __log2f(l)) * 0.69314718055994531f;
+        if (p.dbg && h == 0) {
+          int32_t* dp = p.dbg + ((int64_t)it.b * p.T + t) * 3;
+          dp[0] = nc_row;
+          dp[1] = lo_row;
+          dp[2] = t;
+        }
+      }
+      g += it.ntiles;
+      ++nitem;
+    }
+    if (!ok) raise_timeout(p, bars);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+bool prefill_tc_supported(const hca_desc& d, const hca_cache& c) {
+  if (d.dtype != HCA_BF16 || d.head_dim != kD || d.hkv != 1) return false;
+  if (d.hq < 8 || d.hq > 128 || (128 % d.hq) != 0) return false;
+  if (d.window < 1 || d.window > 128 || d.block < 1) return false;
+  if (c.page_entries % kBN != 0) return false;
+  if (d.gate) {
+    const uintptr_t ga = reinterpret_cast<uintptr_t>(d.gate);
+    if (ga % 16 || d.gate_strides[0] % 8 || d.gate_strides[1] % 8 || d.gate_strides[2] % 8)
+      return false;
+  }
+  return true;
+}
+
+cudaError_t launch_prefill_tc(const hca_desc& d, const void* Q, const void* K, const void* V,
+                              const hca_cache& c, void* O, float* lse, int32_t* dbg_mask,
+                              cudaStream_t s) {
+  Params p;
+  memset(&p, 0, sizeof(p));
+  const uint64_t rowsQ = (uint64_t)d.batch * d.seqlen * d.hq;
+  const uint64_t rowsK = (uint64_t)d.batch * d.seqlen;
+  const uint64_t rowsC = (uint64_t)c.num_pages * c.page_entries;
+  cudaError_t e;
+  if ((e = encode_bf16_rows(&p.tmQ, Q, rowsQ, kD, kKC, kBM)) != cudaSuccess) return e;
+  if ((e = encode_bf16_rows(&p.tmK, K, rowsK, kD, kKC, kBN)) != cudaSuccess) return e;
+  if ((e = encode_bf16_rows(&p.tmV, V, rowsK, kD, kKC, kBN)) != cudaSuccess) return e;
+  if ((e = encode_bf16_rows(&p.tmK16, K, rowsK, kD, kKC, 16)) != cudaSuccess) return e;
+  if ((e = encode_bf16_rows(&p.tmV16, V, rowsK, kD, kKC, 16)) != cudaSuccess) return e;
+  if ((e = encode_bf16_rows(&p.tmKc, c.kc_pool, rowsC, kD, kKC, kBN)) != cudaSuccess) return e;
+  if ((e = encode_bf16_rows(&p.tmVc, c.vc_pool, rowsC, kD, kKC, kBN)) != cudaSuccess) return e;
+  p.O = static_cast<__nv_bfloat16*>(O);
+  p.lse = lse;
+  p.dbg = dbg_mask;
+  p.gate = static_cast<const __nv_bfloat16*>(d.gate);
+  p.gs0 = d.gate_strides[0];
+  p.gs1 = d.gate_strides[1];
+  p.gs2 = d.gate_strides[2];
+  p.page_table = c.page_table;
+  p.n_entries = c.n_entries;
+  p.err_word = c.err_word;
+  p.batch = d.batch;
+  p.T = d.seqlen;
+  p.hq = d.hq;
+  p.P = kBM / d.hq;
+  p.W = d.window;
+  p.block = d.block;
+  p.PE = c.page_entries;
+  p.max_pages = c.max_pages;
+  p.num_pages = c.num_pages;
+  p.n_rt = (d.seqlen + p.P - 1) / p.P;
+  p.n_items = 2 * d.batch * p.n_rt;
+  p.scale_log2 = d.scale * 1.4426950408889634f;
+  if (p.n_items == 0) return cudaSuccess;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  const int grid = min(p.n_items, device_sm_count());
+  prefill_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace hca

@@ -1,0 +1,16 @@
+// tmap.h -- TMA tensor-map encoding through the driver entry point (no -lcuda needed).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace hca {
+
+// 2-D bf16 map over a row-major [rows, cols] array, 128-byte swizzle, box
+// [box_rows, box_cols] (box_cols * 2 bytes must be 128). Loads that fall outside the
+// array are zero-filled by the hardware.
+cudaError_t encode_bf16_rows(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                             uint32_t box_cols, uint32_t box_rows);
+
+}  // namespace hca

@@ -1,0 +1,91 @@
+"""torch-tensor front end over the C ABI (shapes, pointers, streams; no arithmetic).
+
+Every function here calls straight into libhca through ``binding`` and raises
+``binding.HcaError`` on a non-zero status. Tensors must live on the current CUDA
+device and be contiguous.
+"""
+
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import binding as B
+
+
+def _ptr(t: Optional[torch.Tensor]) -> int:
+    return 0 if t is None else t.data_ptr()
+
+
+def _stream(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def desc_for_prefill(Q: torch.Tensor, K: torch.Tensor, block: int = 128, window: int = 128,
+                     scale: Optional[float] = None) -> B.HcaDesc:
+    b, T, hq, D = Q.shape
+    return B.make_desc(b, T, hq, K.shape[2], D, block, window, scale, B.dtype_code(Q))
+
+
+def attach_gate(desc: B.HcaDesc, G: Optional[torch.Tensor]) -> None:
+    """G: [b, T, hq, D] (prefill) or [nseq, hq, D] (decode), head_dim contiguous."""
+    if G is None:
+        B.check(B.hca_set_gate(desc, 0, None), "hca_set_gate")
+        return
+    st = G.stride()
+    strides = (st[0], st[1], st[2]) if G.dim() == 4 else (st[0], 0, st[1])
+    B.check(B.hca_set_gate(desc, G.data_ptr(), strides), "hca_set_gate")
+
+
+def compress(desc: B.HcaDesc, K: torch.Tensor, V: torch.Tensor, cache: B.PagedCache,
+             first_block: int = 0, n_blocks: Optional[int] = None,
+             batch_stride_tokens: Optional[int] = None, stream=None) -> None:
+    """Compress blocks [first_block, first_block + n_blocks) of K/V [b, T, hkv, D]."""
+    T = desc.seqlen
+    if n_blocks is None:
+        n_blocks = -(-T // desc.block) - first_block
+    if batch_stride_tokens is None:
+        batch_stride_tokens = K.shape[1]
+    off = first_block * desc.block * K.shape[2] * K.shape[3] * K.element_size()
+    st = B.hca_compress(desc, K.data_ptr() + off, V.data_ptr() + off, batch_stride_tokens,
+                        first_block, n_blocks, cache.c, _stream(stream))
+    B.check(st, "hca_compress")
+
+
+def prefill(desc: B.HcaDesc, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
+            cache: B.PagedCache, O: Optional[torch.Tensor] = None, want_lse: bool = False,
+            want_mask: bool = False, stream=None):
+    """HCA prefill; returns (O, lse or None, dbg_mask or None)."""
+    if O is None:
+        O = torch.empty_like(Q)
+    b, T, hq, _ = Q.shape
+    lse = torch.empty((b, T, hq), dtype=torch.float32, device=Q.device) if want_lse else None
+    dbg = torch.full((b, T, 3), -1, dtype=torch.int32, device=Q.device) if want_mask else None
+    st = B.hca_attn_prefill(desc, Q.data_ptr(), K.data_ptr(), V.data_ptr(), cache.c,
+                            O.data_ptr(), _ptr(lse), _ptr(dbg), _stream(stream))
+    B.check(st, "hca_attn_prefill")
+    return O, lse, dbg
+
+
+def decode_workspace(desc: B.HcaDesc, device="cuda") -> torch.Tensor:
+    n = B.hca_decode_workspace_bytes(desc)
+    return torch.empty(max(16, n), dtype=torch.uint8, device=device)
+
+
+def decode(desc: B.HcaDesc, q: torch.Tensor, ctx_len: torch.Tensor, cache: B.PagedCache,
+           ring_k: torch.Tensor, ring_v: torch.Tensor, O: Optional[torch.Tensor] = None,
+           workspace: Optional[torch.Tensor] = None, want_lse: bool = False, stream=None):
+    """One decode step; q [nseq, hq, D], ring [nseq, W, hkv, D]. Returns (O, lse or None)."""
+    if O is None:
+        O = torch.empty_like(q)
+    if workspace is None:
+        workspace = decode_workspace(desc, q.device)
+    lse = (torch.empty(q.shape[:2], dtype=torch.float32, device=q.device) if want_lse
+           else None)
+    st = B.hca_attn_decode(desc, q.data_ptr(), ctx_len.data_ptr(), cache.c, ring_k.data_ptr(),
+                           ring_v.data_ptr(), O.data_ptr(), _ptr(lse), workspace.data_ptr(),
+                           workspace.numel(), _stream(stream))
+    B.check(st, "hca_attn_decode")
+    return O, lse

@@ -1,0 +1,167 @@
+/*
+ * hca.h -- C ABI of libhca: Heavily Compressed Attention (HCA) on sm_100a.
+ *
+ * The operation (sources are two pages about ERNIE-5.5-Flash-Base):
+ *   [news 二.1]     "280B总参数、14B激活！百度开源文心5.5 Flash Base" (aitest123.com),
+ *                   section 二.1 "Latent-Gated Sparse Attention": an HCA layer stores one
+ *                   cache entry per 128 tokens and attends only to those entries plus a
+ *                   window of the most recent uncompressed tokens.
+ *   [analysis 1]    "百度 ERNIE 5.5 Flash Base 完整解析" (communeify.com), architecture item 1
+ *                   (HCA): 128 consecutive tokens become one entry, the layer attends to all
+ *                   compressed history entries and a short window of recent raw tokens, and
+ *                   its heads are 512 wide.
+ *   [gate]          both pages, "Low-Rank Gated Attention" paragraph: the attention output
+ *                   is multiplied by a learned gate.
+ *
+ * Readings where the pages are silent: mean pooling over the tokens present in a block;
+ * window = the last `window` tokens up to and including the query; compressed entry j is
+ * visible to position t iff (j+1)*block <= t+1-window (blocks that end before the window);
+ * one softmax over both key sets; the gate arrives already passed through the sigmoid.
+ *
+ * Conventions for every entry point:
+ *   - All tensors are caller-owned DEVICE memory unless stated; the library allocates
+ *     nothing, keeps no global state between calls, and never frees caller memory.
+ *   - Layouts are dense row-major with head_dim innermost:
+ *       Q, O        [batch, seqlen, hq,  head_dim]
+ *       K, V        [batch, seqlen, hkv, head_dim]
+ *       cache pools [num_pages, page_entries, hkv, head_dim]
+ *     Element type is desc->dtype (HCA_BF16 or HCA_F32) for all of them; LSE is float32.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream) and the
+ *     call returns before it runs. The return value reports argument validation and
+ *     launch failures only. Kernels that meet an out-of-range page id or a cache holding
+ *     fewer entries than a query needs skip that access and OR a bit into *cache->err_word
+ *     (if non-NULL); the caller reads it after synchronising.
+ *   - No entry point throws across the ABI or aborts the process.
+ */
+#ifndef HCA_H_
+#define HCA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same handle type as cudaStream_t, declared here so this header needs no CUDA header. */
+typedef struct CUstream_st* hca_stream_t;
+
+typedef enum {
+  HCA_OK = 0,
+  HCA_EINVAL = -1,        /* NULL pointer, negative size, inconsistent shapes */
+  HCA_EUNSUPPORTED = -2,  /* valid HCA problem that this build has no kernel for */
+  HCA_ENOSPACE = -3,      /* cache pages or workspace too small for the request */
+  HCA_ECUDA = -4          /* a CUDA runtime/driver call failed (launch, tensor map) */
+} hca_status;
+
+typedef enum { HCA_BF16 = 0, HCA_F32 = 1 } hca_dtype;
+
+/* Bits OR-ed into *hca_cache.err_word by kernels. */
+#define HCA_ERR_PAGE_RANGE 1   /* a page-table entry outside [0, num_pages) was skipped */
+#define HCA_ERR_CACHE_SHORT 2  /* a query needed more entries than n_entries[b] holds */
+
+/* Problem description. Plain data filled by the caller; copied by value into launches. */
+typedef struct {
+  int32_t batch;       /* sequences in the call (prefill: b; decode: number of sequences) */
+  int32_t seqlen;      /* prefill: tokens per sequence T. decode: largest context length in
+                          the batch (bounds the split count and the workspace size) */
+  int32_t hq;          /* query heads (64 in the pages' model) */
+  int32_t hkv;         /* key/value heads; hq % hkv == 0; query head h reads kv head h*hkv/hq */
+  int32_t head_dim;    /* 512 in [analysis 1] */
+  int32_t block;       /* tokens pooled into one entry: 128 in [news 二.1] */
+  int32_t window;      /* raw tokens each query sees, itself included (reading: 128) */
+  float scale;         /* softmax scale applied to q.k (reading: 1/sqrt(head_dim)) */
+  int32_t dtype;       /* hca_dtype of Q, K, V, O, the pools, the ring and the gate */
+  int32_t decode_splits; /* decode only: key-range splits per sequence, 0 = automatic */
+  const void* gate;    /* optional gate G (post-sigmoid), dtype as above; NULL = no gate.
+                          Set through hca_set_gate. */
+  int64_t gate_strides[3]; /* element strides of G: prefill [batch, token, head];
+                              decode [sequence, unused, head]; head_dim is contiguous */
+} hca_desc;
+
+/* Paged compressed-KV cache. Entry j of sequence b lives in pool row
+ *   page_table[b * max_pages + j / page_entries] * page_entries + j % page_entries. */
+typedef struct {
+  void* kc_pool;              /* [num_pages, page_entries, hkv, head_dim] */
+  void* vc_pool;              /* same shape */
+  const int32_t* page_table;  /* device [batch, max_pages] */
+  int32_t* n_entries;         /* device [batch]; hca_compress stores first_block + n_blocks */
+  int32_t page_entries;       /* entries per page; the bf16 kernels need a multiple of 128 */
+  int32_t max_pages;          /* columns of page_table */
+  int32_t num_pages;          /* pages in each pool */
+  int32_t* err_word;          /* optional device int32 error bits (HCA_ERR_*), may be NULL */
+} hca_cache;
+
+/* ABI version of this header (bumped on any layout change of the structs above). */
+#define HCA_ABI_VERSION 1
+int32_t hca_abi_version(void);
+
+/* Human-readable name of a status code. Static string, never NULL. */
+const char* hca_status_string(int32_t status);
+
+/* Attach (gate != NULL) or detach (gate == NULL) the output gate of [gate].
+ * Host-only: writes d->gate and d->gate_strides; no device work. `strides` (3 elements)
+ * may be NULL only when gate is NULL.
+ * Returns HCA_EINVAL for d == NULL or a non-NULL gate without strides. */
+int32_t hca_set_gate(hca_desc* d, const void* gate, const int64_t* strides);
+
+/* Block compression of [news 二.1] / [analysis 1] (mean pooling, the reading above).
+ * For every sequence b < d->batch and block j in [first_block, first_block + n_blocks):
+ *   Kc[j] = mean of K rows of tokens [j*block, min((j+1)*block, d->seqlen)), same for V,
+ * accumulated in float32 and rounded once to d->dtype, stored into the cache pools at the
+ * row the page table gives; then n_entries[b] = first_block + n_blocks.
+ * K, V point at the first token of block `first_block` of sequence 0; the token rows of
+ * sequence b start `b * batch_stride_tokens` token rows later (prefill: batch_stride_tokens
+ * = seqlen with K advanced by first_block*block rows; a decode ring of `block` slots:
+ * batch_stride_tokens = block).
+ * Errors: HCA_EINVAL (NULL pointer, n_blocks < 0, first_block < 0, a block starting at or
+ * past seqlen), HCA_ENOSPACE (first_block + n_blocks > max_pages * page_entries),
+ * HCA_EUNSUPPORTED (head_dim not a multiple of 8), HCA_ECUDA. */
+int32_t hca_compress(const hca_desc* d, const void* K, const void* V,
+                     int64_t batch_stride_tokens, int32_t first_block, int32_t n_blocks,
+                     const hca_cache* cache, hca_stream_t stream);
+
+/* HCA prefill attention of [news 二.1] / [analysis 1] with the optional gate of [gate].
+ * For every sequence b, position t < seqlen and head h:
+ *   keys  = compressed entries j < n_c(t) of sequence b, then raw tokens u in
+ *           [max(0, t-window+1), t];  n_c(t) = max(0, floor((t+1-window)/block))
+ *   O[b,t,h] = softmax(scale * q . keys) . values  (one softmax over both sets)
+ *   O[b,t,h] *= G[b,t,h] when a gate is attached
+ *   lse[b,t,h] = natural log of the softmax denominator incl. the max (if lse != NULL)
+ *   dbg_mask[(b*seqlen+t)*3 + {0,1,2}] = (n_c(t), window lo, window hi) (if non-NULL)
+ * Compressed entries are read from `cache` (hca_compress must have written them).
+ * Kernels: bf16 -> tcgen05/TMEM tensor-core kernel (needs head_dim 512, hkv 1, hq in
+ * {8,16,32,64,128}, window <= 128, page_entries % 128 == 0); f32 -> CUDA-core kernel
+ * (head_dim % 32 == 0, head_dim <= 512, any block/window).
+ * Errors: HCA_EINVAL, HCA_EUNSUPPORTED, HCA_ECUDA. */
+int32_t hca_attn_prefill(const hca_desc* d, const void* Q, const void* K, const void* V,
+                         const hca_cache* cache, void* O, float* lse, int32_t* dbg_mask,
+                         hca_stream_t stream);
+
+/* Bytes of device workspace hca_attn_decode needs for `d` (split partials of O, max and
+ * sum). 0 if d is invalid. */
+size_t hca_decode_workspace_bytes(const hca_desc* d);
+
+/* One HCA decode step for d->batch sequences ([news 二.1]; the query is the newest token).
+ *   Q        [batch, hq, head_dim]   query of the new token of each sequence
+ *   ctx_len  device int32 [batch]    context length including the new token; the query
+ *                                    position is t = ctx_len - 1, 1 <= ctx_len <= seqlen
+ *   ring_k/v [batch, window, hkv, head_dim]  raw tokens; token u sits in slot u % window
+ *   O        [batch, hq, head_dim];  lse [batch, hq] float32 (optional)
+ * Keys are exactly the prefill key set of position t. The key list is cut into splits
+ * (d->decode_splits, 0 = automatic), each split writes float32 partial (O, max, sum) into
+ * `workspace`, and a merge kernel combines them, applies the gate and casts.
+ * Kernels: bf16 -> tcgen05/TMEM kernel (head_dim 512, hkv 1, hq <= 64, window <= 128,
+ * page_entries % 128 == 0); f32 -> CUDA-core kernel.
+ * Errors: HCA_EINVAL, HCA_EUNSUPPORTED, HCA_ENOSPACE (workspace_bytes too small),
+ * HCA_ECUDA. */
+int32_t hca_attn_decode(const hca_desc* d, const void* Q, const int32_t* ctx_len,
+                        const hca_cache* cache, const void* ring_k, const void* ring_v,
+                        void* O, float* lse, void* workspace, size_t workspace_bytes,
+                        hca_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HCA_H_ */

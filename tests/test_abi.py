@@ -1,0 +1,146 @@
+"""Host-side checks of the C ABI (CPU only: no kernel is launched).
+
+The library must load, export every symbol include/hca.h declares, agree with the
+binding on struct layouts, and reject bad arguments before touching the GPU.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from compressed_long_context_hca_b200 import binding as B
+from compressed_long_context_hca_b200 import build as build_mod
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hca.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build_mod.build()
+    return B.lib()
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\**\s+\**(hca_[a-z_0-9]+)\s*\(", src, re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_binding_names():
+    assert _declared_functions() == sorted(B.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in _declared_functions():
+        assert hasattr(L, name), name
+    out = os.popen(f"nm -D --defined-only {B.LIB_PATH}").read()
+    for name in _declared_functions():
+        assert re.search(rf"\bT {name}\b", out), name
+
+
+def test_abi_version_and_strings(L):
+    assert B.hca_abi_version() == B.ABI_VERSION
+    for code in (0, -1, -2, -3, -4):
+        assert B.hca_status_string(code).startswith("HCA_")
+    assert "unknown" in B.hca_status_string(7)
+
+
+def test_struct_layouts_match_header():
+    # offsets follow the C rules for the field order in hca.h
+    assert ctypes.sizeof(B.HcaDesc) == 72
+    assert B.HcaDesc.gate.offset == 40
+    assert B.HcaDesc.gate_strides.offset == 48
+    assert ctypes.sizeof(B.HcaCache) == 56
+    assert B.HcaCache.err_word.offset == 48
+
+
+def _cache():
+    c = B.HcaCache()
+    c.kc_pool = c.vc_pool = c.page_table = c.n_entries = 0x1000
+    c.page_entries, c.max_pages, c.num_pages = 128, 4, 4
+    return c
+
+
+def test_validation_rejects_before_launch(L):
+    d = B.make_desc(1, 256, 64, 1, 512)
+    c = _cache()
+    # NULL descriptor / cache / tensors
+    assert L.hca_compress(None, 1, 1, 0, 0, 1, ctypes.byref(c), None) == B.HCA_EINVAL
+    assert B.hca_compress(d, 0, 0, 256, 0, 1, c) == B.HCA_EINVAL
+    assert B.hca_attn_prefill(d, 0, 0, 0, c, 0) == B.HCA_EINVAL
+    # hq not a multiple of hkv
+    bad = B.make_desc(1, 256, 6, 4, 512)
+    assert B.hca_attn_prefill(bad, 16, 16, 16, c, 16) == B.HCA_EINVAL
+    # negative sizes
+    neg = B.make_desc(1, -1, 64, 1, 512)
+    assert B.hca_attn_prefill(neg, 16, 16, 16, c, 16) == B.HCA_EINVAL
+    # unsupported dtype code
+    d2 = B.make_desc(1, 256, 64, 1, 512, dtype=7)
+    assert B.hca_attn_prefill(d2, 16, 16, 16, c, 16) == B.HCA_EUNSUPPORTED
+    # bf16 tensor path needs head_dim 512 and hkv 1
+    d3 = B.make_desc(1, 256, 64, 1, 256)
+    assert B.hca_attn_prefill(d3, 16, 16, 16, c, 16) == B.HCA_EUNSUPPORTED
+    d4 = B.make_desc(1, 256, 64, 2, 512)
+    assert B.hca_attn_prefill(d4, 16, 16, 16, c, 16) == B.HCA_EUNSUPPORTED
+    # window above what the tensor-core tiles cover
+    d5 = B.make_desc(1, 256, 64, 1, 512, window=200)
+    assert B.hca_attn_prefill(d5, 16, 16, 16, c, 16) == B.HCA_EUNSUPPORTED
+    # page size not a multiple of 128 for the bf16 kernels
+    c2 = _cache()
+    c2.page_entries = 64
+    assert B.hca_attn_prefill(d, 16, 16, 16, c2, 16) == B.HCA_EUNSUPPORTED
+    # f32 path: head_dim must be a multiple of 32, <= 512
+    d6 = B.make_desc(1, 256, 4, 1, 520, dtype=B.HCA_F32)
+    assert B.hca_attn_prefill(d6, 16, 16, 16, c, 16) == B.HCA_EUNSUPPORTED
+    # misaligned pointer
+    assert B.hca_attn_prefill(d, 16 + 2, 16, 16, c, 16) == B.HCA_EINVAL
+
+
+def test_compress_space_and_range_checks(L):
+    d = B.make_desc(2, 1000, 64, 1, 512)
+    c = _cache()  # 4 pages x 128 entries
+    # blocks past the sequence
+    assert B.hca_compress(d, 16, 16, 1000, 7, 2, c) == B.HCA_EINVAL
+    # more entries than the page table can address
+    c.max_pages = 0
+    assert B.hca_compress(d, 16, 16, 1000, 0, 1, c) == B.HCA_EINVAL
+    c.max_pages = 1
+    c.page_entries = 4
+    assert B.hca_compress(d, 16, 16, 1000, 0, 7, c) == B.HCA_ENOSPACE
+    # zero blocks / empty batch: nothing to do
+    assert B.hca_compress(d, 16, 16, 1000, 0, 0, c) == B.HCA_OK
+    assert B.hca_compress(B.make_desc(0, 1000, 64, 1, 512), 16, 16, 1000, 0, 1, c) == B.HCA_OK
+
+
+def test_decode_workspace_and_space(L):
+    d = B.make_desc(16, 1 << 20, 64, 1, 512, decode_splits=9)
+    n = B.hca_decode_workspace_bytes(d)
+    assert n == 16 * 9 * 64 * (512 + 2) * 4
+    assert B.hca_decode_workspace_bytes(B.make_desc(1, 1, 64, 1, 512, dtype=B.HCA_F32)) == 0
+    c = _cache()
+    st = B.hca_attn_decode(d, 16, 16, c, 16, 16, 16, 0, 16, n - 1)
+    assert st == B.HCA_ENOSPACE
+
+
+def test_set_gate(L):
+    d = B.make_desc(1, 8, 64, 1, 512)
+    assert B.hca_set_gate(d, 0x2000, (1, 2, 3)) == B.HCA_OK
+    assert d.gate == 0x2000 and list(d.gate_strides) == [1, 2, 3]
+    assert B.hca_set_gate(d, 0x2000, None) == B.HCA_EINVAL
+    assert B.hca_set_gate(d, 0, None) == B.HCA_OK
+    assert not d.gate and list(d.gate_strides) == [0, 0, 0]
+
+
+def test_product_path_has_no_oracle_import():
+    # the package must never import the oracle (test infrastructure only)
+    pkg = os.path.join(ROOT, "compressed_long_context_hca_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                txt = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(import|from)\s+oracle\b", txt, re.M), f
+                assert "hca_oracle" not in txt, f

@@ -1,0 +1,112 @@
+"""GPU decode (hca_attn_decode) against the float64 oracle, plus cross-path checks."""
+
+import numpy as np
+import pytest
+import torch
+
+from compressed_long_context_hca_b200 import binding as B
+from compressed_long_context_hca_b200 import inputs, ops
+from oracle import hca_oracle as orc
+from tests.gpu_helpers import (BF16_MAX, BF16_MEAN, F32_MAX, compare, default_scale,
+                               ensure_built, run_prefill, to64)
+
+pytestmark = pytest.mark.gpu
+
+
+def _setup(nseq, ctx_lo, ctx_hi, dtype="bf16", gate=False, seed=0, hq=64, D=512, W=128,
+           block=128, splits=0, pe=128):
+    ensure_built()
+    dev = torch.device("cuda")
+    max_ent = max(1, (ctx_hi - W) // block + 1)
+    x = inputs.decode_inputs(nseq, hq, 1, D, W, block, ctx_lo, ctx_hi, max_ent, dtype, seed,
+                             gate)
+    mp = -(-max_ent // pe)
+    cache = B.PagedCache(nseq, max_ent, 1, D, x.q.dtype, pe,
+                         page_table=inputs.page_table(nseq, mp), device=dev)
+    for b in range(nseq):
+        cache.fill(b, x.entries_k[b].to(dev), x.entries_v[b].to(dev))
+    desc = B.make_desc(nseq, ctx_hi, hq, 1, D, block, W, None,
+                       B.HCA_BF16 if dtype == "bf16" else B.HCA_F32, splits)
+    G = None if x.G is None else x.G.to(dev)
+    ops.attach_gate(desc, G)
+    return x, cache, desc
+
+
+def _run(x, cache, desc):
+    dev = torch.device("cuda")
+    O, lse = ops.decode(desc, x.q.to(dev), x.ctx_len.to(dev), cache, x.ring_k.to(dev),
+                        x.ring_v.to(dev), want_lse=True)
+    torch.cuda.synchronize()
+    return O, lse
+
+
+def _oracle(x, b, block=128, W=128):
+    D = x.q.shape[-1]
+    G = None if x.G is None else to64(x.G[b])
+    return orc.hca_decode(to64(x.q[b]), to64(x.entries_k[b]), to64(x.entries_v[b]),
+                          to64(x.ring_k[b]), to64(x.ring_v[b]), int(x.ctx_len[b]), block, W,
+                          default_scale(D), gate=G)
+
+
+@pytest.mark.parametrize("nseq,lo,hi,gate", [
+    (4, 1, 127, False),            # window only, partly filled ring
+    (6, 128, 700, True),           # 0..4 entries
+    (8, 8192, 40000, False),       # many tiles, several splits
+    (3, 70000, 70000, True),       # equal lengths
+])
+def test_decode_bf16(nseq, lo, hi, gate):
+    x, cache, desc = _setup(nseq, lo, hi, gate=gate)
+    O, lse = _run(x, cache, desc)
+    for b in range(nseq):
+        ref, rl = _oracle(x, b)
+        compare(to64(O[b]), ref, BF16_MAX, BF16_MEAN, what=f"O[{b}]")
+        compare(to64(lse[b]), rl, 2e-2, what=f"lse[{b}]")
+    assert int(cache.err.item()) == 0
+
+
+def test_decode_batched_config_sampled():
+    """128 sequences with context lengths uniform in [8192, 131072], one query each,
+    64 heads, head_dim 512, paged cache + last 128 raw tokens, N(0,1)."""
+    x, cache, desc = _setup(128, 8192, 131072, seed=0)
+    O, _ = _run(x, cache, desc)
+    for b in list(range(0, 128, 9)) + [127]:
+        ref, _ = _oracle(x, b)
+        compare(to64(O[b]), ref, BF16_MAX, BF16_MEAN, what=f"O[{b}]")
+
+
+@pytest.mark.parametrize("splits", [1, 2, 3, 7, 0])
+def test_decode_split_invariance(splits):
+    x, cache, desc = _setup(5, 20000, 60000, seed=3, splits=splits)
+    O, _ = _run(x, cache, desc)
+    for b in range(5):
+        ref, _ = _oracle(x, b)
+        compare(to64(O[b]), ref, BF16_MAX, BF16_MEAN, what=f"splits={splits} O[{b}]")
+
+
+def test_decode_fp32():
+    x, cache, desc = _setup(3, 1, 5000, dtype="f32", gate=True, seed=4, hq=4)
+    O, lse = _run(x, cache, desc)
+    for b in range(3):
+        ref, rl = _oracle(x, b)
+        compare(to64(O[b]), ref, F32_MAX, what=f"O[{b}]")
+        compare(to64(lse[b]), rl, 1e-5, what=f"lse[{b}]")
+
+
+def test_decode_equals_prefill_row():
+    """The decode step at position t sees exactly the prefill key set of t."""
+    T, D, W = 1200, 512, 128
+    x = inputs.prefill_inputs(1, T, 64, 1, D, "bf16", seed=9)
+    r = run_prefill(x)
+    dev = torch.device("cuda")
+    K, V, Q = x.K.to(dev), x.V.to(dev), x.Q.to(dev)
+    for t in (0, 100, 127, 128, 255, 256, 1000, T - 1):
+        rk = torch.zeros((1, W, 1, D), dtype=torch.bfloat16, device=dev)
+        rv = torch.zeros_like(rk)
+        for u in range(max(0, t - W + 1), t + 1):
+            rk[0, u % W] = K[0, u]
+            rv[0, u % W] = V[0, u]
+        desc = B.make_desc(1, T, 64, 1, D)
+        ctx = torch.tensor([t + 1], dtype=torch.int32, device=dev)
+        Od, _ = ops.decode(desc, Q[:, t].contiguous(), ctx, r["cache"], rk, rv)
+        torch.cuda.synchronize()
+        compare(to64(Od[0]), to64(r["O"][0, t]), 1.6e-2, 1e-3, what=f"t={t}")

@@ -1,0 +1,133 @@
+"""GPU prefill (hca_attn_prefill) against the float64 oracle."""
+
+import numpy as np
+import pytest
+import torch
+
+from compressed_long_context_hca_b200 import binding as B
+from compressed_long_context_hca_b200 import inputs
+from oracle import hca_oracle as orc
+from tests.gpu_helpers import (BF16_MAX, BF16_MEAN, F32_MAX, compare, default_scale,
+                               run_prefill, to64)
+
+pytestmark = pytest.mark.gpu
+
+
+def _oracle(x, bi, positions, block=128, window=128, scale=None):
+    D = x.Q.shape[-1]
+    s = default_scale(D) if scale is None else scale
+    G = None if x.G is None else to64(x.G[bi])
+    return orc.hca_prefill(to64(x.Q[bi]), to64(x.K[bi]), to64(x.V[bi]), block, window, s,
+                           gate=G, positions=positions)
+
+
+# ---------------------------------------------------------------------------- float32
+def test_tiny_fp32_config():
+    """1 sequence, T=1024, 4 query heads sharing 1 KV head, head_dim 512, block 128,
+    window 128, N(0,1) from seed 0, gate off: max |err| <= 1e-5, masks bit-exact."""
+    x = inputs.prefill_inputs(1, 1024, 4, 1, 512, "f32", seed=0)
+    r = run_prefill(x, dtype="f32", want_lse=True, want_mask=True)
+    ref, lse = _oracle(x, 0, None)
+    compare(to64(r["O"][0]), ref, F32_MAX, what="O")
+    compare(to64(r["lse"][0]), lse, 1e-5, what="lse")
+    assert np.array_equal(r["dbg"][0].cpu().numpy(), orc.mask_table(1024, 128, 128))
+    assert int(r["cache"].err.item()) == 0
+
+
+@pytest.mark.parametrize("T,hq,hkv,D,block,window,gate", [
+    (37, 2, 1, 32, 4, 3, False),       # tiny ragged, window < block
+    (300, 6, 2, 64, 16, 40, True),     # grouped heads, gate
+    (513, 3, 1, 128, 128, 128, False),  # ragged tail past 4 blocks
+    (64, 1, 1, 32, 1, 5, False),       # block 1 = full causal attention
+    (50, 2, 1, 32, 8, 64, False),      # window >= T = plain causal attention
+])
+def test_fp32_shapes(T, hq, hkv, D, block, window, gate):
+    x = inputs.prefill_inputs(2, T, hq, hkv, D, "f32", seed=11, gate=gate, block=block)
+    r = run_prefill(x, block=block, window=window, dtype="f32", page_entries=4,
+                    want_lse=True, want_mask=True)
+    for bi in range(2):
+        ref, lse = _oracle(x, bi, None, block, window)
+        compare(to64(r["O"][bi]), ref, F32_MAX, what=f"O[{bi}]")
+        compare(to64(r["lse"][bi]), lse, 1e-5, what=f"lse[{bi}]")
+        assert np.array_equal(r["dbg"][bi].cpu().numpy(), orc.mask_table(T, block, window))
+
+
+# ---------------------------------------------------------------------------- bf16
+@pytest.mark.parametrize("T,hq,gate,hetero", [
+    (1, 64, False, False),       # a single token
+    (127, 64, False, False),     # window only
+    (129, 64, True, False),      # first position with a 16-key straggler tile
+    (256, 64, False, True),
+    (700, 64, True, True),       # ragged, several compressed tiles? (no: 4 entries)
+    (2048, 64, False, False),    # compressed tiles of partial width
+    (1500, 16, True, False),     # 8 positions per tile
+    (1000, 8, False, True),      # 16 positions per tile
+    (999, 128, False, False),    # 1 position per tile
+])
+def test_bf16_prefill(T, hq, gate, hetero):
+    x = inputs.prefill_inputs(1, T, hq, 1, 512, "bf16", seed=1, gate=gate,
+                              hetero_blocks=hetero)
+    r = run_prefill(x, want_lse=True, want_mask=True)
+    ref, lse = _oracle(x, 0, None)
+    compare(to64(r["O"][0]), ref, BF16_MAX, BF16_MEAN, what="O")
+    compare(to64(r["lse"][0]), lse, 2e-2, 2e-3, what="lse")
+    assert np.array_equal(r["dbg"][0].cpu().numpy(), orc.mask_table(T, 128, 128))
+    assert int(r["cache"].err.item()) == 0
+
+
+def test_bf16_two_sequences_many_compressed_tiles():
+    """b=2, T=20000: >128 visible entries (several compressed tiles per row tile)."""
+    T = 20000
+    x = inputs.prefill_inputs(2, T, 64, 1, 512, "bf16", seed=2, gate=True,
+                              hetero_blocks=True)
+    r = run_prefill(x, page_entries=256)
+    rng = np.random.default_rng(0)
+    pos = sorted(set([0, 1, 126, 127, 128, 129, 255, 256, 16511, 16512, 16639, 16640,
+                      T - 2, T - 1] + rng.integers(0, T, 40).tolist()))
+    for bi in range(2):
+        ref, _ = _oracle(x, bi, pos)
+        compare(to64(r["O"][bi, pos]), ref, BF16_MAX, BF16_MEAN, what=f"O[{bi}]")
+
+
+def test_bf16_full_32k_config_sampled():
+    """Prefill bf16: batch 1, T=32768, 64 query heads sharing 1 KV head, head_dim 512,
+    block 128, window 128, scale 1/sqrt(512), N(0,1) rounded to bf16, gate off.
+    Every position of a sample of 128-position tiles (first, last, block edges, random)."""
+    T = 32768
+    x = inputs.prefill_inputs(1, T, 64, 1, 512, "bf16", seed=0)
+    r = run_prefill(x, want_mask=True)
+    rng = np.random.default_rng(1)
+    tiles = sorted(set([0, 1, 2, 127, 128, 255] + rng.integers(0, 256, 6).tolist()))
+    pos = [t * 128 + k for t in tiles for k in range(0, 128, 3)] + [T - 1]
+    ref, _ = _oracle(x, 0, pos)
+    compare(to64(r["O"][0, pos]), ref, BF16_MAX, BF16_MEAN, what="O")
+    assert np.array_equal(r["dbg"][0].cpu().numpy(), orc.mask_table(T, 128, 128))
+    # property at any size: every output row is finite
+    assert torch.isfinite(r["O"].float()).all()
+
+
+def test_bf16_constant_values_give_constant_output():
+    """Closed form at full width: V constant per dim -> O equals that constant."""
+    T = 3000
+    x = inputs.prefill_inputs(1, T, 64, 1, 512, "bf16", seed=4)
+    c = torch.randn(512).to(torch.bfloat16)
+    x.V[:] = c
+    r = run_prefill(x)
+    got = r["O"][0].float().cpu()
+    assert (got - c.float()).abs().max().item() <= 1e-2
+
+
+def test_bf16_missing_cache_entries_flagged():
+    """A cache holding fewer entries than the queries need: the kernel skips the missing
+    entries and raises HCA_ERR_CACHE_SHORT instead of reading past them."""
+    from compressed_long_context_hca_b200 import ops
+    T, D = 1024, 512
+    x = inputs.prefill_inputs(1, T, 64, 1, D, "bf16", seed=8)
+    dev = torch.device("cuda")
+    Q, K, V = x.Q.to(dev), x.K.to(dev), x.V.to(dev)
+    desc = ops.desc_for_prefill(Q, K)
+    cache = B.PagedCache(1, 8, 1, D, Q.dtype, 128, device=dev)
+    ops.compress(desc, K, V, cache, first_block=0, n_blocks=2)
+    ops.prefill(desc, Q, K, V, cache)
+    torch.cuda.synchronize()
+    assert int(cache.err.item()) & B.HCA_ERR_CACHE_SHORT
