@@ -1,0 +1,603 @@
+#!/usr/bin/env python
+"""HCA benchmark: prefill TFLOP/s and decode tokens/s at head_dim 512 on B200.
+
+Main line (the step): compress + prefill of one batch of the bf16 prefill workload
+(batch 1, T = 32768, 64 query heads sharing 1 KV head, head_dim 512, block 128,
+window 128, scale 1/sqrt(512), N(0,1) inputs rounded to bf16, gate off). The value is
+algorithmic TFLOP/s (visible query-key pairs only) over all ranks. Inputs (Q alone is
+2.1 GB) are larger than the 126 MB L2, so no flush runs between steps.
+
+Extra results in the same JSON line:
+  decode_batched  128 sequences, context lengths uniform in [8192, 131072]: tokens/s
+  decode_1m       16 sequences at 1,048,576 context, 4 decode steps each, gate on, with
+                  the compress call of the block the first step completes: tokens/s
+  prefill_128k    batch 2 x 131072, heterogeneous blocks, fused gate: TFLOP/s
+  e2e             the main metric with host-resident inputs and output (pinned host
+                  memory, H2D + D2H inside the timed region)
+  roofline        prefill kernel vs the measured bf16 dense peak (and HBM)
+  cpu_baseline    the float64 oracle on a bounded sample of the same workload
+
+Multi-GPU (torchrun): every rank runs its own replica of the workload (independent
+sequences, no data-path collective); the time is the max over ranks.
+``--impl reference`` times the float64 oracle (rank 0 only) on bounded samples.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+D, HQ, BLOCK, WIN = 512, 64, 128, 128
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def visible_pairs(T: int, block: int = BLOCK, W: int = WIN):
+    """Closed-form count of visible (query, key) pairs per head of one sequence."""
+    c = 0
+    # sum_t max(0, floor((t + 1 - W) / block)) for t in [0, T)
+    for x in range(1, T - W + 1):
+        c += x // block
+    w = sum(min(W, t + 1) for t in range(min(T, W))) + max(0, T - W) * W
+    return c, w
+
+
+def prefill_flops(T: int, batch: int = 1) -> float:
+    c, w = visible_pairs(T)
+    return 4.0 * D * HQ * (c + w) * batch
+
+
+# ------------------------------------------------------------------ clocks sampler
+class Clocks:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        time.sleep(0.12)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        sm.sort()
+        med = sm[len(sm) // 2] if sm else None
+        return {"sm_mhz": med, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ oracle timing
+def oracle_sample_prefill(seconds: float, T: int = 32768, seed: int = 0):
+    """Time the float64 oracle on random query positions of the 32K workload.
+
+    Returns (tflops, positions_done, wall_s, threads). Inputs are regenerated on the CPU
+    with the same recipe (values differ from the GPU's generator; the cost does not)."""
+    import numpy as np
+    from compressed_long_context_hca_b200 import inputs
+    from oracle import hca_oracle as orc
+    x = inputs.prefill_inputs(1, T, HQ, 1, D, "bf16", seed=seed)
+    Q = x.Q[0].float().numpy().astype(np.float64)
+    K = x.K[0].float().numpy().astype(np.float64)
+    V = x.V[0].float().numpy().astype(np.float64)
+    s = 1.0 / math.sqrt(D)
+    Kc, Vc = orc.compress_blocks(K, BLOCK), orc.compress_blocks(V, BLOCK)
+    rng = np.random.default_rng(seed)
+    done, flops = 0, 0.0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < seconds:
+        t = int(rng.integers(0, T))
+        orc.attend_position(Q[t], Kc, Vc, K, V, t, BLOCK, WIN, s)
+        n = orc.visible_compressed_count(t, BLOCK, WIN) + (t - max(0, t - WIN + 1) + 1)
+        flops += 4.0 * D * HQ * n
+        done += 1
+    wall = time.perf_counter() - t0
+    threads = blas_threads()
+    return flops / wall / 1e12, done, wall, threads
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = max([i.get("num_threads", 1) for i in info] or [1])
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------ GPU workloads
+def gpu_main(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from compressed_long_context_hca_b200 import binding as B
+    from compressed_long_context_hca_b200 import build as build_mod
+    from compressed_long_context_hca_b200 import ops
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: no CUDA device (the product has no CPU path)")
+    build_mod.build()
+    B.lib()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    peaks, peak_kind = load_peaks()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---------------------------------------------------------------- main: 32K prefill
+    T = args.seqlen
+    g = torch.Generator(device=dev)
+    g.manual_seed(1000 + rank)
+    Q = torch.randn((1, T, HQ, D), generator=g, device=dev).to(torch.bfloat16)
+    K = torch.randn((1, T, 1, D), generator=g, device=dev).to(torch.bfloat16)
+    V = torch.randn((1, T, 1, D), generator=g, device=dev).to(torch.bfloat16)
+    O = torch.empty_like(Q)
+    desc = ops.desc_for_prefill(Q, K)
+    cache = B.PagedCache(1, -(-T // BLOCK), 1, D, torch.bfloat16, 128, device=dev)
+
+    def step():
+        ops.compress(desc, K, V, cache)
+        ops.prefill(desc, Q, K, V, cache, O=O)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    flops = prefill_flops(T)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    clocks = Clocks(local_rank)
+    clocks.start()
+    time.sleep(0.1)
+    barrier()
+    torch.cuda.synchronize()
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    e_start.record(stream)
+    for i in range(args.steps):
+        ops.compress(desc, K, V, cache)
+        ev[i][0].record(stream)
+        ops.prefill(desc, Q, K, V, cache, O=O)
+        ev[i][1].record(stream)
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    total_ms = max_over_ranks(e_start.elapsed_time(e_end))
+    ms_step = total_ms / args.steps
+    prefill_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    launches = 2 * args.steps
+    assert int(cache.err.item()) == 0, "kernel raised an error bit"
+
+    value = world * flops / (ms_step * 1e-3) / 1e12
+    achieved = flops / (prefill_ms * 1e-3) / 1e12
+    bytes_prefill = (2 * Q.numel() + 2 * K.numel() + 2 * V.numel()) * 2  # Q,O + K,V
+    hbm_achieved = bytes_prefill / (prefill_ms * 1e-3) / 1e9
+    result = {
+        "metric": "HCA prefill TFLOP/s at d=512 (32K bf16, compress+prefill step); "
+                  "decode tokens/s in decode_batched / decode_1m",
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic N(0,1) rounded to bf16, seeded",
+        "config": {"workload": "HCA prefill bf16: batch 1, T=32768, 64 query heads, 1 KV head, "
+                               "head_dim 512, block 128, window 128, gate off",
+                   "global_batch": world, "seq_len": T, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (Q 2.1 GB), no flush"},
+        "gpu_launches": launches,
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 1),
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": round(achieved / peaks["bf16_tflops"], 4),
+                     "traffic": args.traffic, "kernel": "prefill_tc_kernel",
+                     "peak_source": f"{peak_kind} bf16 dense burst",
+                     "hbm": {"achieved": round(hbm_achieved, 1), "peak": peaks["hbm_gbs"],
+                             "unit": "GB/s", "frac": round(hbm_achieved / peaks["hbm_gbs"], 4),
+                             "bytes_per_launch": bytes_prefill}},
+        "clocks": clk,
+    }
+
+    # ---------------------------------------------------------------- e2e (host buffers)
+    if not args.no_e2e:
+        hQ = Q.cpu().pin_memory()
+        hK = K.cpu().pin_memory()
+        hV = V.cpu().pin_memory()
+        hO = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+        e2e_steps = max(1, min(args.steps, args.e2e_steps))
+
+        def e2e_step():
+            Q.copy_(hQ, non_blocking=True)
+            K.copy_(hK, non_blocking=True)
+            V.copy_(hV, non_blocking=True)
+            ops.compress(desc, K, V, cache)
+            ops.prefill(desc, Q, K, V, cache, O=O)
+            hO.copy_(O, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(a.elapsed_time(b)) / e2e_steps
+        result["e2e"] = {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3),
+                         "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 3),
+                         "h2d_bytes_per_step": (hQ.numel() + hK.numel() + hV.numel()) * 2,
+                         "d2h_bytes_per_step": hO.numel() * 2}
+        del hQ, hK, hV, hO
+
+    del Q, K, V, O, cache
+    torch.cuda.empty_cache()
+
+    # ---------------------------------------------------------------- decode workloads
+    if not args.no_decode:
+        result["decode_batched"] = bench_decode_batched(args, dev, rank, world, barrier,
+                                                        max_over_ranks, peaks)
+        result["decode_1m"] = bench_decode_1m(args, dev, rank, world, barrier, max_over_ranks,
+                                              peaks)
+    if args.with_128k:
+        result["prefill_128k"] = bench_prefill_128k(args, dev, rank, world, barrier,
+                                                    max_over_ranks, peaks)
+
+    # ---------------------------------------------------------------- CPU baseline
+    if rank == 0 and world == 1 and not args.no_cpu:
+        tf, n, wall, threads = oracle_sample_prefill(args.cpu_seconds, T)
+        result["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": threads,
+                                  "kind": "oracle",
+                                  "sample": f"{n} random query positions x 64 heads of the 32K "
+                                            f"workload, {wall:.1f} s float64 NumPy"}
+    return result
+
+
+def _time_loop(fn, steps, warmup, barrier, max_over_ranks, stream):
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    return max_over_ranks(a.elapsed_time(b)) / steps
+
+
+def bench_decode_batched(args, dev, rank, world, barrier, max_over_ranks, peaks):
+    import torch
+    from compressed_long_context_hca_b200 import binding as B
+    from compressed_long_context_hca_b200 import ops
+    nseq, lo, hi = 128, 8192, 131072
+    g = torch.Generator(device=dev)
+    g.manual_seed(2000 + rank)
+    ctx = torch.randint(lo, hi + 1, (nseq,), generator=g, device=dev, dtype=torch.int64)
+    ctx = ctx.to(torch.int32)
+    max_ent = (hi - WIN) // BLOCK + 1
+    cache = B.PagedCache(nseq, max_ent, 1, D, torch.bfloat16, 128, device=dev)
+    cache.kc.normal_(generator=g)
+    cache.vc.normal_(generator=g)
+    cache.n_entries.fill_(max_ent)
+    q = torch.randn((nseq, HQ, D), generator=g, device=dev).to(torch.bfloat16)
+    rk = torch.randn((nseq, WIN, 1, D), generator=g, device=dev).to(torch.bfloat16)
+    rv = torch.randn((nseq, WIN, 1, D), generator=g, device=dev).to(torch.bfloat16)
+    desc = B.make_desc(nseq, hi, HQ, 1, D)
+    ws = ops.decode_workspace(desc, dev)
+    O = torch.empty_like(q)
+    stream = torch.cuda.current_stream()
+    clocks = Clocks(dev.index)
+    fn = lambda: ops.decode(desc, q, ctx, cache, rk, rv, O=O, workspace=ws)  # noqa: E731
+    clocks.start()
+    ms = _time_loop(fn, args.decode_steps, 3, barrier, max_over_ranks, stream)
+    clk = clocks.stop()
+    ctx_h = ctx.cpu().tolist()
+    keys = sum((c - WIN) // BLOCK + min(WIN, c) for c in ctx_h)
+    byts = keys * D * 2 * 2 + nseq * HQ * D * 2 * 2
+    nsplit = B.hca_decode_workspace_bytes(desc) // (nseq * HQ * (D + 2) * 4)
+    return {"value": round(world * nseq / (ms * 1e-3), 1), "unit": "tokens/s",
+            "ms_per_step": round(ms, 4),
+            "workload": "128 sequences, context U[8192,131072], 1 query each, 64 heads, "
+                        "head_dim 512, paged cache + 128-token ring, N(0,1) bf16",
+            "gpu_launches_per_step": 2, "splits": int(nsplit),
+            "roofline": {"bound": "hbm", "achieved": round(byts / (ms * 1e-3) / 1e9, 1),
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                         "bytes_per_step": byts},
+            "clocks": clk}
+
+
+def bench_decode_1m(args, dev, rank, world, barrier, max_over_ranks, peaks):
+    import torch
+    from compressed_long_context_hca_b200 import binding as B
+    from compressed_long_context_hca_b200 import ops
+    nseq, ctx0, steps_per = 16, 1048576, 4
+    n_ent = (ctx0 - WIN) // BLOCK  # 8191 visible entries at the first step
+    g = torch.Generator(device=dev)
+    g.manual_seed(3000 + rank)
+    cache = B.PagedCache(nseq, n_ent + 2, 1, D, torch.bfloat16, 128, device=dev)
+    cache.kc.normal_(generator=g)
+    cache.vc.normal_(generator=g)
+    cache.n_entries.fill_(n_ent)
+    q = torch.randn((steps_per, nseq, HQ, D), generator=g, device=dev).to(torch.bfloat16)
+    G = torch.sigmoid(torch.randn((steps_per, nseq, HQ, D), generator=g, device=dev))
+    G = G.to(torch.bfloat16)
+    new_k = torch.randn((steps_per, nseq, 1, 1, D), generator=g, device=dev).to(torch.bfloat16)
+    new_v = torch.randn((steps_per, nseq, 1, 1, D), generator=g, device=dev).to(torch.bfloat16)
+    rk = torch.randn((nseq, WIN, 1, D), generator=g, device=dev).to(torch.bfloat16)
+    rv = torch.randn((nseq, WIN, 1, D), generator=g, device=dev).to(torch.bfloat16)
+    ctx = [torch.full((nseq,), ctx0 + s, dtype=torch.int32, device=dev) for s in range(steps_per)]
+    descs = []
+    for s in range(steps_per):
+        d = B.make_desc(nseq, ctx0 + steps_per, HQ, 1, D)
+        ops.attach_gate(d, G[s])
+        descs.append(d)
+    ws = ops.decode_workspace(descs[0], dev)
+    cdesc = B.make_desc(nseq, ctx0, HQ, 1, D)  # compress of the block ending at ctx0 - 1
+    O = torch.empty((nseq, HQ, D), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def four_steps():
+        for s in range(steps_per):
+            p = ctx0 - 1 + s                 # position of the new token
+            slot = p % WIN
+            rk[:, slot].copy_(new_k[s, :, 0])
+            rv[:, slot].copy_(new_v[s, :, 0])
+            if (p + 1) % BLOCK == 0:         # token completes block p // BLOCK
+                B.check(B.hca_compress(cdesc, rk.data_ptr(), rv.data_ptr(), WIN, p // BLOCK,
+                                       1, cache.c, stream.cuda_stream), "hca_compress")
+            ops.decode(descs[s], q[s], ctx[s], cache, rk, rv, O=O, workspace=ws)
+
+    clocks = Clocks(dev.index)
+    clocks.start()
+    ms = _time_loop(four_steps, args.decode_steps, 3, barrier, max_over_ranks, stream)
+    clk = clocks.stop()
+    keys = n_ent + WIN
+    byts_step = nseq * (keys * D * 2 * 2 + 3 * HQ * D * 2)
+    byts = steps_per * byts_step + nseq * BLOCK * D * 2 * 2
+    nsplit = B.hca_decode_workspace_bytes(descs[0]) // (nseq * HQ * (D + 2) * 4)
+    return {"value": round(world * nseq * steps_per / (ms * 1e-3), 1), "unit": "tokens/s",
+            "ms_per_step": round(ms, 4), "ms_per_decode_step": round(ms / steps_per, 4),
+            "workload": "16 sequences at context 1,048,576 (8191 entries + 128 raw), 64 heads, "
+                        "head_dim 512, 4 decode steps each incl. one hca_compress, gate on",
+            "gpu_launches_per_step": 4 * 2 + 1, "splits": int(nsplit),
+            "roofline": {"bound": "hbm", "achieved": round(byts / (ms * 1e-3) / 1e9, 1),
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                         "bytes_per_step": byts},
+            "clocks": clk}
+
+
+def bench_prefill_128k(args, dev, rank, world, barrier, max_over_ranks, peaks):
+    import torch
+    from compressed_long_context_hca_b200 import binding as B
+    from compressed_long_context_hca_b200 import ops
+    b, T = 2, 131072
+    g = torch.Generator(device=dev)
+    g.manual_seed(4000 + rank)
+    blk = ((torch.arange(T, device=dev) // BLOCK) % 4 == 3)
+
+    def draw(h):
+        x = torch.randn((b, T, h, D), generator=g, device=dev)
+        x[:, blk] *= 4.0
+        return x.to(torch.bfloat16)
+
+    Q, K, V = draw(HQ), draw(1), draw(1)
+    G = torch.sigmoid(torch.randn((b, T, HQ, D), generator=g, device=dev)).to(torch.bfloat16)
+    O = torch.empty_like(Q)
+    desc = ops.desc_for_prefill(Q, K)
+    ops.attach_gate(desc, G)
+    cache = B.PagedCache(b, T // BLOCK, 1, D, torch.bfloat16, 128, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ops.compress(desc, K, V, cache)
+        ops.prefill(desc, Q, K, V, cache, O=O)
+
+    clocks = Clocks(dev.index)
+    clocks.start()
+    ms = _time_loop(step, args.steps_128k, 3, barrier, max_over_ranks, stream)
+    clk = clocks.stop()
+    flops = prefill_flops(T, b)
+    tf = world * flops / (ms * 1e-3) / 1e12
+    return {"value": round(tf, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 3),
+            "workload": "batch 2 x 131072, 64 heads, 1 KV head, head_dim 512, every 4th block "
+                        "x4, fused gate", "frac_of_sustained_peak":
+                round(tf / world / peaks["bf16_tflops_sustained"], 4), "clocks": clk}
+
+
+# ------------------------------------------------------------------ reference arm
+def reference_main(args, rank, world):
+    if rank != 0:
+        return None
+    per_step = max(1.0, args.ref_seconds)
+    vals = []
+    threads = blas_threads()
+    for _ in range(args.warmup):
+        oracle_sample_prefill(min(1.0, per_step), args.seqlen)
+    n_tot, wall_tot = 0, 0.0
+    for _ in range(args.steps):
+        tf, n, wall, threads = oracle_sample_prefill(per_step, args.seqlen)
+        vals.append(tf)
+        n_tot += n
+        wall_tot += wall
+    v = sum(vals) / len(vals)
+    return {"metric": "HCA prefill TFLOP/s at d=512 (32K bf16, compress+prefill step); "
+                      "decode tokens/s in decode_batched / decode_1m",
+            "value": v, "unit": "TFLOP/s", "impl": "reference", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * wall_tot / args.steps, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "HCA prefill bf16: batch 1, T=32768, 64 query heads, 1 KV "
+                                   "head, head_dim 512, block 128, window 128, gate off",
+                       "global_batch": 1, "seq_len": args.seqlen, "parallelism": "host cores"},
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                             "sample": f"{n_tot} random query positions x 64 heads in "
+                                       f"{args.steps} steps of {per_step:.0f} s"},
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def profile_case(args):
+    """Small fixed case for ncu captures: compress + 2 prefill launches (or 2 decode
+    launches); no timing. ``--profile prefill --seqlen T`` or ``--profile decode
+    --nseq N --ctx C``."""
+    import torch
+    from compressed_long_context_hca_b200 import binding as B
+    from compressed_long_context_hca_b200 import build as build_mod
+    from compressed_long_context_hca_b200 import ops
+    build_mod.build()
+    dev = torch.device("cuda")
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    if args.profile == "prefill":
+        T = args.seqlen
+        Q = torch.randn((1, T, HQ, D), generator=g, device=dev).to(torch.bfloat16)
+        K = torch.randn((1, T, 1, D), generator=g, device=dev).to(torch.bfloat16)
+        V = torch.randn((1, T, 1, D), generator=g, device=dev).to(torch.bfloat16)
+        desc = ops.desc_for_prefill(Q, K)
+        cache = B.PagedCache(1, -(-T // BLOCK), 1, D, torch.bfloat16, 128, device=dev)
+        O = torch.empty_like(Q)
+        ops.compress(desc, K, V, cache)
+        for _ in range(2):
+            ops.prefill(desc, Q, K, V, cache, O=O)
+    else:
+        nseq, ctx = args.nseq, args.ctx
+        nent = (ctx - WIN) // BLOCK + 1
+        cache = B.PagedCache(nseq, nent, 1, D, torch.bfloat16, 128, device=dev)
+        cache.kc.normal_(generator=g)
+        cache.vc.normal_(generator=g)
+        cache.n_entries.fill_(nent)
+        q = torch.randn((nseq, HQ, D), generator=g, device=dev).to(torch.bfloat16)
+        rk = torch.randn((nseq, WIN, 1, D), generator=g, device=dev).to(torch.bfloat16)
+        rv = torch.randn((nseq, WIN, 1, D), generator=g, device=dev).to(torch.bfloat16)
+        ctx_t = torch.full((nseq,), ctx, dtype=torch.int32, device=dev)
+        desc = B.make_desc(nseq, ctx, HQ, 1, D)
+        ws = ops.decode_workspace(desc, dev)
+        for _ in range(2):
+            ops.decode(desc, q, ctx_t, cache, rk, rv, workspace=ws)
+    torch.cuda.synchronize()
+    assert int(cache.err.item()) == 0
+    print(f"profile case {args.profile} done")
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--seqlen", type=int, default=32768)
+    ap.add_argument("--decode-steps", type=int, default=50)
+    ap.add_argument("--steps-128k", type=int, default=10)
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-seconds", type=float, default=10.0)
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="dram bytes per prefill launch from an ncu capture of this build")
+    ap.add_argument("--with-128k", action="store_true", default=True)
+    ap.add_argument("--no-128k", dest="with_128k", action="store_false")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--profile", choices=["prefill", "decode"], default=None,
+                    help="run a small fixed case for ncu and exit")
+    ap.add_argument("--nseq", type=int, default=16)
+    ap.add_argument("--ctx", type=int, default=1048576)
+    args = ap.parse_args()
+    if args.profile:
+        profile_case(args)
+        return
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        res = reference_main(args, rank, world)
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        res = gpu_main(args, rank, world, local_rank)
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -170,6 +170,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     // ------------------------------------------------------------------ TMA producer
     if (elect_one()) {
       bool ok = true;
+      if (split == 0 && p.err_word) {
+        const int x = sq.t + 1 - p.W;
+        if ((x < 0 ? 0 : x / p.block) > p.n_entries[b]) atomicOr(p.err_word, kErrCacheShort);
+      }
       mbar_expect_tx(&bars->q_full, kQBytes);
       for (int ch = 0; ch < kNCh; ++ch)
         tma_load_2d(sQ + ch * kQChunkBytes, &p.tmQ, &bars->q_full, ch * kKC, b * p.hq);

@@ -221,6 +221,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         const int k = r * G + ((r & 1) ? (G - 1 - c) : c);
         if (k >= p.n_items) break;
         const Item it = make_item(p, k);
+        if (p.err_word && visible_count(it.tl, p.block, p.W) > p.n_entries[it.b])
+          atomicOr(p.err_word, kErrCacheShort);
         // Q tile
         if (nitem > 0 && !(ok = mbar_wait(&bars->q_empty, (nitem - 1) & 1, abort))) break;
         mbar_expect_tx(&bars->q_full, kQBytes);

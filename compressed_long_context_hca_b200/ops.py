@@ -33,10 +33,12 @@ def attach_gate(desc: B.HcaDesc, G: Optional[torch.Tensor]) -> None:
     """G: [b, T, hq, D] (prefill) or [nseq, hq, D] (decode), head_dim contiguous."""
     if G is None:
         B.check(B.hca_set_gate(desc, 0, None), "hca_set_gate")
+        desc._gate_ref = None
         return
     st = G.stride()
     strides = (st[0], st[1], st[2]) if G.dim() == 4 else (st[0], 0, st[1])
     B.check(B.hca_set_gate(desc, G.data_ptr(), strides), "hca_set_gate")
+    desc._gate_ref = G  # the descriptor holds a raw pointer: keep the tensor alive
 
 
 def compress(desc: B.HcaDesc, K: torch.Tensor, V: torch.Tensor, cache: B.PagedCache,
