@@ -31,7 +31,9 @@ HCA_ERR_TIMEOUT = 4
 ABI_VERSION = 1
 
 EXPORTED = ("hca_abi_version", "hca_status_string", "hca_set_gate", "hca_compress",
-            "hca_attn_prefill", "hca_decode_workspace_bytes", "hca_attn_decode")
+            "hca_attn_prefill", "hca_decode_workspace_bytes", "hca_attn_decode",
+            "hca_attn_decode_noalloc")
+HCA_DECODE_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 class HcaDesc(ctypes.Structure):
@@ -83,6 +85,10 @@ def lib() -> ctypes.CDLL:
     L.hca_attn_decode.argtypes = [POINTER(HcaDesc), c_void_p, c_void_p, POINTER(HcaCache),
                                   c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                                   c_void_p]
+    L.hca_attn_decode_noalloc.restype = c_int32
+    L.hca_attn_decode_noalloc.argtypes = [POINTER(HcaDesc), c_void_p, c_void_p,
+                                          POINTER(HcaCache), c_void_p, c_void_p, c_void_p,
+                                          c_void_p, c_void_p]
     if L.hca_abi_version() != ABI_VERSION:
         raise RuntimeError("libhca.so ABI version does not match this binding")
     _lib = L
@@ -138,6 +144,16 @@ def hca_attn_decode(desc: HcaDesc, Q: int, ctx_len: int, cache: HcaCache, ring_k
                                  ctypes.byref(cache), ring_k or None, ring_v or None,
                                  O or None, lse or None, workspace or None, workspace_bytes,
                                  stream or None)
+
+
+def hca_attn_decode_noalloc(desc: HcaDesc, Q: int, ctx_len: int, cache: HcaCache,
+                            ring_k: int, ring_v: int, O: int, lse: int = 0,
+                            stream: int = 0) -> int:
+    """Decode step whose split partials live in the library's own fixed device array, for
+    callers that cannot lend it device memory (see include/hca.h)."""
+    return lib().hca_attn_decode_noalloc(ctypes.byref(desc), Q or None, ctx_len or None,
+                                         ctypes.byref(cache), ring_k or None, ring_v or None,
+                                         O or None, lse or None, stream or None)
 
 
 def check(status: int, what: str) -> None:

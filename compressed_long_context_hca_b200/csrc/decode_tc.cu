@@ -554,4 +554,48 @@ cudaError_t launch_decode_tc(const hca_desc& d, const void* Q, const int32_t* ct
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------------------
+// Decode without a caller-provided workspace.
+//
+// Some callers cannot hand this library a workspace: their device memory belongs to
+// another allocator (a framework's caching pool, or a serving engine that reserves all of
+// HBM up front and has no free block to lend), or their decode loop must not call the CUDA
+// allocator at all, because cudaMalloc/cudaFree can synchronise the device and stall every
+// other stream. For them the split partials live in one fixed array inside the library,
+// sized for HCA_DECODE_NOALLOC_SCRATCH_BYTES (include/hca.h). The array is created when the
+// library's device code is loaded on a GPU and stays allocated on that GPU until the
+// process exits. Every call reuses it, so two calls whose kernels overlap on the GPU (two
+// streams, or two host threads) overwrite each other's partials; callers must serialise
+// them. Nothing in it has to start at zero: each split writes its partial before the merge
+// reads it.
+static __device__ __align__(256) unsigned char g_decode_scratch[HCA_DECODE_NOALLOC_SCRATCH_BYTES];
+
+// The array's name is only a host-side stand-in; its device address is looked up once per
+// device (on that device's first call) and cached.
+static cudaError_t decode_scratch_address(void** out) {
+  static void* cached[64] = {nullptr};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64 && cached[dev]) {
+    *out = cached[dev];
+    return cudaSuccess;
+  }
+  void* ptr = nullptr;
+  e = cudaGetSymbolAddress(&ptr, g_decode_scratch);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64) cached[dev] = ptr;
+  *out = ptr;
+  return cudaSuccess;
+}
+
+cudaError_t launch_decode_tc_noalloc(const hca_desc& d, const void* Q, const int32_t* ctx_len,
+                                     const hca_cache& c, const void* ring_k,
+                                     const void* ring_v, void* O, float* lse, cudaStream_t s) {
+  void* ws = nullptr;
+  cudaError_t e = decode_scratch_address(&ws);
+  if (e != cudaSuccess) return e;
+  return launch_decode_tc(d, Q, ctx_len, c, ring_k, ring_v, O, lse, ws, s);
+}
+
 }  // namespace hca

@@ -185,4 +185,23 @@ int32_t hca_attn_decode(const hca_desc* d, const void* Q, const int32_t* ctx_len
       launch_decode_tc(*d, Q, ctx_len, *cache, ring_k, ring_v, O, lse, workspace, s));
 }
 
+int32_t hca_attn_decode_noalloc(const hca_desc* d, const void* Q, const int32_t* ctx_len,
+                                const hca_cache* cache, const void* ring_k, const void* ring_v,
+                                void* O, float* lse, hca_stream_t stream) {
+  int32_t st = check_desc(d);
+  if (st != HCA_OK) return st;
+  if ((st = check_cache(cache)) != HCA_OK) return st;
+  if (d->batch == 0) return HCA_OK;
+  if (!Q || !ctx_len || !ring_k || !ring_v || !O) return HCA_EINVAL;
+  if (d->seqlen < 1) return HCA_EINVAL;
+  if (d->dtype != HCA_BF16 || !decode_tc_supported(*d, *cache)) return HCA_EUNSUPPORTED;
+  if (decode_tc_workspace_bytes(*d) > (size_t)HCA_DECODE_NOALLOC_SCRATCH_BYTES)
+    return HCA_ENOSPACE;
+  if (!aligned16(Q) || !aligned16(ring_k) || !aligned16(ring_v) || !aligned16(O) ||
+      !aligned16(cache->kc_pool) || !aligned16(cache->vc_pool))
+    return HCA_EINVAL;
+  return from_cuda(launch_decode_tc_noalloc(*d, Q, ctx_len, *cache, ring_k, ring_v, O, lse,
+                                            reinterpret_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

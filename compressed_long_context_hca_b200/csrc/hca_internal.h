@@ -36,5 +36,8 @@ size_t decode_tc_workspace_bytes(const hca_desc& d);
 cudaError_t launch_decode_tc(const hca_desc& d, const void* Q, const int32_t* ctx_len,
                              const hca_cache& c, const void* ring_k, const void* ring_v,
                              void* O, float* lse, void* ws, cudaStream_t s);
+cudaError_t launch_decode_tc_noalloc(const hca_desc& d, const void* Q, const int32_t* ctx_len,
+                                     const hca_cache& c, const void* ring_k,
+                                     const void* ring_v, void* O, float* lse, cudaStream_t s);
 
 }  // namespace hca

@@ -20,7 +20,8 @@
  *
  * Conventions for every entry point:
  *   - All tensors are caller-owned DEVICE memory unless stated; the library allocates
- *     nothing, keeps no global state between calls, and never frees caller memory.
+ *     nothing, keeps no global state between calls (the one exception is the fixed
+ *     scratch array behind hca_attn_decode_noalloc, below), and never frees caller memory.
  *   - Layouts are dense row-major with head_dim innermost:
  *       Q, O        [batch, seqlen, hq,  head_dim]
  *       K, V        [batch, seqlen, hkv, head_dim]
@@ -159,6 +160,30 @@ int32_t hca_attn_decode(const hca_desc* d, const void* Q, const int32_t* ctx_len
                         const hca_cache* cache, const void* ring_k, const void* ring_v,
                         void* O, float* lse, void* workspace, size_t workspace_bytes,
                         hca_stream_t stream);
+
+/* Bytes of device memory the library keeps for hca_attn_decode_noalloc (64 MiB). */
+#define HCA_DECODE_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/* hca_attn_decode without a caller-provided workspace. The pages have no counterpart to
+ * this entry point: it exists for callers that cannot give the library device memory --
+ * their memory is owned by another allocator (a framework's caching pool, or a serving
+ * engine that reserves all of HBM at start-up), or their decode loop must not call the CUDA
+ * allocator, whose cudaMalloc/cudaFree can synchronise the device.
+ * Same arguments and results as hca_attn_decode minus workspace/workspace_bytes, bf16 only.
+ * The split partials go to a fixed HCA_DECODE_NOALLOC_SCRATCH_BYTES array inside the
+ * library, allocated on every GPU that loads the library's device code and held until the
+ * process exits. It allocates nothing, and calls no cudaMalloc or cudaFree.
+ *   - The first call on a device looks up the array's device address (once per device, with
+ *     that device current); make that first call before any stream capture.
+ *   - All calls share the array and it keeps the last call's contents; nothing in it needs
+ *     to start at zero. Calls whose work overlaps on the GPU (different streams or host
+ *     threads) race on it: serialise them.
+ * Errors: as hca_attn_decode; HCA_ENOSPACE when the partials this call needs
+ * (hca_decode_workspace_bytes(d)) exceed HCA_DECODE_NOALLOC_SCRATCH_BYTES;
+ * HCA_EUNSUPPORTED for f32 (its kernel needs no workspace: call hca_attn_decode). */
+int32_t hca_attn_decode_noalloc(const hca_desc* d, const void* Q, const int32_t* ctx_len,
+                                const hca_cache* cache, const void* ring_k, const void* ring_v,
+                                void* O, float* lse, hca_stream_t stream);
 
 #ifdef __cplusplus
 }
