@@ -300,22 +300,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       if (!(ok = mbar_wait(&bars->s_full[sb], (j >> 1) & 1, abort))) break;
       tc_fence_after();
       const uint32_t s_addr = tmem + lane_addr + sb * kTN;  // lanes 16-31 hold the scores
-      auto valid = [&](int col) -> bool {
-        if (col >= tl.n) return false;
-        if (tl.kind == kCompressed) return tl.key0 + col < sq.nc;
-        return col < W && (t >= W - 1 || col <= t);
-      };
-      // pass 1: row max
-      float mt = -INFINITY;
+      // visible columns form one range [vlo, vhi): a prefix of a compressed tile, or the
+      // ring slots 0..min(W, t+1)-1
+      const int vhi = tl.kind == kCompressed ? min(tl.n, sq.nc - tl.key0) : min(W, t + 1);
+      const uint32_t vlen = vhi > 0 ? (uint32_t)vhi : 0u;
+      // pass 1: row max (branch-free selects, tree reduction)
+      float mraw = -INFINITY;
       for (int q = 0; q < kTN / 32; ++q) {
         if (q * 32 >= tl.n) break;
         uint32_t v[32];
         tmem_ld32(s_addr + q * 32, v);
         tmem_wait_ld();
+        float mx[8];
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if (valid(q * 32 + e)) mt = fmaxf(mt, __uint_as_float(v[e]) * p.scale_log2);
+        for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const bool in = (uint32_t)(q * 32 + e) < vlen;
+          mx[e & 7] = fmaxf(mx[e & 7], in ? __uint_as_float(v[e]) : -INFINITY);
+        }
+        mraw = fmaxf(mraw, fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))));
       }
+      const float mt = mraw * p.scale_log2;
       const float mn = fmaxf(m, mt);
       float ref = m, alpha = 1.f;
       bool rescale = false;
@@ -353,8 +360,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         }
         tmem_wait_st();
       }
-      // pass 2: P = exp2(s - ref) -> bf16, K-major 128B-swizzled rows of sP
-      float psum = 0.f;
+      // pass 2: P = exp2(s * scale - ref) -> bf16, K-major 128B-swizzled rows of sP
+      float ps[4] = {0.f, 0.f, 0.f, 0.f};
       for (int q = 0; q < kTN / 32; ++q) {
         if (q * 32 >= tl.n) break;
         uint32_t v[32];
@@ -365,12 +372,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int c0 = q * 32 + 2 * e;
-            const float x0 = valid(c0) ? __uint_as_float(v[2 * e]) * p.scale_log2 : -INFINITY;
-            const float x1 =
-                valid(c0 + 1) ? __uint_as_float(v[2 * e + 1]) * p.scale_log2 : -INFINITY;
-            pk[e] = pack_bf16x2(fast_exp2(x0 - base), fast_exp2(x1 - base));
-            const float2 f2 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&pk[e]));
-            psum += f2.x + f2.y;
+            const float p0 = (uint32_t)c0 < vlen
+                                 ? fast_exp2(fmaf(__uint_as_float(v[2 * e]), p.scale_log2, -base))
+                                 : 0.f;
+            const float p1 = (uint32_t)(c0 + 1) < vlen
+                                 ? fast_exp2(fmaf(__uint_as_float(v[2 * e + 1]), p.scale_log2, -base))
+                                 : 0.f;
+            pk[e] = pack_bf16x2(p0, p1);
+            ps[e & 3] += p0 + p1;
           }
           // keys q*32 .. q*32+31 -> chunk (q/2), 16-byte units u = (q&1)*4 + w
           uint8_t* rowp = sP + (q >> 1) * kPChunkBytes + hrow * 128;
@@ -383,6 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           }
         }
       }
+      const float psum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
       l = l * alpha + psum;
       m = ref;
       fence_proxy_async_smem();

@@ -58,6 +58,21 @@ cudaError_t encode_bf16_rows(CUtensorMap* map, const void* base, uint64_t rows, 
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+cudaError_t encode_bf16_chunks(CUtensorMap* map, const void* base, uint64_t rows,
+                               uint32_t box_rows, uint32_t box_chunks) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  if (rows == 0) rows = 1;
+  cuuint64_t dims[3] = {64, rows, 8};
+  cuuint64_t strides[2] = {1024, 128};
+  cuuint32_t box[3] = {64, box_rows, box_chunks};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 }  // namespace hca
 
 using namespace hca;

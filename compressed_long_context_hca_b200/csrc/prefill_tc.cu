@@ -43,14 +43,15 @@ namespace {
 constexpr int kBM = 128;               // rows per tile
 constexpr int kD = 512;                // head_dim
 constexpr int kDH = 256;               // output half per CTA
-constexpr int kKC = 64;                // elements per 128-byte swizzle row
+constexpr int kKC = 64;                // elements per 128-byte swizzle row (one "chunk")
 constexpr int kNCh = kD / kKC;         // 8 chunks of Q / K
-constexpr int kNVCh = kDH / kKC;       // 4 chunks of V per half
 constexpr int kBN = 128;               // max keys per tile
-constexpr uint32_t kChunkBytes = kBN * kKC * 2;   // 16 KB
-constexpr uint32_t kChunk16Bytes = 16 * kKC * 2;  // 2 KB
-constexpr int kStages = 5;
-constexpr uint32_t kQBytes = kNCh * kBM * kKC * 2;  // 128 KB
+constexpr uint32_t kChunk128 = kBN * kKC * 2;  // 16 KB: 128 rows x one chunk
+constexpr uint32_t kChunk16 = 16 * kKC * 2;    // 2 KB: 16 rows x one chunk
+constexpr uint32_t kSlotBytes = 2 * kChunk128;  // 32 KB: 128 rows x two chunks
+constexpr int kStages = 3;
+constexpr int kQPairs = 4;                     // Q loaded as 4 boxes of two chunks
+constexpr uint32_t kQBytes = kNCh * kChunk128;  // 128 KB
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmS0 = 0, kTmO = 256;
 constexpr int kThreads = 192;
@@ -59,6 +60,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 enum TileKind { kCompressed = 0, kRaw16 = 1, kRaw128 = 2 };
 
 struct Params {
+  // 3-D maps {64 elements, rows, 8 chunks}: one box = rows x (chunks x 128 B)
   CUtensorMap tmQ, tmK, tmV, tmK16, tmV16, tmKc, tmVc;
   __nv_bfloat16* O;
   float* lse;
@@ -97,6 +99,10 @@ __device__ __forceinline__ int round16(int x) { return (x + 15) & ~15; }
 __device__ __forceinline__ int visible_count(int t, int block, int W) {
   const int x = t + 1 - W;
   return x < 0 ? 0 : x / block;
+}
+
+__device__ __forceinline__ int item_index(int r, int G, int c) {
+  return r * G + ((r & 1) ? (G - 1 - c) : c);  // snake over the CTAs
 }
 
 __device__ __forceinline__ Item make_item(const Params& p, int k) {
@@ -141,14 +147,19 @@ __device__ __forceinline__ Tile tile_of(const Item& it, int j) {
   return t;
 }
 
+// K slots of a tile: 4 boxes of two chunks (128-row kinds) or 1 box of all 8 chunks
+// (16-row kind); V slots: 2 boxes of two chunks of this CTA's half, or 1 box of its 4.
+__device__ __forceinline__ int k_slots(const Tile& t) { return t.kind == kRaw16 ? 1 : 4; }
+__device__ __forceinline__ int v_slots(const Tile& t) { return t.kind == kRaw16 ? 1 : 2; }
+
 // Shared-memory carve-up (offsets from a 1024-byte aligned base).
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffRing = kQBytes;
-constexpr uint32_t kOffBar = kOffRing + kStages * kChunkBytes;
+constexpr uint32_t kOffBar = kOffRing + kStages * kSlotBytes;
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // + barriers + alignment slack
 
 struct Bars {
-  uint64_t q_full, q_empty;
+  uint64_t q_full[kQPairs], q_empty[kQPairs];
   uint64_t ring_full[kStages], ring_empty[kStages];
   uint64_t s_full[2], p_full[2];
   uint64_t o_done, o_free, drain;
@@ -160,6 +171,15 @@ static_assert(sizeof(Bars) <= 256, "barrier block too large");
 __device__ __forceinline__ void raise_timeout(const Params& p, Bars* bars) {
   bars->abort = 1;
   if (p.err_word) atomicOr(p.err_word, kErrTimeout);
+}
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int32_t row, int32_t chunk) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(0), "r"(row), "r"(chunk)
+      : "memory");
 }
 
 __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_constant__ Params p) {
@@ -175,8 +195,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
   const int lane = threadIdx.x % 32;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars->q_full, 1);
-    mbar_init(&bars->q_empty, 1);
+    for (int q = 0; q < kQPairs; ++q) {
+      mbar_init(&bars->q_full[q], 1);
+      mbar_init(&bars->q_empty[q], 1);
+    }
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars->ring_full[s], 1);
       mbar_init(&bars->ring_empty[s], 1);
@@ -217,54 +239,73 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       uint32_t cnt = 0;  // ring loads issued
       int nitem = 0;
       bool ok = true;
+      // Q of an item: 4 boxes of two chunks, each reloaded as soon as the previous item's
+      // last score UMMA on it has finished
+      auto load_q = [&](const Item& it, int which) -> bool {
+        const int qrow = (it.b * p.T + it.t0) * p.hq;
+        for (int q = 0; q < kQPairs; ++q) {
+          if (which > 0 && !mbar_wait(&bars->q_empty[q], (which - 1) & 1, abort)) return false;
+          mbar_expect_tx(&bars->q_full[q], kSlotBytes);
+          tma_load_3d(sQ + q * kSlotBytes, &p.tmQ, &bars->q_full[q], qrow, 2 * q);
+        }
+        return true;
+      };
+      auto next_slot = [&](uint32_t bytes) -> int {
+        const uint32_t s = cnt % kStages;
+        const uint32_t round = cnt / kStages;
+        if (round > 0 && !mbar_wait(&bars->ring_empty[s], (round - 1) & 1, abort)) return -1;
+        mbar_expect_tx(&bars->ring_full[s], bytes);
+        ++cnt;
+        return (int)s;
+      };
       for (int r = 0; ok; ++r) {
-        const int k = r * G + ((r & 1) ? (G - 1 - c) : c);
+        const int k = item_index(r, G, c);
         if (k >= p.n_items) break;
         const Item it = make_item(p, k);
         if (p.err_word && visible_count(it.tl, p.block, p.W) > p.n_entries[it.b])
           atomicOr(p.err_word, kErrCacheShort);
-        // Q tile
-        if (nitem > 0 && !(ok = mbar_wait(&bars->q_empty, (nitem - 1) & 1, abort))) break;
-        mbar_expect_tx(&bars->q_full, kQBytes);
-        const int qrow = (it.b * p.T + it.t0) * p.hq;
-        for (int ch = 0; ch < kNCh; ++ch)
-          tma_load_2d(sQ + ch * (kBM * kKC * 2), &p.tmQ, &bars->q_full, ch * kKC, qrow);
+        if (nitem == 0 && !(ok = load_q(it, 0))) break;
         // ring, in the order the MMA warp consumes it: K0, K1, V0, K2, V1, ..., V(n-1)
         auto load_tile = [&](int j, bool is_v) -> bool {
           const Tile t = tile_of(it, j);
-          const int nch = is_v ? kNVCh : kNCh;
-          for (int ch = 0; ch < nch; ++ch) {
-            const uint32_t s = cnt % kStages;
-            const uint32_t round = cnt / kStages;
-            if (round > 0 && !mbar_wait(&bars->ring_empty[s], (round - 1) & 1, abort)) return false;
-            const int x = is_v ? it.half * kDH + ch * kKC : ch * kKC;
-            uint8_t* dst = sRing + s * kChunkBytes;
+          const int nsl = is_v ? v_slots(t) : k_slots(t);
+          for (int q = 0; q < nsl; ++q) {
+            if (t.kind == kRaw16) {
+              const int s = next_slot(is_v ? 4 * kChunk16 : kNCh * kChunk16);
+              if (s < 0) return false;
+              tma_load_3d(sRing + s * kSlotBytes, is_v ? &p.tmV16 : &p.tmK16,
+                          &bars->ring_full[s], it.b * p.T + t.key0, is_v ? it.half * 4 : 0);
+              continue;
+            }
+            const int s = next_slot(kSlotBytes);
+            if (s < 0) return false;
+            const int chunk = is_v ? it.half * 4 + 2 * q : 2 * q;
+            int row;
+            const CUtensorMap* map;
             if (t.kind == kCompressed) {
               int page = p.page_table[(int64_t)it.b * p.max_pages + t.key0 / p.PE];
               if (page < 0 || page >= p.num_pages) {
                 if (p.err_word) atomicOr(p.err_word, kErrPageRange);
                 page = 0;
               }
-              const int y = page * p.PE + (t.key0 % p.PE);
-              mbar_expect_tx(&bars->ring_full[s], kChunkBytes);
-              tma_load_2d(dst, is_v ? &p.tmVc : &p.tmKc, &bars->ring_full[s], x, y);
-            } else if (t.kind == kRaw16) {
-              mbar_expect_tx(&bars->ring_full[s], kChunk16Bytes);
-              tma_load_2d(dst, is_v ? &p.tmV16 : &p.tmK16, &bars->ring_full[s], x,
-                          it.b * p.T + t.key0);
+              row = page * p.PE + (t.key0 % p.PE);
+              map = is_v ? &p.tmVc : &p.tmKc;
             } else {
-              mbar_expect_tx(&bars->ring_full[s], kChunkBytes);
-              tma_load_2d(dst, is_v ? &p.tmV : &p.tmK, &bars->ring_full[s], x,
-                          it.b * p.T + it.hi - kBN + 1);
+              row = it.b * p.T + it.hi - kBN + 1;
+              map = is_v ? &p.tmV : &p.tmK;
             }
-            ++cnt;
+            tma_load_3d(sRing + s * kSlotBytes, map, &bars->ring_full[s], row, chunk);
           }
           return true;
         };
+        const int kn = item_index(r + 1, G, c);
+        const bool has_next = kn < p.n_items;
         for (int j = 0; j < it.ntiles && ok; ++j) {
           ok = load_tile(j, false);
           if (ok && j >= 1) ok = load_tile(j - 1, true);
         }
+        // next item's Q goes in while the last tile's softmax and P.V run
+        if (ok && has_next) ok = load_q(make_item(p, kn), nitem + 1);
         if (ok) ok = load_tile(it.ntiles - 1, true);
         ++nitem;
       }
@@ -275,46 +316,59 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         const uint32_t first = cnt > kStages ? cnt - kStages : 0;
         for (uint32_t q = first; q < cnt; ++q)
           mbar_wait(&bars->ring_full[q % kStages], (q / kStages) & 1, &no_abort, 100000000ull);
+        for (int q = 0; q < kQPairs; ++q)
+          mbar_wait(&bars->q_full[q], nitem & 1, &no_abort, 100000000ull);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ UMMA issuer
     if (elect_one()) {
-      uint32_t cnt = 0;   // ring chunks consumed
+      uint32_t cnt = 0;   // ring slots consumed
       uint32_t g = 0;     // tiles processed (score buffer / phase counter)
       int nitem = 0;
       bool ok = true;
       const uint32_t qbase = smem_u32(sQ);
       const uint32_t rbase = smem_u32(sRing);
       for (int r = 0; ok; ++r) {
-        const int k = r * G + ((r & 1) ? (G - 1 - c) : c);
+        const int k = item_index(r, G, c);
         if (k >= p.n_items) break;
         const Item it = make_item(p, k);
-        if (!(ok = mbar_wait(&bars->q_full, nitem & 1, abort))) break;
-        tc_fence_after();
+        const int last = it.ntiles - 1;
 
         auto issue_s = [&](int j) -> bool {
           const Tile t = tile_of(it, j);
           const uint32_t sb = (g + j) & 1;
           const uint32_t d_tmem = tmem + kTmS0 + sb * 128;
           const uint32_t idesc = idesc_bf16_f32(kBM, t.n, false);
-          for (int ch = 0; ch < kNCh; ++ch) {
+          if (j == 0) {
+            for (int q = 0; q < kQPairs; ++q)
+              if (!mbar_wait(&bars->q_full[q], nitem & 1, abort)) return false;
+          }
+          const int nsl = k_slots(t);
+          for (int q = 0; q < nsl; ++q) {
             const uint32_t s = cnt % kStages;
             if (!mbar_wait(&bars->ring_full[s], (cnt / kStages) & 1, abort)) return false;
             tc_fence_after();
-            const uint32_t kaddr = rbase + s * kChunkBytes + t.rowoff * 128;
-            const uint32_t qaddr = qbase + ch * (kBM * kKC * 2);
+            const uint32_t sbase = rbase + s * kSlotBytes;
+            // chunks of this slot: 2 (128-row kinds, chunk pair q) or all 8 (16-row kind)
+            const int nchunks = t.kind == kRaw16 ? kNCh : 2;
+            const uint32_t cstride = t.kind == kRaw16 ? kChunk16 : kChunk128;
+            for (int cc = 0; cc < nchunks; ++cc) {
+              const int d = t.kind == kRaw16 ? cc : 2 * q + cc;
+              const uint32_t qaddr = qbase + d * kChunk128;
+              const uint32_t kaddr = sbase + cc * cstride + t.rowoff * 128;
 #pragma unroll
-            for (int kk = 0; kk < kKC / 16; ++kk) {
-              const uint64_t ad = sdesc_sw128(qaddr + kk * 32, 16, 1024);
-              const uint64_t bd = sdesc_sw128(kaddr + kk * 32, 16, 1024);
-              umma_ss(d_tmem, ad, bd, idesc, (ch | kk) != 0);
+              for (int kk = 0; kk < kKC / 16; ++kk) {
+                const uint64_t ad = sdesc_sw128(qaddr + kk * 32, 16, 1024);
+                const uint64_t bd = sdesc_sw128(kaddr + kk * 32, 16, 1024);
+                umma_ss(d_tmem, ad, bd, idesc, (d | kk) != 0);
+              }
             }
             umma_commit(&bars->ring_empty[s]);
+            if (j == last) umma_commit(&bars->q_empty[q]);  // the last tile is 128-row
             ++cnt;
           }
           umma_commit(&bars->s_full[sb]);
-          if (j == it.ntiles - 1) umma_commit(&bars->q_empty);
           return true;
         };
         auto issue_pv = [&](int j) -> bool {
@@ -326,16 +380,22 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             return false;
           tc_fence_after();
           const uint32_t a_tmem = tmem + kTmS0 + sb * 128;
-          const uint32_t idesc = idesc_bf16_f32(kBM, kKC, true);
-          for (int ch = 0; ch < kNVCh; ++ch) {
+          const int nsl = v_slots(t);
+          for (int q = 0; q < nsl; ++q) {
             const uint32_t s = cnt % kStages;
             if (!mbar_wait(&bars->ring_full[s], (cnt / kStages) & 1, abort)) return false;
             tc_fence_after();
-            const uint32_t vaddr = rbase + s * kChunkBytes + t.rowoff * 128;
+            const uint32_t vaddr = rbase + s * kSlotBytes + t.rowoff * 128;
+            // 16-row kind: one N=256 MMA over the 4 chunks (stride 2 KB); 128-row kinds:
+            // N=128 over the slot's 2 chunks (stride 16 KB) into columns 128q..128q+127
+            const uint32_t ncols = t.kind == kRaw16 ? 256 : 128;
+            const uint32_t lbo = t.kind == kRaw16 ? kChunk16 : kChunk128;
+            const uint32_t idesc = idesc_bf16_f32(kBM, ncols, true);
+            const uint32_t d_tmem = tmem + kTmO + q * 128;
             for (int kk = 0; kk < t.n / 16; ++kk) {
-              // 16 keys = two 8-row swizzle atoms = 2 KB; N-major, one 64-wide block
-              const uint64_t bd = sdesc_sw128(vaddr + kk * 2048, kChunkBytes, 1024);
-              umma_ts(tmem + kTmO + ch * kKC, a_tmem + kk * 8, bd, idesc, (j > 0 || kk > 0));
+              // 16 keys = two 8-row swizzle atoms = 2 KB
+              const uint64_t bd = sdesc_sw128(vaddr + kk * 2048, lbo, 1024);
+              umma_ts(d_tmem, a_tmem + kk * 8, bd, idesc, (j > 0 || kk > 0));
             }
             umma_commit(&bars->ring_empty[s]);
             ++cnt;
@@ -347,7 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           ok = issue_s(j);
           if (ok && j >= 1) ok = issue_pv(j - 1);
         }
-        if (ok) ok = issue_pv(it.ntiles - 1);
+        if (ok) ok = issue_pv(last);
         g += it.ntiles;
         ++nitem;
       }
@@ -366,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     int nitem = 0;
     bool ok = true;
     for (int r = 0; ok; ++r) {
-      const int k = r * G + ((r & 1) ? (G - 1 - c) : c);
+      const int k = item_index(r, G, c);
       if (k >= p.n_items) break;
       const Item it = make_item(p, k);
       const int pos = it.t0 + row / p.hq;
@@ -384,23 +444,37 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         if (!(ok = mbar_wait(&bars->s_full[sb], (gg >> 1) & 1, abort))) break;
         tc_fence_after();
         const uint32_t s_addr = tmem + lane_addr + kTmS0 + sb * 128;
-        auto valid = [&](int e) -> bool {
-          const int key = tl.key0 + e;
-          return e < tl.n &&
-                 (tl.kind == kCompressed ? (key < nc_row) : (key >= lo_row && key <= t));
-        };
-        // pass 1: row max of the masked, scaled scores
-        float mt = -INFINITY;
+        // visible columns of this row form one range [vlo, vhi) of the tile
+        int vlo, vhi;
+        if (tl.kind == kCompressed) {
+          vlo = 0;
+          vhi = min(tl.n, nc_row - tl.key0);
+        } else {
+          vlo = max(0, lo_row - tl.key0);
+          vhi = min(tl.n, t - tl.key0 + 1);
+        }
+        const uint32_t vlen = vhi > vlo ? (uint32_t)(vhi - vlo) : 0u;
+        // pass 1: row max of the raw scores over the visible range (scale > 0 is applied
+        // after the max); branch-free selects, tree reduction
+        float mraw = -INFINITY;
 #pragma unroll 1
         for (int q = 0; q < kBN / 32; ++q) {
           if (q * 32 >= tl.n) break;
           uint32_t v[32];
           tmem_ld32(s_addr + q * 32, v);
           tmem_wait_ld();
+          float mx[8];
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (valid(q * 32 + e)) mt = fmaxf(mt, __uint_as_float(v[e]) * p.scale_log2);
+          for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const bool in = (uint32_t)(q * 32 + e - vlo) < vlen;
+            mx[e & 7] = fmaxf(mx[e & 7], in ? __uint_as_float(v[e]) : -INFINITY);
+          }
+          mraw = fmaxf(mraw, fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))));
         }
+        const float mt = mraw * p.scale_log2;
         const float mn = fmaxf(m, mt);
         float ref = m;
         float alpha = 1.f;
@@ -413,10 +487,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           rescale = true;
         }
         const float base = ref == -INFINITY ? 0.f : ref;
-        // pass 2: P = exp2(s - ref) in bf16, written over the score columns (A of P.V).
-        // Piece q reads score columns [32q, 32q+32) and writes P columns [16q, 16q+16),
-        // which were read in an earlier piece (or this one).
-        float psum = 0.f;
+        // pass 2: P = exp2(s * scale - ref) in bf16, written over the score columns (A of
+        // P.V). Piece q reads score columns [32q, 32q+32) and writes P columns
+        // [16q, 16q+16), which were read in an earlier piece (or this one).
+        float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
         for (int q = 0; q < kBN / 32; ++q) {
           if (q * 32 >= tl.n) break;
@@ -427,21 +501,28 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int c0 = q * 32 + 2 * e;
-            const float x0 = valid(c0) ? __uint_as_float(v[2 * e]) * p.scale_log2 : -INFINITY;
-            const float x1 =
-                valid(c0 + 1) ? __uint_as_float(v[2 * e + 1]) * p.scale_log2 : -INFINITY;
-            pk[e] = pack_bf16x2(fast_exp2(x0 - base), fast_exp2(x1 - base));
-            const float2 f2 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&pk[e]));
-            psum += f2.x + f2.y;
+            const bool in0 = (uint32_t)(c0 - vlo) < vlen;
+            const bool in1 = (uint32_t)(c0 + 1 - vlo) < vlen;
+            const float p0 = in0 ? fast_exp2(fmaf(__uint_as_float(v[2 * e]), p.scale_log2, -base)) : 0.f;
+            const float p1 =
+                in1 ? fast_exp2(fmaf(__uint_as_float(v[2 * e + 1]), p.scale_log2, -base)) : 0.f;
+            pk[e] = pack_bf16x2(p0, p1);
+            ps[e & 3] += p0 + p1;
           }
           tmem_st16(s_addr + q * 16, pk);
         }
+        const float psum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
         l = l * alpha + psum;
         m = ref;
-        // rescale O (all lanes of the warp take part in the TMEM round trip)
-        if (__any_sync(0xffffffffu, rescale) && j > 0) {
+        // Observe the completion of P.V of the previous tile. Every o_done phase is
+        // consumed in order (a parity wait is only exact while the barrier is at most one
+        // phase away), and a rescale of O must not race that UMMA.
+        if (j > 0) {
           if (!(ok = mbar_wait(&bars->o_done, (gg - 1) & 1, abort))) break;
           tc_fence_after();
+        }
+        // rescale O (all lanes of the warp take part in the TMEM round trip)
+        if (__any_sync(0xffffffffu, rescale) && j > 0) {
           const uint32_t o_addr = tmem + lane_addr + kTmO;
 #pragma unroll 1
           for (int q = 0; q < kDH / 32; ++q) {
@@ -557,13 +638,13 @@ cudaError_t launch_prefill_tc(const hca_desc& d, const void* Q, const void* K, c
   const uint64_t rowsK = (uint64_t)d.batch * d.seqlen;
   const uint64_t rowsC = (uint64_t)c.num_pages * c.page_entries;
   cudaError_t e;
-  if ((e = encode_bf16_rows(&p.tmQ, Q, rowsQ, kD, kKC, kBM)) != cudaSuccess) return e;
-  if ((e = encode_bf16_rows(&p.tmK, K, rowsK, kD, kKC, kBN)) != cudaSuccess) return e;
-  if ((e = encode_bf16_rows(&p.tmV, V, rowsK, kD, kKC, kBN)) != cudaSuccess) return e;
-  if ((e = encode_bf16_rows(&p.tmK16, K, rowsK, kD, kKC, 16)) != cudaSuccess) return e;
-  if ((e = encode_bf16_rows(&p.tmV16, V, rowsK, kD, kKC, 16)) != cudaSuccess) return e;
-  if ((e = encode_bf16_rows(&p.tmKc, c.kc_pool, rowsC, kD, kKC, kBN)) != cudaSuccess) return e;
-  if ((e = encode_bf16_rows(&p.tmVc, c.vc_pool, rowsC, kD, kKC, kBN)) != cudaSuccess) return e;
+  if ((e = encode_bf16_chunks(&p.tmQ, Q, rowsQ, kBM, 2)) != cudaSuccess) return e;
+  if ((e = encode_bf16_chunks(&p.tmK, K, rowsK, kBN, 2)) != cudaSuccess) return e;
+  if ((e = encode_bf16_chunks(&p.tmV, V, rowsK, kBN, 2)) != cudaSuccess) return e;
+  if ((e = encode_bf16_chunks(&p.tmK16, K, rowsK, 16, 8)) != cudaSuccess) return e;
+  if ((e = encode_bf16_chunks(&p.tmV16, V, rowsK, 16, 4)) != cudaSuccess) return e;
+  if ((e = encode_bf16_chunks(&p.tmKc, c.kc_pool, rowsC, kBN, 2)) != cudaSuccess) return e;
+  if ((e = encode_bf16_chunks(&p.tmVc, c.vc_pool, rowsC, kBN, 2)) != cudaSuccess) return e;
   p.O = static_cast<__nv_bfloat16*>(O);
   p.lse = lse;
   p.dbg = dbg_mask;

@@ -13,4 +13,11 @@ namespace hca {
 cudaError_t encode_bf16_rows(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                              uint32_t box_cols, uint32_t box_rows);
 
+// 3-D bf16 map over a row-major [rows, 512] array seen as {64 elements, rows, 8 chunks}
+// (row stride 1024 B, chunk stride 128 B), 128-byte swizzle. One box = box_rows rows x
+// box_chunks consecutive 64-element chunks, landing in shared memory chunk-major:
+// [box_chunks][box_rows][64], each chunk a stack of 128-byte swizzled rows.
+cudaError_t encode_bf16_chunks(CUtensorMap* map, const void* base, uint64_t rows,
+                               uint32_t box_rows, uint32_t box_chunks);
+
 }  // namespace hca
