@@ -6,6 +6,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include "hca_internal.h"
@@ -79,7 +81,14 @@ using namespace hca;
 
 namespace {
 
-int32_t from_cuda(cudaError_t e) { return e == cudaSuccess ? HCA_OK : HCA_ECUDA; }
+// HCA_ECUDA carries no detail across the ABI; with HCA_DEBUG set in the environment the
+// CUDA error string is also written to stderr.
+int32_t from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return HCA_OK;
+  static const bool debug = getenv("HCA_DEBUG") != nullptr;
+  if (debug) fprintf(stderr, "libhca: CUDA error %d: %s\n", (int)e, cudaGetErrorString(e));
+  return HCA_ECUDA;
+}
 
 int32_t check_desc(const hca_desc* d) {
   if (!d) return HCA_EINVAL;

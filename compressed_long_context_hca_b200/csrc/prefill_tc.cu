@@ -54,7 +54,7 @@ constexpr int kQPairs = 4;                     // Q loaded as 4 boxes of two chu
 constexpr uint32_t kQBytes = kNCh * kChunk128;  // 128 KB
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmS0 = 0, kTmO = 256;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // TMA, UMMA, 4 softmax warps, 4 epilogue warps
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 enum TileKind { kCompressed = 0, kRaw16 = 1, kRaw128 = 2 };
@@ -156,13 +156,14 @@ __device__ __forceinline__ int v_slots(const Tile& t) { return t.kind == kRaw16 
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffRing = kQBytes;
 constexpr uint32_t kOffBar = kOffRing + kStages * kSlotBytes;
-constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // + barriers + alignment slack
+constexpr uint32_t kOffL = kOffBar + 256;               // row sums l, 2 items x 128 rows
+constexpr uint32_t kSmemBytes = kOffL + 2 * kBM * 4 + 1024;  // + alignment slack
 
 struct Bars {
   uint64_t q_full[kQPairs], q_empty[kQPairs];
   uint64_t ring_full[kStages], ring_empty[kStages];
   uint64_t s_full[2], p_full[2];
-  uint64_t o_done, o_free, drain;
+  uint64_t o_done, o_free, o_final, l_full, drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -174,12 +175,38 @@ __device__ __forceinline__ void raise_timeout(const Params& p, Bars* bars) {
 }
 
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
-                                            int32_t row, int32_t chunk) {
+                                            int32_t row, int32_t chunk, uint64_t policy) {
   asm volatile(
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(0), "r"(row), "r"(chunk)
+      ".L2::cache_hint [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(0), "r"(row), "r"(chunk),
+      "l"(policy)
       : "memory");
+}
+
+// L2 policies: streams read or written once (Q, gate, O) leave L2 first; K/V tiles, read
+// by every row tile of a sequence, stay.
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ uint4 ld_stream_hint(const void* ptr, uint64_t pol) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(ptr), "l"(pol));
+  return v;
+}
+__device__ __forceinline__ void st_stream_hint(void* ptr, const uint4& v, uint64_t pol) {
+  asm volatile("st.global.L1::no_allocate.L2::cache_hint.v4.u32 [%0], {%1,%2,%3,%4}, %5;" ::"l"(ptr),
+               "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "l"(pol)
+               : "memory");
 }
 
 __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_constant__ Params p) {
@@ -189,6 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
   uint8_t* sQ = smem + kOffQ;
   uint8_t* sRing = smem + kOffRing;
   Bars* bars = reinterpret_cast<Bars*>(smem + kOffBar);
+  float* sL = reinterpret_cast<float*>(smem + kOffL);
   volatile int* abort = &bars->abort;
 
   const int warp = threadIdx.x / 32;
@@ -209,6 +237,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     }
     mbar_init(&bars->o_done, 1);
     mbar_init(&bars->o_free, 4);
+    mbar_init(&bars->o_final, 1);
+    mbar_init(&bars->l_full, 4);
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
     fence_mbar_init();
@@ -236,6 +266,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (elect_one()) {
+      const uint64_t pol_q = policy_evict_first();
+      const uint64_t pol_kv = policy_evict_last();
       uint32_t cnt = 0;  // ring loads issued
       int nitem = 0;
       bool ok = true;
@@ -246,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         for (int q = 0; q < kQPairs; ++q) {
           if (which > 0 && !mbar_wait(&bars->q_empty[q], (which - 1) & 1, abort)) return false;
           mbar_expect_tx(&bars->q_full[q], kSlotBytes);
-          tma_load_3d(sQ + q * kSlotBytes, &p.tmQ, &bars->q_full[q], qrow, 2 * q);
+          tma_load_3d(sQ + q * kSlotBytes, &p.tmQ, &bars->q_full[q], qrow, 2 * q, pol_q);
         }
         return true;
       };
@@ -274,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
               const int s = next_slot(is_v ? 4 * kChunk16 : kNCh * kChunk16);
               if (s < 0) return false;
               tma_load_3d(sRing + s * kSlotBytes, is_v ? &p.tmV16 : &p.tmK16,
-                          &bars->ring_full[s], it.b * p.T + t.key0, is_v ? it.half * 4 : 0);
+                          &bars->ring_full[s], it.b * p.T + t.key0, is_v ? it.half * 4 : 0, pol_kv);
               continue;
             }
             const int s = next_slot(kSlotBytes);
@@ -294,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
               row = it.b * p.T + it.hi - kBN + 1;
               map = is_v ? &p.tmV : &p.tmK;
             }
-            tma_load_3d(sRing + s * kSlotBytes, map, &bars->ring_full[s], row, chunk);
+            tma_load_3d(sRing + s * kSlotBytes, map, &bars->ring_full[s], row, chunk, pol_kv);
           }
           return true;
         };
@@ -408,6 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           if (ok && j >= 1) ok = issue_pv(j - 1);
         }
         if (ok) ok = issue_pv(last);
+        if (ok) umma_commit(&bars->o_final);
         g += it.ntiles;
         ++nitem;
       }
@@ -417,8 +450,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       umma_commit(&bars->drain);
       mbar_wait(&bars->drain, 0, &no_abort, 100000000ull);
     }
-  } else {
-    // ------------------------------------------------------------------ softmax + epilogue
+  } else if (warp < 6) {
+    // ------------------------------------------------------------------ softmax
     const int quad = warp & 3;               // TMEM lane quadrant of this warp
     const int row = quad * 32 + lane;        // tile row == TMEM lane
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
@@ -433,7 +466,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       const int h = row % p.hq;
       const bool row_valid = pos < p.T;
       const int t = min(pos, p.T - 1);
-      const int nc_row = min(visible_count(t, p.block, p.W), min(p.n_entries[it.b], p.max_pages * p.PE));
+      const int nc_row =
+          min(visible_count(t, p.block, p.W), min(p.n_entries[it.b], p.max_pages * p.PE));
       const int lo_row = max(0, t - p.W + 1);
       float m = -INFINITY;  // reference of the stored P / O (log2 domain)
       float l = 0.f;
@@ -444,6 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         if (!(ok = mbar_wait(&bars->s_full[sb], (gg >> 1) & 1, abort))) break;
         tc_fence_after();
         const uint32_t s_addr = tmem + lane_addr + kTmS0 + sb * 128;
+        // all scores of the tile in registers (one TMEM pass)
         // visible columns of this row form one range [vlo, vhi) of the tile
         int vlo, vhi;
         if (tl.kind == kCompressed) {
@@ -454,27 +489,30 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           vhi = min(tl.n, t - tl.key0 + 1);
         }
         const uint32_t vlen = vhi > vlo ? (uint32_t)(vhi - vlo) : 0u;
-        // pass 1: row max of the raw scores over the visible range (scale > 0 is applied
-        // after the max); branch-free selects, tree reduction
-        float mraw = -INFINITY;
-#pragma unroll 1
-        for (int q = 0; q < kBN / 32; ++q) {
-          if (q * 32 >= tl.n) break;
-          uint32_t v[32];
-          tmem_ld32(s_addr + q * 32, v);
-          tmem_wait_ld();
-          float mx[8];
+        const int npieces = (tl.n + 31) >> 5;
+        // pass 1: row max of the raw scores (scale > 0 applies after); 32-column pieces,
+        // the next piece's TMEM load in flight while this one is reduced
+        float mx[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
+        for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
+        uint32_t cur[32], nxt[32];
+        tmem_ld32(s_addr, cur);
+        tmem_wait_ld();
+#pragma unroll 1
+        for (int q = 0; q < npieces; ++q) {
+          if (q + 1 < npieces) tmem_ld32(s_addr + (q + 1) * 32, nxt);
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const bool in = (uint32_t)(q * 32 + e - vlo) < vlen;
-            mx[e & 7] = fmaxf(mx[e & 7], in ? __uint_as_float(v[e]) : -INFINITY);
+            mx[e & 7] = fmaxf(mx[e & 7], in ? __uint_as_float(cur[e]) : -INFINITY);
           }
-          mraw = fmaxf(mraw, fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))));
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) cur[e] = nxt[e];
         }
-        const float mt = mraw * p.scale_log2;
+        const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) *
+                         p.scale_log2;
         const float mn = fmaxf(m, mt);
         float ref = m;
         float alpha = 1.f;
@@ -487,37 +525,39 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           rescale = true;
         }
         const float base = ref == -INFINITY ? 0.f : ref;
-        // pass 2: P = exp2(s * scale - ref) in bf16, written over the score columns (A of
-        // P.V). Piece q reads score columns [32q, 32q+32) and writes P columns
-        // [16q, 16q+16), which were read in an earlier piece (or this one).
+        // P = exp2(s * scale - ref) in bf16, written over the score columns (A of P.V).
+        // The scores are re-read 32 columns at a time, the next piece's load in flight while
+        // this one is converted; piece q writes P columns [16q, 16q+16), already read.
         float ps[4] = {0.f, 0.f, 0.f, 0.f};
+        tmem_ld32(s_addr, cur);
+        tmem_wait_ld();
 #pragma unroll 1
-        for (int q = 0; q < kBN / 32; ++q) {
-          if (q * 32 >= tl.n) break;
-          uint32_t v[32];
-          tmem_ld32(s_addr + q * 32, v);
-          tmem_wait_ld();
+        for (int q = 0; q < npieces; ++q) {
+          if (q + 1 < npieces) tmem_ld32(s_addr + (q + 1) * 32, nxt);
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int c0 = q * 32 + 2 * e;
             const bool in0 = (uint32_t)(c0 - vlo) < vlen;
             const bool in1 = (uint32_t)(c0 + 1 - vlo) < vlen;
-            const float p0 = in0 ? fast_exp2(fmaf(__uint_as_float(v[2 * e]), p.scale_log2, -base)) : 0.f;
+            const float p0 =
+                in0 ? fast_exp2(fmaf(__uint_as_float(cur[2 * e]), p.scale_log2, -base)) : 0.f;
             const float p1 =
-                in1 ? fast_exp2(fmaf(__uint_as_float(v[2 * e + 1]), p.scale_log2, -base)) : 0.f;
+                in1 ? fast_exp2(fmaf(__uint_as_float(cur[2 * e + 1]), p.scale_log2, -base)) : 0.f;
             pk[e] = pack_bf16x2(p0, p1);
             ps[e & 3] += p0 + p1;
           }
           tmem_st16(s_addr + q * 16, pk);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) cur[e] = nxt[e];
         }
-        const float psum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
-        l = l * alpha + psum;
+        l = l * alpha + (ps[0] + ps[1]) + (ps[2] + ps[3]);
         m = ref;
-        // Observe the completion of P.V of the previous tile. Every o_done phase is
-        // consumed in order (a parity wait is only exact while the barrier is at most one
-        // phase away), and a rescale of O must not race that UMMA.
-        if (j > 0) {
+        // Observe the completion of the previous P.V (of this item, or the previous item's
+        // last one). Every o_done phase is consumed in order: a parity wait is exact only
+        // while the barrier is at most one phase away. A rescale of O must not race it.
+        if (gg > 0) {
           if (!(ok = mbar_wait(&bars->o_done, (gg - 1) & 1, abort))) break;
           tc_fence_after();
         }
@@ -526,25 +566,60 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           const uint32_t o_addr = tmem + lane_addr + kTmO;
 #pragma unroll 1
           for (int q = 0; q < kDH / 32; ++q) {
-            uint32_t v[32];
-            tmem_ld32(o_addr + q * 32, v);
+            uint32_t o[32];
+            tmem_ld32(o_addr + q * 32, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-            tmem_st32(o_addr + q * 32, v);
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(o_addr + q * 32, o);
           }
+        }
+        if (j == it.ntiles - 1) {
+          // hand the row sum to the epilogue warps; LSE and the debug mask go out here
+          sL[(nitem & 1) * kBM + row] = l;
+          if (row_valid && it.half == 0) {
+            const int64_t orow = ((int64_t)it.b * p.T + t) * p.hq + h;
+            if (p.lse) p.lse[orow] = (m + __log2f(l)) * 0.69314718055994531f;
+            if (p.dbg && h == 0) {
+              int32_t* dp = p.dbg + ((int64_t)it.b * p.T + t) * 3;
+              dp[0] = nc_row;
+              dp[1] = lo_row;
+              dp[2] = t;
+            }
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->l_full);
         }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->p_full[sb]);
       }
-      if (!ok) break;
-      // epilogue: O half / l (* gate) -> bf16
-      const uint32_t glast = g + it.ntiles - 1;
-      if (!(ok = mbar_wait(&bars->o_done, glast & 1, abort))) break;
+      g += it.ntiles;
+      ++nitem;
+    }
+    if (!ok) raise_timeout(p, bars);
+  } else {
+    // ------------------------------------------------------------------ epilogue
+    // O half / l (* gate) -> bf16, overlapping the next item's softmax
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+    const uint64_t pol_stream = policy_evict_first();
+    int nitem = 0;
+    bool ok = true;
+    for (int r = 0; ok; ++r) {
+      const int k = item_index(r, G, c);
+      if (k >= p.n_items) break;
+      const Item it = make_item(p, k);
+      const int pos = it.t0 + row / p.hq;
+      const int h = row % p.hq;
+      const bool row_valid = pos < p.T;
+      const int t = min(pos, p.T - 1);
+      if (!(ok = mbar_wait(&bars->o_final, nitem & 1, abort))) break;
+      if (!(ok = mbar_wait(&bars->l_full, nitem & 1, abort))) break;
       tc_fence_after();
-      const float inv = 1.f / l;
+      const float inv = 1.f / sL[(nitem & 1) * kBM + row];
       const int64_t orow = ((int64_t)it.b * p.T + t) * p.hq + h;
       __nv_bfloat16* op = p.O + orow * kD + it.half * kDH;
       const __nv_bfloat16* gp =
@@ -554,6 +629,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       const uint32_t o_addr = tmem + lane_addr + kTmO;
 #pragma unroll 1
       for (int q = 0; q < kDH / 32; ++q) {
+        uint4 gv[4];
+        if (gp) {
+#pragma unroll
+          for (int w = 0; w < 4; ++w) gv[w] = ld_stream_hint(gp + q * 32 + w * 8, pol_stream);
+        }
         uint32_t v[32];
         tmem_ld32(o_addr + q * 32, v);
         tmem_wait_ld();
@@ -561,11 +641,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
 #pragma unroll
         for (int e = 0; e < 32; ++e) o[e] = __uint_as_float(v[e]) * inv;
         if (gp) {
-          const uint4* g4 = reinterpret_cast<const uint4*>(gp + q * 32);
 #pragma unroll
           for (int w = 0; w < 4; ++w) {
-            const uint4 gv = g4[w];
-            const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
+            const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv[w]);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const float2 f = __bfloat1622float2(g2[e]);
@@ -575,7 +653,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           }
         }
         if (row_valid) {
-          uint4* o4 = reinterpret_cast<uint4*>(op + q * 32);
 #pragma unroll
           for (int w = 0; w < 4; ++w) {
             uint4 pk;
@@ -583,23 +660,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             pk.y = pack_bf16x2(o[w * 8 + 2], o[w * 8 + 3]);
             pk.z = pack_bf16x2(o[w * 8 + 4], o[w * 8 + 5]);
             pk.w = pack_bf16x2(o[w * 8 + 6], o[w * 8 + 7]);
-            o4[w] = pk;
+            st_stream_hint(op + q * 32 + w * 8, pk, pol_stream);
           }
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->o_free);
-      if (row_valid && it.half == 0) {
-        if (p.lse) p.lse[orow] = (m + __log2f(l)) * 0.69314718055994531f;
-        if (p.dbg && h == 0) {
-          int32_t* dp = p.dbg + ((int64_t)it.b * p.T + t) * 3;
-          dp[0] = nc_row;
-          dp[1] = lo_row;
-          dp[2] = t;
-        }
-      }
-      g += it.ntiles;
       ++nitem;
     }
     if (!ok) raise_timeout(p, bars);
