@@ -54,7 +54,7 @@ constexpr int kQPairs = 4;                     // Q loaded as 4 boxes of two chu
 constexpr uint32_t kQBytes = kNCh * kChunk128;  // 128 KB
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmS0 = 0, kTmO = 256;
-constexpr int kThreads = 320;  // TMA, UMMA, 4 softmax warps, 4 epilogue warps
+constexpr int kThreads = 384;  // 3 TMA warps, UMMA, 4 softmax warps, 4 epilogue warps
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 enum TileKind { kCompressed = 0, kRaw16 = 1, kRaw128 = 2 };
@@ -263,54 +263,49 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
   const int G = gridDim.x;
   const int c = blockIdx.x;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
+  if (warp == 0 || warp == 10) {
+    // ------------------------------------------------------------------ K/V TMA producers
+    // Two producer warps walk the same load sequence and take turns (even / odd loads):
+    // one issuing thread's bulk-tensor copies are served one after another, so two
+    // issuers double the fill rate. The sequence is the order the UMMA warp consumes:
+    // K0, K1, V0, K2, V1, ..., V(n-1) per item.
     if (elect_one()) {
-      const uint64_t pol_q = policy_evict_first();
+      const uint32_t mine = warp == 0 ? 0u : 1u;
       const uint64_t pol_kv = policy_evict_last();
-      uint32_t cnt = 0;  // ring loads issued
-      int nitem = 0;
+      uint32_t cnt = 0;  // ring loads in the sequence so far (both producers)
       bool ok = true;
-      // Q of an item: 4 boxes of two chunks, each reloaded as soon as the previous item's
-      // last score UMMA on it has finished
-      auto load_q = [&](const Item& it, int which) -> bool {
-        const int qrow = (it.b * p.T + it.t0) * p.hq;
-        for (int q = 0; q < kQPairs; ++q) {
-          if (which > 0 && !mbar_wait(&bars->q_empty[q], (which - 1) & 1, abort)) return false;
-          mbar_expect_tx(&bars->q_full[q], kSlotBytes);
-          tma_load_3d(sQ + q * kSlotBytes, &p.tmQ, &bars->q_full[q], qrow, 2 * q, pol_q);
-        }
-        return true;
-      };
+      // returns the slot to fill, -2 when the other producer owns this load, -1 on time-out
       auto next_slot = [&](uint32_t bytes) -> int {
-        const uint32_t s = cnt % kStages;
-        const uint32_t round = cnt / kStages;
+        const uint32_t n = cnt++;
+        if ((n & 1u) != mine) return -2;
+        const uint32_t s = n % kStages;
+        const uint32_t round = n / kStages;
         if (round > 0 && !mbar_wait(&bars->ring_empty[s], (round - 1) & 1, abort)) return -1;
         mbar_expect_tx(&bars->ring_full[s], bytes);
-        ++cnt;
         return (int)s;
       };
       for (int r = 0; ok; ++r) {
         const int k = item_index(r, G, c);
         if (k >= p.n_items) break;
         const Item it = make_item(p, k);
-        if (p.err_word && visible_count(it.tl, p.block, p.W) > p.n_entries[it.b])
+        if (mine == 0 && p.err_word && visible_count(it.tl, p.block, p.W) > p.n_entries[it.b])
           atomicOr(p.err_word, kErrCacheShort);
-        if (nitem == 0 && !(ok = load_q(it, 0))) break;
-        // ring, in the order the MMA warp consumes it: K0, K1, V0, K2, V1, ..., V(n-1)
         auto load_tile = [&](int j, bool is_v) -> bool {
           const Tile t = tile_of(it, j);
           const int nsl = is_v ? v_slots(t) : k_slots(t);
           for (int q = 0; q < nsl; ++q) {
             if (t.kind == kRaw16) {
               const int s = next_slot(is_v ? 4 * kChunk16 : kNCh * kChunk16);
-              if (s < 0) return false;
-              tma_load_3d(sRing + s * kSlotBytes, is_v ? &p.tmV16 : &p.tmK16,
-                          &bars->ring_full[s], it.b * p.T + t.key0, is_v ? it.half * 4 : 0, pol_kv);
+              if (s == -1) return false;
+              if (s >= 0)
+                tma_load_3d(sRing + s * kSlotBytes, is_v ? &p.tmV16 : &p.tmK16,
+                            &bars->ring_full[s], it.b * p.T + t.key0, is_v ? it.half * 4 : 0,
+                            pol_kv);
               continue;
             }
             const int s = next_slot(kSlotBytes);
-            if (s < 0) return false;
+            if (s == -1) return false;
+            if (s < 0) continue;
             const int chunk = is_v ? it.half * 4 + 2 * q : 2 * q;
             int row;
             const CUtensorMap* map;
@@ -330,26 +325,47 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           }
           return true;
         };
-        const int kn = item_index(r + 1, G, c);
-        const bool has_next = kn < p.n_items;
         for (int j = 0; j < it.ntiles && ok; ++j) {
           ok = load_tile(j, false);
           if (ok && j >= 1) ok = load_tile(j - 1, true);
         }
-        // next item's Q goes in while the last tile's softmax and P.V run
-        if (ok && has_next) ok = load_q(make_item(p, kn), nitem + 1);
         if (ok) ok = load_tile(it.ntiles - 1, true);
+      }
+      if (!ok) {
+        raise_timeout(p, bars);
+        // let this producer's loads already in flight land before shared memory goes away
+        volatile int no_abort = 0;
+        const uint32_t first = cnt > kStages ? cnt - kStages : 0;
+        for (uint32_t q = first; q < cnt; ++q)
+          if ((q & 1u) == mine)
+            mbar_wait(&bars->ring_full[q % kStages], (q / kStages) & 1, &no_abort, 100000000ull);
+      }
+    }
+  } else if (warp == 11) {
+    // ------------------------------------------------------------------ Q TMA producer
+    // Q of an item: 4 boxes of two chunks, each reloaded as soon as the previous item's
+    // last score UMMA on that pair has finished.
+    if (elect_one()) {
+      const uint64_t pol_q = policy_evict_first();
+      int nitem = 0;
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int k = item_index(r, G, c);
+        if (k >= p.n_items) break;
+        const Item it = make_item(p, k);
+        const int qrow = (it.b * p.T + it.t0) * p.hq;
+        for (int q = 0; q < kQPairs && ok; ++q) {
+          if (nitem > 0 && !(ok = mbar_wait(&bars->q_empty[q], (nitem - 1) & 1, abort))) break;
+          mbar_expect_tx(&bars->q_full[q], kSlotBytes);
+          tma_load_3d(sQ + q * kSlotBytes, &p.tmQ, &bars->q_full[q], qrow, 2 * q, pol_q);
+        }
         ++nitem;
       }
       if (!ok) {
         raise_timeout(p, bars);
-        // let loads already in flight land before the CTA's shared memory goes away
         volatile int no_abort = 0;
-        const uint32_t first = cnt > kStages ? cnt - kStages : 0;
-        for (uint32_t q = first; q < cnt; ++q)
-          mbar_wait(&bars->ring_full[q % kStages], (q / kStages) & 1, &no_abort, 100000000ull);
         for (int q = 0; q < kQPairs; ++q)
-          mbar_wait(&bars->q_full[q], nitem & 1, &no_abort, 100000000ull);
+          mbar_wait(&bars->q_full[q], (nitem - 1) & 1, &no_abort, 100000000ull);
       }
     }
   } else if (warp == 1) {
@@ -450,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       umma_commit(&bars->drain);
       mbar_wait(&bars->drain, 0, &no_abort, 100000000ull);
     }
-  } else if (warp < 6) {
+  } else if (warp >= 2 && warp < 6) {
     // ------------------------------------------------------------------ softmax
     const int quad = warp & 3;               // TMEM lane quadrant of this warp
     const int row = quad * 32 + lane;        // tile row == TMEM lane
@@ -599,7 +615,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       ++nitem;
     }
     if (!ok) raise_timeout(p, bars);
-  } else {
+  } else if (warp >= 6 && warp < 10) {
     // ------------------------------------------------------------------ epilogue
     // O half / l (* gate) -> bf16, overlapping the next item's softmax
     const int quad = warp & 3;
