@@ -163,15 +163,18 @@ struct Bars {
   uint64_t q_full[kQPairs], q_empty[kQPairs];
   uint64_t ring_full[kStages], ring_empty[kStages];
   uint64_t s_full[2], p_full[2];
-  uint64_t o_done, o_free, o_final, l_full, drain;
+  uint64_t o_done, o_free, o_final, drain;
+  uint64_t l_full[2];  // per item parity: a single barrier could run two phases ahead
   uint32_t tmem_base;
   int abort;
 };
 static_assert(sizeof(Bars) <= 256, "barrier block too large");
 
-__device__ __forceinline__ void raise_timeout(const Params& p, Bars* bars) {
+// role: 1 K/V producer, 2 Q producer, 3 UMMA issuer, 4 softmax, 5 epilogue; recorded in
+// bit (8 + role) next to HCA_ERR_TIMEOUT so a report names the role that gave up first.
+__device__ __forceinline__ void raise_timeout(const Params& p, Bars* bars, int role) {
   bars->abort = 1;
-  if (p.err_word) atomicOr(p.err_word, kErrTimeout);
+  if (p.err_word) atomicOr(p.err_word, kErrTimeout | (1 << (8 + role)));
 }
 
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
@@ -238,7 +241,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     mbar_init(&bars->o_done, 1);
     mbar_init(&bars->o_free, 4);
     mbar_init(&bars->o_final, 1);
-    mbar_init(&bars->l_full, 4);
+    mbar_init(&bars->l_full[0], 4);
+    mbar_init(&bars->l_full[1], 4);
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
     fence_mbar_init();
@@ -267,8 +271,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     // ------------------------------------------------------------------ K/V TMA producers
     // Two producer warps walk the same load sequence and take turns (even / odd loads):
     // one issuing thread's bulk-tensor copies are served one after another, so two
-    // issuers double the fill rate. The sequence is the order the UMMA warp consumes:
-    // K0, K1, V0, K2, V1, ..., V(n-1) per item.
+    // issuers double the fill rate. The sequence is the order the UMMA warp consumes,
+    // one stream over all items of the CTA: K of tile g, then V of tile g-1.
     if (elect_one()) {
       const uint32_t mine = warp == 0 ? 0u : 1u;
       const uint64_t pol_kv = policy_evict_last();
@@ -284,55 +288,62 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         mbar_expect_tx(&bars->ring_full[s], bytes);
         return (int)s;
       };
+      auto load_tile = [&](const Item& it, int j, bool is_v) -> bool {
+        const Tile t = tile_of(it, j);
+        const int nsl = is_v ? v_slots(t) : k_slots(t);
+        for (int q = 0; q < nsl; ++q) {
+          if (t.kind == kRaw16) {
+            const int s = next_slot(is_v ? 4 * kChunk16 : kNCh * kChunk16);
+            if (s == -1) return false;
+            if (s >= 0)
+              tma_load_3d(sRing + s * kSlotBytes, is_v ? &p.tmV16 : &p.tmK16,
+                          &bars->ring_full[s], it.b * p.T + t.key0, is_v ? it.half * 4 : 0,
+                          pol_kv);
+            continue;
+          }
+          const int s = next_slot(kSlotBytes);
+          if (s == -1) return false;
+          if (s < 0) continue;
+          const int chunk = is_v ? it.half * 4 + 2 * q : 2 * q;
+          int row;
+          const CUtensorMap* map;
+          if (t.kind == kCompressed) {
+            int page = p.page_table[(int64_t)it.b * p.max_pages + t.key0 / p.PE];
+            if (page < 0 || page >= p.num_pages) {
+              if (p.err_word) atomicOr(p.err_word, kErrPageRange);
+              page = 0;
+            }
+            row = page * p.PE + (t.key0 % p.PE);
+            map = is_v ? &p.tmVc : &p.tmKc;
+          } else {
+            row = it.b * p.T + it.hi - kBN + 1;
+            map = is_v ? &p.tmV : &p.tmK;
+          }
+          tma_load_3d(sRing + s * kSlotBytes, map, &bars->ring_full[s], row, chunk, pol_kv);
+        }
+        return true;
+      };
+      // The UMMA warp consumes one stream across items: K of tile g, then V of tile g-1
+      // (which may belong to the previous item), so the next item's first K tile does not
+      // wait for the current item's last softmax.
+      Item pit;
+      int pj = -1;
       for (int r = 0; ok; ++r) {
         const int k = item_index(r, G, c);
         if (k >= p.n_items) break;
         const Item it = make_item(p, k);
         if (mine == 0 && p.err_word && visible_count(it.tl, p.block, p.W) > p.n_entries[it.b])
           atomicOr(p.err_word, kErrCacheShort);
-        auto load_tile = [&](int j, bool is_v) -> bool {
-          const Tile t = tile_of(it, j);
-          const int nsl = is_v ? v_slots(t) : k_slots(t);
-          for (int q = 0; q < nsl; ++q) {
-            if (t.kind == kRaw16) {
-              const int s = next_slot(is_v ? 4 * kChunk16 : kNCh * kChunk16);
-              if (s == -1) return false;
-              if (s >= 0)
-                tma_load_3d(sRing + s * kSlotBytes, is_v ? &p.tmV16 : &p.tmK16,
-                            &bars->ring_full[s], it.b * p.T + t.key0, is_v ? it.half * 4 : 0,
-                            pol_kv);
-              continue;
-            }
-            const int s = next_slot(kSlotBytes);
-            if (s == -1) return false;
-            if (s < 0) continue;
-            const int chunk = is_v ? it.half * 4 + 2 * q : 2 * q;
-            int row;
-            const CUtensorMap* map;
-            if (t.kind == kCompressed) {
-              int page = p.page_table[(int64_t)it.b * p.max_pages + t.key0 / p.PE];
-              if (page < 0 || page >= p.num_pages) {
-                if (p.err_word) atomicOr(p.err_word, kErrPageRange);
-                page = 0;
-              }
-              row = page * p.PE + (t.key0 % p.PE);
-              map = is_v ? &p.tmVc : &p.tmKc;
-            } else {
-              row = it.b * p.T + it.hi - kBN + 1;
-              map = is_v ? &p.tmV : &p.tmK;
-            }
-            tma_load_3d(sRing + s * kSlotBytes, map, &bars->ring_full[s], row, chunk, pol_kv);
-          }
-          return true;
-        };
         for (int j = 0; j < it.ntiles && ok; ++j) {
-          ok = load_tile(j, false);
-          if (ok && j >= 1) ok = load_tile(j - 1, true);
+          ok = load_tile(it, j, false);
+          if (ok && pj >= 0) ok = load_tile(pit, pj, true);
+          pit = it;
+          pj = j;
         }
-        if (ok) ok = load_tile(it.ntiles - 1, true);
       }
+      if (ok && pj >= 0) ok = load_tile(pit, pj, true);
       if (!ok) {
-        raise_timeout(p, bars);
+        raise_timeout(p, bars, 1);
         // let this producer's loads already in flight land before shared memory goes away
         volatile int no_abort = 0;
         const uint32_t first = cnt > kStages ? cnt - kStages : 0;
@@ -362,7 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         ++nitem;
       }
       if (!ok) {
-        raise_timeout(p, bars);
+        raise_timeout(p, bars, 2);
         volatile int no_abort = 0;
         for (int q = 0; q < kQPairs; ++q)
           mbar_wait(&bars->q_full[q], (nitem - 1) & 1, &no_abort, 100000000ull);
@@ -377,90 +388,97 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       bool ok = true;
       const uint32_t qbase = smem_u32(sQ);
       const uint32_t rbase = smem_u32(sRing);
+      auto issue_s = [&](const Item& it, int j, uint32_t gg, int ni) -> bool {
+        const Tile t = tile_of(it, j);
+        const int last = it.ntiles - 1;
+        const uint32_t sb = gg & 1;
+        const uint32_t d_tmem = tmem + kTmS0 + sb * 128;
+        const uint32_t idesc = idesc_bf16_f32(kBM, t.n, false);
+        if (j == 0) {
+          for (int q = 0; q < kQPairs; ++q)
+            if (!mbar_wait(&bars->q_full[q], ni & 1, abort)) return false;
+        }
+        const int nsl = k_slots(t);
+        for (int q = 0; q < nsl; ++q) {
+          const uint32_t s = cnt % kStages;
+          if (!mbar_wait(&bars->ring_full[s], (cnt / kStages) & 1, abort)) return false;
+          tc_fence_after();
+          const uint32_t sbase = rbase + s * kSlotBytes;
+          // chunks of this slot: 2 (128-row kinds, chunk pair q) or all 8 (16-row kind)
+          const int nchunks = t.kind == kRaw16 ? kNCh : 2;
+          const uint32_t cstride = t.kind == kRaw16 ? kChunk16 : kChunk128;
+          for (int cc = 0; cc < nchunks; ++cc) {
+            const int d = t.kind == kRaw16 ? cc : 2 * q + cc;
+            const uint32_t qaddr = qbase + d * kChunk128;
+            const uint32_t kaddr = sbase + cc * cstride + t.rowoff * 128;
+#pragma unroll
+            for (int kk = 0; kk < kKC / 16; ++kk) {
+              const uint64_t ad = sdesc_sw128(qaddr + kk * 32, 16, 1024);
+              const uint64_t bd = sdesc_sw128(kaddr + kk * 32, 16, 1024);
+              umma_ss(d_tmem, ad, bd, idesc, (d | kk) != 0);
+            }
+          }
+          umma_commit(&bars->ring_empty[s]);
+          if (j == last) umma_commit(&bars->q_empty[q]);  // the last tile is 128-row
+          ++cnt;
+        }
+        umma_commit(&bars->s_full[sb]);
+        return true;
+      };
+      auto issue_pv = [&](const Item& it, int j, uint32_t gg, int ni) -> bool {
+        const Tile t = tile_of(it, j);
+        const uint32_t sb = gg & 1;
+        if (!mbar_wait(&bars->p_full[sb], (gg >> 1) & 1, abort)) return false;
+        // the first P.V of an item overwrites O: the epilogue must have read the last one
+        if (j == 0 && ni > 0 && !mbar_wait(&bars->o_free, (ni - 1) & 1, abort)) return false;
+        tc_fence_after();
+        const uint32_t a_tmem = tmem + kTmS0 + sb * 128;
+        const int nsl = v_slots(t);
+        for (int q = 0; q < nsl; ++q) {
+          const uint32_t s = cnt % kStages;
+          if (!mbar_wait(&bars->ring_full[s], (cnt / kStages) & 1, abort)) return false;
+          tc_fence_after();
+          const uint32_t vaddr = rbase + s * kSlotBytes + t.rowoff * 128;
+          // 16-row kind: one N=256 MMA over the 4 chunks (stride 2 KB); 128-row kinds:
+          // N=128 over the slot's 2 chunks (stride 16 KB) into columns 128q..128q+127
+          const uint32_t ncols = t.kind == kRaw16 ? 256 : 128;
+          const uint32_t lbo = t.kind == kRaw16 ? kChunk16 : kChunk128;
+          const uint32_t idesc = idesc_bf16_f32(kBM, ncols, true);
+          const uint32_t d_tmem = tmem + kTmO + q * 128;
+          for (int kk = 0; kk < t.n / 16; ++kk) {
+            // 16 keys = two 8-row swizzle atoms = 2 KB
+            const uint64_t bd = sdesc_sw128(vaddr + kk * 2048, lbo, 1024);
+            umma_ts(d_tmem, a_tmem + kk * 8, bd, idesc, (j > 0 || kk > 0));
+          }
+          umma_commit(&bars->ring_empty[s]);
+          ++cnt;
+        }
+        umma_commit(&bars->o_done);
+        if (j == it.ntiles - 1) umma_commit(&bars->o_final);
+        return true;
+      };
+      // One stream across items: S of tile g, then P.V of tile g-1 (possibly of the
+      // previous item), so the tensor pipe keeps working over item boundaries.
+      Item pit;
+      int pj = -1, pni = 0;
+      uint32_t pgg = 0;
       for (int r = 0; ok; ++r) {
         const int k = item_index(r, G, c);
         if (k >= p.n_items) break;
         const Item it = make_item(p, k);
-        const int last = it.ntiles - 1;
-
-        auto issue_s = [&](int j) -> bool {
-          const Tile t = tile_of(it, j);
-          const uint32_t sb = (g + j) & 1;
-          const uint32_t d_tmem = tmem + kTmS0 + sb * 128;
-          const uint32_t idesc = idesc_bf16_f32(kBM, t.n, false);
-          if (j == 0) {
-            for (int q = 0; q < kQPairs; ++q)
-              if (!mbar_wait(&bars->q_full[q], nitem & 1, abort)) return false;
-          }
-          const int nsl = k_slots(t);
-          for (int q = 0; q < nsl; ++q) {
-            const uint32_t s = cnt % kStages;
-            if (!mbar_wait(&bars->ring_full[s], (cnt / kStages) & 1, abort)) return false;
-            tc_fence_after();
-            const uint32_t sbase = rbase + s * kSlotBytes;
-            // chunks of this slot: 2 (128-row kinds, chunk pair q) or all 8 (16-row kind)
-            const int nchunks = t.kind == kRaw16 ? kNCh : 2;
-            const uint32_t cstride = t.kind == kRaw16 ? kChunk16 : kChunk128;
-            for (int cc = 0; cc < nchunks; ++cc) {
-              const int d = t.kind == kRaw16 ? cc : 2 * q + cc;
-              const uint32_t qaddr = qbase + d * kChunk128;
-              const uint32_t kaddr = sbase + cc * cstride + t.rowoff * 128;
-#pragma unroll
-              for (int kk = 0; kk < kKC / 16; ++kk) {
-                const uint64_t ad = sdesc_sw128(qaddr + kk * 32, 16, 1024);
-                const uint64_t bd = sdesc_sw128(kaddr + kk * 32, 16, 1024);
-                umma_ss(d_tmem, ad, bd, idesc, (d | kk) != 0);
-              }
-            }
-            umma_commit(&bars->ring_empty[s]);
-            if (j == last) umma_commit(&bars->q_empty[q]);  // the last tile is 128-row
-            ++cnt;
-          }
-          umma_commit(&bars->s_full[sb]);
-          return true;
-        };
-        auto issue_pv = [&](int j) -> bool {
-          const Tile t = tile_of(it, j);
-          const uint32_t gg = g + j;
-          const uint32_t sb = gg & 1;
-          if (!mbar_wait(&bars->p_full[sb], (gg >> 1) & 1, abort)) return false;
-          if (j == 0 && nitem > 0 && !mbar_wait(&bars->o_free, (nitem - 1) & 1, abort))
-            return false;
-          tc_fence_after();
-          const uint32_t a_tmem = tmem + kTmS0 + sb * 128;
-          const int nsl = v_slots(t);
-          for (int q = 0; q < nsl; ++q) {
-            const uint32_t s = cnt % kStages;
-            if (!mbar_wait(&bars->ring_full[s], (cnt / kStages) & 1, abort)) return false;
-            tc_fence_after();
-            const uint32_t vaddr = rbase + s * kSlotBytes + t.rowoff * 128;
-            // 16-row kind: one N=256 MMA over the 4 chunks (stride 2 KB); 128-row kinds:
-            // N=128 over the slot's 2 chunks (stride 16 KB) into columns 128q..128q+127
-            const uint32_t ncols = t.kind == kRaw16 ? 256 : 128;
-            const uint32_t lbo = t.kind == kRaw16 ? kChunk16 : kChunk128;
-            const uint32_t idesc = idesc_bf16_f32(kBM, ncols, true);
-            const uint32_t d_tmem = tmem + kTmO + q * 128;
-            for (int kk = 0; kk < t.n / 16; ++kk) {
-              // 16 keys = two 8-row swizzle atoms = 2 KB
-              const uint64_t bd = sdesc_sw128(vaddr + kk * 2048, lbo, 1024);
-              umma_ts(d_tmem, a_tmem + kk * 8, bd, idesc, (j > 0 || kk > 0));
-            }
-            umma_commit(&bars->ring_empty[s]);
-            ++cnt;
-          }
-          umma_commit(&bars->o_done);
-          return true;
-        };
         for (int j = 0; j < it.ntiles && ok; ++j) {
-          ok = issue_s(j);
-          if (ok && j >= 1) ok = issue_pv(j - 1);
+          ok = issue_s(it, j, g + j, nitem);
+          if (ok && pj >= 0) ok = issue_pv(pit, pj, pgg, pni);
+          pit = it;
+          pj = j;
+          pgg = g + j;
+          pni = nitem;
         }
-        if (ok) ok = issue_pv(last);
-        if (ok) umma_commit(&bars->o_final);
         g += it.ntiles;
         ++nitem;
       }
-      if (!ok) raise_timeout(p, bars);
+      if (ok && pj >= 0) ok = issue_pv(pit, pj, pgg, pni);
+      if (!ok) raise_timeout(p, bars, 3);
       // drain: every UMMA issued above has finished before TMEM is released
       volatile int no_abort = 0;
       umma_commit(&bars->drain);
@@ -604,7 +622,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             }
           }
           __syncwarp();
-          if (lane == 0) mbar_arrive(&bars->l_full);
+          if (lane == 0) mbar_arrive(&bars->l_full[nitem & 1]);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -614,7 +632,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       g += it.ntiles;
       ++nitem;
     }
-    if (!ok) raise_timeout(p, bars);
+    if (!ok) raise_timeout(p, bars, 4);
   } else if (warp >= 6 && warp < 10) {
     // ------------------------------------------------------------------ epilogue
     // O half / l (* gate) -> bf16, overlapping the next item's softmax
@@ -633,7 +651,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       const bool row_valid = pos < p.T;
       const int t = min(pos, p.T - 1);
       if (!(ok = mbar_wait(&bars->o_final, nitem & 1, abort))) break;
-      if (!(ok = mbar_wait(&bars->l_full, nitem & 1, abort))) break;
+      if (!(ok = mbar_wait(&bars->l_full[nitem & 1], (nitem >> 1) & 1, abort))) break;
       tc_fence_after();
       const float inv = 1.f / sL[(nitem & 1) * kBM + row];
       const int64_t orow = ((int64_t)it.b * p.T + t) * p.hq + h;
@@ -685,7 +703,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       if (lane == 0) mbar_arrive(&bars->o_free);
       ++nitem;
     }
-    if (!ok) raise_timeout(p, bars);
+    if (!ok) raise_timeout(p, bars, 5);
   }
 
   tc_fence_before();

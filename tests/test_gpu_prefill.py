@@ -68,6 +68,7 @@ def test_bf16_prefill(T, hq, gate, hetero):
     x = inputs.prefill_inputs(1, T, hq, 1, 512, "bf16", seed=1, gate=gate,
                               hetero_blocks=hetero)
     r = run_prefill(x, want_lse=True, want_mask=True)
+    assert int(r["cache"].err.item()) == 0
     ref, lse = _oracle(x, 0, None)
     if hetero:
         compare_peaked(to64(r["O"][0]), ref, p_rounding_bound(x, 0, range(T)), what="O")
@@ -135,3 +136,19 @@ def test_bf16_missing_cache_entries_flagged():
     ops.prefill(desc, Q, K, V, cache)
     torch.cuda.synchronize()
     assert int(cache.err.item()) & B.HCA_ERR_CACHE_SHORT
+
+
+def test_bf16_many_short_items_with_gate_repeated():
+    """Stress the hand-offs between the softmax and the epilogue warps: 16 sequences of
+    200 tokens give each CTA ~20 consecutive items of one or two key tiles, and the gate
+    makes every epilogue slower than the softmax of the next item. No wait may time out
+    (error word 0) and the output must match the oracle on every run."""
+    T, b = 200, 16
+    x = inputs.prefill_inputs(b, T, 64, 1, 512, "bf16", seed=21, gate=True)
+    pos = [0, 1, 63, 127, 128, 129, 150, 199]
+    refs = [_oracle(x, bi, pos)[0] for bi in (0, 7, 15)]
+    for _ in range(4):
+        r = run_prefill(x)
+        assert int(r["cache"].err.item()) == 0
+        for bi, ref in zip((0, 7, 15), refs):
+            compare(to64(r["O"][bi, pos]), ref, BF16_MAX, BF16_MEAN, what=f"O[{bi}]")
