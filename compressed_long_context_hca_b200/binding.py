@@ -28,6 +28,7 @@ HCA_F32 = 1
 HCA_ERR_PAGE_RANGE = 1
 HCA_ERR_CACHE_SHORT = 2
 HCA_ERR_TIMEOUT = 4
+HCA_ERR_CTX_RANGE = 8
 ABI_VERSION = 1
 
 EXPORTED = ("hca_abi_version", "hca_status_string", "hca_set_gate", "hca_compress",

@@ -9,17 +9,16 @@
 //  * The hq <= 64 query heads of a sequence share its KV head, so they form the M = 64 rows
 //    of every UMMA. An M = 64 accumulator occupies TMEM lanes 0-15 of each 32-lane
 //    subpartition; a second one sits at lane offset 16. O (64 x 512 f32) takes lanes
-//    0-15 x 512 columns and the double-buffered scores (64 x 256 each) take lanes 16-31.
-//  * The key list (compressed tiles of up to 256 entries, then the ring tile) is cut into
-//    `nsplit` contiguous ranges; grid = (nsplit, sequences). Each CTA streams its K/V tiles
-//    through a 4-deep ring of 32 KB TMA chunks (256 rows x 64 elements, 128-byte swizzle),
-//    runs S = Q K^T (both operands in shared memory), a two-pass softmax per tile (max,
-//    then exp and the bf16 P written to shared memory in the UMMA K-major swizzled layout),
-//    and O += P V with V N-major.
-//  * Lazy rescaling as in prefill (reference moves when the max grows by more than 8 in
-//    log2 units). A rescale reads and writes whole 32-lane rows of TMEM, so it first waits
-//    until no UMMA is in flight.
-//  * Each CTA writes float32 partials (unnormalised O, reference m in log2 units, sum l) to
+//    0-15 x 512 columns; two score buffers of 256 keys take lanes 16-31.
+//  * The key list (compressed tiles of 128 entries, then the ring tile) is cut into
+//    `nsplit` contiguous splits; grid = (nsplit, sequences). A split is walked in chunks
+//    of two tiles (256 keys) with a running softmax (lazy rescale).
+//  * One load stream per CTA, in the order K(0), K(1), V(0), K(2), V(1), ...: the scores of
+//    chunk c + 1 are computed while the softmax of chunk c runs, and V(c) arrives after it,
+//    so the stream of 3-D TMA boxes (128 rows x two 128-byte chunks, two issuing warps)
+//    does not wait on the softmax. P goes to shared memory in bf16 (two buffers, UMMA
+//    K-major swizzled layout); O += P V with V N-major.
+//  * Each CTA writes float32 partials (unnormalised O, base max m in log2 units, sum l) to
 //    the workspace; merge_kernel combines them per head, applies the gate and casts.
 //  * All mbarrier waits are bounded (HCA_ERR_TIMEOUT on give-up).
 #include <cuda.h>
@@ -36,31 +35,34 @@ namespace {
 
 constexpr int kM = 64;                    // head rows
 constexpr int kD = 512;
-constexpr int kKC = 64;
+constexpr int kKC = 64;                   // elements per 128-byte swizzle row ("chunk")
 constexpr int kNCh = kD / kKC;            // 8
-constexpr int kTN = 256;                  // keys per compressed tile
-constexpr int kRingRows = 128;            // rows of the ring box (window <= 128)
-constexpr uint32_t kChunkBytes = kTN * kKC * 2;         // 32 KB
-constexpr uint32_t kHalfChunkBytes = 128 * kKC * 2;     // 16 KB
+constexpr int kTN = 128;                  // keys per tile (compressed or ring)
+constexpr uint32_t kChunk128 = 128 * kKC * 2;           // 16 KB: 128 rows x one chunk
+constexpr uint32_t kSlotBytes = 2 * kChunk128;          // 32 KB: one 3-D box, 2 chunks
+constexpr int kSlotsPerTile = kNCh / 2;                 // 4 for K, 4 for V
 constexpr uint32_t kQChunkBytes = kM * kKC * 2;         // 8 KB
-constexpr uint32_t kQBytes = kNCh * kQChunkBytes;       // 64 KB
+constexpr uint32_t kQBytes = kNCh * kQChunkBytes;       // 64 KB (two 32 KB boxes)
 constexpr uint32_t kPChunkBytes = kM * kKC * 2;         // 8 KB (64 rows x 64 keys)
-constexpr uint32_t kPBytes = (kTN / kKC) * kPChunkBytes;  // 32 KB
-constexpr int kStages = 4;
-constexpr int kThreads = 192;
+constexpr int kCT = 2;                    // tiles per softmax chunk (256 keys)
+constexpr uint32_t kPBufBytes = kCT * (kTN / kKC) * kPChunkBytes;  // 32 KB per P buffer
+constexpr uint32_t kPBytes = 2 * kPBufBytes;                       // 64 KB
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays below 2^8 between rescales
+constexpr int kStages = 3;
+constexpr int kThreads = 224;             // 2 TMA warps, UMMA warp, 4 softmax warps
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kLaneS = 16u << 16;   // lane offset of the score accumulator
-constexpr float kRescaleThreshold = 8.0f;
 
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffP = kQBytes;
 constexpr uint32_t kOffRing = kOffP + kPBytes;
-constexpr uint32_t kOffBar = kOffRing + kStages * kChunkBytes;
+constexpr uint32_t kOffBar = kOffRing + kStages * kSlotBytes;
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
 
 enum { kCompressed = 0, kRing = 1 };
 
 struct Params {
+  // 3-D maps {64 elements, rows, 8 chunks}
   CUtensorMap tmQ, tmKc, tmVc, tmRk, tmRv;
   const int32_t* ctx_len;
   const int32_t* page_table;
@@ -68,15 +70,15 @@ struct Params {
   int32_t* err_word;
   float* ws_ml;   // [nseq, nsplit, hq, 2]
   float* ws_o;    // [nseq, nsplit, hq, 512]
-  int32_t nseq, hq, W, block, PE, max_pages, num_pages, nsplit;
+  int32_t nseq, seqlen, hq, W, block, PE, max_pages, num_pages, nsplit;
   float scale_log2;
 };
 
 struct Bars {
   uint64_t q_full;
   uint64_t ring_full[kStages], ring_empty[kStages];
-  uint64_t s_full[2], p_full;
-  uint64_t o_done, drain;
+  uint64_t s_full[2], p_full[2], o_done[2];
+  uint64_t drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -94,7 +96,10 @@ __device__ __forceinline__ int round16(int x) { return (x + 15) & ~15; }
 
 __device__ __forceinline__ Seq make_seq(const Params& p, int b, int split) {
   Seq s;
-  s.t = max(p.ctx_len[b] - 1, 0);
+  // ctx_len is clamped into [1, seqlen]: the host sized the splits (and with them the TMEM
+  // columns a split's scores take) for seqlen
+  const int ctx = p.ctx_len[b];
+  s.t = min(max(ctx, 1), p.seqlen) - 1;
   int x = s.t + 1 - p.W;
   int nc = x < 0 ? 0 : x / p.block;
   s.nc = min(nc, min(p.n_entries[b], p.max_pages * p.PE));
@@ -120,6 +125,22 @@ __device__ __forceinline__ Tile tile_of(const Params& p, const Seq& s, int j) {
   return t;
 }
 
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int32_t row, int32_t chunk, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(0), "r"(row), "r"(chunk),
+      "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
 __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -140,10 +161,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       mbar_init(&bars->ring_full[s], 1);
       mbar_init(&bars->ring_empty[s], 1);
     }
-    mbar_init(&bars->s_full[0], 1);
-    mbar_init(&bars->s_full[1], 1);
-    mbar_init(&bars->p_full, 4);
-    mbar_init(&bars->o_done, 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&bars->s_full[x], 1);
+      mbar_init(&bars->p_full[x], 4);
+      mbar_init(&bars->o_done[x], 1);
+    }
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
     fence_mbar_init();
@@ -158,6 +180,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   const uint32_t tmem = bars->tmem_base;
   const Seq sq = make_seq(p, b, split);
   const int ntiles = sq.j1 - sq.j0;
+  const int nchunks = (ntiles + kCT - 1) / kCT;
+  // tiles [chunk_t0(c), chunk_t1(c)) of the split form chunk c
+  auto chunk_t0 = [&](int c) { return sq.j0 + c * kCT; };
+  auto chunk_t1 = [&](int c) { return min(sq.j0 + (c + 1) * kCT, sq.j1); };
 
   if (ntiles <= 0) {
     // empty split: an all-zero partial that the merge skips
@@ -166,62 +192,74 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       ml[0] = -INFINITY;
       ml[1] = 0.f;
     }
-  } else if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
+  } else if (warp == 0 || warp == 6) {
+    // ------------------------------------------------------------------ TMA producers
+    // Two producer warps take turns over one load sequence (even / odd loads): one issuing
+    // thread's bulk-tensor copies are served one after another.
     if (elect_one()) {
+      const uint32_t mine = warp == 0 ? 0u : 1u;
+      const uint64_t pol = policy_evict_first();  // every cache row is read once
       bool ok = true;
-      if (split == 0 && p.err_word) {
-        const int x = sq.t + 1 - p.W;
-        if ((x < 0 ? 0 : x / p.block) > p.n_entries[b]) atomicOr(p.err_word, kErrCacheShort);
+      if (mine == 0) {
+        if (split == 0 && p.err_word) {
+          const int ctx = p.ctx_len[b];
+          if (ctx < 1 || ctx > p.seqlen) atomicOr(p.err_word, kErrCtxRange);
+          const int x = sq.t + 1 - p.W;
+          if ((x < 0 ? 0 : x / p.block) > p.n_entries[b]) atomicOr(p.err_word, kErrCacheShort);
+        }
+        mbar_expect_tx(&bars->q_full, kQBytes);
+        for (int h = 0; h < 2; ++h)
+          tma_load_3d(sQ + h * (kQBytes / 2), &p.tmQ, &bars->q_full, b * p.hq, 4 * h, pol);
       }
-      mbar_expect_tx(&bars->q_full, kQBytes);
-      for (int ch = 0; ch < kNCh; ++ch)
-        tma_load_2d(sQ + ch * kQChunkBytes, &p.tmQ, &bars->q_full, ch * kKC, b * p.hq);
       uint32_t cnt = 0;
       auto load_tile = [&](int j, bool is_v) -> bool {
         const Tile t = tile_of(p, sq, j);
-        for (int ch = 0; ch < kNCh; ++ch) {
-          const uint32_t s = cnt % kStages;
-          const uint32_t round = cnt / kStages;
-          if (round > 0 && !mbar_wait(&bars->ring_empty[s], (round - 1) & 1, abort)) return false;
-          uint8_t* dst = sRing + s * kChunkBytes;
-          if (t.kind == kCompressed) {
-            const int halves = t.key0 + 128 < sq.nc ? 2 : 1;
-            mbar_expect_tx(&bars->ring_full[s], halves * kHalfChunkBytes);
-            for (int hh = 0; hh < halves; ++hh) {
-              const int e = t.key0 + hh * 128;
-              int page = p.page_table[(int64_t)b * p.max_pages + e / p.PE];
-              if (page < 0 || page >= p.num_pages) {
-                if (p.err_word) atomicOr(p.err_word, kErrPageRange);
-                page = 0;
-              }
-              tma_load_2d(dst + hh * kHalfChunkBytes, is_v ? &p.tmVc : &p.tmKc,
-                          &bars->ring_full[s], ch * kKC, page * p.PE + e % p.PE);
-            }
-          } else {
-            mbar_expect_tx(&bars->ring_full[s], kHalfChunkBytes);
-            tma_load_2d(dst, is_v ? &p.tmRv : &p.tmRk, &bars->ring_full[s], ch * kKC, b * p.W);
+        int row;
+        if (t.kind == kCompressed) {
+          int page = p.page_table[(int64_t)b * p.max_pages + t.key0 / p.PE];
+          if (page < 0 || page >= p.num_pages) {
+            if (p.err_word) atomicOr(p.err_word, kErrPageRange);
+            page = 0;
           }
-          ++cnt;
+          row = page * p.PE + t.key0 % p.PE;
+        } else {
+          row = b * p.W;
+        }
+        const CUtensorMap* map = t.kind == kCompressed ? (is_v ? &p.tmVc : &p.tmKc)
+                                                       : (is_v ? &p.tmRv : &p.tmRk);
+        for (int q = 0; q < kSlotsPerTile; ++q) {
+          const uint32_t n = cnt++;
+          if ((n & 1u) != mine) continue;
+          const uint32_t s = n % kStages;
+          const uint32_t round = n / kStages;
+          if (round > 0 && !mbar_wait(&bars->ring_empty[s], (round - 1) & 1, abort)) return false;
+          mbar_expect_tx(&bars->ring_full[s], kSlotBytes);
+          tma_load_3d(sRing + s * kSlotBytes, map, &bars->ring_full[s], row, 2 * q, pol);
         }
         return true;
       };
-      for (int j = 0; j < ntiles && ok; ++j) {
-        ok = load_tile(sq.j0 + j, false);
-        if (ok && j >= 1) ok = load_tile(sq.j0 + j - 1, true);
+      // K(0), then per step c >= 1: K(c) (if any), V(c - 1)
+      for (int c = 0; c <= nchunks && ok; ++c) {
+        if (c < nchunks)
+          for (int j = chunk_t0(c); j < chunk_t1(c) && ok; ++j) ok = load_tile(j, false);
+        if (c >= 1)
+          for (int j = chunk_t0(c - 1); j < chunk_t1(c - 1) && ok; ++j) ok = load_tile(j, true);
       }
-      if (ok) ok = load_tile(sq.j0 + ntiles - 1, true);
       if (!ok) {
         bars->abort = 1;
-        if (p.err_word) atomicOr(p.err_word, kErrTimeout);
+        if (p.err_word) atomicOr(p.err_word, kErrTimeout | (1 << 9));
         volatile int no_abort = 0;
         const uint32_t first = cnt > kStages ? cnt - kStages : 0;
         for (uint32_t q = first; q < cnt; ++q)
-          mbar_wait(&bars->ring_full[q % kStages], (q / kStages) & 1, &no_abort, 100000000ull);
+          if ((q & 1u) == mine)
+            mbar_wait(&bars->ring_full[q % kStages], (q / kStages) & 1, &no_abort, 100000000ull);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ UMMA issuer
+    // Same order as the loads: S(0), then per step c >= 1: S(c) (if any), PV(c - 1).
+    // S(c) writes score buffer c & 1, which the softmax of chunk c - 2 has released:
+    // PV(c - 2), issued earlier, waited for that softmax's p_full.
     if (elect_one()) {
       bool ok = mbar_wait(&bars->q_full, 0, abort);
       tc_fence_after();
@@ -229,181 +267,203 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       const uint32_t qbase = smem_u32(sQ);
       const uint32_t pbase = smem_u32(sP);
       const uint32_t rbase = smem_u32(sRing);
-      auto issue_s = [&](int j) -> bool {
-        const Tile t = tile_of(p, sq, sq.j0 + j);
-        const uint32_t sb = j & 1;
-        const uint32_t d_tmem = tmem + kLaneS + sb * kTN;
-        const uint32_t idesc = idesc_bf16_f32(kM, t.n, false);
-        for (int ch = 0; ch < kNCh; ++ch) {
-          const uint32_t s = cnt % kStages;
-          if (!mbar_wait(&bars->ring_full[s], (cnt / kStages) & 1, abort)) return false;
-          tc_fence_after();
-          const uint32_t kaddr = rbase + s * kChunkBytes;
-          const uint32_t qaddr = qbase + ch * kQChunkBytes;
+      const uint32_t idesc_pv = idesc_bf16_f32(kM, 128, true);
+      for (int c = 0; c <= nchunks && ok; ++c) {
+        if (c < nchunks) {
+          const uint32_t sbuf = tmem + kLaneS + (c & 1) * (kCT * kTN);
+          for (int j = chunk_t0(c); j < chunk_t1(c) && ok; ++j) {
+            const Tile t = tile_of(p, sq, j);
+            const uint32_t d_tmem = sbuf + (j - chunk_t0(c)) * kTN;
+            const uint32_t idesc = idesc_bf16_f32(kM, t.n, false);
+            for (int q = 0; q < kSlotsPerTile && ok; ++q) {
+              const uint32_t s = cnt % kStages;
+              if (!(ok = mbar_wait(&bars->ring_full[s], (cnt / kStages) & 1, abort))) break;
+              tc_fence_after();
+              const uint32_t sbase = rbase + s * kSlotBytes;
+              for (int cc = 0; cc < 2; ++cc) {
+                const int d = 2 * q + cc;
+                const uint32_t kaddr = sbase + cc * kChunk128;
+                const uint32_t qaddr = qbase + d * kQChunkBytes;
 #pragma unroll
-          for (int kk = 0; kk < kKC / 16; ++kk)
-            umma_ss(d_tmem, sdesc_sw128(qaddr + kk * 32, 16, 1024),
-                    sdesc_sw128(kaddr + kk * 32, 16, 1024), idesc, (ch | kk) != 0);
-          umma_commit(&bars->ring_empty[s]);
-          ++cnt;
-        }
-        umma_commit(&bars->s_full[sb]);
-        return true;
-      };
-      auto issue_pv = [&](int j) -> bool {
-        const Tile t = tile_of(p, sq, sq.j0 + j);
-        if (!mbar_wait(&bars->p_full, j & 1, abort)) return false;
-        tc_fence_after();
-        const uint32_t idesc = idesc_bf16_f32(kM, kKC, true);
-        for (int ch = 0; ch < kNCh; ++ch) {
-          const uint32_t s = cnt % kStages;
-          if (!mbar_wait(&bars->ring_full[s], (cnt / kStages) & 1, abort)) return false;
-          tc_fence_after();
-          const uint32_t vaddr = rbase + s * kChunkBytes;
-          for (int kk = 0; kk < t.n / 16; ++kk) {
-            const uint32_t paddr = pbase + (kk >> 2) * kPChunkBytes + (kk & 3) * 32;
-            umma_ss(tmem + ch * kKC, sdesc_sw128(paddr, 16, 1024),
-                    sdesc_sw128(vaddr + kk * 2048, kChunkBytes, 1024), idesc, (j > 0 || kk > 0));
+                for (int kk = 0; kk < kKC / 16; ++kk)
+                  umma_ss(d_tmem, sdesc_sw128(qaddr + kk * 32, 16, 1024),
+                          sdesc_sw128(kaddr + kk * 32, 16, 1024), idesc, (d | kk) != 0);
+              }
+              umma_commit(&bars->ring_empty[s]);
+              ++cnt;
+            }
           }
-          umma_commit(&bars->ring_empty[s]);
-          ++cnt;
+          if (ok) umma_commit(&bars->s_full[c & 1]);
         }
-        umma_commit(&bars->o_done);
-        return true;
-      };
-      for (int j = 0; j < ntiles && ok; ++j) {
-        ok = issue_s(j);
-        if (ok && j >= 1) ok = issue_pv(j - 1);
+        if (c >= 1 && ok) {
+          const int pc = c - 1;
+          if (!(ok = mbar_wait(&bars->p_full[pc & 1], (pc >> 1) & 1, abort))) break;
+          tc_fence_after();
+          const uint32_t pbuf = pbase + (pc & 1) * kPBufBytes;
+          // O[:, 128 q .. 128 q + 127] += P(tile) V(tile, slot q)
+          for (int j = chunk_t0(pc); j < chunk_t1(pc) && ok; ++j) {
+            const Tile t = tile_of(p, sq, j);
+            const int jt = j - chunk_t0(pc);
+            for (int q = 0; q < kSlotsPerTile && ok; ++q) {
+              const uint32_t s = cnt % kStages;
+              if (!(ok = mbar_wait(&bars->ring_full[s], (cnt / kStages) & 1, abort))) break;
+              tc_fence_after();
+              const uint32_t vaddr = rbase + s * kSlotBytes;
+              for (int kk = 0; kk < t.n / 16; ++kk) {
+                const int key16 = jt * (kTN / 16) + kk;  // 16-key group within the chunk
+                const uint32_t paddr = pbuf + (key16 >> 2) * kPChunkBytes + (key16 & 3) * 32;
+                umma_ss(tmem + q * 128, sdesc_sw128(paddr, 16, 1024),
+                        sdesc_sw128(vaddr + kk * 2048, kChunk128, 1024), idesc_pv,
+                        (pc > 0 || jt > 0 || kk > 0));
+              }
+              umma_commit(&bars->ring_empty[s]);
+              ++cnt;
+            }
+          }
+          if (ok) umma_commit(&bars->o_done[pc & 1]);
+        }
       }
-      if (ok) ok = issue_pv(ntiles - 1);
       if (!ok) {
         bars->abort = 1;
-        if (p.err_word) atomicOr(p.err_word, kErrTimeout);
+        if (p.err_word) atomicOr(p.err_word, kErrTimeout | (1 << 11));
       }
       volatile int no_abort = 0;
       umma_commit(&bars->drain);
       mbar_wait(&bars->drain, 0, &no_abort, 100000000ull);
     }
-  } else {
+  } else if (warp >= 2 && warp < 6) {
     // ------------------------------------------------------------------ softmax + partials
+    // Lane l + 16 of a warp holds score row quad * 16 + l; lane l (< 16) holds the O row of
+    // the same head. Per chunk c: wait S(c); row max; lazy rescale; P(c) -> buffer c & 1
+    // (free once PV(c - 2) is done); arrive p_full. Every o_done[x] phase is awaited in
+    // order (PV(c - 2) before chunk c writes P), so a parity wait never sees a barrier that
+    // is two phases away.
     const int quad = warp & 3;
-    const bool s_lane = lane >= 16;           // this thread holds a score row
-    const int hrow = quad * 16 + (lane & 15);  // head row of both the score and O lanes
+    const bool s_lane = lane >= 16;
+    const int hrow = quad * 16 + (lane & 15);
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
     const int t = sq.t;
     const int W = p.W;
-    float m = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < ntiles && ok; ++j) {
-      const Tile tl = tile_of(p, sq, sq.j0 + j);
-      const uint32_t sb = j & 1;
-      if (!(ok = mbar_wait(&bars->s_full[sb], (j >> 1) & 1, abort))) break;
+    float base = -INFINITY, l = 0.f;
+    for (int c = 0; c < nchunks && ok; ++c) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[c & 1], (c >> 1) & 1, abort));
+      if (!ok) break;
       tc_fence_after();
-      const uint32_t s_addr = tmem + lane_addr + sb * kTN;  // lanes 16-31 hold the scores
-      // visible columns form one range [vlo, vhi): a prefix of a compressed tile, or the
-      // ring slots 0..min(W, t+1)-1
-      const int vhi = tl.kind == kCompressed ? min(tl.n, sq.nc - tl.key0) : min(W, t + 1);
-      const uint32_t vlen = vhi > 0 ? (uint32_t)vhi : 0u;
-      // pass 1: row max (branch-free selects, tree reduction)
-      float mraw = -INFINITY;
-      for (int q = 0; q < kTN / 32; ++q) {
-        if (q * 32 >= tl.n) break;
-        uint32_t v[32];
-        tmem_ld32(s_addr + q * 32, v);
-        tmem_wait_ld();
-        float mx[8];
+      const uint32_t sbuf = tmem + lane_addr + (c & 1) * (kCT * kTN);
+      // pass 1: row max over the visible keys of the chunk (branch-free selects)
+      float mx[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
+      for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
+      for (int j = chunk_t0(c); j < chunk_t1(c); ++j) {
+        const Tile tl = tile_of(p, sq, j);
+        // visible columns: a prefix of a compressed tile, or ring slots 0..min(W,t+1)-1
+        const int vhi = tl.kind == kCompressed ? min(tl.n, sq.nc - tl.key0) : min(W, t + 1);
+        const uint32_t vlen = vhi > 0 ? (uint32_t)vhi : 0u;
+        const uint32_t col0 = (j - chunk_t0(c)) * kTN;
+        for (int q = 0; q < kTN / 32; ++q) {
+          if (q * 32 >= tl.n) break;
+          uint32_t v[32];
+          tmem_ld32(sbuf + col0 + q * 32, v);
+          tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const bool in = (uint32_t)(q * 32 + e) < vlen;
-          mx[e & 7] = fmaxf(mx[e & 7], in ? __uint_as_float(v[e]) : -INFINITY);
+          for (int e = 0; e < 32; ++e) {
+            const bool in = (uint32_t)(q * 32 + e) < vlen;
+            mx[e & 7] = fmaxf(mx[e & 7], in ? __uint_as_float(v[e]) : -INFINITY);
+          }
         }
-        mraw = fmaxf(mraw, fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))));
       }
-      const float mt = mraw * p.scale_log2;
-      const float mn = fmaxf(m, mt);
-      float ref = m, alpha = 1.f;
-      bool rescale = false;
-      if (m == -INFINITY) {
-        ref = mn;
-      } else if (mn > m + kRescaleThreshold) {
-        ref = mn;
-        alpha = fast_exp2(m - mn);
-        rescale = true;
+      const float cmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) *
+                         p.scale_log2;
+      // lazy rescale: move the base only when the max grew by more than the threshold
+      const bool grow = s_lane && (c == 0 || cmax > base + kRescaleThreshold);
+      float factor = 1.f;
+      if (grow) {
+        factor = c == 0 ? 1.f : fast_exp2(base - cmax);
+        l *= factor;
+        base = cmax;
       }
-      if (!s_lane) rescale = false;
-      const float base = ref == -INFINITY ? 0.f : ref;
-      // P of the previous tile must have been consumed before P is overwritten
-      if (j > 0) {
-        if (!(ok = mbar_wait(&bars->o_done, (j - 1) & 1, abort))) break;
+      if (c > 0 && __any_sync(0xffffffffu, grow)) {
+        // O rows live in lanes 0-15 next to score lanes 16-31 of the same columns: the
+        // 32-lane read-modify-write below is safe only with no UMMA in flight, i.e. after
+        // PV(c - 1) and (if issued) S(c + 1) have completed. PV(c) waits for our p_full.
+        ok = mbar_wait(&bars->o_done[(c - 1) & 1], ((c - 1) >> 1) & 1, abort);
+        if (ok && c + 1 < nchunks)
+          ok = mbar_wait(&bars->s_full[(c + 1) & 1], ((c + 1) >> 1) & 1, abort);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
         tc_fence_after();
-      }
-      if (__any_sync(0xffffffffu, rescale)) {
-        // no UMMA may write TMEM during the read-modify-write of whole lanes
-        if (j + 1 < ntiles && !(ok = mbar_wait(&bars->s_full[sb ^ 1], ((j + 1) >> 1) & 1, abort)))
-          break;
-        tc_fence_after();
-        const float a_o = __shfl_sync(0xffffffffu, alpha, (lane & 15) + 16);
-        const float a_me = s_lane ? 1.f : a_o;
+        const float f_o = __shfl_sync(0xffffffffu, factor, (lane & 15) + 16);
+        const float f = s_lane ? 1.f : f_o;
 #pragma unroll 1
         for (int q = 0; q < kD / 32; ++q) {
           uint32_t v[32];
           tmem_ld32(tmem + lane_addr + q * 32, v);
           tmem_wait_ld();
-          if (!s_lane) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * a_me);
-          }
+          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
           tmem_st32(tmem + lane_addr + q * 32, v);
         }
         tmem_wait_st();
       }
-      // pass 2: P = exp2(s * scale - ref) -> bf16, K-major 128B-swizzled rows of sP
+      // P buffer c & 1 is free once PV(c - 2) is done
+      if (c >= 2) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done[c & 1], ((c - 2) >> 1) & 1, abort));
+        if (!ok) break;
+      }
+      // pass 2: P = exp2(s * scale - base) -> bf16, K-major 128B-swizzled rows of the buffer
+      uint8_t* pbuf = sP + (c & 1) * kPBufBytes;
+      const float bb = base == -INFINITY ? 0.f : base;
       float ps[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int q = 0; q < kTN / 32; ++q) {
-        if (q * 32 >= tl.n) break;
-        uint32_t v[32];
-        tmem_ld32(s_addr + q * 32, v);
-        tmem_wait_ld();
-        if (s_lane) {
-          uint32_t pk[16];
+      for (int j = chunk_t0(c); j < chunk_t1(c); ++j) {
+        const Tile tl = tile_of(p, sq, j);
+        const int vhi = tl.kind == kCompressed ? min(tl.n, sq.nc - tl.key0) : min(W, t + 1);
+        const uint32_t vlen = vhi > 0 ? (uint32_t)vhi : 0u;
+        const int jt = j - chunk_t0(c);
+        for (int q = 0; q < kTN / 32; ++q) {
+          if (q * 32 >= tl.n) break;
+          uint32_t v[32];
+          tmem_ld32(sbuf + jt * kTN + q * 32, v);
+          tmem_wait_ld();
+          if (s_lane) {
+            uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int c0 = q * 32 + 2 * e;
-            const float p0 = (uint32_t)c0 < vlen
-                                 ? fast_exp2(fmaf(__uint_as_float(v[2 * e]), p.scale_log2, -base))
-                                 : 0.f;
-            const float p1 = (uint32_t)(c0 + 1) < vlen
-                                 ? fast_exp2(fmaf(__uint_as_float(v[2 * e + 1]), p.scale_log2, -base))
-                                 : 0.f;
-            pk[e] = pack_bf16x2(p0, p1);
-            ps[e & 3] += p0 + p1;
-          }
-          // keys q*32 .. q*32+31 -> chunk (q/2), 16-byte units u = (q&1)*4 + w
-          uint8_t* rowp = sP + (q >> 1) * kPChunkBytes + hrow * 128;
+            for (int e = 0; e < 16; ++e) {
+              const int c0 = q * 32 + 2 * e;
+              const float p0 = (uint32_t)c0 < vlen
+                                   ? fast_exp2(fmaf(__uint_as_float(v[2 * e]), p.scale_log2, -bb))
+                                   : 0.f;
+              const float p1 = (uint32_t)(c0 + 1) < vlen
+                                   ? fast_exp2(fmaf(__uint_as_float(v[2 * e + 1]), p.scale_log2, -bb))
+                                   : 0.f;
+              pk[e] = pack_bf16x2(p0, p1);
+              ps[e & 3] += p0 + p1;
+            }
+            // chunk keys jt*128 + q*32 .. -> 64-key P chunk (jt*2 + q/2), units (q&1)*4 + w
+            uint8_t* rowp = pbuf + (jt * 2 + (q >> 1)) * kPChunkBytes + hrow * 128;
 #pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            const int u = (q & 1) * 4 + w;
-            const int us = u ^ (hrow & 7);
-            *reinterpret_cast<uint4*>(rowp + us * 16) =
-                make_uint4(pk[4 * w], pk[4 * w + 1], pk[4 * w + 2], pk[4 * w + 3]);
+            for (int w = 0; w < 4; ++w) {
+              const int u = (q & 1) * 4 + w;
+              const int us = u ^ (hrow & 7);
+              *reinterpret_cast<uint4*>(rowp + us * 16) =
+                  make_uint4(pk[4 * w], pk[4 * w + 1], pk[4 * w + 2], pk[4 * w + 3]);
+            }
           }
         }
       }
-      const float psum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
-      l = l * alpha + psum;
-      m = ref;
+      l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_full);
+      if (lane == 0) mbar_arrive(&bars->p_full[c & 1]);
     }
-    if (ok) ok = mbar_wait(&bars->o_done, (ntiles - 1) & 1, abort);
+    // the last PV's commit covers every earlier UMMA of this CTA
+    if (ok) ok = mbar_wait(&bars->o_done[(nchunks - 1) & 1], ((nchunks - 1) >> 1) & 1, abort);
+    ok = __all_sync(0xffffffffu, ok);
     if (ok) {
       tc_fence_after();
-      const float m_o = __shfl_sync(0xffffffffu, m, (lane & 15) + 16);
+      const float m_o = __shfl_sync(0xffffffffu, base, (lane & 15) + 16);
       const float l_o = __shfl_sync(0xffffffffu, l, (lane & 15) + 16);
       const bool store = !s_lane && hrow < p.hq;
       const int64_t slot = ((int64_t)b * p.nsplit + split) * p.hq + hrow;
@@ -427,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       }
     } else {
       bars->abort = 1;
-      if (p.err_word) atomicOr(p.err_word, kErrTimeout);
+      if (p.err_word) atomicOr(p.err_word, kErrTimeout | (1 << 12));
     }
   }
 
@@ -486,7 +546,7 @@ __global__ void __launch_bounds__(256) merge_kernel(const float* ws_ml, const fl
 bool decode_tc_supported(const hca_desc& d, const hca_cache& c) {
   if (d.dtype != HCA_BF16 || d.head_dim != kD || d.hkv != 1) return false;
   if (d.hq < 1 || d.hq > kM) return false;
-  if (d.window < 1 || d.window > kRingRows || d.block < 1) return false;
+  if (d.window < 1 || d.window > kTN || d.block < 1) return false;
   if (c.page_entries % 128 != 0) return false;
   if (d.gate) {
     const uintptr_t ga = reinterpret_cast<uintptr_t>(d.gate);
@@ -495,15 +555,18 @@ bool decode_tc_supported(const hca_desc& d, const hca_cache& c) {
   return true;
 }
 
+// Splits per sequence. Automatic rule: size a split so that, if every sequence had the
+// largest context, all splits would fill the SMs once (tiles per split
+// = ceil(tiles * batch / SMs)); shorter sequences leave some splits empty.
 int decode_num_splits(const hca_desc& d) {
   const int64_t x = (int64_t)d.seqlen - d.window;
   const int64_t nc = x < 0 ? 0 : x / d.block;
   const int tiles = (int)((nc + kTN - 1) / kTN) + 1;
   if (d.decode_splits > 0) return d.decode_splits < tiles ? d.decode_splits : tiles;
-  const int sms = device_sm_count();
-  int s = d.batch >= sms ? 1 : (2 * sms + d.batch / 2) / (d.batch > 0 ? d.batch : 1);
-  if (d.batch < sms && d.batch * 2 > sms) s = 2;
-  if (d.batch <= sms / 2) s = sms / (d.batch > 0 ? d.batch : 1);
+  const int64_t sms = device_sm_count();
+  const int64_t batch = d.batch > 0 ? d.batch : 1;
+  const int64_t tps = (tiles * batch + sms - 1) / sms;
+  int s = (int)((tiles + tps - 1) / tps);
   if (s < 1) s = 1;
   if (s > tiles) s = tiles;
   return s;
@@ -522,13 +585,13 @@ cudaError_t launch_decode_tc(const hca_desc& d, const void* Q, const int32_t* ct
   const int nsplit = decode_num_splits(d);
   cudaError_t e;
   const uint64_t rowsC = (uint64_t)c.num_pages * c.page_entries;
-  if ((e = encode_bf16_rows(&p.tmQ, Q, (uint64_t)d.batch * d.hq, kD, kKC, kM)) != cudaSuccess)
+  if ((e = encode_bf16_chunks(&p.tmQ, Q, (uint64_t)d.batch * d.hq, kM, 4)) != cudaSuccess)
     return e;
-  if ((e = encode_bf16_rows(&p.tmKc, c.kc_pool, rowsC, kD, kKC, 128)) != cudaSuccess) return e;
-  if ((e = encode_bf16_rows(&p.tmVc, c.vc_pool, rowsC, kD, kKC, 128)) != cudaSuccess) return e;
+  if ((e = encode_bf16_chunks(&p.tmKc, c.kc_pool, rowsC, kTN, 2)) != cudaSuccess) return e;
+  if ((e = encode_bf16_chunks(&p.tmVc, c.vc_pool, rowsC, kTN, 2)) != cudaSuccess) return e;
   const uint64_t rowsR = (uint64_t)d.batch * d.window;
-  if ((e = encode_bf16_rows(&p.tmRk, ring_k, rowsR, kD, kKC, kRingRows)) != cudaSuccess) return e;
-  if ((e = encode_bf16_rows(&p.tmRv, ring_v, rowsR, kD, kKC, kRingRows)) != cudaSuccess) return e;
+  if ((e = encode_bf16_chunks(&p.tmRk, ring_k, rowsR, kTN, 2)) != cudaSuccess) return e;
+  if ((e = encode_bf16_chunks(&p.tmRv, ring_v, rowsR, kTN, 2)) != cudaSuccess) return e;
   p.ctx_len = ctx_len;
   p.page_table = c.page_table;
   p.n_entries = c.n_entries;
@@ -536,6 +599,7 @@ cudaError_t launch_decode_tc(const hca_desc& d, const void* Q, const int32_t* ct
   p.ws_ml = static_cast<float*>(ws);
   p.ws_o = p.ws_ml + (size_t)d.batch * nsplit * d.hq * 2;
   p.nseq = d.batch;
+  p.seqlen = d.seqlen;
   p.hq = d.hq;
   p.W = d.window;
   p.block = d.block;

@@ -151,8 +151,11 @@ __global__ void __launch_bounds__(kWarps * 32) decode_simt_kernel(SimtArgs a) {
   if (row >= rows) return;
   const int h = (int)(row % a.hq);
   const int b = (int)(row / a.hq);
-  const int t = a.ctx_len[b] - 1;
-  if (t < 0) return;
+  // ctx_len is clamped into [1, seqlen] (flagged), the same rule as the tensor-core decode
+  const int ctx = a.ctx_len[b];
+  if ((ctx < 1 || ctx > a.T) && h == 0 && (threadIdx.x & 31) == 0 && a.err_word)
+    atomicOr(a.err_word, kErrCtxRange);
+  const int t = min(max(ctx, 1), a.T) - 1;
   const int64_t goff = (int64_t)b * a.gs0 + (int64_t)h * a.gs2;
   attend_row<true>(a, b, t, h, row, goff);
 }

@@ -14,6 +14,7 @@ namespace hca {
 constexpr int kErrPageRange = 1;
 constexpr int kErrCacheShort = 2;
 constexpr int kErrTimeout = 4;
+constexpr int kErrCtxRange = 8;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

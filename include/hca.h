@@ -60,6 +60,9 @@ typedef enum { HCA_BF16 = 0, HCA_F32 = 1 } hca_dtype;
 /* Bits OR-ed into *hca_cache.err_word by kernels. */
 #define HCA_ERR_PAGE_RANGE 1   /* a page-table entry outside [0, num_pages) was skipped */
 #define HCA_ERR_CACHE_SHORT 2  /* a query needed more entries than n_entries[b] holds */
+#define HCA_ERR_TIMEOUT 4      /* a kernel gave up waiting on one of its own pipeline stages
+                                  (bits 8 and up then name the stage); outputs are invalid */
+#define HCA_ERR_CTX_RANGE 8    /* decode: a ctx_len[b] outside [1, seqlen] was clamped into it */
 
 /* Problem description. Plain data filled by the caller; copied by value into launches. */
 typedef struct {
@@ -146,7 +149,9 @@ size_t hca_decode_workspace_bytes(const hca_desc* d);
 /* One HCA decode step for d->batch sequences ([news 二.1]; the query is the newest token).
  *   Q        [batch, hq, head_dim]   query of the new token of each sequence
  *   ctx_len  device int32 [batch]    context length including the new token; the query
- *                                    position is t = ctx_len - 1, 1 <= ctx_len <= seqlen
+ *                                    position is t = ctx_len - 1, 1 <= ctx_len <= seqlen;
+ *                                    a value outside is clamped into that range and sets
+ *                                    HCA_ERR_CTX_RANGE in *cache->err_word
  *   ring_k/v [batch, window, hkv, head_dim]  raw tokens; token u sits in slot u % window
  *   O        [batch, hq, head_dim];  lse [batch, hq] float32 (optional)
  * Keys are exactly the prefill key set of position t. The key list is cut into splits

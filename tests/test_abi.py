@@ -120,6 +120,11 @@ def test_decode_workspace_and_space(L):
     d = B.make_desc(16, 1 << 20, 64, 1, 512, decode_splits=9)
     n = B.hca_decode_workspace_bytes(d)
     assert n == 16 * 9 * 64 * (512 + 2) * 4
+    # 1M context: 8191 entries -> 64 tiles of 128 + the ring tile = 65 tiles; more splits
+    # than tiles are capped at one tile each
+    d.decode_splits = 100
+    assert B.hca_decode_workspace_bytes(d) == 16 * 65 * 64 * (512 + 2) * 4
+    d.decode_splits = 9
     assert B.hca_decode_workspace_bytes(B.make_desc(1, 1, 64, 1, 512, dtype=B.HCA_F32)) == 0
     c = _cache()
     st = B.hca_attn_decode(d, 16, 16, c, 16, 16, 16, 0, 16, n - 1)

@@ -7,19 +7,26 @@ import torch
 from compressed_long_context_hca_b200 import binding as B
 from compressed_long_context_hca_b200 import inputs, ops
 from oracle import hca_oracle as orc
-from tests.gpu_helpers import (BF16_MAX, BF16_MEAN, F32_MAX, compare, default_scale,
-                               ensure_built, run_prefill, to64)
+from tests.gpu_helpers import (BF16_MAX, BF16_MEAN, F32_MAX, compare, compare_peaked,
+                               default_scale, ensure_built, run_prefill, to64)
 
 pytestmark = pytest.mark.gpu
 
 
 def _setup(nseq, ctx_lo, ctx_hi, dtype="bf16", gate=False, seed=0, hq=64, D=512, W=128,
-           block=128, splits=0, pe=128):
+           block=128, splits=0, pe=128, k_ramp=None):
     ensure_built()
     dev = torch.device("cuda")
     max_ent = max(1, (ctx_hi - W) // block + 1)
     x = inputs.decode_inputs(nseq, hq, 1, D, W, block, ctx_lo, ctx_hi, max_ent, dtype, seed,
                              gate)
+    if k_ramp is not None:
+        # compressed keys of 128-entry tile j scaled by k_ramp**j (then rounded again), so
+        # the running row max grows from one 256-key chunk to the next
+        for b in range(nseq):
+            ek = x.entries_k[b]
+            f = k_ramp ** (torch.arange(ek.shape[0], dtype=torch.float64) // 128)
+            x.entries_k[b] = (ek.double() * f[:, None, None]).to(ek.dtype)
     mp = -(-max_ent // pe)
     cache = B.PagedCache(nseq, max_ent, 1, D, x.q.dtype, pe,
                          page_table=inputs.page_table(nseq, mp), device=dev)
@@ -110,3 +117,41 @@ def test_decode_equals_prefill_row():
         Od, _ = ops.decode(desc, Q[:, t].contiguous(), ctx, r["cache"], rk, rv)
         torch.cuda.synchronize()
         compare(to64(Od[0]), to64(r["O"][0, t]), 1.6e-2, 1e-3, what=f"t={t}")
+
+
+@pytest.mark.parametrize("dtype,hq", [("bf16", 64), ("f32", 4)])
+def test_decode_ctx_len_out_of_range_is_clamped_and_flagged(dtype, hq):
+    """ctx_len outside [1, seqlen] is clamped into that range and raises HCA_ERR_CTX_RANGE;
+    the result then equals a call with the clamped lengths."""
+    x, cache, desc = _setup(3, 300, 9000, dtype=dtype, seed=6, hq=hq)
+    dev = torch.device("cuda")
+    args = (x.q.to(dev), cache, x.ring_k.to(dev), x.ring_v.to(dev))
+    bad = torch.tensor([0, int(x.ctx_len[1]), desc.seqlen + 777], dtype=torch.int32)
+    good = torch.tensor([1, int(x.ctx_len[1]), desc.seqlen], dtype=torch.int32)
+    O_bad, _ = ops.decode(desc, args[0], bad.to(dev), *args[1:])
+    torch.cuda.synchronize()
+    assert int(cache.err.item()) & B.HCA_ERR_CTX_RANGE
+    cache.err.zero_()
+    O_good, _ = ops.decode(desc, args[0], good.to(dev), *args[1:])
+    torch.cuda.synchronize()
+    assert int(cache.err.item()) == 0
+    assert torch.equal(O_bad, O_good)
+
+
+def test_decode_running_max_grows_across_chunks():
+    """Keys whose scale grows tile by tile: the row max rises by far more than the lazy
+    rescale threshold at every 256-key chunk of a split, so O is rescaled in tensor memory
+    between chunks. The softmax is nearly one-hot, so the error bound is the bf16 P
+    rounding bound on the spread of the visible values."""
+    x, cache, desc = _setup(2, 100000, 110000, seed=8, splits=1, k_ramp=1.8)
+    O, lse = _run(x, cache, desc)
+    for b in range(2):
+        ref, rl = _oracle(x, b)
+        t = int(x.ctx_len[b]) - 1
+        nc = max(0, (t + 1 - 128) // 128)
+        ring = [x.ring_v[b, u % 128, 0] for u in range(max(0, t - 127), t + 1)]
+        vals = torch.cat([x.entries_v[b][:nc, 0], torch.stack(ring)]).double()
+        spread = (vals.max(0).values - vals.min(0).values).numpy()[None, :]
+        compare_peaked(to64(O[b]), ref, np.broadcast_to(spread, ref.shape), what=f"O[{b}]")
+        compare(to64(lse[b]), rl, 2e-2, what=f"lse[{b}]", out_bf16=False)
+    assert int(cache.err.item()) == 0
