@@ -12,6 +12,7 @@ Extra results in the same JSON line:
   decode_1m       16 sequences at 1,048,576 context, 4 decode steps each, gate on, with
                   the compress call of the block the first step completes: tokens/s
   prefill_128k    batch 2 x 131072, heterogeneous blocks, fused gate: TFLOP/s
+  compress_2x128k hca_compress of the K and V of 2 x 131072 tokens alone: GB/s vs HBM
   e2e             the main metric with host-resident inputs and output (pinned host
                   memory, H2D + D2H inside the timed region)
   roofline        prefill kernel vs the measured bf16 dense peak (and HBM)
@@ -311,6 +312,8 @@ def gpu_main(args, rank, world, local_rank):
         result["decode_1m"] = bench_decode_1m(args, dev, rank, world, barrier, max_over_ranks,
                                               peaks)
     if args.with_128k:
+        result["compress_2x128k"] = bench_compress_2x128k(args, dev, rank, world, barrier,
+                                                          max_over_ranks, peaks)
         result["prefill_128k"] = bench_prefill_128k(args, dev, rank, world, barrier,
                                                     max_over_ranks, peaks)
 
@@ -443,6 +446,38 @@ def bench_decode_1m(args, dev, rank, world, barrier, max_over_ranks, peaks):
             "clocks": clk}
 
 
+def bench_compress_2x128k(args, dev, rank, world, barrier, max_over_ranks, peaks):
+    """hca_compress alone on the K and V of the training-context prefill workload
+    (2 x 131072 tokens, 2048 entries per sequence): read K + V once, write the entries."""
+    import torch
+    from compressed_long_context_hca_b200 import binding as B
+    from compressed_long_context_hca_b200 import ops
+    b, T = 2, 131072
+    g = torch.Generator(device=dev)
+    g.manual_seed(5000 + rank)
+    K = torch.randn((b, T, 1, D), generator=g, device=dev).to(torch.bfloat16)
+    V = torch.randn((b, T, 1, D), generator=g, device=dev).to(torch.bfloat16)
+    desc = ops.desc_for_prefill(K, K)
+    cache = B.PagedCache(b, T // BLOCK, 1, D, torch.bfloat16, 128, device=dev)
+    stream = torch.cuda.current_stream()
+    clocks = Clocks(dev.index)
+    clocks.start()
+    ms = _time_loop(lambda: ops.compress(desc, K, V, cache), args.decode_steps, 3, barrier,
+                    max_over_ranks, stream)
+    clk = clocks.stop()
+    assert int(cache.err.item()) == 0, "kernel raised an error bit"
+    byts = (K.numel() + V.numel()) * 2 + 2 * b * (T // BLOCK) * D * 2
+    gbs = byts / (ms * 1e-3) / 1e9
+    return {"value": round(world * gbs, 1), "unit": "GB/s", "ms_per_step": round(ms, 4),
+            "workload": "hca_compress of K and V, batch 2 x 131072 tokens, head_dim 512, bf16 "
+                        "(536 MB read, larger than L2)",
+            "gpu_launches_per_step": 1,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+                         "bytes_per_step": byts},
+            "clocks": clk}
+
+
 def bench_prefill_128k(args, dev, rank, world, barrier, max_over_ranks, peaks):
     import torch
     from compressed_long_context_hca_b200 import binding as B
@@ -515,8 +550,8 @@ def reference_main(args, rank, world):
 
 def profile_case(args):
     """Small fixed case for ncu captures: compress + 2 prefill launches (or 2 decode
-    launches); no timing. ``--profile prefill --seqlen T`` or ``--profile decode
-    --nseq N --ctx C``."""
+    launches, or 2 compress launches over 2 sequences); no timing. ``--profile prefill
+    --seqlen T``, ``--profile decode --nseq N --ctx C`` or ``--profile compress --seqlen T``."""
     import torch
     from compressed_long_context_hca_b200 import binding as B
     from compressed_long_context_hca_b200 import build as build_mod
@@ -525,7 +560,15 @@ def profile_case(args):
     dev = torch.device("cuda")
     g = torch.Generator(device=dev)
     g.manual_seed(0)
-    if args.profile == "prefill":
+    if args.profile == "compress":
+        T = args.seqlen
+        K = torch.randn((2, T, 1, D), generator=g, device=dev).to(torch.bfloat16)
+        V = torch.randn((2, T, 1, D), generator=g, device=dev).to(torch.bfloat16)
+        desc = ops.desc_for_prefill(K, K)
+        cache = B.PagedCache(2, -(-T // BLOCK), 1, D, torch.bfloat16, 128, device=dev)
+        for _ in range(2):
+            ops.compress(desc, K, V, cache)
+    elif args.profile == "prefill":
         T = args.seqlen
         Q = torch.randn((1, T, HQ, D), generator=g, device=dev).to(torch.bfloat16)
         K = torch.randn((1, T, 1, D), generator=g, device=dev).to(torch.bfloat16)
@@ -575,7 +618,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--profile", choices=["prefill", "decode"], default=None,
+    ap.add_argument("--profile", choices=["prefill", "decode", "compress"], default=None,
                     help="run a small fixed case for ncu and exit")
     ap.add_argument("--nseq", type=int, default=16)
     ap.add_argument("--ctx", type=int, default=1048576)

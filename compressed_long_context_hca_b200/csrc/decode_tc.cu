@@ -16,8 +16,9 @@
 //  * One load stream per CTA, in the order K(0), K(1), V(0), K(2), V(1), ...: the scores of
 //    chunk c + 1 are computed while the softmax of chunk c runs, and V(c) arrives after it,
 //    so the stream of 3-D TMA boxes (128 rows x two 128-byte chunks, two issuing warps)
-//    does not wait on the softmax. P goes to shared memory in bf16 (two buffers, UMMA
-//    K-major swizzled layout); O += P V with V N-major.
+//    does not wait on the softmax. P goes to shared memory in bf16 (UMMA K-major swizzled
+//    layout); one buffer is enough: P(c) is written once PV(c - 1) is done, and V(c) only
+//    arrives after K(c + 1). O += P V with V N-major.
 //  * Each CTA writes float32 partials (unnormalised O, base max m in log2 units, sum l) to
 //    the workspace; merge_kernel combines them per head, applies the gate and casts.
 //  * All mbarrier waits are bounded (HCA_ERR_TIMEOUT on give-up).
@@ -45,10 +46,9 @@ constexpr uint32_t kQChunkBytes = kM * kKC * 2;         // 8 KB
 constexpr uint32_t kQBytes = kNCh * kQChunkBytes;       // 64 KB (two 32 KB boxes)
 constexpr uint32_t kPChunkBytes = kM * kKC * 2;         // 8 KB (64 rows x 64 keys)
 constexpr int kCT = 2;                    // tiles per softmax chunk (256 keys)
-constexpr uint32_t kPBufBytes = kCT * (kTN / kKC) * kPChunkBytes;  // 32 KB per P buffer
-constexpr uint32_t kPBytes = 2 * kPBufBytes;                       // 64 KB
+constexpr uint32_t kPBytes = kCT * (kTN / kKC) * kPChunkBytes;  // 32 KB: P of one chunk
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays below 2^8 between rescales
-constexpr int kStages = 3;
+constexpr int kStages = 4;
 constexpr int kThreads = 224;             // 2 TMA warps, UMMA warp, 4 softmax warps
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kLaneS = 16u << 16;   // lane offset of the score accumulator
@@ -58,6 +58,12 @@ constexpr uint32_t kOffP = kQBytes;
 constexpr uint32_t kOffRing = kOffP + kPBytes;
 constexpr uint32_t kOffBar = kOffRing + kStages * kSlotBytes;
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
+// End of a CTA: O (64 x 512 f32) is staged row-major in the P + ring region (free once the
+// last PV is done) with a padded row stride, then written out coalesced.
+constexpr int kORow = kD + 4;  // floats per staged row: rows r and r + 8 share banks only
+constexpr uint32_t kOffStage = kOffP;
+static_assert(kOffRing == kOffP + kPBytes, "P and ring must be adjacent");
+static_assert(kM * kORow * 4 + 3 * kM * 4 <= kPBytes + kStages * kSlotBytes, "staging space");
 
 enum { kCompressed = 0, kRing = 1 };
 
@@ -70,6 +76,11 @@ struct Params {
   int32_t* err_word;
   float* ws_ml;   // [nseq, nsplit, hq, 2]
   float* ws_o;    // [nseq, nsplit, hq, 512]
+  // nsplit == 1: the CTA writes the final output itself (no merge launch)
+  __nv_bfloat16* O;
+  float* lse;
+  const __nv_bfloat16* gate;
+  int64_t gs0, gs2;
   int32_t nseq, seqlen, hq, W, block, PE, max_pages, num_pages, nsplit;
   float scale_log2;
 };
@@ -178,6 +189,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
+  // launched as a programmatic dependent: the previous grid on the stream (a merge reading
+  // this workspace, or whatever wrote the inputs) must be complete before the first global
+  // access; then the merge grid may be scheduled as SMs free up
+  pdl_wait();
+  pdl_trigger();
   const Seq sq = make_seq(p, b, split);
   const int ntiles = sq.j1 - sq.j0;
   const int nchunks = (ntiles + kCT - 1) / kCT;
@@ -299,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           const int pc = c - 1;
           if (!(ok = mbar_wait(&bars->p_full[pc & 1], (pc >> 1) & 1, abort))) break;
           tc_fence_after();
-          const uint32_t pbuf = pbase + (pc & 1) * kPBufBytes;
+          const uint32_t pbuf = pbase;
           // O[:, 128 q .. 128 q + 127] += P(tile) V(tile, slot q)
           for (int j = chunk_t0(pc); j < chunk_t1(pc) && ok; ++j) {
             const Tile t = tile_of(p, sq, j);
@@ -334,10 +350,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   } else if (warp >= 2 && warp < 6) {
     // ------------------------------------------------------------------ softmax + partials
     // Lane l + 16 of a warp holds score row quad * 16 + l; lane l (< 16) holds the O row of
-    // the same head. Per chunk c: wait S(c); row max; lazy rescale; P(c) -> buffer c & 1
-    // (free once PV(c - 2) is done); arrive p_full. Every o_done[x] phase is awaited in
-    // order (PV(c - 2) before chunk c writes P), so a parity wait never sees a barrier that
-    // is two phases away.
+    // the same head. Per chunk c: wait S(c); row max; wait PV(c - 1) (frees P, and lets O
+    // be rescaled); lazy rescale; P(c); arrive p_full. PV(c - 1) is awaited at every chunk,
+    // so each o_done[x] phase is awaited in order and a parity wait never sees a barrier
+    // that is two phases away.
     const int quad = warp & 3;
     const bool s_lane = lane >= 16;
     const int hrow = quad * 16 + (lane & 15);
@@ -384,12 +400,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         l *= factor;
         base = cmax;
       }
+      if (c > 0) {
+        // PV(c - 1) done: the P buffer is free and O holds every earlier chunk
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait(&bars->o_done[(c - 1) & 1], ((c - 1) >> 1) & 1, abort));
+        if (!ok) break;
+      }
       if (c > 0 && __any_sync(0xffffffffu, grow)) {
         // O rows live in lanes 0-15 next to score lanes 16-31 of the same columns: the
-        // 32-lane read-modify-write below is safe only with no UMMA in flight, i.e. after
-        // PV(c - 1) and (if issued) S(c + 1) have completed. PV(c) waits for our p_full.
-        ok = mbar_wait(&bars->o_done[(c - 1) & 1], ((c - 1) >> 1) & 1, abort);
-        if (ok && c + 1 < nchunks)
+        // 32-lane read-modify-write below is safe only with no UMMA in flight, i.e. also
+        // after S(c + 1) (if issued) has completed. PV(c) waits for our p_full.
+        if (c + 1 < nchunks)
           ok = mbar_wait(&bars->s_full[(c + 1) & 1], ((c + 1) >> 1) & 1, abort);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
@@ -407,13 +428,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         }
         tmem_wait_st();
       }
-      // P buffer c & 1 is free once PV(c - 2) is done
-      if (c >= 2) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done[c & 1], ((c - 2) >> 1) & 1, abort));
-        if (!ok) break;
-      }
-      // pass 2: P = exp2(s * scale - base) -> bf16, K-major 128B-swizzled rows of the buffer
-      uint8_t* pbuf = sP + (c & 1) * kPBufBytes;
+      // pass 2: P = exp2(s * scale - base) -> bf16, K-major 128B-swizzled rows
+      uint8_t* pbuf = sP;
       const float bb = base == -INFINITY ? 0.f : base;
       float ps[4] = {0.f, 0.f, 0.f, 0.f};
       for (int j = chunk_t0(c); j < chunk_t1(c); ++j) {
@@ -461,33 +477,83 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     // the last PV's commit covers every earlier UMMA of this CTA
     if (ok) ok = mbar_wait(&bars->o_done[(nchunks - 1) & 1], ((nchunks - 1) >> 1) & 1, abort);
     ok = __all_sync(0xffffffffu, ok);
+    float* sO = reinterpret_cast<float*>(smem + kOffStage);  // [64][kORow]
+    float* sM = sO + kM * kORow;                               // row max (log2 units)
+    float* sL = sM + kM;                                       // row sum
+    float* sInv = sL + kM;                                     // 1 / row sum
     if (ok) {
       tc_fence_after();
-      const float m_o = __shfl_sync(0xffffffffu, base, (lane & 15) + 16);
-      const float l_o = __shfl_sync(0xffffffffu, l, (lane & 15) + 16);
-      const bool store = !s_lane && hrow < p.hq;
-      const int64_t slot = ((int64_t)b * p.nsplit + split) * p.hq + hrow;
-      float* op = p.ws_o + slot * kD;
+      if (s_lane) {
+        sM[hrow] = base;
+        sL[hrow] = l;
+        sInv[hrow] = 1.f / l;
+      }
+      float* orow = sO + hrow * kORow;
 #pragma unroll 1
       for (int q = 0; q < kD / 32; ++q) {
         uint32_t v[32];
         tmem_ld32(tmem + lane_addr + q * 32, v);
         tmem_wait_ld();
-        if (store) {
-          float4* o4 = reinterpret_cast<float4*>(op + q * 32);
+        if (!s_lane) {
+          float4* o4 = reinterpret_cast<float4*>(orow + q * 32);
 #pragma unroll
           for (int w = 0; w < 8; ++w)
             o4[w] = make_float4(__uint_as_float(v[4 * w]), __uint_as_float(v[4 * w + 1]),
                                 __uint_as_float(v[4 * w + 2]), __uint_as_float(v[4 * w + 3]));
         }
       }
-      if (store) {
-        p.ws_ml[slot * 2] = m_o;
-        p.ws_ml[slot * 2 + 1] = l_o;
-      }
     } else {
       bars->abort = 1;
       if (p.err_word) atomicOr(p.err_word, kErrTimeout | (1 << 12));
+    }
+    // every softmax warp arrives here exactly once (also after a time-out: the output is
+    // then invalid and flagged)
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    const int tid = threadIdx.x - 64;  // 0..127 over the four softmax warps
+    if (p.nsplit == 1) {
+      // final output: O / l, gate, bf16 in 16-byte units; lse in natural log
+      __nv_bfloat16* ob = p.O + (int64_t)b * p.hq * kD;
+#pragma unroll 4
+      for (int i = tid; i < p.hq * (kD / 8); i += 128) {
+        const int h = i / (kD / 8);
+        const int c = 8 * (i % (kD / 8));
+        const float4 x0 = *reinterpret_cast<const float4*>(sO + h * kORow + c);
+        const float4 x1 = *reinterpret_cast<const float4*>(sO + h * kORow + c + 4);
+        const float inv = sInv[h];
+        float o[8] = {x0.x * inv, x0.y * inv, x0.z * inv, x0.w * inv,
+                      x1.x * inv, x1.y * inv, x1.z * inv, x1.w * inv};
+        if (p.gate) {
+          // the gate is only guaranteed 4-byte aligned: four bf16x2 loads
+          const __nv_bfloat162* gp = reinterpret_cast<const __nv_bfloat162*>(
+              p.gate + (int64_t)b * p.gs0 + (int64_t)h * p.gs2 + c);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 g = __bfloat1622float2(gp[k]);
+            o[2 * k] *= g.x;
+            o[2 * k + 1] *= g.y;
+          }
+        }
+        *reinterpret_cast<uint4*>(ob + (int64_t)h * kD + c) =
+            make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
+                       pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
+      }
+      if (p.lse)
+        for (int h = tid; h < p.hq; h += 128)
+          p.lse[(int64_t)b * p.hq + h] = (sM[h] + __log2f(sL[h])) * 0.69314718055994531f;
+    } else {
+      // split partial: unnormalised O, (max, sum) per head
+      const int64_t slot0 = ((int64_t)b * p.nsplit + split) * p.hq;
+      float* ob = p.ws_o + slot0 * kD;
+      for (int i = tid; i < p.hq * (kD / 4); i += 128) {
+        const int h = i / (kD / 4);
+        const int c = 4 * (i % (kD / 4));
+        *reinterpret_cast<float4*>(ob + (int64_t)h * kD + c) =
+            *reinterpret_cast<const float4*>(sO + h * kORow + c);
+      }
+      for (int h = tid; h < p.hq; h += 128) {
+        p.ws_ml[(slot0 + h) * 2] = sM[h];
+        p.ws_ml[(slot0 + h) * 2 + 1] = sL[h];
+      }
     }
   }
 
@@ -502,43 +568,110 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
 
 // Combine the split partials of one sequence: per head, O = sum_s 2^(m_s - M) O_s /
 // sum_s 2^(m_s - M) l_s, then the gate and the cast to bf16; lse in natural log.
-__global__ void __launch_bounds__(256) merge_kernel(const float* ws_ml, const float* ws_o,
-                                                    int nsplit, int hq,
-                                                    const __nv_bfloat16* gate, int64_t gs0,
-                                                    int64_t gs2, __nv_bfloat16* O, float* lse) {
+// One block per (head, sequence), 4 output columns per thread. The non-empty splits are
+// listed in split order (ballot compaction, so the sums are deterministic) with their
+// weights in shared memory; every thread then walks the list with independent loads.
+constexpr int kMergeThreads = kD / 4;  // 128
+
+__global__ void __launch_bounds__(kMergeThreads) merge_kernel(const float* ws_ml,
+                                                              const float* ws_o, int nsplit,
+                                                              int hq, const __nv_bfloat16* gate,
+                                                              int64_t gs0, int64_t gs2,
+                                                              __nv_bfloat16* O, float* lse) {
+  __shared__ float s_w[kMergeThreads], s_l[kMergeThreads];
+  __shared__ int s_idx[kMergeThreads];
+  __shared__ float s_red[kMergeThreads / 32];
+  __shared__ int s_cnt[kMergeThreads / 32];
+  pdl_wait();  // the decode grid's partials are complete and visible
+  pdl_trigger();
   const int b = blockIdx.y;
   const int h = blockIdx.x;
-  const int d = threadIdx.x * 2;
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int wid = tid >> 5;
+  const int64_t mstride = (int64_t)hq * 2;   // floats between splits in ws_ml
+  const int64_t ostride = (int64_t)hq * kD;  // floats between splits in ws_o
   const float* ml = ws_ml + ((int64_t)b * nsplit * hq + h) * 2;
-  float M = -INFINITY;
-  for (int s = 0; s < nsplit; ++s) {
-    const float ms = ml[(int64_t)s * hq * 2];
-    const float ls = ml[(int64_t)s * hq * 2 + 1];
-    if (ls > 0.f) M = fmaxf(M, ms);
+  const float* ob = ws_o + ((int64_t)b * nsplit * hq + h) * kD + tid * 4;
+
+  float m = -INFINITY;
+  for (int s = tid; s < nsplit; s += kMergeThreads) {
+    const float2 v = *reinterpret_cast<const float2*>(ml + s * mstride);
+    if (v.y > 0.f) m = fmaxf(m, v.x);
   }
-  float L = 0.f, o0 = 0.f, o1 = 0.f;
-  for (int s = 0; s < nsplit; ++s) {
-    const float ms = ml[(int64_t)s * hq * 2];
-    const float ls = ml[(int64_t)s * hq * 2 + 1];
-    if (!(ls > 0.f)) continue;
-    const float w = exp2f(ms - M);
-    L += w * ls;
-    const float2 ov = *reinterpret_cast<const float2*>(
-        ws_o + (((int64_t)b * nsplit + s) * hq + h) * kD + d);
-    o0 += w * ov.x;
-    o1 += w * ov.y;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) s_red[wid] = m;
+  __syncthreads();
+  float M = s_red[0];
+#pragma unroll
+  for (int w = 1; w < kMergeThreads / 32; ++w) M = fmaxf(M, s_red[w]);
+
+  float L = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s0 = 0; s0 < nsplit; s0 += kMergeThreads) {
+    const int s = s0 + tid;
+    float2 v = make_float2(-INFINITY, 0.f);
+    if (s < nsplit) v = *reinterpret_cast<const float2*>(ml + s * mstride);
+    const bool live = v.y > 0.f;
+    const unsigned bal = __ballot_sync(0xffffffffu, live);
+    __syncthreads();  // the previous chunk's list has been consumed
+    if (lane == 0) s_cnt[wid] = __popc(bal);
+    __syncthreads();
+    int off = 0, n = 0;
+#pragma unroll
+    for (int w = 0; w < kMergeThreads / 32; ++w) {
+      off += w < wid ? s_cnt[w] : 0;
+      n += s_cnt[w];
+    }
+    if (live) {
+      const int k = off + __popc(bal & ((1u << lane) - 1u));
+      s_w[k] = exp2f(v.x - M);
+      s_l[k] = v.y;
+      s_idx[k] = s;
+    }
+    __syncthreads();
+    int k = 0;
+    for (; k + 4 <= n; k += 4) {
+      float4 x[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        x[u] = *reinterpret_cast<const float4*>(ob + s_idx[k + u] * ostride);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float w = s_w[k + u];
+        acc.x = fmaf(w, x[u].x, acc.x);
+        acc.y = fmaf(w, x[u].y, acc.y);
+        acc.z = fmaf(w, x[u].z, acc.z);
+        acc.w = fmaf(w, x[u].w, acc.w);
+        L = fmaf(w, s_l[k + u], L);
+      }
+    }
+    for (; k < n; ++k) {
+      const float4 x = *reinterpret_cast<const float4*>(ob + s_idx[k] * ostride);
+      const float w = s_w[k];
+      acc.x = fmaf(w, x.x, acc.x);
+      acc.y = fmaf(w, x.y, acc.y);
+      acc.z = fmaf(w, x.z, acc.z);
+      acc.w = fmaf(w, x.w, acc.w);
+      L = fmaf(w, s_l[k], L);
+    }
   }
   const float inv = 1.f / L;
-  o0 *= inv;
-  o1 *= inv;
+  float o[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
+  const int d = tid * 4;
   if (gate) {
-    const float2 g = __bfloat1622float2(
-        *reinterpret_cast<const __nv_bfloat162*>(gate + (int64_t)b * gs0 + (int64_t)h * gs2 + d));
-    o0 *= g.x;
-    o1 *= g.y;
+    const __nv_bfloat16* gp = gate + (int64_t)b * gs0 + (int64_t)h * gs2 + d;
+    const float2 g0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(gp));
+    const float2 g1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(gp + 2));
+    o[0] *= g0.x;
+    o[1] *= g0.y;
+    o[2] *= g1.x;
+    o[3] *= g1.y;
   }
-  *reinterpret_cast<uint32_t*>(O + ((int64_t)b * hq + h) * kD + d) = pack_bf16x2(o0, o1);
-  if (lse && threadIdx.x == 0) lse[(int64_t)b * hq + h] = (M + __log2f(L)) * 0.69314718055994531f;
+  *reinterpret_cast<uint2*>(O + ((int64_t)b * hq + h) * kD + d) =
+      make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
+  if (lse && tid == 0) lse[(int64_t)b * hq + h] = (M + __log2f(L)) * 0.69314718055994531f;
 }
 
 }  // namespace
@@ -572,9 +705,17 @@ int decode_num_splits(const hca_desc& d) {
   return s;
 }
 
+// Workspace layout: ws_ml [batch, nsplit, hq, 2] float, padded to a multiple of 4 floats so
+// that ws_o [batch, nsplit, hq, 512] float (read and written as float4) starts 16-byte
+// aligned whatever batch * nsplit * hq is.
+static size_t ml_floats(const hca_desc& d, int nsplit) {
+  const size_t n = (size_t)d.batch * nsplit * d.hq * 2;
+  return (n + 3) & ~size_t(3);
+}
+
 size_t decode_tc_workspace_bytes(const hca_desc& d) {
-  const size_t ns = (size_t)decode_num_splits(d);
-  return (size_t)d.batch * ns * d.hq * (kD + 2) * sizeof(float);
+  const int ns = decode_num_splits(d);
+  return (ml_floats(d, ns) + (size_t)d.batch * ns * d.hq * kD) * sizeof(float);
 }
 
 cudaError_t launch_decode_tc(const hca_desc& d, const void* Q, const int32_t* ctx_len,
@@ -597,7 +738,7 @@ cudaError_t launch_decode_tc(const hca_desc& d, const void* Q, const int32_t* ct
   p.n_entries = c.n_entries;
   p.err_word = c.err_word;
   p.ws_ml = static_cast<float*>(ws);
-  p.ws_o = p.ws_ml + (size_t)d.batch * nsplit * d.hq * 2;
+  p.ws_o = p.ws_ml + ml_floats(d, nsplit);
   p.nseq = d.batch;
   p.seqlen = d.seqlen;
   p.hq = d.hq;
@@ -608,6 +749,11 @@ cudaError_t launch_decode_tc(const hca_desc& d, const void* Q, const int32_t* ct
   p.num_pages = c.num_pages;
   p.nsplit = nsplit;
   p.scale_log2 = d.scale * 1.4426950408889634f;
+  p.O = static_cast<__nv_bfloat16*>(O);
+  p.lse = lse;
+  p.gate = static_cast<const __nv_bfloat16*>(d.gate);
+  p.gs0 = d.gate_strides[0];
+  p.gs2 = d.gate_strides[2];
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -617,15 +763,29 @@ cudaError_t launch_decode_tc(const hca_desc& d, const void* Q, const int32_t* ct
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  dim3 grid(nsplit, d.batch);
-  decode_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(p);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  dim3 mgrid(d.hq, d.batch);
-  merge_kernel<<<mgrid, kD / 2, 0, s>>>(p.ws_ml, p.ws_o, nsplit, d.hq,
-                                        static_cast<const __nv_bfloat16*>(d.gate),
-                                        d.gate_strides[0], d.gate_strides[2],
-                                        static_cast<__nv_bfloat16*>(O), lse);
-  return cudaGetLastError();
+  // both grids are programmatic dependents of the grid before them on the stream (each
+  // waits for it with griddepcontrol.wait before touching memory): the merge is scheduled
+  // while decode CTAs drain, and a following decode step's prologue overlaps the merge
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(nsplit, d.batch);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = s;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  if ((e = cudaLaunchKernelEx(&cfg, decode_tc_kernel, p)) != cudaSuccess) return e;
+  if (nsplit == 1) return cudaSuccess;  // the decode CTAs wrote O and lse themselves
+  cudaLaunchConfig_t mcfg = cfg;
+  mcfg.gridDim = dim3(d.hq, d.batch);
+  mcfg.blockDim = dim3(kMergeThreads);
+  mcfg.dynamicSmemBytes = 0;
+  return cudaLaunchKernelEx(&mcfg, merge_kernel, (const float*)p.ws_ml, (const float*)p.ws_o,
+                            nsplit, (int)d.hq, static_cast<const __nv_bfloat16*>(d.gate),
+                            (int64_t)d.gate_strides[0], (int64_t)d.gate_strides[2],
+                            static_cast<__nv_bfloat16*>(O), lse);
 }
 
 // ---------------------------------------------------------------------------------------

@@ -126,6 +126,9 @@ def test_decode_workspace_and_space(L):
     assert B.hca_decode_workspace_bytes(d) == 16 * 65 * 64 * (512 + 2) * 4
     d.decode_splits = 9
     assert B.hca_decode_workspace_bytes(B.make_desc(1, 1, 64, 1, 512, dtype=B.HCA_F32)) == 0
+    # one split of 3 heads: 6 floats of (max, sum) padded to 8 so the float4 partials of O
+    # start 16-byte aligned
+    assert B.hca_decode_workspace_bytes(B.make_desc(1, 100, 3, 1, 512)) == (8 + 3 * 512) * 4
     c = _cache()
     st = B.hca_attn_decode(d, 16, 16, c, 16, 16, 16, 0, 16, n - 1)
     assert st == B.HCA_ENOSPACE

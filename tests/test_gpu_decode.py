@@ -155,3 +155,16 @@ def test_decode_running_max_grows_across_chunks():
         compare_peaked(to64(O[b]), ref, np.broadcast_to(spread, ref.shape), what=f"O[{b}]")
         compare(to64(lse[b]), rl, 2e-2, what=f"lse[{b}]", out_bf16=False)
     assert int(cache.err.item()) == 0
+
+
+@pytest.mark.parametrize("nseq,hq,gate", [(1, 5, True), (3, 33, False), (2, 1, True)])
+def test_decode_bf16_odd_head_counts(nseq, hq, gate):
+    """hq below 64 and odd: the M = 64 UMMA rows past hq are padding, and the split
+    partials of an odd number of heads still start 16-byte aligned in the workspace."""
+    x, cache, desc = _setup(nseq, 9000, 40000, seed=10 + hq, hq=hq, gate=gate)
+    O, lse = _run(x, cache, desc)
+    for b in range(nseq):
+        ref, rl = _oracle(x, b)
+        compare(to64(O[b]), ref, BF16_MAX, BF16_MEAN, what=f"O[{b}]")
+        compare(to64(lse[b]), rl, 2e-2, what=f"lse[{b}]", out_bf16=False)
+    assert int(cache.err.item()) == 0
