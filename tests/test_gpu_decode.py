@@ -81,8 +81,10 @@ def test_decode_batched_config_sampled():
         compare(to64(O[b]), ref, BF16_MAX, BF16_MEAN, what=f"O[{b}]")
 
 
-@pytest.mark.parametrize("splits", [1, 2, 3, 7, 0])
+@pytest.mark.parametrize("splits", [1, 2, 3, 7, 40, 0])
 def test_decode_split_invariance(splits):
+    """Each key list cut into `splits` splits (40: more than the tiles, capped at one tile
+    per split) and merged."""
     x, cache, desc = _setup(5, 20000, 60000, seed=3, splits=splits)
     O, _ = _run(x, cache, desc)
     for b in range(5):
@@ -168,3 +170,14 @@ def test_decode_bf16_odd_head_counts(nseq, hq, gate):
         compare(to64(O[b]), ref, BF16_MAX, BF16_MEAN, what=f"O[{b}]")
         compare(to64(lse[b]), rl, 2e-2, what=f"lse[{b}]", out_bf16=False)
     assert int(cache.err.item()) == 0
+
+
+def test_decode_more_splits_than_tiles():
+    """Short contexts (1 or 2 tiles each) with 50 splits requested: the splits are capped
+    at the tiles of the longest context and the empty ones are skipped by the merge."""
+    x, cache, desc = _setup(3, 100, 300, seed=12, gate=True, splits=50)
+    O, lse = _run(x, cache, desc)
+    for b in range(3):
+        ref, rl = _oracle(x, b)
+        compare(to64(O[b]), ref, BF16_MAX, BF16_MEAN, what=f"O[{b}]")
+        compare(to64(lse[b]), rl, 2e-2, what=f"lse[{b}]", out_bf16=False)
