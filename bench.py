@@ -271,36 +271,69 @@ def gpu_main(args, rank, world, local_rank):
     }
 
     # ---------------------------------------------------------------- e2e (host buffers)
+    # Every step copies its inputs from pinned host memory, runs compress + prefill and
+    # copies its output back. Steps are pipelined over three streams with two device
+    # buffer sets: the upload of step i + 1 and the download of step i - 1 run while step i
+    # computes (PCIe is full duplex). The timed region runs from the first upload to the
+    # last download.
     if not args.no_e2e:
         hQ = Q.cpu().pin_memory()
         hK = K.cpu().pin_memory()
         hV = V.cpu().pin_memory()
         hO = torch.empty(O.shape, dtype=O.dtype).pin_memory()
-        e2e_steps = max(1, min(args.steps, args.e2e_steps))
+        e2e_steps = max(2, min(args.steps, args.e2e_steps))
+        bufs = [(Q, K, V, O), (torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V),
+                               torch.empty_like(O))]
+        up, comp, down = torch.cuda.Stream(), stream, torch.cuda.Stream()
+        ev = lambda: torch.cuda.Event()  # noqa: E731
+        inputs_free = [ev(), ev()]   # compute of the buffer set's last step is done
+        out_free = [ev(), ev()]      # download of the buffer set's last output is done
+        uploaded = [ev(), ev()]
+        computed = [ev(), ev()]
 
-        def e2e_step():
-            Q.copy_(hQ, non_blocking=True)
-            K.copy_(hK, non_blocking=True)
-            V.copy_(hV, non_blocking=True)
-            ops.compress(desc, K, V, cache)
-            ops.prefill(desc, Q, K, V, cache, O=O)
-            hO.copy_(O, non_blocking=True)
+        def run(n):
+            for i in range(n):
+                x = i % 2
+                q_, k_, v_, o_ = bufs[x]
+                with torch.cuda.stream(up):
+                    if i >= 2:
+                        up.wait_event(inputs_free[x])
+                    q_.copy_(hQ, non_blocking=True)
+                    k_.copy_(hK, non_blocking=True)
+                    v_.copy_(hV, non_blocking=True)
+                    uploaded[x].record(up)
+                comp.wait_event(uploaded[x])
+                if i >= 2:
+                    comp.wait_event(out_free[x])
+                with torch.cuda.stream(comp):
+                    ops.compress(desc, k_, v_, cache)
+                    ops.prefill(desc, q_, k_, v_, cache, O=o_)
+                computed[x].record(comp)
+                inputs_free[x].record(comp)
+                with torch.cuda.stream(down):
+                    down.wait_event(computed[x])
+                    hO.copy_(o_, non_blocking=True)
+                    out_free[x].record(down)
 
-        e2e_step()
+        run(2)
         torch.cuda.synchronize()
         barrier()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(e2e_steps):
-            e2e_step()
-        b.record(stream)
+        a.record(up)
+        comp.wait_stream(up)
+        down.wait_stream(up)
+        run(e2e_steps)
+        comp.wait_stream(down)
+        b.record(comp)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(a.elapsed_time(b)) / e2e_steps
         result["e2e"] = {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3),
                          "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 3),
                          "h2d_bytes_per_step": (hQ.numel() + hK.numel() + hV.numel()) * 2,
-                         "d2h_bytes_per_step": hO.numel() * 2}
-        del hQ, hK, hV, hO
+                         "d2h_bytes_per_step": hO.numel() * 2,
+                         "overlap": "uploads / compute / downloads of consecutive steps on "
+                                    "three streams, two device buffer sets"}
+        del hQ, hK, hV, hO, bufs
 
     del Q, K, V, O, cache
     torch.cuda.empty_cache()
@@ -325,6 +358,27 @@ def gpu_main(args, rank, world, local_rank):
                                   "sample": f"{n} random query positions x 64 heads of the 32K "
                                             f"workload, {wall:.1f} s float64 NumPy"}
     return result
+
+
+def _time_graph(fn, steps, warmup, barrier, max_over_ranks, stream):
+    """Capture one call of `fn` (every launch of a decode step) in a CUDA graph and time
+    `steps` replays back to back, as a serving loop replays its decode step: the host's
+    per-launch work is left out, the device work is the same."""
+    import torch
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        for _ in range(warmup):
+            fn()
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    ms = _time_loop(g.replay, steps, warmup, barrier, max_over_ranks, stream)
+    del g
+    return ms
 
 
 def _time_loop(fn, steps, warmup, barrier, max_over_ranks, stream):
@@ -367,7 +421,7 @@ def bench_decode_batched(args, dev, rank, world, barrier, max_over_ranks, peaks)
     clocks = Clocks(dev.index)
     fn = lambda: ops.decode(desc, q, ctx, cache, rk, rv, O=O, workspace=ws)  # noqa: E731
     clocks.start()
-    ms = _time_loop(fn, args.decode_steps, 3, barrier, max_over_ranks, stream)
+    ms = _time_graph(fn, args.decode_steps, 3, barrier, max_over_ranks, stream)
     clk = clocks.stop()
     ctx_h = ctx.cpu().tolist()
     keys = sum((c - WIN) // BLOCK + min(WIN, c) for c in ctx_h)
@@ -423,12 +477,13 @@ def bench_decode_1m(args, dev, rank, world, barrier, max_over_ranks, peaks):
             rv[:, slot].copy_(new_v[s, :, 0])
             if (p + 1) % BLOCK == 0:         # token completes block p // BLOCK
                 B.check(B.hca_compress(cdesc, rk.data_ptr(), rv.data_ptr(), WIN, p // BLOCK,
-                                       1, cache.c, stream.cuda_stream), "hca_compress")
+                                       1, cache.c, torch.cuda.current_stream().cuda_stream),
+                        "hca_compress")
             ops.decode(descs[s], q[s], ctx[s], cache, rk, rv, O=O, workspace=ws)
 
     clocks = Clocks(dev.index)
     clocks.start()
-    ms = _time_loop(four_steps, args.decode_steps, 3, barrier, max_over_ranks, stream)
+    ms = _time_graph(four_steps, args.decode_steps, 3, barrier, max_over_ranks, stream)
     clk = clocks.stop()
     keys = n_ent + WIN
     byts_step = nseq * (keys * D * 2 * 2 + 3 * HQ * D * 2)
