@@ -112,3 +112,28 @@ def decode_inputs(nseq: int, hq: int, hkv: int, D: int, W: int, block: int,
         G = torch.sigmoid(torch.randn((nseq, hq, D), generator=g,
                                       device=device)).to(dt)
     return DecodeInputs(q, ctx, ek, ev, rk, rv, G)
+
+
+@dataclass
+class DecodeStepTokens:
+    q: torch.Tensor          # [steps, nseq, hq, D] query of each step's new token
+    k: torch.Tensor          # [steps, nseq, hkv, D] its key / value (step 0 is unused: the
+    v: torch.Tensor          #   first step's token is already in the ring)
+    G: Optional[torch.Tensor]  # [steps, nseq, hq, D] or None
+
+
+def decode_step_tokens(nseq: int, hq: int, hkv: int, D: int, steps: int,
+                       dtype: str = "bf16", seed: int = 0, gate: bool = False,
+                       device: str = "cpu") -> DecodeStepTokens:
+    """New tokens of consecutive decode steps (query, key, value, gate), N(0, 1)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    dt = _dtype(dtype)
+    q = torch.randn((steps, nseq, hq, D), generator=g, device=device).to(dt)
+    k = torch.randn((steps, nseq, hkv, D), generator=g, device=device).to(dt)
+    v = torch.randn((steps, nseq, hkv, D), generator=g, device=device).to(dt)
+    G = None
+    if gate:
+        G = torch.sigmoid(torch.randn((steps, nseq, hq, D), generator=g,
+                                      device=device)).to(dt)
+    return DecodeStepTokens(q, k, v, G)

@@ -67,7 +67,8 @@ def compare(got, ref, max_tol, mean_tol=None, what="", out_bf16=None):
     if bf16:
         ulp = bf16_ulp(ref)
         bound = np.maximum(max_tol, ulp)
-        mean_bound = mean_tol + float((ulp * (np.abs(ref) >= 2.0)).mean()) / 4
+        mean_bound = (None if mean_tol is None else
+                      mean_tol + float((ulp * (np.abs(ref) >= 2.0)).mean()) / 4)
     else:
         bound = np.full_like(err, max_tol)
         mean_bound = mean_tol

@@ -181,3 +181,56 @@ def test_decode_more_splits_than_tiles():
         ref, rl = _oracle(x, b)
         compare(to64(O[b]), ref, BF16_MAX, BF16_MEAN, what=f"O[{b}]")
         compare(to64(lse[b]), rl, 2e-2, what=f"lse[{b}]", out_bf16=False)
+
+
+def test_decode_1m_config_four_steps_sampled():
+    """Long-context decode: 16 sequences at context 1,048,576 (8191 entries + 128 raw
+    tokens), 64 heads, head_dim 512, gate on, 4 decode steps; the first step's token
+    completes block 8191, whose entry hca_compress writes from the ring. The entry is
+    checked against the block mean, and sequences 0, 7 and 15 against the oracle at every
+    step (the new entry stays invisible to these queries: it is visible from position
+    1,048,703 on)."""
+    dev = torch.device("cuda")
+    nseq, ctx0, W, blk, steps = 16, 1048576, 128, 128, 4
+    n_ent = (ctx0 - W) // blk  # 8191 visible entries
+    x = inputs.decode_inputs(nseq, 64, 1, 512, W, blk, ctx0, ctx0, n_ent + 1, "bf16", seed=21)
+    tok = inputs.decode_step_tokens(nseq, 64, 1, 512, steps, "bf16", seed=22, gate=True)
+    cache = B.PagedCache(nseq, n_ent + 1, 1, 512, torch.bfloat16, 128,
+                         page_table=inputs.page_table(nseq, -(-(n_ent + 1) // 128), 23),
+                         device=dev)
+    for b in range(nseq):
+        cache.fill(b, x.entries_k[b, :n_ent].to(dev), x.entries_v[b, :n_ent].to(dev))
+    rk, rv = x.ring_k.to(dev), x.ring_v.to(dev)
+    rk_h, rv_h = x.ring_k.clone(), x.ring_v.clone()
+    cdesc = B.make_desc(nseq, ctx0, 64, 1, 512)
+    O = torch.empty((nseq, 64, 512), dtype=torch.bfloat16, device=dev)
+    for s in range(steps):
+        p = ctx0 - 1 + s
+        q = x.q if s == 0 else tok.q[s]
+        if s > 0:
+            rk[:, p % W] = tok.k[s].to(dev)
+            rv[:, p % W] = tok.v[s].to(dev)
+            rk_h[:, p % W] = tok.k[s]
+            rv_h[:, p % W] = tok.v[s]
+        if (p + 1) % blk == 0:
+            B.check(B.hca_compress(cdesc, rk.data_ptr(), rv.data_ptr(), W, p // blk, 1, cache.c,
+                                   torch.cuda.current_stream().cuda_stream), "hca_compress")
+        desc = B.make_desc(nseq, ctx0 + steps, 64, 1, 512)
+        ops.attach_gate(desc, tok.G[s].to(dev))
+        ctx = torch.full((nseq,), p + 1, dtype=torch.int32, device=dev)
+        ops.decode(desc, q.to(dev), ctx, cache, rk, rv, O=O)
+        torch.cuda.synchronize()
+        assert int(cache.err.item()) == 0
+        for b in (0, 7, 15):
+            ref, _ = orc.hca_decode(to64(q[b]), to64(x.entries_k[b, :n_ent]),
+                                    to64(x.entries_v[b, :n_ent]), to64(rk_h[b]), to64(rv_h[b]),
+                                    p + 1, blk, W, default_scale(512), gate=to64(tok.G[s][b]))
+            compare(to64(O[b]), ref, BF16_MAX, BF16_MEAN, what=f"step {s} O[{b}]")
+        if s == 0:
+            # entry 8191 = mean of the ring (tokens 8191*128 .. 1048575), in bf16
+            assert int(cache.n_entries[0].item()) == n_ent + 1
+            row = cache.entry_rows(0, n_ent + 1)[n_ent]
+            got = to64(cache.kc.view(-1, 1, 512)[row])
+            want = orc.compress_blocks(to64(rk_h[0]), blk)[0]
+            # one bf16 rounding of a float32 mean (sum of 128 bf16 values / 128): <= 1 ulp
+            compare(got, want, 0.0, what="entry 8191 (K)", out_bf16=True)

@@ -152,3 +152,37 @@ def test_bf16_many_short_items_with_gate_repeated():
         assert int(r["cache"].err.item()) == 0
         for bi, ref in zip((0, 7, 15), refs):
             compare(to64(r["O"][bi, pos]), ref, BF16_MAX, BF16_MEAN, what=f"O[{bi}]")
+
+
+class _Rows:
+    """Rows t of a [T, H, D] tensor held on the GPU, fetched (as float64) only for the
+    positions the oracle evaluates."""
+
+    def __init__(self, t, positions):
+        self.shape = tuple(t.shape)
+        self._rows = {int(p): to64(t[int(p)]) for p in positions}
+
+    def __getitem__(self, i):
+        return self._rows[int(i)]
+
+
+def test_bf16_training_context_config_sampled():
+    """Prefill bf16 at training context: batch 2, T = 131072, 64 query heads sharing 1 KV
+    head, head_dim 512, block 128, window 128; every 4th 128-token block scaled x4; fused
+    gate G = sigmoid(N(0,1)). Inputs drawn on the GPU (Q alone is 17 GB); sampled
+    positions of both sequences against the oracle (first, block edges, the middle, the
+    end, random), with the bf16 P-rounding bound of the peaked softmax."""
+    T = 131072
+    x = inputs.prefill_inputs(2, T, 64, 1, 512, "bf16", seed=0, hetero_blocks=True,
+                              gate=True, device="cuda")
+    r = run_prefill(x)
+    rng = np.random.default_rng(2)
+    pos = sorted(set([0, 127, 128, 129, 255, 256, 383, 511, 16383, 16384, 65535, 65536,
+                      T - 129, T - 2, T - 1] + rng.integers(0, T, 17).tolist()))
+    for bi in range(2):
+        ref, _ = orc.hca_prefill(_Rows(x.Q[bi], pos), to64(x.K[bi]), to64(x.V[bi]), 128, 128,
+                                 default_scale(512), gate=_Rows(x.G[bi], pos), positions=pos)
+        compare_peaked(to64(r["O"][bi, pos]), ref, p_rounding_bound(x, bi, pos),
+                       what=f"O[{bi}]")
+    assert int(r["cache"].err.item()) == 0
+    assert torch.isfinite(r["O"].float()).all()
