@@ -688,9 +688,12 @@ bool decode_tc_supported(const hca_desc& d, const hca_cache& c) {
   return true;
 }
 
-// Splits per sequence. Automatic rule: size a split so that, if every sequence had the
-// largest context, all splits would fill the SMs once (tiles per split
-// = ceil(tiles * batch / SMs)); shorter sequences leave some splits empty.
+// Splits per sequence (d.decode_splits if > 0, capped at the tiles). Automatic rule: the
+// time of a step is about the largest number of 128-key tiles one CTA streams, plus, once
+// a sequence is split, its float32 partials and the merge (about two tiles' worth,
+// measured). Among the split counts that keep every CTA in one wave (splits x batch <=
+// SMs), take the one with the fewest tiles per CTA + 2 if split; ties go to fewer splits.
+// 16 sequences at 1M context (65 tiles) -> 9 splits; 128 sequences of up to 9 tiles -> 1.
 int decode_num_splits(const hca_desc& d) {
   const int64_t x = (int64_t)d.seqlen - d.window;
   const int64_t nc = x < 0 ? 0 : x / d.block;
@@ -698,11 +701,19 @@ int decode_num_splits(const hca_desc& d) {
   if (d.decode_splits > 0) return d.decode_splits < tiles ? d.decode_splits : tiles;
   const int64_t sms = device_sm_count();
   const int64_t batch = d.batch > 0 ? d.batch : 1;
-  const int64_t tps = (tiles * batch + sms - 1) / sms;
-  int s = (int)((tiles + tps - 1) / tps);
-  if (s < 1) s = 1;
-  if (s > tiles) s = tiles;
-  return s;
+  int64_t smax = sms / batch;
+  if (smax < 1) smax = 1;
+  if (smax > tiles) smax = tiles;
+  int best = 1;
+  int64_t best_cost = tiles;
+  for (int64_t sp = 2; sp <= smax; ++sp) {
+    const int64_t cost = (tiles + sp - 1) / sp + 2;
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = (int)sp;
+    }
+  }
+  return best;
 }
 
 // Workspace layout: ws_ml [batch, nsplit, hq, 2] float, padded to a multiple of 4 floats so
