@@ -24,8 +24,9 @@
 //    position of the tile still sees, then one 128-row raw tile ending at the last position.
 //  * Online softmax in base 2 with lazy rescaling: the running reference only moves when
 //    the row max grows by more than 8 (a factor of 256), so O is rarely touched.
-//  * Persistent grid, one CTA per SM, work items (tile, half) in decreasing-work order and
-//    handed out in a snake so that every CTA gets a similar share.
+//  * Persistent grid, one CTA per SM, row tiles in decreasing-work order handed out in a
+//    snake so that every CTA gets a similar share; a CTA runs both output halves of a row
+//    tile back to back, the second on the Q tile already in shared memory.
 //  * Every mbarrier wait is bounded; on time-out the CTA raises HCA_ERR_TIMEOUT (4) in the
 //    error word and unwinds, releasing its TMEM.
 #include <cuda.h>
@@ -103,6 +104,13 @@ __device__ __forceinline__ int visible_count(int t, int block, int W) {
 
 __device__ __forceinline__ int item_index(int r, int G, int c) {
   return r * G + ((r & 1) ? (G - 1 - c) : c);  // snake over the CTAs
+}
+
+// The r-th item of CTA c: row tiles are dealt out in the snake above, and a CTA takes both
+// output halves of a row tile one after the other (items 2 rt and 2 rt + 1), so the second
+// half reuses the Q tile already in shared memory.
+__device__ __forceinline__ int cta_item(int r, int G, int c) {
+  return 2 * item_index(r >> 1, G, c) + (r & 1);
 }
 
 __device__ __forceinline__ Item make_item(const Params& p, int k) {
@@ -329,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       Item pit;
       int pj = -1;
       for (int r = 0; ok; ++r) {
-        const int k = item_index(r, G, c);
+        const int k = cta_item(r, G, c);
         if (k >= p.n_items) break;
         const Item it = make_item(p, k);
         if (mine == 0 && p.err_word && visible_count(it.tl, p.block, p.W) > p.n_entries[it.b])
@@ -355,20 +363,26 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
   } else if (warp == 11) {
     // ------------------------------------------------------------------ Q TMA producer
     // Q of an item: 4 boxes of two chunks, each reloaded as soon as the previous item's
-    // last score UMMA on that pair has finished.
+    // last score UMMA on that pair has finished. The second half of a row tile has the
+    // same Q: its pairs are only handed over again (an arrival without a copy).
     if (elect_one()) {
       const uint64_t pol_q = policy_evict_first();
       int nitem = 0;
       bool ok = true;
       for (int r = 0; ok; ++r) {
-        const int k = item_index(r, G, c);
+        const int k = cta_item(r, G, c);
         if (k >= p.n_items) break;
         const Item it = make_item(p, k);
         const int qrow = (it.b * p.T + it.t0) * p.hq;
+        const bool reuse = (r & 1) != 0;  // same row tile as the previous item
         for (int q = 0; q < kQPairs && ok; ++q) {
           if (nitem > 0 && !(ok = mbar_wait(&bars->q_empty[q], (nitem - 1) & 1, abort))) break;
-          mbar_expect_tx(&bars->q_full[q], kSlotBytes);
-          tma_load_3d(sQ + q * kSlotBytes, &p.tmQ, &bars->q_full[q], qrow, 2 * q, pol_q);
+          if (reuse) {
+            mbar_arrive(&bars->q_full[q]);
+          } else {
+            mbar_expect_tx(&bars->q_full[q], kSlotBytes);
+            tma_load_3d(sQ + q * kSlotBytes, &p.tmQ, &bars->q_full[q], qrow, 2 * q, pol_q);
+          }
         }
         ++nitem;
       }
@@ -463,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       int pj = -1, pni = 0;
       uint32_t pgg = 0;
       for (int r = 0; ok; ++r) {
-        const int k = item_index(r, G, c);
+        const int k = cta_item(r, G, c);
         if (k >= p.n_items) break;
         const Item it = make_item(p, k);
         for (int j = 0; j < it.ntiles && ok; ++j) {
@@ -493,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     int nitem = 0;
     bool ok = true;
     for (int r = 0; ok; ++r) {
-      const int k = item_index(r, G, c);
+      const int k = cta_item(r, G, c);
       if (k >= p.n_items) break;
       const Item it = make_item(p, k);
       const int pos = it.t0 + row / p.hq;
@@ -643,7 +657,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     int nitem = 0;
     bool ok = true;
     for (int r = 0; ok; ++r) {
-      const int k = item_index(r, G, c);
+      const int k = cta_item(r, G, c);
       if (k >= p.n_items) break;
       const Item it = make_item(p, k);
       const int pos = it.t0 + row / p.hq;
@@ -778,7 +792,7 @@ cudaError_t launch_prefill_tc(const hca_desc& d, const void* Q, const void* K, c
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  const int grid = min(p.n_items, device_sm_count());
+  const int grid = min(p.n_items / 2, device_sm_count());  // row tiles (pairs of items)
   prefill_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(p);
   return cudaGetLastError();
 }
