@@ -13,9 +13,11 @@
 //    output half (256 columns) and two 128-column score buffers. Both halves compute the
 //    full scores (the price of the split: 1.5x tensor work; a later design removes it).
 //  * Q (128 x 512 bf16, 128 KB) stays in shared memory for the tile; K and V stream through
-//    a ring of 16 KB TMA chunks (128 rows x 64 elements, 128-byte swizzle).
-//  * Warp roles: warp 0 issues TMA, warp 1 issues UMMA (single thread), warps 2-5 run the
-//    online softmax (one row per thread, TMEM lane = row) and the epilogue.
+//    a ring of three 32 KB slots (3-D TMA boxes of 128 rows x two 128-byte chunks, 128-byte
+//    swizzle).
+//  * Warp roles: warps 0 and 10 stream K/V and warp 11 streams Q through TMA, warp 1 issues
+//    UMMA (single thread), warps 2-5 run the online softmax (one row per thread, TMEM
+//    lane = row), warps 6-9 the epilogue (O / l, gate, bf16) of the previous item.
 //  * S = Q K^T runs as kind::f16 with both operands in shared memory; P is rounded to bf16
 //    and written back into the score columns of TMEM, and O += P V runs with A from TMEM
 //    and V (N-major) from shared memory.
