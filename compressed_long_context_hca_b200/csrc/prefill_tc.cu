@@ -738,6 +738,9 @@ bool prefill_tc_supported(const hca_desc& d, const hca_cache& c) {
   if (d.hq < 8 || d.hq > 128 || (128 % d.hq) != 0) return false;
   if (d.window < 1 || d.window > 128 || d.block < 1) return false;
   if (c.page_entries % kBN != 0) return false;
+  // TMA row coordinates and row indices are 32-bit
+  if ((int64_t)d.batch * d.seqlen * d.hq >= (int64_t(1) << 31)) return false;
+  if ((int64_t)c.num_pages * c.page_entries >= (int64_t(1) << 31)) return false;
   if (d.gate) {
     const uintptr_t ga = reinterpret_cast<uintptr_t>(d.gate);
     if (ga % 16 || d.gate_strides[0] % 8 || d.gate_strides[1] % 8 || d.gate_strides[2] % 8)

@@ -135,7 +135,8 @@ int32_t hca_compress(const hca_desc* d, const void* K, const void* V,
  *   dbg_mask[(b*seqlen+t)*3 + {0,1,2}] = (n_c(t), window lo, window hi) (if non-NULL)
  * Compressed entries are read from `cache` (hca_compress must have written them).
  * Kernels: bf16 -> tcgen05/TMEM tensor-core kernel (needs head_dim 512, hkv 1, hq in
- * {8,16,32,64,128}, window <= 128, page_entries % 128 == 0); f32 -> CUDA-core kernel
+ * {8,16,32,64,128}, window <= 128, page_entries % 128 == 0, batch*seqlen*hq and
+ * num_pages*page_entries below 2^31); f32 -> CUDA-core kernel
  * (head_dim % 32 == 0, head_dim <= 512, any block/window).
  * Errors: HCA_EINVAL, HCA_EUNSUPPORTED, HCA_ECUDA. */
 int32_t hca_attn_prefill(const hca_desc* d, const void* Q, const void* K, const void* V,
@@ -158,7 +159,7 @@ size_t hca_decode_workspace_bytes(const hca_desc* d);
  * (d->decode_splits, 0 = automatic), each split writes float32 partial (O, max, sum) into
  * `workspace`, and a merge kernel combines them, applies the gate and casts.
  * Kernels: bf16 -> tcgen05/TMEM kernel (head_dim 512, hkv 1, hq <= 64, window <= 128,
- * page_entries % 128 == 0); f32 -> CUDA-core kernel.
+ * page_entries % 128 == 0, num_pages*page_entries below 2^31); f32 -> CUDA-core kernel.
  * Errors: HCA_EINVAL, HCA_EUNSUPPORTED, HCA_ENOSPACE (workspace_bytes too small),
  * HCA_ECUDA. */
 int32_t hca_attn_decode(const hca_desc* d, const void* Q, const int32_t* ctx_len,

@@ -98,6 +98,15 @@ def test_validation_rejects_before_launch(L):
     assert B.hca_attn_prefill(d6, 16, 16, 16, c, 16) == B.HCA_EUNSUPPORTED
     # misaligned pointer
     assert B.hca_attn_prefill(d, 16 + 2, 16, 16, c, 16) == B.HCA_EINVAL
+    # 32-bit row coordinates of the tensor-core kernels: batch * seqlen * hq and the pool's
+    # rows must stay below 2^31
+    big = B.make_desc(64, 1 << 20, 64, 1, 512)
+    assert B.hca_attn_prefill(big, 16, 16, 16, c, 16) == B.HCA_EUNSUPPORTED
+    c3 = _cache()
+    c3.page_entries, c3.num_pages = 1 << 16, 1 << 15
+    assert B.hca_attn_prefill(d, 16, 16, 16, c3, 16) == B.HCA_EUNSUPPORTED
+    dd = B.make_desc(1, 1000, 64, 1, 512)
+    assert B.hca_attn_decode(dd, 16, 16, c3, 16, 16, 16, 0, 16, 1 << 30) == B.HCA_EUNSUPPORTED
 
 
 def test_compress_space_and_range_checks(L):
