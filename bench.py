@@ -159,9 +159,28 @@ def blas_threads() -> int:
 
 
 # ------------------------------------------------------------------ GPU workloads
-def gpu_main(args, rank, world, local_rank):
+def rank_tools(world, device):
+    """The two collectives of a timed region: a barrier on both sides, and the max over
+    ranks of the measured time (NCCL tensors on the GPU; CPU tensors under gloo)."""
     import torch
     import torch.distributed as dist
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    return barrier, max_over_ranks
+
+
+def gpu_main(args, rank, world, local_rank):
+    import torch
     from compressed_long_context_hca_b200 import binding as B
     from compressed_long_context_hca_b200 import build as build_mod
     from compressed_long_context_hca_b200 import ops
@@ -175,16 +194,7 @@ def gpu_main(args, rank, world, local_rank):
     stream = torch.cuda.current_stream()
     peaks, peak_kind = load_peaks()
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    barrier, max_over_ranks = rank_tools(world, dev)
 
     # ---------------------------------------------------------------- main: 32K prefill
     T = args.seqlen
