@@ -73,6 +73,7 @@ struct CompressArgs {
   int32_t* err_word;
   int64_t batch_stride_rows;  // token rows between sequences
   int32_t row_vecs;           // 16-byte vectors per token row (hkv * head_dim)
+  int32_t part_vecs;          // of which one CTA handles (row_vecs / column parts)
   int32_t groups;             // row groups per CTA
   int32_t seqlen, block, first_block, n_blocks;
   int32_t page_entries, max_pages, num_pages;
@@ -84,7 +85,8 @@ __global__ void __launch_bounds__(kThreads) compress_kernel(CompressArgs a) {
   constexpr int N = V16::N;
   const int jrel = blockIdx.x;
   const int b = blockIdx.y;
-  const int which = blockIdx.z;  // 0: K, 1: V
+  const int which = blockIdx.z & 1;          // 0: K, 1: V
+  const int vofs = (blockIdx.z >> 1) * a.part_vecs;  // this CTA's columns of the row
   const int j = a.first_block + jrel;
   const int tok0 = j * a.block;
   const int count = min(a.block, a.seqlen - tok0);
@@ -93,36 +95,37 @@ __global__ void __launch_bounds__(kThreads) compress_kernel(CompressArgs a) {
 
   const uint4* src = reinterpret_cast<const uint4*>(a.src[which]) +
                      ((int64_t)b * a.batch_stride_rows + (int64_t)jrel * a.block) * a.row_vecs;
-  const int lanes = a.row_vecs < kThreads ? a.row_vecs : kThreads;
+  const int lanes = a.part_vecs < kThreads ? a.part_vecs : kThreads;
   const int g = threadIdx.x / lanes;
   const int v0 = threadIdx.x % lanes;
   const bool active = g < a.groups;
 
-  for (int vbase = 0; vbase < a.row_vecs; vbase += lanes) {
+  for (int vbase = 0; vbase < a.part_vecs; vbase += lanes) {
     const int v = vbase + v0;
     float acc[N];
 #pragma unroll
     for (int i = 0; i < N; ++i) acc[i] = 0.f;
-    if (active && v < a.row_vecs) {
+    if (active && v < a.part_vecs) {
       int r = g;
       // 4 independent 16-byte loads in flight per thread
       for (; r + 3 * a.groups < count; r += 4 * a.groups) {
-        uint4 x0 = ld_stream(src + (int64_t)r * a.row_vecs + v);
-        uint4 x1 = ld_stream(src + (int64_t)(r + a.groups) * a.row_vecs + v);
-        uint4 x2 = ld_stream(src + (int64_t)(r + 2 * a.groups) * a.row_vecs + v);
-        uint4 x3 = ld_stream(src + (int64_t)(r + 3 * a.groups) * a.row_vecs + v);
+        uint4 x0 = ld_stream(src + (int64_t)r * a.row_vecs + vofs + v);
+        uint4 x1 = ld_stream(src + (int64_t)(r + a.groups) * a.row_vecs + vofs + v);
+        uint4 x2 = ld_stream(src + (int64_t)(r + 2 * a.groups) * a.row_vecs + vofs + v);
+        uint4 x3 = ld_stream(src + (int64_t)(r + 3 * a.groups) * a.row_vecs + vofs + v);
         V16::add(x0, acc);
         V16::add(x1, acc);
         V16::add(x2, acc);
         V16::add(x3, acc);
       }
-      for (; r < count; r += a.groups) V16::add(ld_stream(src + (int64_t)r * a.row_vecs + v), acc);
+      for (; r < count; r += a.groups)
+        V16::add(ld_stream(src + (int64_t)r * a.row_vecs + vofs + v), acc);
       float* dst = red + ((int64_t)g * lanes + v0) * N;
 #pragma unroll
       for (int i = 0; i < N; ++i) dst[i] = acc[i];
     }
     __syncthreads();
-    if (g == 0 && v < a.row_vecs) {
+    if (g == 0 && v < a.part_vecs) {
       float sum[N];
 #pragma unroll
       for (int i = 0; i < N; ++i) sum[i] = 0.f;
@@ -139,13 +142,13 @@ __global__ void __launch_bounds__(kThreads) compress_kernel(CompressArgs a) {
         if (a.err_word) atomicOr(a.err_word, kErrPageRange);
       } else {
         const int64_t row = (int64_t)page * a.page_entries + j % a.page_entries;
-        uint4* dst = reinterpret_cast<uint4*>(a.pool[which]) + row * a.row_vecs + v;
+        uint4* dst = reinterpret_cast<uint4*>(a.pool[which]) + row * a.row_vecs + vofs + v;
         *dst = V16::pack(sum);
       }
     }
     __syncthreads();
   }
-  if (which == 0 && jrel == a.n_blocks - 1 && threadIdx.x == 0)
+  if (which == 0 && vofs == 0 && jrel == a.n_blocks - 1 && threadIdx.x == 0)
     a.n_entries[b] = a.first_block + a.n_blocks;
 }
 
@@ -172,12 +175,20 @@ cudaError_t launch_compress(const hca_desc& d, const void* K, const void* V,
   a.page_entries = c.page_entries;
   a.max_pages = c.max_pages;
   a.num_pages = c.num_pages;
-  const int lanes = a.row_vecs < kThreads ? a.row_vecs : kThreads;
+  // Few blocks (a decode step completing one block per sequence): split each row's columns
+  // over up to 8 CTAs until there are about two CTAs per SM, so that enough loads are in
+  // flight; each CTA then walks the block's rows over fewer columns.
+  int csplit = 1;
+  const int64_t ctas = (int64_t)n_blocks * d.batch * 2;
+  const int64_t want = 2 * (int64_t)device_sm_count();
+  while (csplit < 8 && ctas * csplit < want && a.row_vecs % (2 * csplit) == 0) csplit *= 2;
+  a.part_vecs = a.row_vecs / csplit;
+  const int lanes = a.part_vecs < kThreads ? a.part_vecs : kThreads;
   a.groups = kThreads / lanes;
   if (a.groups > d.block) a.groups = d.block;
   const int vec_elems = 16 / esize;
   const size_t smem = (size_t)a.groups * lanes * vec_elems * sizeof(float);
-  dim3 grid(n_blocks, d.batch, 2);
+  dim3 grid(n_blocks, d.batch, 2 * csplit);
   if (d.dtype == HCA_BF16) {
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(compress_kernel<__nv_bfloat16>,
