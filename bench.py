@@ -40,10 +40,11 @@ if ROOT not in sys.path:
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM bytes (read + write) of one prefill launch of the 32K workload, from an ncu capture
-# of the 8K case (profiles/prefill_tc_kernel_8k_bf16.md: 1.038 GB) scaled by query
-# positions (x4; Q and O dominate, K/V stay in L2). Keyed by the SHA-1 prefix of the kernel
-# source the capture was made on: any change to the kernel makes the figure null.
-PREFILL_TRAFFIC = {"05e476ddcd2f": 4.151e9}
+# of the 8K case scaled by query positions (x4; Q and O dominate, K/V stay in L2). Keyed by
+# the SHA-1 prefix of the kernel source the capture was made on: any change to the kernel
+# makes the figure null.
+PREFILL_KERNEL_SRC = "prefill_pair.cu"
+PREFILL_TRAFFIC = {}
 D, HQ, BLOCK, WIN = 512, 64, 128, 128
 
 
@@ -246,7 +247,7 @@ def gpu_main(args, rank, world, local_rank):
     traffic = args.traffic
     if traffic is None and T == 32768:
         import hashlib
-        src = os.path.join(ROOT, "compressed_long_context_hca_b200", "csrc", "prefill_tc.cu")
+        src = os.path.join(ROOT, "compressed_long_context_hca_b200", "csrc", PREFILL_KERNEL_SRC)
         with open(src, "rb") as f:
             traffic = PREFILL_TRAFFIC.get(hashlib.sha1(f.read()).hexdigest()[:12])
     hbm_achieved = bytes_prefill / (prefill_ms * 1e-3) / 1e9
@@ -272,7 +273,7 @@ def gpu_main(args, rank, world, local_rank):
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1),
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": round(achieved / peaks["bf16_tflops"], 4),
-                     "traffic": traffic, "kernel": "prefill_tc_kernel",
+                     "traffic": traffic, "kernel": "prefill_pair_kernel",
                      "peak_source": f"{peak_kind} bf16 dense burst",
                      "hbm": {"achieved": round(hbm_achieved, 1), "peak": peaks["hbm_gbs"],
                              "unit": "GB/s", "frac": round(hbm_achieved / peaks["hbm_gbs"], 4),

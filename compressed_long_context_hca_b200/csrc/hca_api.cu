@@ -175,6 +175,8 @@ int32_t hca_attn_prefill(const hca_desc* d, const void* Q, const void* K, const 
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) ||
       !aligned16(cache->kc_pool) || !aligned16(cache->vc_pool))
     return HCA_EINVAL;
+  if (prefill_pair_supported(*d, *cache))
+    return from_cuda(launch_prefill_pair(*d, Q, K, V, *cache, O, lse, dbg_mask, s));
   return from_cuda(launch_prefill_tc(*d, Q, K, V, *cache, O, lse, dbg_mask, s));
 }
 

@@ -29,6 +29,11 @@ bool prefill_tc_supported(const hca_desc& d, const hca_cache& c);
 cudaError_t launch_prefill_tc(const hca_desc& d, const void* Q, const void* K, const void* V,
                               const hca_cache& c, void* O, float* lse, int32_t* dbg_mask,
                               cudaStream_t s);
+// bf16, 2-CTA clusters on the 2-SM UMMA (hq in 16..128); preferred over the one-CTA kernel
+bool prefill_pair_supported(const hca_desc& d, const hca_cache& c);
+cudaError_t launch_prefill_pair(const hca_desc& d, const void* Q, const void* K, const void* V,
+                                const hca_cache& c, void* O, float* lse, int32_t* dbg_mask,
+                                cudaStream_t s);
 
 bool decode_tc_supported(const hca_desc& d, const hca_cache& c);
 int decode_num_splits(const hca_desc& d);

@@ -134,9 +134,11 @@ int32_t hca_compress(const hca_desc* d, const void* K, const void* V,
  *   lse[b,t,h] = natural log of the softmax denominator incl. the max (if lse != NULL)
  *   dbg_mask[(b*seqlen+t)*3 + {0,1,2}] = (n_c(t), window lo, window hi) (if non-NULL)
  * Compressed entries are read from `cache` (hca_compress must have written them).
- * Kernels: bf16 -> tcgen05/TMEM tensor-core kernel (needs head_dim 512, hkv 1, hq in
+ * Kernels: bf16 -> tcgen05/TMEM tensor-core kernels (need head_dim 512, hkv 1, hq in
  * {8,16,32,64,128}, window <= 128, page_entries % 128 == 0, batch*seqlen*hq and
- * num_pages*page_entries below 2^31); f32 -> CUDA-core kernel
+ * num_pages*page_entries below 2^31). hq >= 16 runs on clusters of two CTAs sharing the
+ * 2-SM UMMA (each SM loads half of every K/V tile; needs (batch*seqlen + 256)*hq below
+ * 2^31, else the one-CTA kernel runs); hq = 8 on one CTA per tile. f32 -> CUDA-core kernel
  * (head_dim % 32 == 0, head_dim <= 512, any block/window).
  * Errors: HCA_EINVAL, HCA_EUNSUPPORTED, HCA_ECUDA. */
 int32_t hca_attn_prefill(const hca_desc* d, const void* Q, const void* K, const void* V,
