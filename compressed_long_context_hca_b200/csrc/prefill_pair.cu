@@ -28,6 +28,11 @@
 //    softmax (TMEM lane = row), warps 6-9 the epilogue (O / l, gate, bf16). The peer's TMA
 //    loads complete on the leader's barriers; the leader's UMMA commits arrive on the same
 //    barrier of both CTAs; the peer's softmax and epilogue warps arrive on the leader's.
+//  * One UMMA stream across items: S of tile g, then P.V of tile g-1. The softmax hands
+//    P(g) over before it observes the completion of P.V(g-1) unless O must be rescaled
+//    (lazy rescale: only when the row max grows by more than 2^8), so P.V(g) queues behind
+//    P.V(g-1) instead of waiting for a round trip through the softmax warps. The epilogue
+//    hands O back as soon as its last TMEM piece is in registers.
 //  * Every mbarrier wait is bounded; on time-out a CTA raises HCA_ERR_TIMEOUT (4) and
 //    unwinds. Both CTAs leave through one cluster barrier, after the leader's last UMMA has
 //    completed, so neither's shared memory or TMEM goes away while the other can reach it.
@@ -519,8 +524,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t g = 0;    // tiles processed (score buffer / phase counter)
       int nitem = 0;
       bool ok = true;
-      const uint32_t qbase = smem_u32(sQ);
       const uint32_t rbase = smem_u32(sRing);
+      const uint64_t qd0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
       auto issue_s = [&](const Item& it, int j, uint32_t gg, int ni) -> bool {
         const Tile t = tile_of(it, j);
         const int last = it.ntiles - 1;
@@ -536,20 +541,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t s = cnt % kStages;
           if (!mbar_wait(&bars->ring_full[s], (cnt / kStages) & 1, abort)) return false;
           tc_fence_after();
-          const uint32_t sbase = rbase + s * kSlotBytes;
-          // chunks of this slot: 4 (128-key kinds, chunks 4q .. 4q+3) or all 8 (16-key kind)
-          const int nchunks = t.kind == kRaw16 ? kNCh : 4;
-          const uint32_t cstride = t.kind == kRaw16 ? kK8Chunk : kKChunk;
-          for (int cc = 0; cc < nchunks; ++cc) {
-            const int d = t.kind == kRaw16 ? cc : 4 * q + cc;
-            const uint32_t qaddr = qbase + d * kQChunk;
-            const uint32_t kaddr = sbase + cc * cstride;
+          // Descriptors are built once per slot and stepped by constant offsets (the start
+          // address field is address >> 4; every shared address here is below 256 KB, so the
+          // addition never carries out of the field).
+          const uint64_t kd0 = sdesc_sw128(rbase + s * kSlotBytes, 16, 1024);
+          if (t.kind == kRaw16) {
+            // all 8 chunks of 8 keys in one slot
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = sdesc_sw128(qaddr + kk * 32, 16, 1024);
-              const uint64_t bd = sdesc_sw128(kaddr + kk * 32, 16, 1024);
-              umma2_ss(d_tmem, ad, bd, idesc, (d | kk) != 0);
-            }
+            for (int cc = 0; cc < kNCh; ++cc)
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                umma2_ss(d_tmem, qd0 + ((cc * kQChunk + kk * 32) >> 4),
+                         kd0 + ((cc * kK8Chunk + kk * 32) >> 4), idesc, (cc | kk) != 0);
+          } else {
+            // chunks 4q .. 4q+3 of 64 keys
+            const uint64_t qdq = qd0 + ((uint32_t)(4 * q) * (kQChunk >> 4));
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                umma2_ss(d_tmem, qdq + ((cc * kQChunk + kk * 32) >> 4),
+                         kd0 + ((cc * kKChunk + kk * 32) >> 4), idesc, (q | cc | kk) != 0);
           }
           umma2_commit_both(&bars->ring_empty[s]);
           if (j == last) {  // the last tile is a 128-key kind: slot q held Q pairs 2q, 2q+1
@@ -572,14 +584,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t s = cnt % kStages;
         if (!mbar_wait(&bars->ring_full[s], (cnt / kStages) & 1, abort)) return false;
         tc_fence_after();
-        const uint32_t vaddr = rbase + s * kSlotBytes;
-        // N = 256 output columns, 128 in each CTA (two chunks, N-major, chunk stride lbo)
+        // N = 256 output columns, 128 in each CTA (two chunks, N-major, chunk stride lbo);
+        // 16 keys = two 8-row swizzle atoms = 2 KB of each chunk
         const uint32_t lbo = t.kind == kRaw16 ? kV16Chunk : kVChunk;
         const uint32_t idesc = idesc_bf16_f32(2 * kBM, kDH, true);
-        for (int kk = 0; kk < t.n / 16; ++kk) {
-          // 16 keys = two 8-row swizzle atoms = 2 KB
-          const uint64_t bd = sdesc_sw128(vaddr + kk * 2048, lbo, 1024);
-          umma2_ts(tmem + kTmO, a_tmem + kk * 8, bd, idesc, (j > 0 || kk > 0));
+        const uint64_t vd0 = sdesc_sw128(rbase + s * kSlotBytes, lbo, 1024);
+        const uint32_t acc0 = j > 0 ? 1u : 0u;
+        if (t.n == kBN) {
+#pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk)
+            umma2_ts(tmem + kTmO, a_tmem + kk * 8, vd0 + kk * (2048 >> 4), idesc, acc0 | kk);
+        } else {
+          for (int kk = 0; kk < t.n / 16; ++kk)
+            umma2_ts(tmem + kTmO, a_tmem + kk * 8, vd0 + kk * (2048 >> 4), idesc, acc0 | kk);
         }
         umma2_commit_both(&bars->ring_empty[s]);
         ++cnt;
@@ -665,10 +682,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
         for (int q = 0; q < npieces; ++q) {
           if (q + 1 < npieces) tmem_ld32(s_addr + (q + 1) * 32, nxt);
+          // a piece is visible in full for most rows (every compressed tile, all but the
+          // last piece of the raw tile): the masks are only applied where some lane needs them
+          const int c0 = q * 32;
+          if (__all_sync(0xffffffffu, c0 >= vlo && c0 + 32 <= vhi)) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const bool in = (uint32_t)(q * 32 + e - vlo) < vlen;
-            mx[e & 7] = fmaxf(mx[e & 7], in ? __uint_as_float(cur[e]) : -INFINITY);
+            for (int e = 0; e < 32; ++e) mx[e & 7] = fmaxf(mx[e & 7], __uint_as_float(cur[e]));
+          } else if (!__all_sync(0xffffffffu, c0 >= vhi || c0 + 32 <= vlo)) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const bool in = (uint32_t)(c0 + e - vlo) < vlen;
+              mx[e & 7] = fmaxf(mx[e & 7], in ? __uint_as_float(cur[e]) : -INFINITY);
+            }
           }
           tmem_wait_ld();
 #pragma unroll
@@ -698,17 +723,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int q = 0; q < npieces; ++q) {
           if (q + 1 < npieces) tmem_ld32(s_addr + (q + 1) * 32, nxt);
           uint32_t pk[16];
+          const int c0 = q * 32;
+          if (__all_sync(0xffffffffu, c0 >= vlo && c0 + 32 <= vhi)) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int c0 = q * 32 + 2 * e;
-            const bool in0 = (uint32_t)(c0 - vlo) < vlen;
-            const bool in1 = (uint32_t)(c0 + 1 - vlo) < vlen;
-            const float p0 =
-                in0 ? fast_exp2(fmaf(__uint_as_float(cur[2 * e]), p.scale_log2, -base)) : 0.f;
-            const float p1 =
-                in1 ? fast_exp2(fmaf(__uint_as_float(cur[2 * e + 1]), p.scale_log2, -base)) : 0.f;
-            pk[e] = pack_bf16x2(p0, p1);
-            ps[e & 3] += p0 + p1;
+            for (int e = 0; e < 16; ++e) {
+              const float p0 = fast_exp2(fmaf(__uint_as_float(cur[2 * e]), p.scale_log2, -base));
+              const float p1 =
+                  fast_exp2(fmaf(__uint_as_float(cur[2 * e + 1]), p.scale_log2, -base));
+              pk[e] = pack_bf16x2(p0, p1);
+              ps[e & 3] += p0 + p1;
+            }
+          } else if (__all_sync(0xffffffffu, c0 >= vhi || c0 + 32 <= vlo)) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) pk[e] = 0u;
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int cc = c0 + 2 * e;
+              const bool in0 = (uint32_t)(cc - vlo) < vlen;
+              const bool in1 = (uint32_t)(cc + 1 - vlo) < vlen;
+              const float p0 =
+                  in0 ? fast_exp2(fmaf(__uint_as_float(cur[2 * e]), p.scale_log2, -base)) : 0.f;
+              const float p1 =
+                  in1 ? fast_exp2(fmaf(__uint_as_float(cur[2 * e + 1]), p.scale_log2, -base))
+                      : 0.f;
+              pk[e] = pack_bf16x2(p0, p1);
+              ps[e & 3] += p0 + p1;
+            }
           }
           tmem_st16(s_addr + q * 16, pk);
           tmem_wait_ld();
@@ -794,23 +835,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                        it.half * kDH
                  : nullptr;
       const uint32_t o_addr = tmem + lane_addr + kTmO;
+      // 32-column pieces; the next piece's TMEM (and gate) loads are in flight while this
+      // one is scaled, rounded and stored. O is handed back to the UMMA warp as soon as the
+      // last piece is in registers.
+      uint32_t cur[32], nxt[32];
+      uint4 gcur[4], gnxt[4];
+      tmem_ld32(o_addr, cur);
+      if (gp) {
+#pragma unroll
+        for (int w = 0; w < 4; ++w) gcur[w] = ld_stream_hint(gp + w * 8, pol_stream);
+      }
+      tmem_wait_ld();
 #pragma unroll 1
       for (int q = 0; q < kDH / 32; ++q) {
-        uint4 gv[4];
-        if (gp) {
+        const bool more = q + 1 < kDH / 32;
+        if (more) {
+          tmem_ld32(o_addr + (q + 1) * 32, nxt);
+          if (gp) {
 #pragma unroll
-          for (int w = 0; w < 4; ++w) gv[w] = ld_stream_hint(gp + q * 32 + w * 8, pol_stream);
+            for (int w = 0; w < 4; ++w)
+              gnxt[w] = ld_stream_hint(gp + (q + 1) * 32 + w * 8, pol_stream);
+          }
         }
-        uint32_t v[32];
-        tmem_ld32(o_addr + q * 32, v);
-        tmem_wait_ld();
         float o[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) o[e] = __uint_as_float(v[e]) * inv;
+        for (int e = 0; e < 32; ++e) o[e] = __uint_as_float(cur[e]) * inv;
         if (gp) {
 #pragma unroll
           for (int w = 0; w < 4; ++w) {
-            const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv[w]);
+            const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gcur[w]);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const float2 f = __bfloat1622float2(g2[e]);
@@ -830,10 +883,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             st_stream_hint(op + q * 32 + w * 8, pk, pol_stream);
           }
         }
+        if (more) {
+          tmem_wait_ld();
+          if (q + 2 == kDH / 32) {
+            // every TMEM read of this warp has completed
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cl(ofree_cl);
+          }
+#pragma unroll
+          for (int e = 0; e < 32; ++e) cur[e] = nxt[e];
+#pragma unroll
+          for (int w = 0; w < 4; ++w) gcur[w] = gnxt[w];
+        }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cl(ofree_cl);
       ++nitem;
     }
     if (!ok) raise_timeout(p, bars, 5);
