@@ -79,6 +79,25 @@ def test_bf16_prefill(T, hq, gate, hetero):
     assert int(r["cache"].err.item()) == 0
 
 
+@pytest.mark.parametrize("b,T,hq,block,window,gate", [
+    (2, 777, 32, 128, 128, True),   # 4 positions per CTA, 8 per pair row tile, ragged tail
+    (1, 1000, 32, 64, 32, False),   # narrow window: no 16-key tile, a 48-key raw tile
+    (2, 613, 16, 200, 100, True),   # block not a power of two, window 100, 16 positions per pair
+    (1, 300, 128, 32, 128, False),  # one position per CTA, many small blocks
+])
+def test_bf16_block_window_shapes(b, T, hq, block, window, gate):
+    """Tensor-core prefill at other block sizes, windows and head counts, every position
+    against the oracle (masks bit-exact)."""
+    x = inputs.prefill_inputs(b, T, hq, 1, 512, "bf16", seed=12, gate=gate, block=block)
+    r = run_prefill(x, block=block, window=window, want_lse=True, want_mask=True)
+    assert int(r["cache"].err.item()) == 0
+    for bi in range(b):
+        ref, lse = _oracle(x, bi, None, block, window)
+        compare(to64(r["O"][bi]), ref, BF16_MAX, BF16_MEAN, what=f"O[{bi}]")
+        compare(to64(r["lse"][bi]), lse, 2e-2, 2e-3, what=f"lse[{bi}]", out_bf16=False)
+        assert np.array_equal(r["dbg"][bi].cpu().numpy(), orc.mask_table(T, block, window))
+
+
 def test_bf16_two_sequences_many_compressed_tiles():
     """b=2, T=20000: >128 visible entries (several compressed tiles per row tile)."""
     T = 20000
