@@ -88,6 +88,7 @@ struct Params {
   const int32_t* n_entries;
   int32_t* err_word;
   int32_t batch, T, hq, P, W, block, PE, max_pages, num_pages;
+  int32_t o32;      // O is 32-byte aligned: the epilogue stores 32 bytes per lane
   int32_t n_pt;     // pair row tiles per sequence (2 P positions each)
   int32_t n_items;  // 2 * batch * n_pt
   float scale_log2;
@@ -305,6 +306,16 @@ __device__ __forceinline__ void st_stream_hint(void* ptr, const uint4& v, uint64
   asm volatile("st.global.L1::no_allocate.L2::cache_hint.v4.u32 [%0], {%1,%2,%3,%4}, %5;" ::"l"(ptr),
                "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "l"(pol)
                : "memory");
+}
+// 32-byte store (ptr 32-byte aligned): each lane of an epilogue warp writes its own row, so
+// a warp's store touches 32 rows; wider stores halve the instructions the LSU processes
+__device__ __forceinline__ void st_stream_hint32(void* ptr, const uint32_t* v, uint64_t pol) {
+  asm volatile(
+      "st.global.L1::no_allocate.L2::cache_hint.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8}, %9;" ::"l"(
+          ptr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "l"(pol)
+      : "memory");
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -873,14 +884,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (row_valid) {
+          uint32_t pk[16];
 #pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            uint4 pk;
-            pk.x = pack_bf16x2(o[w * 8 + 0], o[w * 8 + 1]);
-            pk.y = pack_bf16x2(o[w * 8 + 2], o[w * 8 + 3]);
-            pk.z = pack_bf16x2(o[w * 8 + 4], o[w * 8 + 5]);
-            pk.w = pack_bf16x2(o[w * 8 + 6], o[w * 8 + 7]);
-            st_stream_hint(op + q * 32 + w * 8, pk, pol_stream);
+          for (int w = 0; w < 16; ++w) pk[w] = pack_bf16x2(o[2 * w], o[2 * w + 1]);
+          if (p.o32) {
+            st_stream_hint32(op + q * 32, pk, pol_stream);
+            st_stream_hint32(op + q * 32 + 16, pk + 8, pol_stream);
+          } else {
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+              st_stream_hint(op + q * 32 + w * 8,
+                             make_uint4(pk[4 * w], pk[4 * w + 1], pk[4 * w + 2], pk[4 * w + 3]),
+                             pol_stream);
           }
         }
         if (more) {
@@ -965,6 +980,7 @@ cudaError_t launch_prefill_pair(const hca_desc& d, const void* Q, const void* K,
   if ((e = encode_bf16_chunks(&p.tmKc, c.kc_pool, rowsC, kBN / 2, 4)) != cudaSuccess) return e;
   if ((e = encode_bf16_chunks(&p.tmVc, c.vc_pool, rowsC, kBN, 2)) != cudaSuccess) return e;
   p.O = static_cast<__nv_bfloat16*>(O);
+  p.o32 = (reinterpret_cast<uintptr_t>(O) % 32) == 0 ? 1 : 0;
   p.lse = lse;
   p.dbg = dbg_mask;
   p.gate = static_cast<const __nv_bfloat16*>(d.gate);

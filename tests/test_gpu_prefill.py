@@ -98,6 +98,27 @@ def test_bf16_block_window_shapes(b, T, hq, block, window, gate):
         assert np.array_equal(r["dbg"][bi].cpu().numpy(), orc.mask_table(T, block, window))
 
 
+def test_bf16_output_alignment_paths_agree():
+    """O at a 32-byte boundary (32-byte stores) and O 16 bytes past one (16-byte stores):
+    the same inputs give bit-identical outputs, and both match the oracle."""
+    from compressed_long_context_hca_b200 import ops
+    T, hq, D = 700, 64, 512
+    x = inputs.prefill_inputs(1, T, hq, 1, D, "bf16", seed=13, gate=True)
+    r = run_prefill(x)
+    dev = torch.device("cuda")
+    Q, K, V = x.Q.to(dev), x.K.to(dev), x.V.to(dev)
+    buf = torch.zeros(T * hq * D + 16, dtype=torch.bfloat16, device=dev)
+    O16 = buf[8:8 + T * hq * D].view(1, T, hq, D)  # 16 bytes past the 32-byte aligned base
+    assert buf.data_ptr() % 32 == 0 and O16.data_ptr() % 32 == 16
+    assert r["O"].data_ptr() % 32 == 0
+    ops.prefill(r["desc"], Q, K, V, r["cache"], O=O16)
+    torch.cuda.synchronize()
+    assert torch.equal(O16, r["O"])
+    pos = [0, 1, 127, 128, 129, 255, 256, 511, T - 2, T - 1]
+    ref, _ = _oracle(x, 0, pos)
+    compare(to64(O16[0, pos]), ref, BF16_MAX, BF16_MEAN, what="O")
+
+
 def test_bf16_two_sequences_many_compressed_tiles():
     """b=2, T=20000: >128 visible entries (several compressed tiles per row tile)."""
     T = 20000
