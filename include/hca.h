@@ -27,6 +27,10 @@
  *       K, V        [batch, seqlen, hkv, head_dim]
  *       cache pools [num_pages, page_entries, hkv, head_dim]
  *     Element type is desc->dtype (HCA_BF16 or HCA_F32) for all of them; LSE is float32.
+ *   - The bf16 tensor-core paths read and write through TMA and vector accesses: Q, K, V, O,
+ *     the cache pools and the gate must start on a 16-byte boundary (HCA_EINVAL otherwise).
+ *     Prefill writes O with 32-byte stores when O starts on a 32-byte boundary (faster;
+ *     same result).
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream) and the
  *     call returns before it runs. The return value reports argument validation and
  *     launch failures only. Kernels that meet an out-of-range page id or a cache holding
