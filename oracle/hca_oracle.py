@@ -19,6 +19,10 @@ What it restates (each function cites its passage):
   recent raw tokens; head dimension 512.
 * Both pages, "Low-Rank Gated Attention" paragraph: the attention output is
   multiplied by a learned gate.
+* The same communeify.com page, section "33.5T 預訓練資料工程與分散式訓練基礎設施"
+  item 3 (the FlashMask-4 attention kernel for the 512-wide HCA heads) -- cited below
+  as [analysis infra 3]: the operator has a training backward pass (the page quotes
+  its speed-up, not its formulas).
 
 Readings taken where the pages are silent:
 
@@ -34,6 +38,11 @@ Everything is float64 NumPy.  The per-position loop is the definition written
 out: for each query position, gather its visible keys, one softmax, one
 weighted sum.  All heads of a position are handled by one matmul (a library
 primitive); there is no tiling across positions.
+
+``hca_prefill_backward`` restates the gradients of the prefill output (dQ, dK, dV
+through both the window and the mean pooling, dG); it is pinned by central finite
+differences of the forward, torch autograd of an independent dense formulation and
+two reductions to causal attention in ``tests/test_oracle_backward.py``.
 
 Parity status: exact values for random inputs are not printed by the pages
 ("parity unpinned" in that narrow sense); every function below is pinned by
@@ -225,6 +234,117 @@ def hca_decode(q: np.ndarray, Kc: np.ndarray, Vc: np.ndarray,
     if gate is not None:
         o = o * np.asarray(gate, dtype=np.float64)
     return o, lse
+
+
+# ---------------------------------------------------------------------------
+# Backward (gradients of the prefill output)
+# ---------------------------------------------------------------------------
+#
+# The pages give the operator and note that it is trained: the attention kernel has a
+# backward pass whose speed-up they quote ([analysis infra 3]); they print no backward
+# formulas.  The backward here is the derivative of the forward
+# definition above, taken step by step: gate, weighted sum, softmax, scores, and the
+# mean pooling that made the compressed entries.
+
+def pool_backward(dXc: np.ndarray, T: int, block: int) -> np.ndarray:
+    """Gradient of ``compress_blocks`` with respect to its input.
+
+    dXc: [n_entries, H, D] gradient of the entries.  Entry j is the mean of the
+    tokens of block j, so each of those tokens receives dXc[j] / count_j.
+    Returns [T, H, D].
+    """
+    dXc = np.asarray(dXc, dtype=np.float64)
+    out = np.zeros((T,) + dXc.shape[1:], dtype=np.float64)
+    for j in range(dXc.shape[0]):
+        a, b = j * block, min((j + 1) * block, T)
+        if a < b:
+            out[a:b] += dXc[j] / (b - a)
+    return out
+
+
+def _softmax_backward(w: np.ndarray, dw: np.ndarray) -> np.ndarray:
+    """Gradient of the scores through a row softmax: w (dw - sum_k w dw)."""
+    return w * (dw - (w * dw).sum(axis=1, keepdims=True))
+
+
+def attend_position_backward(q: np.ndarray, do: np.ndarray, Kc: np.ndarray,
+                             Vc: np.ndarray, K: np.ndarray, V: np.ndarray, t: int,
+                             block: int, window: int, scale: float):
+    """Gradients of the (ungated) output of ``attend_position`` at position ``t``.
+
+    do: [Hq, D] gradient of that output.  Returns (dq [Hq, D], dkey, dval) where
+    dkey / dval are lists over KV heads g of arrays [n_c + window length, D]: the
+    gradient of every key / value row of that head, visible compressed entries first,
+    then the raw window in token order -- the key order of the forward.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    do = np.asarray(do, dtype=np.float64)
+    Hq = q.shape[0]
+    Hkv = K.shape[1]
+    nc = visible_compressed_count(t, block, window)
+    lo, hi = window_bounds(t, window)
+    dq = np.zeros_like(q)
+    dkey, dval = [], []
+    for g in range(Hkv):
+        heads = [h for h in range(Hq) if h * Hkv // Hq == g]
+        keys = np.concatenate([np.asarray(Kc[:nc, g], np.float64),
+                               np.asarray(K[lo:hi + 1, g], np.float64)], axis=0)
+        vals = np.concatenate([np.asarray(Vc[:nc, g], np.float64),
+                               np.asarray(V[lo:hi + 1, g], np.float64)], axis=0)
+        scores = (q[heads] @ keys.T) * scale
+        _, _, w = _softmax_weighted(scores, vals)
+        dw = do[heads] @ vals.T                    # d(out)/d(weights)
+        ds = _softmax_backward(w, dw) * scale      # d/d(q.k), scale folded in
+        dq[heads] = ds @ keys
+        dkey.append(ds.T @ q[heads])               # summed over the heads of group g
+        dval.append(w.T @ do[heads])
+    return dq, dkey, dval
+
+
+def hca_prefill_backward(Q: np.ndarray, K: np.ndarray, V: np.ndarray, dO: np.ndarray,
+                         block: int, window: int, scale: float,
+                         gate: Optional[np.ndarray] = None):
+    """Gradients of ``hca_prefill`` (all positions) for an output gradient dO.
+
+    Q, dO: [T, Hq, D]; K, V: [T, Hkv, D]; gate: [T, Hq, D] (already sigmoided) or None.
+    Returns (dQ [T, Hq, D], dK [T, Hkv, D], dV [T, Hkv, D], dG [T, Hq, D] or None) in
+    float64.  Raw keys and values receive their window gradients directly and, through
+    the mean pooling, 1/count of the gradient of the compressed entry of their block.
+    """
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    dO = np.asarray(dO, dtype=np.float64)
+    T, Hq, _ = Q.shape
+    Hkv = K.shape[1]
+    Kc = compress_blocks(K, block)
+    Vc = compress_blocks(V, block)
+    dQ = np.zeros_like(Q)
+    dK = np.zeros_like(K)
+    dV = np.zeros_like(V)
+    dKc = np.zeros_like(Kc)
+    dVc = np.zeros_like(Vc)
+    dG = None if gate is None else np.zeros_like(Q)
+    for t in range(T):
+        do = dO[t]
+        if gate is not None:
+            g_t = np.asarray(gate[t], dtype=np.float64)
+            o, _ = attend_position(Q[t], Kc, Vc, K, V, t, block, window, scale)
+            dG[t] = dO[t] * o                      # O = o * G
+            do = dO[t] * g_t
+        dq, dkey, dval = attend_position_backward(Q[t], do, Kc, Vc, K, V, t, block,
+                                                  window, scale)
+        dQ[t] = dq
+        nc = visible_compressed_count(t, block, window)
+        lo, hi = window_bounds(t, window)
+        for g in range(Hkv):
+            dKc[:nc, g] += dkey[g][:nc]
+            dVc[:nc, g] += dval[g][:nc]
+            dK[lo:hi + 1, g] += dkey[g][nc:]
+            dV[lo:hi + 1, g] += dval[g][nc:]
+    dK += pool_backward(dKc, T, block)
+    dV += pool_backward(dVc, T, block)
+    return dQ, dK, dV, dG
 
 
 def visible_pairs(T: int, block: int, window: int) -> Tuple[int, int]:
