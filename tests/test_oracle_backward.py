@@ -135,6 +135,17 @@ def pin_dense_autograd(orc):
         _close(a, b, 1e-10, f"d{name} vs dense autograd")
 
 
+def pin_dense_autograd_64_heads(orc):
+    """The operator's head layout: 64 query heads share one KV head, so dK and dV sum the
+    contributions of all 64 (torch autograd of the dense formulation, gate on)."""
+    T, B, W, Hq, Hkv, D, scale = 160, 16, 24, 64, 1, 16, 0.25
+    Q, K, V, dO, G = _case(T, Hq, Hkv, D, seed=61)
+    want = _torch_grads(lambda q, k, v, g: _dense_hca(q, k, v, g, B, W, scale), Q, K, V, G, dO)
+    got = orc.hca_prefill_backward(Q, K, V, dO, B, W, scale, gate=G)
+    for name, a, b in zip("QKVG", got, want):
+        _close(a, b, 1e-9, f"d{name} vs dense autograd (64 heads on one KV head)")
+
+
 def pin_full_window_is_causal(orc):
     """window >= T: no compressed entry is visible, gradients of causal attention."""
     T, B, W, Hq, Hkv, D, scale = 40, 4, 64, 2, 1, 8, 0.3
@@ -156,8 +167,8 @@ def pin_block1_is_causal(orc):
         _close(a, b, 1e-10, f"d{name} vs causal SDPA (block 1)")
 
 
-PINS = [pin_finite_differences, pin_dense_autograd, pin_full_window_is_causal,
-        pin_block1_is_causal]
+PINS = [pin_finite_differences, pin_dense_autograd, pin_dense_autograd_64_heads,
+        pin_full_window_is_causal, pin_block1_is_causal]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
