@@ -32,8 +32,9 @@ HCA_ERR_CTX_RANGE = 8
 ABI_VERSION = 1
 
 EXPORTED = ("hca_abi_version", "hca_status_string", "hca_set_gate", "hca_compress",
-            "hca_attn_prefill", "hca_decode_workspace_bytes", "hca_attn_decode",
-            "hca_attn_decode_noalloc")
+            "hca_attn_prefill", "hca_attn_prefill_range", "hca_decode_workspace_bytes",
+            "hca_attn_decode", "hca_decode_partial_bytes", "hca_attn_decode_partial",
+            "hca_decode_merge", "hca_attn_decode_noalloc")
 HCA_DECODE_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
@@ -80,6 +81,20 @@ def lib() -> ctypes.CDLL:
     L.hca_attn_prefill.restype = c_int32
     L.hca_attn_prefill.argtypes = [POINTER(HcaDesc), c_void_p, c_void_p, c_void_p,
                                    POINTER(HcaCache), c_void_p, c_void_p, c_void_p, c_void_p]
+    L.hca_attn_prefill_range.restype = c_int32
+    L.hca_attn_prefill_range.argtypes = [POINTER(HcaDesc), c_int32, c_int32, c_int32, c_void_p,
+                                         c_void_p, c_void_p, POINTER(HcaCache), c_void_p,
+                                         c_void_p, c_void_p, c_void_p]
+    L.hca_decode_partial_bytes.restype = c_size_t
+    L.hca_decode_partial_bytes.argtypes = [POINTER(HcaDesc)]
+    L.hca_attn_decode_partial.restype = c_int32
+    L.hca_attn_decode_partial.argtypes = [POINTER(HcaDesc), c_void_p, c_void_p,
+                                          POINTER(HcaCache), c_void_p, c_void_p, c_int32,
+                                          c_int32, c_int32, c_void_p, c_void_p, c_size_t,
+                                          c_void_p]
+    L.hca_decode_merge.restype = c_int32
+    L.hca_decode_merge.argtypes = [POINTER(HcaDesc), c_void_p, c_int32, c_int64, c_void_p,
+                                   c_void_p, c_void_p]
     L.hca_decode_workspace_bytes.restype = c_size_t
     L.hca_decode_workspace_bytes.argtypes = [POINTER(HcaDesc)]
     L.hca_attn_decode.restype = c_int32
@@ -132,6 +147,34 @@ def hca_attn_prefill(desc: HcaDesc, Q: int, K: int, V: int, cache: HcaCache, O: 
     return lib().hca_attn_prefill(ctypes.byref(desc), Q or None, K or None, V or None,
                                   ctypes.byref(cache), O or None, lse or None,
                                   dbg_mask or None, stream or None)
+
+
+def hca_attn_prefill_range(desc: HcaDesc, q_pos0: int, kv_pos0: int, kv_len: int, Q: int,
+                           K: int, V: int, cache: HcaCache, O: int, lse: int = 0,
+                           dbg_mask: int = 0, stream: int = 0) -> int:
+    return lib().hca_attn_prefill_range(ctypes.byref(desc), q_pos0, kv_pos0, kv_len, Q or None,
+                                        K or None, V or None, ctypes.byref(cache), O or None,
+                                        lse or None, dbg_mask or None, stream or None)
+
+
+def hca_decode_partial_bytes(desc: HcaDesc) -> int:
+    return lib().hca_decode_partial_bytes(ctypes.byref(desc))
+
+
+def hca_attn_decode_partial(desc: HcaDesc, Q: int, ctx_len: int, cache: HcaCache, ring_k: int,
+                            ring_v: int, entry_begin: int, entry_end: int, with_window: int,
+                            partial: int, workspace: int, workspace_bytes: int,
+                            stream: int = 0) -> int:
+    return lib().hca_attn_decode_partial(ctypes.byref(desc), Q or None, ctx_len or None,
+                                         ctypes.byref(cache), ring_k or None, ring_v or None,
+                                         entry_begin, entry_end, with_window, partial or None,
+                                         workspace or None, workspace_bytes, stream or None)
+
+
+def hca_decode_merge(desc: HcaDesc, parts: int, n_parts: int, part_stride: int, O: int,
+                     lse: int = 0, stream: int = 0) -> int:
+    return lib().hca_decode_merge(ctypes.byref(desc), parts or None, n_parts, part_stride,
+                                  O or None, lse or None, stream or None)
 
 
 def hca_decode_workspace_bytes(desc: HcaDesc) -> int:

@@ -9,16 +9,18 @@
 //  * The hq <= 64 query heads of a sequence share its KV head, so they form the M = 64 rows
 //    of every UMMA. An M = 64 accumulator occupies TMEM lanes 0-15 of each 32-lane
 //    subpartition; a second one sits at lane offset 16. O (64 x 512 f32) takes lanes
-//    0-15 x 512 columns; two score buffers of 256 keys take lanes 16-31.
+//    0-15 x 512 columns; two score buffers of 128 keys take lanes 16-31.
 //  * The key list (compressed tiles of 128 entries, then the ring tile) is cut into
 //    `nsplit` contiguous splits; grid = (nsplit, sequences). A split is walked in chunks
-//    of two tiles (256 keys) with a running softmax (lazy rescale).
+//    of one tile (128 keys) with a running softmax (lazy rescale).
 //  * One load stream per CTA, in the order K(0), K(1), V(0), K(2), V(1), ...: the scores of
 //    chunk c + 1 are computed while the softmax of chunk c runs, and V(c) arrives after it,
 //    so the stream of 3-D TMA boxes (128 rows x two 128-byte chunks, two issuing warps)
-//    does not wait on the softmax. P goes to shared memory in bf16 (UMMA K-major swizzled
-//    layout); one buffer is enough: P(c) is written once PV(c - 1) is done, and V(c) only
-//    arrives after K(c + 1). O += P V with V N-major.
+//    does not wait on the softmax. P goes to shared memory as two bf16 parts, P_hi = bf16(P)
+//    and P_lo = bf16(P - P_hi) (UMMA K-major swizzled layout), and O += P_hi V + P_lo V runs
+//    as two UMMAs with V N-major: the rounding of P costs ~2^-17 of the value spread instead
+//    of 2^-9. One buffer pair is enough: P(c) is written once PV(c - 1) is done, and V(c)
+//    only arrives after K(c + 1).
 //  * Each CTA writes float32 partials (unnormalised O, base max m in log2 units, sum l) to
 //    the workspace; merge_kernel combines them per head, applies the gate and casts.
 //  * All mbarrier waits are bounded (HCA_ERR_TIMEOUT on give-up).
@@ -45,25 +47,26 @@ constexpr int kSlotsPerTile = kNCh / 2;                 // 4 for K, 4 for V
 constexpr uint32_t kQChunkBytes = kM * kKC * 2;         // 8 KB
 constexpr uint32_t kQBytes = kNCh * kQChunkBytes;       // 64 KB (two 32 KB boxes)
 constexpr uint32_t kPChunkBytes = kM * kKC * 2;         // 8 KB (64 rows x 64 keys)
-constexpr int kCT = 2;                    // tiles per softmax chunk (256 keys)
-constexpr uint32_t kPBytes = kCT * (kTN / kKC) * kPChunkBytes;  // 32 KB: P of one chunk
+constexpr int kCT = 1;                    // tiles per softmax chunk (128 keys)
+constexpr uint32_t kPBytes = kCT * (kTN / kKC) * kPChunkBytes;  // 16 KB: one part of P
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays below 2^8 between rescales
-constexpr int kStages = 4;
+constexpr int kStages = 4;  // = kSlotsPerTile: the slots of a tile are ring slots 0..3
+static_assert(kStages == kSlotsPerTile, "P.V pairs ring slots (0,1) and (2,3) of a V tile");
 constexpr int kThreads = 224;             // 2 TMA warps, UMMA warp, 4 softmax warps
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kLaneS = 16u << 16;   // lane offset of the score accumulator
 
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffP = kQBytes;
-constexpr uint32_t kOffRing = kOffP + kPBytes;
+constexpr uint32_t kOffRing = kOffP + 2 * kPBytes;  // P_hi, then P_lo
 constexpr uint32_t kOffBar = kOffRing + kStages * kSlotBytes;
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
 // End of a CTA: O (64 x 512 f32) is staged row-major in the P + ring region (free once the
 // last PV is done) with a padded row stride, then written out coalesced.
 constexpr int kORow = kD + 4;  // floats per staged row: rows r and r + 8 share banks only
 constexpr uint32_t kOffStage = kOffP;
-static_assert(kOffRing == kOffP + kPBytes, "P and ring must be adjacent");
-static_assert(kM * kORow * 4 + 3 * kM * 4 <= kPBytes + kStages * kSlotBytes, "staging space");
+static_assert(kOffRing == kOffP + 2 * kPBytes, "P and ring must be adjacent");
+static_assert(kM * kORow * 4 + 3 * kM * 4 <= 2 * kPBytes + kStages * kSlotBytes, "staging space");
 
 enum { kCompressed = 0, kRing = 1 };
 
@@ -82,6 +85,10 @@ struct Params {
   const __nv_bfloat16* gate;
   int64_t gs0, gs2;
   int32_t nseq, seqlen, hq, W, block, PE, max_pages, num_pages, nsplit;
+  // key part of the call: visible compressed entries [e0, e1) (e0 % 128 == 0), and the raw
+  // window if with_ring; partial != 0: the result is an unnormalised float32 partial
+  // (written to ws_ml / ws_o at split 0 when nsplit == 1, else merged into one by the merge)
+  int32_t e0, e1, with_ring, partial;
   float scale_log2;
 };
 
@@ -96,7 +103,9 @@ struct Bars {
 static_assert(sizeof(Bars) <= 256, "barrier block too large");
 
 struct Seq {
-  int t, nc, nct, total, j0, j1;  // tiles [j0, j1) belong to this split
+  int t, nc;      // query position, visible compressed entries
+  int e0, e1;     // compressed entries of the call's part, [e0, e1)
+  int nct, total, j0, j1;  // tiles [j0, j1) belong to this split
 };
 
 struct Tile {
@@ -114,8 +123,10 @@ __device__ __forceinline__ Seq make_seq(const Params& p, int b, int split) {
   int x = s.t + 1 - p.W;
   int nc = x < 0 ? 0 : x / p.block;
   s.nc = min(nc, min(p.n_entries[b], p.max_pages * p.PE));
-  s.nct = (s.nc + kTN - 1) / kTN;
-  s.total = s.nct + 1;
+  s.e0 = min(p.e0, s.nc);
+  s.e1 = max(s.e0, min(p.e1, s.nc));
+  s.nct = (s.e1 - s.e0 + kTN - 1) / kTN;
+  s.total = s.nct + (p.with_ring ? 1 : 0);
   const int tps = (s.total + p.nsplit - 1) / p.nsplit;
   s.j0 = min(s.total, split * tps);
   s.j1 = min(s.total, s.j0 + tps);
@@ -126,8 +137,8 @@ __device__ __forceinline__ Tile tile_of(const Params& p, const Seq& s, int j) {
   Tile t;
   if (j < s.nct) {
     t.kind = kCompressed;
-    t.key0 = j * kTN;
-    t.n = min(kTN, round16(s.nc - j * kTN));
+    t.key0 = s.e0 + j * kTN;
+    t.n = min(kTN, round16(s.e1 - t.key0));
   } else {
     t.kind = kRing;
     t.key0 = 0;
@@ -283,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       const uint32_t qbase = smem_u32(sQ);
       const uint32_t pbase = smem_u32(sP);
       const uint32_t rbase = smem_u32(sRing);
-      const uint32_t idesc_pv = idesc_bf16_f32(kM, 128, true);
+      const uint32_t idesc_pv = idesc_bf16_f32(kM, 256, true);
       for (int c = 0; c <= nchunks && ok; ++c) {
         if (c < nchunks) {
           const uint32_t sbuf = tmem + kLaneS + (c & 1) * (kCT * kTN);
@@ -316,24 +327,31 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           if (!(ok = mbar_wait(&bars->p_full[pc & 1], (pc >> 1) & 1, abort))) break;
           tc_fence_after();
           const uint32_t pbuf = pbase;
-          // O[:, 128 q .. 128 q + 127] += P(tile) V(tile, slot q)
+          // O[:, 256 h .. 256 h + 255] += P(tile) V(tile, slots 2h and 2h + 1): a V tile fills
+          // ring slots 0..3 in order (every tile is 4 loads), so slots 2h and 2h + 1 are
+          // adjacent and their four 128-column chunks have one stride (16 KB): one N = 256
+          // MMA per 16-key group and part of P
           for (int j = chunk_t0(pc); j < chunk_t1(pc) && ok; ++j) {
             const Tile t = tile_of(p, sq, j);
             const int jt = j - chunk_t0(pc);
-            for (int q = 0; q < kSlotsPerTile && ok; ++q) {
-              const uint32_t s = cnt % kStages;
+            for (int h = 0; h < kSlotsPerTile / 2 && ok; ++h) {
+              const uint32_t s = cnt % kStages;  // == 2 h
               if (!(ok = mbar_wait(&bars->ring_full[s], (cnt / kStages) & 1, abort))) break;
+              if (!(ok = mbar_wait(&bars->ring_full[s + 1], ((cnt + 1) / kStages) & 1, abort)))
+                break;
               tc_fence_after();
               const uint32_t vaddr = rbase + s * kSlotBytes;
               for (int kk = 0; kk < t.n / 16; ++kk) {
                 const int key16 = jt * (kTN / 16) + kk;  // 16-key group within the chunk
                 const uint32_t paddr = pbuf + (key16 >> 2) * kPChunkBytes + (key16 & 3) * 32;
-                umma_ss(tmem + q * 128, sdesc_sw128(paddr, 16, 1024),
-                        sdesc_sw128(vaddr + kk * 2048, kChunk128, 1024), idesc_pv,
+                const uint64_t vd = sdesc_sw128(vaddr + kk * 2048, kChunk128, 1024);
+                umma_ss(tmem + h * 256, sdesc_sw128(paddr, 16, 1024), vd, idesc_pv,
                         (pc > 0 || jt > 0 || kk > 0));
+                umma_ss(tmem + h * 256, sdesc_sw128(paddr + kPBytes, 16, 1024), vd, idesc_pv, 1u);
               }
               umma_commit(&bars->ring_empty[s]);
-              ++cnt;
+              umma_commit(&bars->ring_empty[s + 1]);
+              cnt += 2;
             }
           }
           if (ok) umma_commit(&bars->o_done[pc & 1]);
@@ -374,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       for (int j = chunk_t0(c); j < chunk_t1(c); ++j) {
         const Tile tl = tile_of(p, sq, j);
         // visible columns: a prefix of a compressed tile, or ring slots 0..min(W,t+1)-1
-        const int vhi = tl.kind == kCompressed ? min(tl.n, sq.nc - tl.key0) : min(W, t + 1);
+        const int vhi = tl.kind == kCompressed ? min(tl.n, sq.e1 - tl.key0) : min(W, t + 1);
         const uint32_t vlen = vhi > 0 ? (uint32_t)vhi : 0u;
         const uint32_t col0 = (j - chunk_t0(c)) * kTN;
         for (int q = 0; q < kTN / 32; ++q) {
@@ -428,13 +446,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         }
         tmem_wait_st();
       }
-      // pass 2: P = exp2(s * scale - base) -> bf16, K-major 128B-swizzled rows
+      // pass 2: P = exp2(s * scale - base) -> bf16 parts P_hi = bf16(P), P_lo = bf16(P - P_hi)
+      // in two K-major 128B-swizzled buffers; O += P_hi V + P_lo V keeps ~16 bits of P
       uint8_t* pbuf = sP;
       const float bb = base == -INFINITY ? 0.f : base;
       float ps[4] = {0.f, 0.f, 0.f, 0.f};
       for (int j = chunk_t0(c); j < chunk_t1(c); ++j) {
         const Tile tl = tile_of(p, sq, j);
-        const int vhi = tl.kind == kCompressed ? min(tl.n, sq.nc - tl.key0) : min(W, t + 1);
+        const int vhi = tl.kind == kCompressed ? min(tl.n, sq.e1 - tl.key0) : min(W, t + 1);
         const uint32_t vlen = vhi > 0 ? (uint32_t)vhi : 0u;
         const int jt = j - chunk_t0(c);
         for (int q = 0; q < kTN / 32; ++q) {
@@ -443,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           tmem_ld32(sbuf + jt * kTN + q * 32, v);
           tmem_wait_ld();
           if (s_lane) {
-            uint32_t pk[16];
+            uint32_t pk[16], pl[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
               const int c0 = q * 32 + 2 * e;
@@ -453,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
               const float p1 = (uint32_t)(c0 + 1) < vlen
                                    ? fast_exp2(fmaf(__uint_as_float(v[2 * e + 1]), p.scale_log2, -bb))
                                    : 0.f;
-              pk[e] = pack_bf16x2(p0, p1);
+              split_bf16x2(p0, p1, pk[e], pl[e]);
               ps[e & 3] += p0 + p1;
             }
             // chunk keys jt*128 + q*32 .. -> 64-key P chunk (jt*2 + q/2), units (q&1)*4 + w
@@ -464,6 +483,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
               const int us = u ^ (hrow & 7);
               *reinterpret_cast<uint4*>(rowp + us * 16) =
                   make_uint4(pk[4 * w], pk[4 * w + 1], pk[4 * w + 2], pk[4 * w + 3]);
+              *reinterpret_cast<uint4*>(rowp + kPBytes + us * 16) =
+                  make_uint4(pl[4 * w], pl[4 * w + 1], pl[4 * w + 2], pl[4 * w + 3]);
             }
           }
         }
@@ -510,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     // then invalid and flagged)
     asm volatile("bar.sync 1, 128;" ::: "memory");
     const int tid = threadIdx.x - 64;  // 0..127 over the four softmax warps
-    if (p.nsplit == 1) {
+    if (p.nsplit == 1 && !p.partial) {
       // final output: O / l, gate, bf16 in 16-byte units; lse in natural log
       __nv_bfloat16* ob = p.O + (int64_t)b * p.hq * kD;
 #pragma unroll 4
@@ -566,18 +587,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   }
 }
 
-// Combine the split partials of one sequence: per head, O = sum_s 2^(m_s - M) O_s /
-// sum_s 2^(m_s - M) l_s, then the gate and the cast to bf16; lse in natural log.
-// One block per (head, sequence), 4 output columns per thread. The non-empty splits are
-// listed in split order (ballot compaction, so the sums are deterministic) with their
-// weights in shared memory; every thread then walks the list with independent loads.
+// Combine the partials of one sequence: per head, M = max_s m_s over the parts holding keys,
+// L = sum_s 2^(m_s - M) l_s, acc = sum_s 2^(m_s - M) O_s. Final output: acc / L, then the
+// gate and the cast to bf16, lse = (M + log2 L) ln 2. Partial output (one part that stands
+// for all of them): (M, L) and acc, float32. One block per (head, sequence), 4 output
+// columns per thread. The non-empty parts are listed in order (ballot compaction, so the
+// sums are deterministic) with their weights in shared memory; every thread then walks the
+// list with independent loads.
 constexpr int kMergeThreads = kD / 4;  // 128
 
-__global__ void __launch_bounds__(kMergeThreads) merge_kernel(const float* ws_ml,
-                                                              const float* ws_o, int nsplit,
-                                                              int hq, const __nv_bfloat16* gate,
-                                                              int64_t gs0, int64_t gs2,
-                                                              __nv_bfloat16* O, float* lse) {
+struct MergeArgs {
+  const float* ml;             // (m, l) of part s, sequence b, head h at
+  const float* o;              //   ml + s * ml_ss + b * ml_bs + 2 h;  o: + s * o_ss + b * o_bs
+  int64_t ml_ss, ml_bs, o_ss, o_bs;  // + h * 512
+  int nsplit, hq;
+  const __nv_bfloat16* gate;
+  int64_t gs0, gs2;
+  __nv_bfloat16* O;            // final output (when pml == nullptr)
+  float* lse;
+  float* pml;                  // partial output [b, h, 2] and [b, h, 512] (or nullptr)
+  float* po;
+};
+
+__global__ void __launch_bounds__(kMergeThreads) merge_kernel(const MergeArgs a) {
   __shared__ float s_w[kMergeThreads], s_l[kMergeThreads];
   __shared__ int s_idx[kMergeThreads];
   __shared__ float s_red[kMergeThreads / 32];
@@ -589,14 +621,13 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const float* ws_ml
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int wid = tid >> 5;
-  const int64_t mstride = (int64_t)hq * 2;   // floats between splits in ws_ml
-  const int64_t ostride = (int64_t)hq * kD;  // floats between splits in ws_o
-  const float* ml = ws_ml + ((int64_t)b * nsplit * hq + h) * 2;
-  const float* ob = ws_o + ((int64_t)b * nsplit * hq + h) * kD + tid * 4;
+  const int nsplit = a.nsplit;
+  const float* ml = a.ml + (int64_t)b * a.ml_bs + (int64_t)h * 2;
+  const float* ob = a.o + (int64_t)b * a.o_bs + (int64_t)h * kD + tid * 4;
 
   float m = -INFINITY;
   for (int s = tid; s < nsplit; s += kMergeThreads) {
-    const float2 v = *reinterpret_cast<const float2*>(ml + s * mstride);
+    const float2 v = *reinterpret_cast<const float2*>(ml + s * a.ml_ss);
     if (v.y > 0.f) m = fmaxf(m, v.x);
   }
 #pragma unroll
@@ -612,7 +643,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const float* ws_ml
   for (int s0 = 0; s0 < nsplit; s0 += kMergeThreads) {
     const int s = s0 + tid;
     float2 v = make_float2(-INFINITY, 0.f);
-    if (s < nsplit) v = *reinterpret_cast<const float2*>(ml + s * mstride);
+    if (s < nsplit) v = *reinterpret_cast<const float2*>(ml + s * a.ml_ss);
     const bool live = v.y > 0.f;
     const unsigned bal = __ballot_sync(0xffffffffu, live);
     __syncthreads();  // the previous chunk's list has been consumed
@@ -636,7 +667,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const float* ws_ml
       float4 x[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u)
-        x[u] = *reinterpret_cast<const float4*>(ob + s_idx[k + u] * ostride);
+        x[u] = *reinterpret_cast<const float4*>(ob + s_idx[k + u] * a.o_ss);
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const float w = s_w[k + u];
@@ -648,7 +679,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const float* ws_ml
       }
     }
     for (; k < n; ++k) {
-      const float4 x = *reinterpret_cast<const float4*>(ob + s_idx[k] * ostride);
+      const float4 x = *reinterpret_cast<const float4*>(ob + s_idx[k] * a.o_ss);
       const float w = s_w[k];
       acc.x = fmaf(w, x.x, acc.x);
       acc.y = fmaf(w, x.y, acc.y);
@@ -657,11 +688,17 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const float* ws_ml
       L = fmaf(w, s_l[k], L);
     }
   }
+  const int d = tid * 4;
+  const int64_t bh = (int64_t)b * a.hq + h;
+  if (a.pml) {
+    *reinterpret_cast<float4*>(a.po + bh * kD + d) = acc;
+    if (tid == 0) *reinterpret_cast<float2*>(a.pml + bh * 2) = make_float2(M, L);
+    return;
+  }
   const float inv = 1.f / L;
   float o[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
-  const int d = tid * 4;
-  if (gate) {
-    const __nv_bfloat16* gp = gate + (int64_t)b * gs0 + (int64_t)h * gs2 + d;
+  if (a.gate) {
+    const __nv_bfloat16* gp = a.gate + (int64_t)b * a.gs0 + (int64_t)h * a.gs2 + d;
     const float2 g0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(gp));
     const float2 g1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(gp + 2));
     o[0] *= g0.x;
@@ -669,9 +706,9 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const float* ws_ml
     o[2] *= g1.x;
     o[3] *= g1.y;
   }
-  *reinterpret_cast<uint2*>(O + ((int64_t)b * hq + h) * kD + d) =
+  *reinterpret_cast<uint2*>(a.O + bh * kD + d) =
       make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
-  if (lse && tid == 0) lse[(int64_t)b * hq + h] = (M + __log2f(L)) * 0.69314718055994531f;
+  if (a.lse && tid == 0) a.lse[bh] = (M + __log2f(L)) * 0.69314718055994531f;
 }
 
 }  // namespace
@@ -691,16 +728,15 @@ bool decode_tc_supported(const hca_desc& d, const hca_cache& c) {
   return true;
 }
 
-// Splits per sequence (d.decode_splits if > 0, capped at the tiles). Automatic rule: the
-// time of a step is about the largest number of 128-key tiles one CTA streams, plus, once
-// a sequence is split, its float32 partials and the merge (about two tiles' worth,
-// measured). Among the split counts that keep every CTA in one wave (splits x batch <=
-// SMs), take the one with the fewest tiles per CTA + 2 if split; ties go to fewer splits.
-// 16 sequences at 1M context (65 tiles) -> 9 splits; 128 sequences of up to 9 tiles -> 1.
-int decode_num_splits(const hca_desc& d) {
-  const int64_t x = (int64_t)d.seqlen - d.window;
-  const int64_t nc = x < 0 ? 0 : x / d.block;
-  const int tiles = (int)((nc + kTN - 1) / kTN) + 1;
+// Splits per sequence for a key list of `tiles` 128-key tiles (d.decode_splits if > 0,
+// capped at the tiles). Automatic rule: the time of a step is about the largest number of
+// tiles one CTA streams, plus, once a sequence is split, its float32 partials and the merge
+// (about two tiles' worth, measured). Among the split counts that keep every CTA in one
+// wave (splits x batch <= SMs), take the one with the fewest tiles per CTA + 2 if split;
+// ties go to fewer splits. 16 sequences at 1M context (65 tiles) -> 9 splits; 128
+// sequences of up to 9 tiles -> 1.
+static int splits_for_tiles(const hca_desc& d, int tiles) {
+  if (tiles < 1) tiles = 1;
   if (d.decode_splits > 0) return d.decode_splits < tiles ? d.decode_splits : tiles;
   const int64_t sms = device_sm_count();
   const int64_t batch = d.batch > 0 ? d.batch : 1;
@@ -719,9 +755,31 @@ int decode_num_splits(const hca_desc& d) {
   return best;
 }
 
+// visible compressed entries of the longest context d.seqlen
+static int64_t max_visible_entries(const hca_desc& d) {
+  const int64_t x = (int64_t)d.seqlen - d.window;
+  return x < 0 ? 0 : x / d.block;
+}
+
+int decode_num_splits(const hca_desc& d) {
+  return splits_for_tiles(d, (int)((max_visible_entries(d) + kTN - 1) / kTN) + 1);
+}
+
+// Split count of a call over the key part: at most that of the whole key list, so the
+// workspace of hca_decode_workspace_bytes(d) always suffices.
+static int part_num_splits(const hca_desc& d, const DecodePart& part) {
+  const int64_t nc = max_visible_entries(d);
+  const int64_t e1 = part.e1 < nc ? part.e1 : nc;
+  const int64_t n = e1 > part.e0 ? e1 - part.e0 : 0;
+  const int tiles = (int)((n + kTN - 1) / kTN) + (part.with_ring ? 1 : 0);
+  const int ns = splits_for_tiles(d, tiles);
+  const int full = decode_num_splits(d);
+  return ns < full ? ns : full;
+}
+
 // Workspace layout: ws_ml [batch, nsplit, hq, 2] float, padded to a multiple of 4 floats so
 // that ws_o [batch, nsplit, hq, 512] float (read and written as float4) starts 16-byte
-// aligned whatever batch * nsplit * hq is.
+// aligned whatever batch * nsplit * hq is. A partial result is this layout with nsplit 1.
 static size_t ml_floats(const hca_desc& d, int nsplit) {
   const size_t n = (size_t)d.batch * nsplit * d.hq * 2;
   return (n + 3) & ~size_t(3);
@@ -732,12 +790,35 @@ size_t decode_tc_workspace_bytes(const hca_desc& d) {
   return (ml_floats(d, ns) + (size_t)d.batch * ns * d.hq * kD) * sizeof(float);
 }
 
-cudaError_t launch_decode_tc(const hca_desc& d, const void* Q, const int32_t* ctx_len,
-                             const hca_cache& c, const void* ring_k, const void* ring_v,
-                             void* O, float* lse, void* ws, cudaStream_t s) {
+size_t decode_partial_bytes(const hca_desc& d) {
+  return (ml_floats(d, 1) + (size_t)d.batch * d.hq * kD) * sizeof(float);
+}
+
+size_t decode_part_workspace_bytes(const hca_desc& d, const DecodePart& part) {
+  const int ns = part_num_splits(d, part);
+  if (ns == 1 && part.out_partial) return 0;
+  return (ml_floats(d, ns) + (size_t)d.batch * ns * d.hq * kD) * sizeof(float);
+}
+
+static cudaLaunchConfig_t pdl_config(cudaLaunchAttribute* pdl, cudaStream_t s) {
+  // programmatic dependent of the grid before it on the stream (each kernel waits for it
+  // with griddepcontrol.wait before touching memory)
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.stream = s;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+
+cudaError_t launch_decode_part(const hca_desc& d, const void* Q, const int32_t* ctx_len,
+                               const hca_cache& c, const void* ring_k, const void* ring_v,
+                               const DecodePart& part, void* O, float* lse, void* ws,
+                               cudaStream_t s) {
   Params p;
   memset(&p, 0, sizeof(p));
-  const int nsplit = decode_num_splits(d);
+  const int nsplit = part_num_splits(d, part);
   cudaError_t e;
   const uint64_t rowsC = (uint64_t)c.num_pages * c.page_entries;
   if ((e = encode_bf16_chunks(&p.tmQ, Q, (uint64_t)d.batch * d.hq, kM, 4)) != cudaSuccess)
@@ -747,12 +828,19 @@ cudaError_t launch_decode_tc(const hca_desc& d, const void* Q, const int32_t* ct
   const uint64_t rowsR = (uint64_t)d.batch * d.window;
   if ((e = encode_bf16_chunks(&p.tmRk, ring_k, rowsR, kTN, 2)) != cudaSuccess) return e;
   if ((e = encode_bf16_chunks(&p.tmRv, ring_v, rowsR, kTN, 2)) != cudaSuccess) return e;
+  float* pml = static_cast<float*>(part.out_partial);
+  float* po = pml ? pml + ml_floats(d, 1) : nullptr;
   p.ctx_len = ctx_len;
   p.page_table = c.page_table;
   p.n_entries = c.n_entries;
   p.err_word = c.err_word;
-  p.ws_ml = static_cast<float*>(ws);
-  p.ws_o = p.ws_ml + ml_floats(d, nsplit);
+  if (pml && nsplit == 1) {  // the decode CTAs write the partial result themselves
+    p.ws_ml = pml;
+    p.ws_o = po;
+  } else {
+    p.ws_ml = static_cast<float*>(ws);
+    p.ws_o = p.ws_ml + ml_floats(d, nsplit);
+  }
   p.nseq = d.batch;
   p.seqlen = d.seqlen;
   p.hq = d.hq;
@@ -762,44 +850,84 @@ cudaError_t launch_decode_tc(const hca_desc& d, const void* Q, const int32_t* ct
   p.max_pages = c.max_pages;
   p.num_pages = c.num_pages;
   p.nsplit = nsplit;
+  p.e0 = part.e0;
+  p.e1 = part.e1;
+  p.with_ring = part.with_ring ? 1 : 0;
+  p.partial = pml ? 1 : 0;
   p.scale_log2 = d.scale * 1.4426950408889634f;
   p.O = static_cast<__nv_bfloat16*>(O);
   p.lse = lse;
   p.gate = static_cast<const __nv_bfloat16*>(d.gate);
   p.gs0 = d.gate_strides[0];
   p.gs2 = d.gate_strides[2];
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
-  // both grids are programmatic dependents of the grid before them on the stream (each
-  // waits for it with griddepcontrol.wait before touching memory): the merge is scheduled
-  // while decode CTAs drain, and a following decode step's prologue overlaps the merge
+  static PerDevice<int> smem_limit_set;
+  if ((e = set_smem_limit_once(smem_limit_set, (const void*)decode_tc_kernel, (int)kSmemBytes)) !=
+      cudaSuccess)
+    return e;
+  // both grids are programmatic dependents of the grid before them on the stream: the merge
+  // is scheduled while decode CTAs drain, and a following decode step's prologue overlaps
+  // the merge
   cudaLaunchAttribute pdl[1];
-  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  pdl[0].val.programmaticStreamSerializationAllowed = 1;
-  cudaLaunchConfig_t cfg = {};
+  cudaLaunchConfig_t cfg = pdl_config(pdl, s);
   cfg.gridDim = dim3(nsplit, d.batch);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmemBytes;
-  cfg.stream = s;
-  cfg.attrs = pdl;
-  cfg.numAttrs = 1;
   if ((e = cudaLaunchKernelEx(&cfg, decode_tc_kernel, p)) != cudaSuccess) return e;
-  if (nsplit == 1) return cudaSuccess;  // the decode CTAs wrote O and lse themselves
-  cudaLaunchConfig_t mcfg = cfg;
+  if (nsplit == 1) return cudaSuccess;  // the decode CTAs wrote their result themselves
+  MergeArgs m;
+  memset(&m, 0, sizeof(m));
+  m.ml = p.ws_ml;
+  m.o = p.ws_o;
+  m.ml_ss = (int64_t)d.hq * 2;
+  m.ml_bs = (int64_t)nsplit * d.hq * 2;
+  m.o_ss = (int64_t)d.hq * kD;
+  m.o_bs = (int64_t)nsplit * d.hq * kD;
+  m.nsplit = nsplit;
+  m.hq = d.hq;
+  m.gate = static_cast<const __nv_bfloat16*>(d.gate);
+  m.gs0 = d.gate_strides[0];
+  m.gs2 = d.gate_strides[2];
+  m.O = static_cast<__nv_bfloat16*>(O);
+  m.lse = lse;
+  m.pml = pml;
+  m.po = po;
+  cudaLaunchConfig_t mcfg = pdl_config(pdl, s);
   mcfg.gridDim = dim3(d.hq, d.batch);
   mcfg.blockDim = dim3(kMergeThreads);
-  mcfg.dynamicSmemBytes = 0;
-  return cudaLaunchKernelEx(&mcfg, merge_kernel, (const float*)p.ws_ml, (const float*)p.ws_o,
-                            nsplit, (int)d.hq, static_cast<const __nv_bfloat16*>(d.gate),
-                            (int64_t)d.gate_strides[0], (int64_t)d.gate_strides[2],
-                            static_cast<__nv_bfloat16*>(O), lse);
+  return cudaLaunchKernelEx(&mcfg, merge_kernel, m);
+}
+
+cudaError_t launch_decode_tc(const hca_desc& d, const void* Q, const int32_t* ctx_len,
+                             const hca_cache& c, const void* ring_k, const void* ring_v,
+                             void* O, float* lse, void* ws, cudaStream_t s) {
+  const DecodePart whole{0, INT32_MAX, 1, nullptr};
+  return launch_decode_part(d, Q, ctx_len, c, ring_k, ring_v, whole, O, lse, ws, s);
+}
+
+cudaError_t launch_decode_merge(const hca_desc& d, const void* parts, int n_parts,
+                                int64_t part_stride_bytes, void* O, float* lse,
+                                cudaStream_t s) {
+  MergeArgs m;
+  memset(&m, 0, sizeof(m));
+  const int64_t stride = part_stride_bytes / (int64_t)sizeof(float);
+  m.ml = static_cast<const float*>(parts);
+  m.o = m.ml + ml_floats(d, 1);
+  m.ml_ss = stride;
+  m.ml_bs = (int64_t)d.hq * 2;
+  m.o_ss = stride;
+  m.o_bs = (int64_t)d.hq * kD;
+  m.nsplit = n_parts;
+  m.hq = d.hq;
+  m.gate = static_cast<const __nv_bfloat16*>(d.gate);
+  m.gs0 = d.gate_strides[0];
+  m.gs2 = d.gate_strides[2];
+  m.O = static_cast<__nv_bfloat16*>(O);
+  m.lse = lse;
+  cudaLaunchAttribute pdl[1];
+  cudaLaunchConfig_t mcfg = pdl_config(pdl, s);
+  mcfg.gridDim = dim3(d.hq, d.batch);
+  mcfg.blockDim = dim3(kMergeThreads);
+  return cudaLaunchKernelEx(&mcfg, merge_kernel, m);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -819,20 +947,17 @@ cudaError_t launch_decode_tc(const hca_desc& d, const void* Q, const int32_t* ct
 static __device__ __align__(256) unsigned char g_decode_scratch[HCA_DECODE_NOALLOC_SCRATCH_BYTES];
 
 // The array's name is only a host-side stand-in; its device address is looked up once per
-// device (on that device's first call) and cached.
+// device (on that device's first call, with that device current) and memoised.
 static cudaError_t decode_scratch_address(void** out) {
-  static void* cached[64] = {nullptr};
+  static PerDevice<void*> cached;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev >= 0 && dev < 64 && cached[dev]) {
-    *out = cached[dev];
-    return cudaSuccess;
-  }
+  if (cached.get(dev, out)) return cudaSuccess;
   void* ptr = nullptr;
   e = cudaGetSymbolAddress(&ptr, g_decode_scratch);
   if (e != cudaSuccess) return e;
-  if (dev >= 0 && dev < 64) cached[dev] = ptr;
+  cached.put(dev, ptr);
   *out = ptr;
   return cudaSuccess;
 }

@@ -16,15 +16,27 @@
 namespace hca {
 
 int device_sm_count() {
-  static int cache[64] = {0};
+  static PerDevice<int> cache;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
   int n = 0;
+  if (cache.get(dev, &n)) return n;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
     n = 148;
-  if (dev >= 0 && dev < 64) cache[dev] = n;
+  cache.put(dev, n);
   return n;
+}
+
+cudaError_t set_smem_limit_once(PerDevice<int>& done, const void* kernel, int bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  int flag = 0;
+  if (done.get(dev, &flag)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  done.put(dev, 1);
+  return cudaSuccess;
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -33,7 +45,9 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 static EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
+  // looked up once; threads racing on the first lookup store the same pointer
+  static std::atomic<EncodeTiledFn> cached{nullptr};
+  EncodeTiledFn fn = cached.load(std::memory_order_relaxed);
   if (fn) return fn;
   void* ptr = nullptr;
   cudaDriverEntryPointQueryResult q;
@@ -42,6 +56,7 @@ static EncodeTiledFn get_encode_fn() {
       q != cudaDriverEntryPointSuccess)
     return nullptr;
   fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  cached.store(fn, std::memory_order_relaxed);
   return fn;
 }
 
@@ -156,28 +171,44 @@ int32_t hca_compress(const hca_desc* d, const void* K, const void* V,
                                    reinterpret_cast<cudaStream_t>(stream)));
 }
 
-int32_t hca_attn_prefill(const hca_desc* d, const void* Q, const void* K, const void* V,
-                         const hca_cache* cache, void* O, float* lse, int32_t* dbg_mask,
-                         hca_stream_t stream) {
+int32_t hca_attn_prefill_range(const hca_desc* d, int32_t q_pos0, int32_t kv_pos0,
+                               int32_t kv_len, const void* Q, const void* K, const void* V,
+                               const hca_cache* cache, void* O, float* lse, int32_t* dbg_mask,
+                               hca_stream_t stream) {
   int32_t st = check_desc(d);
   if (st != HCA_OK) return st;
   if ((st = check_cache(cache)) != HCA_OK) return st;
+  if (q_pos0 < 0 || kv_pos0 < 0 || kv_len < 0) return HCA_EINVAL;
   if (d->batch == 0 || d->seqlen == 0) return HCA_OK;
   if (!Q || !K || !V || !O) return HCA_EINVAL;
+  if ((int64_t)q_pos0 + d->seqlen > INT32_MAX) return HCA_EINVAL;
+  // the K/V rows must hold every raw token a query row's window reaches
+  const int64_t first_needed = q_pos0 - d->window + 1 > 0 ? q_pos0 - d->window + 1 : 0;
+  if (kv_pos0 > first_needed || (int64_t)kv_pos0 + kv_len < (int64_t)q_pos0 + d->seqlen)
+    return HCA_EINVAL;
   if (d->gate && (d->gate_strides[0] < 0 || d->gate_strides[1] < 0 || d->gate_strides[2] < 0))
     return HCA_EINVAL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const PrefillRange r{q_pos0, kv_pos0, kv_len};
   if (d->dtype == HCA_F32) {
     if (d->head_dim % 32 != 0 || d->head_dim > 512) return HCA_EUNSUPPORTED;
-    return from_cuda(launch_prefill_simt(*d, Q, K, V, *cache, O, lse, dbg_mask, s));
+    return from_cuda(launch_prefill_simt(*d, Q, K, V, *cache, O, lse, dbg_mask, r, s));
   }
   if (!prefill_tc_supported(*d, *cache)) return HCA_EUNSUPPORTED;
+  if ((int64_t)d->batch * kv_len >= (int64_t(1) << 31)) return HCA_EUNSUPPORTED;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) ||
       !aligned16(cache->kc_pool) || !aligned16(cache->vc_pool))
     return HCA_EINVAL;
   if (prefill_pair_supported(*d, *cache))
-    return from_cuda(launch_prefill_pair(*d, Q, K, V, *cache, O, lse, dbg_mask, s));
-  return from_cuda(launch_prefill_tc(*d, Q, K, V, *cache, O, lse, dbg_mask, s));
+    return from_cuda(launch_prefill_pair(*d, Q, K, V, *cache, O, lse, dbg_mask, r, s));
+  return from_cuda(launch_prefill_tc(*d, Q, K, V, *cache, O, lse, dbg_mask, r, s));
+}
+
+int32_t hca_attn_prefill(const hca_desc* d, const void* Q, const void* K, const void* V,
+                         const hca_cache* cache, void* O, float* lse, int32_t* dbg_mask,
+                         hca_stream_t stream) {
+  if (!d) return HCA_EINVAL;
+  return hca_attn_prefill_range(d, 0, 0, d->seqlen, Q, K, V, cache, O, lse, dbg_mask, stream);
 }
 
 size_t hca_decode_workspace_bytes(const hca_desc* d) {
@@ -209,6 +240,57 @@ int32_t hca_attn_decode(const hca_desc* d, const void* Q, const int32_t* ctx_len
     return HCA_EINVAL;
   return from_cuda(
       launch_decode_tc(*d, Q, ctx_len, *cache, ring_k, ring_v, O, lse, workspace, s));
+}
+
+size_t hca_decode_partial_bytes(const hca_desc* d) {
+  if (check_desc(d) != HCA_OK || d->dtype != HCA_BF16) return 0;
+  return decode_partial_bytes(*d);
+}
+
+int32_t hca_attn_decode_partial(const hca_desc* d, const void* Q, const int32_t* ctx_len,
+                                const hca_cache* cache, const void* ring_k, const void* ring_v,
+                                int32_t entry_begin, int32_t entry_end, int32_t with_window,
+                                void* partial, void* workspace, size_t workspace_bytes,
+                                hca_stream_t stream) {
+  int32_t st = check_desc(d);
+  if (st != HCA_OK) return st;
+  if ((st = check_cache(cache)) != HCA_OK) return st;
+  if (entry_begin < 0 || entry_end < entry_begin || entry_begin % 128 != 0) return HCA_EINVAL;
+  if (d->batch == 0) return HCA_OK;
+  if (!Q || !ctx_len || !ring_k || !ring_v || !partial) return HCA_EINVAL;
+  if (d->seqlen < 1) return HCA_EINVAL;
+  if (d->dtype != HCA_BF16 || !decode_tc_supported(*d, *cache)) return HCA_EUNSUPPORTED;
+  const DecodePart part{entry_begin, entry_end, with_window ? 1 : 0, partial};
+  const size_t need = decode_part_workspace_bytes(*d, part);
+  if (need > 0 && (!workspace || workspace_bytes < need)) return HCA_ENOSPACE;
+  if (!aligned16(Q) || !aligned16(ring_k) || !aligned16(ring_v) || !aligned16(partial) ||
+      (need > 0 && !aligned16(workspace)) || !aligned16(cache->kc_pool) ||
+      !aligned16(cache->vc_pool))
+    return HCA_EINVAL;
+  return from_cuda(launch_decode_part(*d, Q, ctx_len, *cache, ring_k, ring_v, part, nullptr,
+                                      nullptr, workspace, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int32_t hca_decode_merge(const hca_desc* d, const void* parts, int32_t n_parts,
+                         int64_t part_stride, void* O, float* lse, hca_stream_t stream) {
+  int32_t st = check_desc(d);
+  if (st != HCA_OK) return st;
+  if (n_parts < 1) return HCA_EINVAL;
+  if (d->batch == 0) return HCA_OK;
+  if (!parts || !O) return HCA_EINVAL;
+  if (d->dtype != HCA_BF16 || d->head_dim != 512 || d->hq < 1 || d->hq > 64)
+    return HCA_EUNSUPPORTED;
+  if (n_parts > 1 && (part_stride < (int64_t)decode_partial_bytes(*d) || part_stride % 16 != 0))
+    return HCA_EINVAL;
+  if (!aligned16(parts) || !aligned16(O)) return HCA_EINVAL;
+  if (d->gate) {
+    const uintptr_t ga = reinterpret_cast<uintptr_t>(d->gate);
+    if (ga % 4 || d->gate_strides[0] % 2 || d->gate_strides[2] % 2 || d->gate_strides[0] < 0 ||
+        d->gate_strides[2] < 0)
+      return HCA_EINVAL;
+  }
+  return from_cuda(launch_decode_merge(*d, parts, n_parts, part_stride, O, lse,
+                                       reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int32_t hca_attn_decode_noalloc(const hca_desc* d, const void* Q, const int32_t* ctx_len,

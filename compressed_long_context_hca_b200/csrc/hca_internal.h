@@ -5,9 +5,35 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/hca.h"
 
 namespace hca {
+
+// Per-device memo of a value that a device's first call computes (a kernel attribute set,
+// a symbol address, a count); T() means "not computed yet". The slots are relaxed atomics:
+// host threads whose first calls on one device race each compute the same value and store
+// it, which is harmless. Devices numbered kMaxDevices and up are not memoised: every call
+// computes the value again.
+constexpr int kMaxDevices = 64;
+template <typename T>
+struct PerDevice {
+  std::atomic<T> slot[kMaxDevices];
+  bool get(int dev, T* out) const {
+    if (dev < 0 || dev >= kMaxDevices) return false;
+    const T v = slot[dev].load(std::memory_order_relaxed);
+    if (v == T()) return false;
+    *out = v;
+    return true;
+  }
+  void put(int dev, T v) {
+    if (dev >= 0 && dev < kMaxDevices) slot[dev].store(v, std::memory_order_relaxed);
+  }
+};
+
+// Raises the dynamic shared-memory limit of `kernel` on the current device, once per device.
+cudaError_t set_smem_limit_once(PerDevice<int>& done, const void* kernel, int bytes);
 
 // Number of SMs of the current device (cached per device).
 int device_sm_count();
@@ -16,10 +42,16 @@ cudaError_t launch_compress(const hca_desc& d, const void* K, const void* V,
                             int64_t batch_stride_tokens, int32_t first_block,
                             int32_t n_blocks, const hca_cache& c, cudaStream_t s);
 
+// Query rows of a prefill call: row t of a sequence is position q_pos0 + t; K/V row u is
+// position kv_pos0 + u, kv_len rows per sequence (a whole sequence: 0, 0, seqlen).
+struct PrefillRange {
+  int32_t q_pos0, kv_pos0, kv_len;
+};
+
 // float32, CUDA cores, any shape with head_dim % 32 == 0 && head_dim <= 512
 cudaError_t launch_prefill_simt(const hca_desc& d, const void* Q, const void* K,
                                 const void* V, const hca_cache& c, void* O, float* lse,
-                                int32_t* dbg_mask, cudaStream_t s);
+                                int32_t* dbg_mask, const PrefillRange& r, cudaStream_t s);
 cudaError_t launch_decode_simt(const hca_desc& d, const void* Q, const int32_t* ctx_len,
                                const hca_cache& c, const void* ring_k, const void* ring_v,
                                void* O, float* lse, cudaStream_t s);
@@ -28,14 +60,30 @@ cudaError_t launch_decode_simt(const hca_desc& d, const void* Q, const int32_t* 
 bool prefill_tc_supported(const hca_desc& d, const hca_cache& c);
 cudaError_t launch_prefill_tc(const hca_desc& d, const void* Q, const void* K, const void* V,
                               const hca_cache& c, void* O, float* lse, int32_t* dbg_mask,
-                              cudaStream_t s);
+                              const PrefillRange& r, cudaStream_t s);
 // bf16, 2-CTA clusters on the 2-SM UMMA (hq in 16..128); preferred over the one-CTA kernel
 bool prefill_pair_supported(const hca_desc& d, const hca_cache& c);
 cudaError_t launch_prefill_pair(const hca_desc& d, const void* Q, const void* K, const void* V,
                                 const hca_cache& c, void* O, float* lse, int32_t* dbg_mask,
-                                cudaStream_t s);
+                                const PrefillRange& r, cudaStream_t s);
+
+// The key part of a decode call: visible compressed entries [e0, e1) (e0 a multiple of 128)
+// and the raw window if with_ring. out_partial == nullptr: the call writes the final output;
+// else it writes an unnormalised float32 partial result there (decode_partial_bytes).
+struct DecodePart {
+  int32_t e0, e1, with_ring;
+  void* out_partial;
+};
 
 bool decode_tc_supported(const hca_desc& d, const hca_cache& c);
+size_t decode_partial_bytes(const hca_desc& d);
+size_t decode_part_workspace_bytes(const hca_desc& d, const DecodePart& part);
+cudaError_t launch_decode_part(const hca_desc& d, const void* Q, const int32_t* ctx_len,
+                               const hca_cache& c, const void* ring_k, const void* ring_v,
+                               const DecodePart& part, void* O, float* lse, void* ws,
+                               cudaStream_t s);
+cudaError_t launch_decode_merge(const hca_desc& d, const void* parts, int n_parts,
+                                int64_t part_stride_bytes, void* O, float* lse, cudaStream_t s);
 int decode_num_splits(const hca_desc& d);
 size_t decode_tc_workspace_bytes(const hca_desc& d);
 cudaError_t launch_decode_tc(const hca_desc& d, const void* Q, const int32_t* ctx_len,

@@ -28,6 +28,10 @@
 //    softmax (TMEM lane = row), warps 6-9 the epilogue (O / l, gate, bf16). The peer's TMA
 //    loads complete on the leader's barriers; the leader's UMMA commits arrive on the same
 //    barrier of both CTAs; the peer's softmax and epilogue warps arrive on the leader's.
+//  * P is carried as two bf16 parts, P = P_hi + P_lo (P_lo the bf16 of the remainder), and
+//    O += P.V runs as two TS-UMMAs per 16-key group, one per part: a peaked softmax (a few
+//    keys of large, far-apart values) then loses ~2^-17 of the value spread to the rounding
+//    of P instead of 2^-9 with one bf16 P.
 //  * One UMMA stream across items: S of tile g, then P.V of tile g-1. The softmax hands
 //    P(g) over before it observes the completion of P.V(g-1) unless O must be rescaled
 //    (lazy rescale: only when the row max grows by more than 2^8), so P.V(g) queues behind
@@ -88,6 +92,8 @@ struct Params {
   const int32_t* n_entries;
   int32_t* err_word;
   int32_t batch, T, hq, P, W, block, PE, max_pages, num_pages;
+  // query row t of a sequence is position q0 + t; K/V row u is position kv0 + u, of Tk rows
+  int32_t q0, kv0, Tk;
   int32_t o32;      // O is 32-byte aligned: the epilogue stores 32 bytes per lane
   int32_t n_pt;     // pair row tiles per sequence (2 P positions each)
   int32_t n_items;  // 2 * batch * n_pt
@@ -96,10 +102,10 @@ struct Params {
 
 struct Item {
   int b, half;
-  int t0, tl;   // first position, last valid position of the pair row tile
+  int t0, tl;   // first query row, last valid query row of the pair row tile
   int nc_last;  // compressed entries visible to the last position (clamped)
   int nct;      // compressed tiles
-  int lo, hi;   // raw key range of the pair row tile
+  int lo, hi;   // raw key range of the pair row tile (positions)
   int rawA_n;   // keys of the last raw tile
   int strag;    // 1 if the 16-key raw tile exists
   int ntiles;
@@ -135,10 +141,10 @@ __device__ __forceinline__ Item make_item(const Params& p, int k) {
   it.t0 = i * 2 * p.P;
   it.tl = min(it.t0 + 2 * p.P - 1, p.T - 1);
   const int have = min(p.n_entries[it.b], p.max_pages * p.PE);
-  it.nc_last = min(visible_count(it.tl, p.block, p.W), have);
+  it.nc_last = min(visible_count(it.tl + p.q0, p.block, p.W), have);
   it.nct = (it.nc_last + kBN - 1) / kBN;
-  it.lo = max(0, it.t0 - p.W + 1);
-  it.hi = it.tl;
+  it.lo = max(0, it.t0 + p.q0 - p.W + 1);
+  it.hi = it.tl + p.q0;
   const int R = it.hi - it.lo + 1;
   it.rawA_n = min(kBN, round16(min(R, kBN)));
   it.strag = R > kBN ? 1 : 0;
@@ -419,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mk = &p.tmKc;
           mv = &p.tmVc;
         } else {
-          row0 = it.b * p.T + t.key0;
+          row0 = it.b * p.Tk + t.key0 - p.kv0;
           mk = &p.tmK;
           mv = &p.tmV;
         }
@@ -459,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (k >= p.n_items) break;
         const Item it = make_item(p, k);
         if (leader && mine == 0 && p.err_word &&
-            visible_count(it.tl, p.block, p.W) > p.n_entries[it.b])
+            visible_count(it.tl + p.q0, p.block, p.W) > p.n_entries[it.b])
           atomicOr(p.err_word, kErrCacheShort);
         for (int j = 0; j < it.ntiles && ok; ++j) {
           ok = load_tile(it, j, false);
@@ -601,13 +607,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t idesc = idesc_bf16_f32(2 * kBM, kDH, true);
         const uint64_t vd0 = sdesc_sw128(rbase + s * kSlotBytes, lbo, 1024);
         const uint32_t acc0 = j > 0 ? 1u : 0u;
+        // per 16-key group: O += P_hi V, then O += P_lo V (A columns 16 kk and 16 kk + 8)
         if (t.n == kBN) {
 #pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk)
-            umma2_ts(tmem + kTmO, a_tmem + kk * 8, vd0 + kk * (2048 >> 4), idesc, acc0 | kk);
+          for (int kk = 0; kk < kBN / 16; ++kk) {
+            umma2_ts(tmem + kTmO, a_tmem + kk * 16, vd0 + kk * (2048 >> 4), idesc, acc0 | kk);
+            umma2_ts(tmem + kTmO, a_tmem + kk * 16 + 8, vd0 + kk * (2048 >> 4), idesc, 1u);
+          }
         } else {
-          for (int kk = 0; kk < t.n / 16; ++kk)
-            umma2_ts(tmem + kTmO, a_tmem + kk * 8, vd0 + kk * (2048 >> 4), idesc, acc0 | kk);
+          for (int kk = 0; kk < t.n / 16; ++kk) {
+            umma2_ts(tmem + kTmO, a_tmem + kk * 16, vd0 + kk * (2048 >> 4), idesc, acc0 | kk);
+            umma2_ts(tmem + kTmO, a_tmem + kk * 16 + 8, vd0 + kk * (2048 >> 4), idesc, 1u);
+          }
         }
         umma2_commit_both(&bars->ring_empty[s]);
         ++cnt;
@@ -658,7 +669,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int pos = it.t0 + (int)rank * p.P + row / p.hq;
       const int h = row % p.hq;
       const bool row_valid = pos < p.T;
-      const int t = min(pos, p.T - 1);
+      const int tq = min(pos, p.T - 1);  // query row
+      const int t = tq + p.q0;           // its position
       const int nc_row =
           min(visible_count(t, p.block, p.W), min(p.n_entries[it.b], p.max_pages * p.PE));
       const int lo_row = max(0, t - p.W + 1);
@@ -725,15 +737,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           rescale = true;
         }
         const float base = ref == -INFINITY ? 0.f : ref;
-        // P = exp2(s * scale - ref) in bf16, written over the score columns (A of P.V);
-        // piece q writes P columns [16q, 16q+16), already read
+        // P = exp2(s * scale - ref) as a bf16 pair hi + lo (A of the two P.V products),
+        // written over the score columns: 16-key group k of the tile keeps hi in columns
+        // [16k, 16k+8) and lo in [16k+8, 16k+16), so piece q (keys 32q .. 32q+31) lands on
+        // its own columns, already read
         float ps[4] = {0.f, 0.f, 0.f, 0.f};
         tmem_ld32(s_addr, cur);
         tmem_wait_ld();
 #pragma unroll 1
         for (int q = 0; q < npieces; ++q) {
           if (q + 1 < npieces) tmem_ld32(s_addr + (q + 1) * 32, nxt);
-          uint32_t pk[16];
+          uint32_t pk[32];
           const int c0 = q * 32;
           if (__all_sync(0xffffffffu, c0 >= vlo && c0 + 32 <= vhi)) {
 #pragma unroll
@@ -741,12 +755,12 @@ __global__ void __launch_bounds__(kThreads, 1)
               const float p0 = fast_exp2(fmaf(__uint_as_float(cur[2 * e]), p.scale_log2, -base));
               const float p1 =
                   fast_exp2(fmaf(__uint_as_float(cur[2 * e + 1]), p.scale_log2, -base));
-              pk[e] = pack_bf16x2(p0, p1);
+              split_bf16x2(p0, p1, pk[(e & 8) * 2 + (e & 7)], pk[(e & 8) * 2 + 8 + (e & 7)]);
               ps[e & 3] += p0 + p1;
             }
           } else if (__all_sync(0xffffffffu, c0 >= vhi || c0 + 32 <= vlo)) {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) pk[e] = 0u;
+            for (int e = 0; e < 32; ++e) pk[e] = 0u;
           } else {
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
@@ -758,11 +772,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               const float p1 =
                   in1 ? fast_exp2(fmaf(__uint_as_float(cur[2 * e + 1]), p.scale_log2, -base))
                       : 0.f;
-              pk[e] = pack_bf16x2(p0, p1);
+              split_bf16x2(p0, p1, pk[(e & 8) * 2 + (e & 7)], pk[(e & 8) * 2 + 8 + (e & 7)]);
               ps[e & 3] += p0 + p1;
             }
           }
-          tmem_st16(s_addr + q * 16, pk);
+          tmem_st32(s_addr + q * 32, pk);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) cur[e] = nxt[e];
@@ -793,10 +807,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           // hand the row sum to the epilogue warps; LSE and the debug mask go out here
           sL[(nitem & 1) * kBM + row] = l;
           if (row_valid && it.half == 0) {
-            const int64_t orow = ((int64_t)it.b * p.T + t) * p.hq + h;
+            const int64_t orow = ((int64_t)it.b * p.T + tq) * p.hq + h;
             if (p.lse) p.lse[orow] = (m + __log2f(l)) * 0.69314718055994531f;
             if (p.dbg && h == 0) {
-              int32_t* dp = p.dbg + ((int64_t)it.b * p.T + t) * 3;
+              int32_t* dp = p.dbg + ((int64_t)it.b * p.T + tq) * 3;
               dp[0] = nc_row;
               dp[1] = lo_row;
               dp[2] = t;
@@ -931,14 +945,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // Clusters of two that fit on the device at once (one CTA per SM); 0 if the query fails.
 int resident_pairs(cudaLaunchConfig_t cfg) {
-  static int cache[64] = {0};
+  static PerDevice<int> cache;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
   int n = 0;
+  if (cache.get(dev, &n)) return n;
   if (cudaOccupancyMaxActiveClusters(&n, (const void*)prefill_pair_kernel, &cfg) != cudaSuccess)
     return 0;
-  if (dev >= 0 && dev < 64 && n > 0) cache[dev] = n;
+  if (n > 0) cache.put(dev, n);
   return n;
 }
 
@@ -965,11 +979,11 @@ bool prefill_pair_supported(const hca_desc& d, const hca_cache& c) {
 
 cudaError_t launch_prefill_pair(const hca_desc& d, const void* Q, const void* K, const void* V,
                                 const hca_cache& c, void* O, float* lse, int32_t* dbg_mask,
-                                cudaStream_t s) {
+                                const PrefillRange& r, cudaStream_t s) {
   Params p;
   memset(&p, 0, sizeof(p));
   const uint64_t rowsQ = (uint64_t)d.batch * d.seqlen * d.hq;
-  const uint64_t rowsK = (uint64_t)d.batch * d.seqlen;
+  const uint64_t rowsK = (uint64_t)d.batch * r.kv_len;
   const uint64_t rowsC = (uint64_t)c.num_pages * c.page_entries;
   cudaError_t e;
   if ((e = encode_bf16_chunks(&p.tmQ, Q, rowsQ, kBM, 2)) != cudaSuccess) return e;
@@ -992,6 +1006,9 @@ cudaError_t launch_prefill_pair(const hca_desc& d, const void* Q, const void* K,
   p.err_word = c.err_word;
   p.batch = d.batch;
   p.T = d.seqlen;
+  p.q0 = r.q_pos0;
+  p.kv0 = r.kv_pos0;
+  p.Tk = r.kv_len;
   p.hq = d.hq;
   p.P = kBM / d.hq;
   p.W = d.window;
@@ -1003,15 +1020,10 @@ cudaError_t launch_prefill_pair(const hca_desc& d, const void* Q, const void* K,
   p.n_items = 2 * d.batch * p.n_pt;
   p.scale_log2 = d.scale * 1.4426950408889634f;
   if (p.n_items == 0) return cudaSuccess;
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    e = cudaFuncSetAttribute(prefill_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  static PerDevice<int> smem_limit_set;
+  if ((e = set_smem_limit_once(smem_limit_set, (const void*)prefill_pair_kernel, (int)kSmemBytes)) !=
+      cudaSuccess)
+    return e;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;

@@ -18,9 +18,10 @@
 //  * Warp roles: warps 0 and 10 stream K/V and warp 11 streams Q through TMA, warp 1 issues
 //    UMMA (single thread), warps 2-5 run the online softmax (one row per thread, TMEM
 //    lane = row), warps 6-9 the epilogue (O / l, gate, bf16) of the previous item.
-//  * S = Q K^T runs as kind::f16 with both operands in shared memory; P is rounded to bf16
-//    and written back into the score columns of TMEM, and O += P V runs with A from TMEM
-//    and V (N-major) from shared memory.
+//  * S = Q K^T runs as kind::f16 with both operands in shared memory; P is split into two
+//    bf16 parts (P_hi = bf16(P), P_lo = bf16(P - P_hi)) written back into the score columns
+//    of TMEM, and O += P_hi V + P_lo V runs as two UMMAs with A from TMEM and V (N-major)
+//    from shared memory, so the rounding of P costs ~2^-17 of the value spread, not 2^-9.
 //  * The key list of a tile is: compressed tiles of up to 128 entries (the last one cut to
 //    a multiple of 16), an optional 16-row raw tile for the keys that only the first
 //    position of the tile still sees, then one 128-row raw tile ending at the last position.
@@ -74,6 +75,8 @@ struct Params {
   const int32_t* n_entries;
   int32_t* err_word;
   int32_t batch, T, hq, P, W, block, PE, max_pages, num_pages;
+  // query row t of a sequence is position q0 + t; K/V row u is position kv0 + u, of Tk rows
+  int32_t q0, kv0, Tk;
   int32_t n_rt;     // row tiles per sequence
   int32_t n_items;  // 2 * batch * n_rt
   float scale_log2;
@@ -81,10 +84,10 @@ struct Params {
 
 struct Item {
   int b, i, half;
-  int t0, tl;       // first / last valid position of the tile
+  int t0, tl;       // first / last valid query row of the tile
   int nc_last;      // compressed entries visible to the last position (clamped)
   int nct;          // compressed tiles
-  int lo, hi;       // raw key range of the tile
+  int lo, hi;       // raw key range of the tile (positions)
   int rawA_n;       // keys used from the 128-row raw tile
   int strag;        // 1 if the 16-row raw tile exists
   int ntiles;
@@ -125,10 +128,10 @@ __device__ __forceinline__ Item make_item(const Params& p, int k) {
   it.tl = min(it.t0 + p.P - 1, p.T - 1);
   // never trust the device count beyond what the page table can address
   const int have = min(p.n_entries[it.b], p.max_pages * p.PE);
-  it.nc_last = min(visible_count(it.tl, p.block, p.W), have);
+  it.nc_last = min(visible_count(it.tl + p.q0, p.block, p.W), have);
   it.nct = (it.nc_last + kBN - 1) / kBN;
-  it.lo = max(0, it.t0 - p.W + 1);
-  it.hi = it.tl;
+  it.lo = max(0, it.t0 + p.q0 - p.W + 1);
+  it.hi = it.tl + p.q0;
   const int R = it.hi - it.lo + 1;
   it.rawA_n = min(kBN, round16(min(R, kBN)));
   it.strag = R > kBN ? 1 : 0;
@@ -307,7 +310,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             if (s == -1) return false;
             if (s >= 0)
               tma_load_3d(sRing + s * kSlotBytes, is_v ? &p.tmV16 : &p.tmK16,
-                          &bars->ring_full[s], it.b * p.T + t.key0, is_v ? it.half * 4 : 0,
+                          &bars->ring_full[s], it.b * p.Tk + t.key0 - p.kv0,
+                          is_v ? it.half * 4 : 0,
                           pol_kv);
             continue;
           }
@@ -326,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             row = page * p.PE + (t.key0 % p.PE);
             map = is_v ? &p.tmVc : &p.tmKc;
           } else {
-            row = it.b * p.T + it.hi - kBN + 1;
+            row = it.b * p.Tk + it.hi - kBN + 1 - p.kv0;
             map = is_v ? &p.tmV : &p.tmK;
           }
           tma_load_3d(sRing + s * kSlotBytes, map, &bars->ring_full[s], row, chunk, pol_kv);
@@ -342,7 +346,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         const int k = cta_item(r, G, c);
         if (k >= p.n_items) break;
         const Item it = make_item(p, k);
-        if (mine == 0 && p.err_word && visible_count(it.tl, p.block, p.W) > p.n_entries[it.b])
+        if (mine == 0 && p.err_word &&
+            visible_count(it.tl + p.q0, p.block, p.W) > p.n_entries[it.b])
           atomicOr(p.err_word, kErrCacheShort);
         for (int j = 0; j < it.ntiles && ok; ++j) {
           ok = load_tile(it, j, false);
@@ -462,9 +467,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           const uint32_t idesc = idesc_bf16_f32(kBM, ncols, true);
           const uint32_t d_tmem = tmem + kTmO + q * 128;
           for (int kk = 0; kk < t.n / 16; ++kk) {
-            // 16 keys = two 8-row swizzle atoms = 2 KB
+            // 16 keys = two 8-row swizzle atoms = 2 KB; P_hi then P_lo of the group
             const uint64_t bd = sdesc_sw128(vaddr + kk * 2048, lbo, 1024);
-            umma_ts(d_tmem, a_tmem + kk * 8, bd, idesc, (j > 0 || kk > 0));
+            umma_ts(d_tmem, a_tmem + kk * 16, bd, idesc, (j > 0 || kk > 0));
+            umma_ts(d_tmem, a_tmem + kk * 16 + 8, bd, idesc, 1u);
           }
           umma_commit(&bars->ring_empty[s]);
           ++cnt;
@@ -515,7 +521,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
       const int pos = it.t0 + row / p.hq;
       const int h = row % p.hq;
       const bool row_valid = pos < p.T;
-      const int t = min(pos, p.T - 1);
+      const int tq = min(pos, p.T - 1);  // query row
+      const int t = tq + p.q0;           // its position
       const int nc_row =
           min(visible_count(t, p.block, p.W), min(p.n_entries[it.b], p.max_pages * p.PE));
       const int lo_row = max(0, t - p.W + 1);
@@ -575,16 +582,18 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           rescale = true;
         }
         const float base = ref == -INFINITY ? 0.f : ref;
-        // P = exp2(s * scale - ref) in bf16, written over the score columns (A of P.V).
-        // The scores are re-read 32 columns at a time, the next piece's load in flight while
-        // this one is converted; piece q writes P columns [16q, 16q+16), already read.
+        // P = exp2(s * scale - ref) as a bf16 pair hi + lo (A of the two P.V products),
+        // written over the score columns. The scores are re-read 32 columns at a time, the
+        // next piece's load in flight while this one is converted; 16-key group k keeps hi
+        // in columns [16k, 16k+8) and lo in [16k+8, 16k+16), so piece q lands on its own
+        // columns, already read.
         float ps[4] = {0.f, 0.f, 0.f, 0.f};
         tmem_ld32(s_addr, cur);
         tmem_wait_ld();
 #pragma unroll 1
         for (int q = 0; q < npieces; ++q) {
           if (q + 1 < npieces) tmem_ld32(s_addr + (q + 1) * 32, nxt);
-          uint32_t pk[16];
+          uint32_t pk[32];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int c0 = q * 32 + 2 * e;
@@ -594,10 +603,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 in0 ? fast_exp2(fmaf(__uint_as_float(cur[2 * e]), p.scale_log2, -base)) : 0.f;
             const float p1 =
                 in1 ? fast_exp2(fmaf(__uint_as_float(cur[2 * e + 1]), p.scale_log2, -base)) : 0.f;
-            pk[e] = pack_bf16x2(p0, p1);
+            split_bf16x2(p0, p1, pk[(e & 8) * 2 + (e & 7)], pk[(e & 8) * 2 + 8 + (e & 7)]);
             ps[e & 3] += p0 + p1;
           }
-          tmem_st16(s_addr + q * 16, pk);
+          tmem_st32(s_addr + q * 32, pk);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) cur[e] = nxt[e];
@@ -628,10 +637,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
           // hand the row sum to the epilogue warps; LSE and the debug mask go out here
           sL[(nitem & 1) * kBM + row] = l;
           if (row_valid && it.half == 0) {
-            const int64_t orow = ((int64_t)it.b * p.T + t) * p.hq + h;
+            const int64_t orow = ((int64_t)it.b * p.T + tq) * p.hq + h;
             if (p.lse) p.lse[orow] = (m + __log2f(l)) * 0.69314718055994531f;
             if (p.dbg && h == 0) {
-              int32_t* dp = p.dbg + ((int64_t)it.b * p.T + t) * 3;
+              int32_t* dp = p.dbg + ((int64_t)it.b * p.T + tq) * 3;
               dp[0] = nc_row;
               dp[1] = lo_row;
               dp[2] = t;
@@ -751,11 +760,11 @@ bool prefill_tc_supported(const hca_desc& d, const hca_cache& c) {
 
 cudaError_t launch_prefill_tc(const hca_desc& d, const void* Q, const void* K, const void* V,
                               const hca_cache& c, void* O, float* lse, int32_t* dbg_mask,
-                              cudaStream_t s) {
+                              const PrefillRange& r, cudaStream_t s) {
   Params p;
   memset(&p, 0, sizeof(p));
   const uint64_t rowsQ = (uint64_t)d.batch * d.seqlen * d.hq;
-  const uint64_t rowsK = (uint64_t)d.batch * d.seqlen;
+  const uint64_t rowsK = (uint64_t)d.batch * r.kv_len;
   const uint64_t rowsC = (uint64_t)c.num_pages * c.page_entries;
   cudaError_t e;
   if ((e = encode_bf16_chunks(&p.tmQ, Q, rowsQ, kBM, 2)) != cudaSuccess) return e;
@@ -777,6 +786,9 @@ cudaError_t launch_prefill_tc(const hca_desc& d, const void* Q, const void* K, c
   p.err_word = c.err_word;
   p.batch = d.batch;
   p.T = d.seqlen;
+  p.q0 = r.q_pos0;
+  p.kv0 = r.kv_pos0;
+  p.Tk = r.kv_len;
   p.hq = d.hq;
   p.P = kBM / d.hq;
   p.W = d.window;
@@ -788,15 +800,10 @@ cudaError_t launch_prefill_tc(const hca_desc& d, const void* Q, const void* K, c
   p.n_items = 2 * d.batch * p.n_rt;
   p.scale_log2 = d.scale * 1.4426950408889634f;
   if (p.n_items == 0) return cudaSuccess;
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  static PerDevice<int> smem_limit_set;
+  if ((e = set_smem_limit_once(smem_limit_set, (const void*)prefill_tc_kernel, (int)kSmemBytes)) !=
+      cudaSuccess)
+    return e;
   const int grid = min(p.n_items / 2, device_sm_count());  // row tiles (pairs of items)
   prefill_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(p);
   return cudaGetLastError();

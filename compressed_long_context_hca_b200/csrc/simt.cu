@@ -36,6 +36,8 @@ struct SimtArgs {
   float* lse;
   int32_t* dbg;
   int32_t batch, T, hq, hkv, D, block, window, page_entries, max_pages, num_pages;
+  // prefill: query row t is position q0 + t; K/V row u is position kv0 + u, of Tk rows
+  int32_t q0, kv0, Tk;
   float scale;
 };
 
@@ -68,10 +70,10 @@ __device__ __forceinline__ void consume_key(RowState& st, const float (&q)[kMaxV
   st.m = mn;
 }
 
-// Shared body: one warp, one row. `raw_row(u)` maps a raw token to its row pointer offset.
+// Shared body: one warp, one row: position t of sequence b, head h, written at out_row.
 template <bool kDecode>
 __device__ void attend_row(const SimtArgs& a, int b, int t, int h, int64_t out_row,
-                           int64_t gate_off) {
+                           int64_t gate_off, int64_t dbg_row) {
   const int lane = threadIdx.x & 31;
   const int vpl = a.D / 32;
   const int g = h * a.hkv / a.hq;
@@ -108,7 +110,7 @@ __device__ void attend_row(const SimtArgs& a, int b, int t, int h, int64_t out_r
     if (kDecode)
       row = ((int64_t)b * a.window + (u % a.window)) * a.hkv + g;
     else
-      row = ((int64_t)b * a.T + u) * a.hkv + g;
+      row = ((int64_t)b * a.Tk + (u - a.kv0)) * a.hkv + g;
     consume_key(st, q, a.K + row * a.D, a.V + row * a.D, lane, vpl, a.scale);
   }
   const float inv = 1.f / st.l;
@@ -125,7 +127,7 @@ __device__ void attend_row(const SimtArgs& a, int b, int t, int h, int64_t out_r
   if (lane == 0) {
     if (a.lse) a.lse[out_row] = st.m + logf(st.l);
     if (!kDecode && a.dbg && h == 0) {
-      int32_t* dp = a.dbg + ((int64_t)b * a.T + t) * 3;
+      int32_t* dp = a.dbg + dbg_row * 3;
       dp[0] = nc;
       dp[1] = lo;
       dp[2] = t;
@@ -139,10 +141,10 @@ __global__ void __launch_bounds__(kWarps * 32) prefill_simt_kernel(SimtArgs a) {
   if (row >= rows) return;
   const int h = (int)(row % a.hq);
   const int64_t bt = row / a.hq;
-  const int t = (int)(bt % a.T);
+  const int tq = (int)(bt % a.T);  // query row; position q0 + tq
   const int b = (int)(bt / a.T);
-  const int64_t goff = (int64_t)b * a.gs0 + (int64_t)t * a.gs1 + (int64_t)h * a.gs2;
-  attend_row<false>(a, b, t, h, row, goff);
+  const int64_t goff = (int64_t)b * a.gs0 + (int64_t)tq * a.gs1 + (int64_t)h * a.gs2;
+  attend_row<false>(a, b, tq + a.q0, h, row, goff, bt);
 }
 
 __global__ void __launch_bounds__(kWarps * 32) decode_simt_kernel(SimtArgs a) {
@@ -157,7 +159,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_simt_kernel(SimtArgs a) {
     atomicOr(a.err_word, kErrCtxRange);
   const int t = min(max(ctx, 1), a.T) - 1;
   const int64_t goff = (int64_t)b * a.gs0 + (int64_t)h * a.gs2;
-  attend_row<true>(a, b, t, h, row, goff);
+  attend_row<true>(a, b, t, h, row, goff, 0);
 }
 
 SimtArgs make_args(const hca_desc& d, const hca_cache& c) {
@@ -189,8 +191,11 @@ SimtArgs make_args(const hca_desc& d, const hca_cache& c) {
 
 cudaError_t launch_prefill_simt(const hca_desc& d, const void* Q, const void* K,
                                 const void* V, const hca_cache& c, void* O, float* lse,
-                                int32_t* dbg_mask, cudaStream_t s) {
+                                int32_t* dbg_mask, const PrefillRange& r, cudaStream_t s) {
   SimtArgs a = make_args(d, c);
+  a.q0 = r.q_pos0;
+  a.kv0 = r.kv_pos0;
+  a.Tk = r.kv_len;
   a.Q = static_cast<const float*>(Q);
   a.K = static_cast<const float*>(K);
   a.V = static_cast<const float*>(V);

@@ -266,6 +266,16 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Split two floats into bf16 pairs: hi = RNE bf16 of each, lo = RNE bf16 of the remainder
+// x - hi (exact in f32). hi + lo carries ~16 significant bits (|x - hi - lo| <= 2^-17 |x|),
+// so a product A.B taken as A_hi.B + A_lo.B over bf16 B keeps that precision of A.
+__device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  hi = pack_bf16x2(a, b);
+  const float ha = __uint_as_float(hi << 16);
+  const float hb = __uint_as_float(hi & 0xffff0000u);
+  lo = pack_bf16x2(a - ha, b - hb);
+}
+
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

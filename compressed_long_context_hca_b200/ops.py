@@ -91,3 +91,57 @@ def decode(desc: B.HcaDesc, q: torch.Tensor, ctx_len: torch.Tensor, cache: B.Pag
                            workspace.numel(), _stream(stream))
     B.check(st, "hca_attn_decode")
     return O, lse
+
+
+def prefill_range(desc: B.HcaDesc, q_pos0: int, kv_pos0: int, Q: torch.Tensor,
+                  K: torch.Tensor, V: torch.Tensor, cache: B.PagedCache,
+                  O: Optional[torch.Tensor] = None, want_lse: bool = False,
+                  want_mask: bool = False, stream=None):
+    """Prefill of query positions q_pos0 .. q_pos0 + Q.shape[1] - 1 with K/V rows of
+    positions kv_pos0 .. kv_pos0 + K.shape[1] - 1 (desc.seqlen = Q.shape[1])."""
+    if O is None:
+        O = torch.empty_like(Q)
+    b, T, hq, _ = Q.shape
+    lse = torch.empty((b, T, hq), dtype=torch.float32, device=Q.device) if want_lse else None
+    dbg = torch.full((b, T, 3), -1, dtype=torch.int32, device=Q.device) if want_mask else None
+    st = B.hca_attn_prefill_range(desc, q_pos0, kv_pos0, K.shape[1], Q.data_ptr(),
+                                  K.data_ptr(), V.data_ptr(), cache.c, O.data_ptr(), _ptr(lse),
+                                  _ptr(dbg), _stream(stream))
+    B.check(st, "hca_attn_prefill_range")
+    return O, lse, dbg
+
+
+def decode_partial_buffer(desc: B.HcaDesc, n_parts: int = 1, device="cuda") -> torch.Tensor:
+    """Device memory for n_parts partial results, part k at byte k * partial_stride(desc)."""
+    return torch.empty((n_parts, partial_stride(desc)), dtype=torch.uint8, device=device)
+
+
+def partial_stride(desc: B.HcaDesc) -> int:
+    n = B.hca_decode_partial_bytes(desc)
+    return (n + 255) // 256 * 256
+
+
+def decode_partial(desc: B.HcaDesc, q: torch.Tensor, ctx_len: torch.Tensor,
+                   cache: B.PagedCache, ring_k: torch.Tensor, ring_v: torch.Tensor,
+                   entry_begin: int, entry_end: int, with_window: bool,
+                   out: torch.Tensor, workspace: Optional[torch.Tensor] = None,
+                   stream=None) -> torch.Tensor:
+    """Partial result of a decode step over entries [entry_begin, entry_end) (+ window)
+    into `out` (a row of decode_partial_buffer)."""
+    if workspace is None:
+        workspace = decode_workspace(desc, q.device)
+    st = B.hca_attn_decode_partial(desc, q.data_ptr(), ctx_len.data_ptr(), cache.c,
+                                   ring_k.data_ptr(), ring_v.data_ptr(), entry_begin,
+                                   entry_end, 1 if with_window else 0, out.data_ptr(),
+                                   workspace.data_ptr(), workspace.numel(), _stream(stream))
+    B.check(st, "hca_attn_decode_partial")
+    return out
+
+
+def decode_merge(desc: B.HcaDesc, parts: torch.Tensor, O: torch.Tensor,
+                 lse: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Decode output from the partial results in the rows of `parts` [n_parts, stride]."""
+    st = B.hca_decode_merge(desc, parts.data_ptr(), parts.shape[0], parts.stride(0),
+                            O.data_ptr(), _ptr(lse), _stream(stream))
+    B.check(st, "hca_decode_merge")
+    return O

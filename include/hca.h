@@ -149,6 +149,26 @@ int32_t hca_attn_prefill(const hca_desc* d, const void* Q, const void* K, const 
                          const hca_cache* cache, void* O, float* lse, int32_t* dbg_mask,
                          hca_stream_t stream);
 
+/* Prefill of a contiguous range of query positions: the operation of hca_attn_prefill for
+ * positions q_pos0 .. q_pos0 + d->seqlen - 1 of every sequence, with the key/value tokens
+ * given as a range too. It serves chunked prefill and the split of one long sequence's
+ * query rows over several GPUs (each GPU holds its own rows plus a window-1 token halo).
+ *   Q, O     [batch, d->seqlen, hq, head_dim]   rows of positions q_pos0 + t
+ *   lse      [batch, d->seqlen, hq];  dbg_mask [batch, d->seqlen, 3] (values are positions)
+ *   gate     rows aligned with Q (token stride over the d->seqlen rows)
+ *   K, V     [batch, kv_len, hkv, head_dim]     rows of positions kv_pos0 + u; they must
+ *            cover every window: kv_pos0 <= max(0, q_pos0 - window + 1) and
+ *            kv_pos0 + kv_len >= q_pos0 + d->seqlen
+ *   cache    compressed entries by absolute block index (entry j = block j of the sequence)
+ * hca_attn_prefill(d, ...) is hca_attn_prefill_range(d, 0, 0, d->seqlen, ...).
+ * Kernels and support as hca_attn_prefill (also needs batch * kv_len below 2^31 for bf16).
+ * Errors: HCA_EINVAL (also: negative positions, K/V rows that miss a window),
+ * HCA_EUNSUPPORTED, HCA_ECUDA. */
+int32_t hca_attn_prefill_range(const hca_desc* d, int32_t q_pos0, int32_t kv_pos0,
+                               int32_t kv_len, const void* Q, const void* K, const void* V,
+                               const hca_cache* cache, void* O, float* lse, int32_t* dbg_mask,
+                               hca_stream_t stream);
+
 /* Bytes of device workspace hca_attn_decode needs for `d` (split partials of O, max and
  * sum). 0 if d is invalid. */
 size_t hca_decode_workspace_bytes(const hca_desc* d);
@@ -172,6 +192,42 @@ int32_t hca_attn_decode(const hca_desc* d, const void* Q, const int32_t* ctx_len
                         const hca_cache* cache, const void* ring_k, const void* ring_v,
                         void* O, float* lse, void* workspace, size_t workspace_bytes,
                         hca_stream_t stream);
+
+/* Bytes of one decode partial result for d (bf16 paths; 0 if d is invalid or f32). */
+size_t hca_decode_partial_bytes(const hca_desc* d);
+
+/* One decode step over a part of every sequence's key list, for splitting a long context
+ * over several GPUs ([news 二.1]: the keys are the compressed entries and the window; one
+ * softmax over all of them is the same as a log-sum-exp combination of softmaxes over
+ * disjoint parts). The part is the visible compressed entries j with
+ * entry_begin <= j < entry_end (entry_begin a multiple of 128), plus the raw window when
+ * with_window != 0. Instead of O it writes, into `partial` (hca_decode_partial_bytes(d)
+ * bytes of device memory, 16-byte aligned), float32 data laid out as
+ *   ml [batch, hq, 2]   (m, l), padded to a multiple of 4 floats, then
+ *   o  [batch, hq, head_dim]
+ * with s_i = scale * q . k_i * log2(e) over the part's keys: l = sum_i 2^(s_i - m) and
+ * o = sum_i 2^(s_i - m) v_i for a reference m near max_i s_i. A part holding no key has
+ * l = 0 (m and o are then unspecified). No gate is applied. workspace: as for
+ * hca_attn_decode; hca_decode_workspace_bytes(d) bytes always suffice (a part that fits one
+ * split per sequence needs none).
+ * Errors: HCA_EINVAL (also: entry_begin not a multiple of 128, entry_end < entry_begin),
+ * HCA_EUNSUPPORTED (f32, or shapes the bf16 decode does not run), HCA_ENOSPACE, HCA_ECUDA. */
+int32_t hca_attn_decode_partial(const hca_desc* d, const void* Q, const int32_t* ctx_len,
+                                const hca_cache* cache, const void* ring_k, const void* ring_v,
+                                int32_t entry_begin, int32_t entry_end, int32_t with_window,
+                                void* partial, void* workspace, size_t workspace_bytes,
+                                hca_stream_t stream);
+
+/* The decode output from n_parts partial results of disjoint key parts that together make
+ * up each sequence's key set (part k at parts + k * part_stride bytes, each laid out as
+ * above): per sequence and head, M = max m_k over the parts with l_k > 0,
+ *   O = sum_k 2^(m_k - M) o_k / sum_k 2^(m_k - M) l_k,
+ * times the gate of d if attached, rounded to bf16; lse (optional, [batch, hq] float32)
+ * = (M + log2 sum_k 2^(m_k - M) l_k) ln 2. At least one part of every sequence must hold a
+ * key. part_stride: a multiple of 16, at least hca_decode_partial_bytes(d) when n_parts > 1.
+ * Errors: HCA_EINVAL, HCA_EUNSUPPORTED (f32, head_dim != 512, hq > 64), HCA_ECUDA. */
+int32_t hca_decode_merge(const hca_desc* d, const void* parts, int32_t n_parts,
+                         int64_t part_stride, void* O, float* lse, hca_stream_t stream);
 
 /* Bytes of device memory the library keeps for hca_attn_decode_noalloc (64 MiB). */
 #define HCA_DECODE_NOALLOC_SCRATCH_BYTES (64u << 20)

@@ -237,6 +237,50 @@ def hca_decode(q: np.ndarray, Kc: np.ndarray, Vc: np.ndarray,
 
 
 # ---------------------------------------------------------------------------
+# Softmax over a key set cut into parts (the split of one sequence's keys over GPUs)
+# ---------------------------------------------------------------------------
+#
+# One softmax over a union of disjoint key sets equals a combination of per-part sums
+# taken relative to each part's own maximum: with s_i the scores of part k,
+# m_k = max_i s_i, l_k = sum_i exp(s_i - m_k) and o_k = sum_i exp(s_i - m_k) v_i, the
+# output over all parts is sum_k exp(m_k - M) o_k / sum_k exp(m_k - M) l_k for any M
+# (M = max_k m_k keeps every factor <= 1), and the log-sum-exp is M + log of the
+# denominator.  This is the algebra behind splitting a decode's keys ([news 二.1]: the
+# keys are the compressed entries plus the window) over several devices.
+
+def attend_part(q: np.ndarray, keys: np.ndarray, vals: np.ndarray, scale: float):
+    """Unnormalised softmax sums of all query heads over one part of the keys.
+
+    q: [Hq, D]; keys, vals: [n, D] (one KV head).  Returns (m [Hq], l [Hq], o [Hq, Dv])
+    with natural-log m; a part with no keys gives m = -inf, l = 0, o = 0.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    keys = np.asarray(keys, dtype=np.float64)
+    vals = np.asarray(vals, dtype=np.float64)
+    Hq = q.shape[0]
+    if keys.shape[0] == 0:
+        return (np.full(Hq, -np.inf), np.zeros(Hq), np.zeros((Hq, vals.shape[-1])))
+    s = (q @ keys.T) * scale
+    m = s.max(axis=1)
+    e = np.exp(s - m[:, None])
+    return m, e.sum(axis=1), e @ vals
+
+
+def merge_parts(ms, ls, os_):
+    """Combine the per-part sums of ``attend_part`` (lists over parts) into the softmax
+    output [Hq, Dv] and its log-sum-exp [Hq]; parts with l = 0 hold no key."""
+    ms = np.stack([np.asarray(m, np.float64) for m in ms])   # [P, Hq]
+    ls = np.stack([np.asarray(x, np.float64) for x in ls])
+    os_ = np.stack([np.asarray(o, np.float64) for o in os_])  # [P, Hq, Dv]
+    live = ls > 0
+    M = np.where(live, ms, -np.inf).max(axis=0)
+    w = np.where(live, np.exp(np.where(live, ms, 0.0) - M[None, :]), 0.0)
+    L = (w * ls).sum(axis=0)
+    O = (w[:, :, None] * os_).sum(axis=0) / L[:, None]
+    return O, M + np.log(L)
+
+
+# ---------------------------------------------------------------------------
 # Backward (gradients of the prefill output)
 # ---------------------------------------------------------------------------
 #

@@ -161,3 +161,37 @@ def test_product_path_has_no_oracle_import():
                 txt = open(os.path.join(dirpath, f)).read()
                 assert not re.search(r"^\s*(import|from)\s+oracle\b", txt, re.M), f
                 assert "hca_oracle" not in txt, f
+
+
+def test_range_partial_and_merge_validation(L):
+    """The query/key range of hca_attn_prefill_range, the key part of
+    hca_attn_decode_partial and the part list of hca_decode_merge are checked before any
+    launch."""
+    d = B.make_desc(1, 256, 64, 1, 512)
+    c = _cache()
+    # K/V rows must cover every window: kv_pos0 <= max(0, q_pos0 - W + 1) ...
+    assert B.hca_attn_prefill_range(d, 1000, 1000 - 126, 500, 16, 16, 16, c, 16) == B.HCA_EINVAL
+    # ... and kv_pos0 + kv_len >= q_pos0 + seqlen
+    assert B.hca_attn_prefill_range(d, 1000, 873, 382, 16, 16, 16, c, 16) == B.HCA_EINVAL
+    assert B.hca_attn_prefill_range(d, -1, 0, 256, 16, 16, 16, c, 16) == B.HCA_EINVAL
+    # decode part: entry_begin a multiple of 128, entry_end >= entry_begin
+    dd = B.make_desc(2, 5000, 64, 1, 512)
+    assert B.hca_attn_decode_partial(dd, 16, 16, c, 16, 16, 64, 256, 1, 16, 16,
+                                     1 << 20) == B.HCA_EINVAL
+    assert B.hca_attn_decode_partial(dd, 16, 16, c, 16, 16, 256, 128, 1, 16, 16,
+                                     1 << 20) == B.HCA_EINVAL
+    assert B.hca_attn_decode_partial(dd, 16, 16, c, 16, 16, 0, 128, 1, 0, 16,
+                                     1 << 20) == B.HCA_EINVAL
+    d32 = B.make_desc(2, 5000, 4, 1, 512, dtype=B.HCA_F32)
+    assert B.hca_attn_decode_partial(d32, 16, 16, c, 16, 16, 0, 128, 1, 16, 16,
+                                     1 << 20) == B.HCA_EUNSUPPORTED
+    assert B.hca_decode_partial_bytes(d32) == 0
+    # partial size: (m, l) padded to 4 floats, then the float32 rows
+    pb = B.hca_decode_partial_bytes(dd)
+    assert pb == (((2 * 64 * 2 + 3) // 4 * 4) + 2 * 64 * 512) * 4
+    # merge: at least one part, stride >= the partial size and a multiple of 16
+    assert B.hca_decode_merge(dd, 16, 0, pb, 16) == B.HCA_EINVAL
+    assert B.hca_decode_merge(dd, 16, 2, pb - 16, 16) == B.HCA_EINVAL
+    assert B.hca_decode_merge(dd, 16, 2, pb + 8, 16) == B.HCA_EINVAL
+    assert B.hca_decode_merge(dd, 0, 2, pb, 16) == B.HCA_EINVAL
+    assert B.hca_decode_merge(d32, 16, 2, pb, 16) == B.HCA_EUNSUPPORTED

@@ -7,8 +7,8 @@ import torch
 from compressed_long_context_hca_b200 import binding as B
 from compressed_long_context_hca_b200 import inputs, ops
 from oracle import hca_oracle as orc
-from tests.gpu_helpers import (BF16_MAX, BF16_MEAN, F32_MAX, compare, compare_peaked,
-                               default_scale, ensure_built, run_prefill, to64)
+from tests.gpu_helpers import (BF16_MAX, BF16_MEAN, F32_MAX, LSE_MAX, LSE_MEAN, bf16_ulp,
+                               compare, default_scale, ensure_built, run_prefill, to64)
 
 pytestmark = pytest.mark.gpu
 
@@ -67,18 +67,30 @@ def test_decode_bf16(nseq, lo, hi, gate):
     for b in range(nseq):
         ref, rl = _oracle(x, b)
         compare(to64(O[b]), ref, BF16_MAX, BF16_MEAN, what=f"O[{b}]")
-        compare(to64(lse[b]), rl, 2e-2, what=f"lse[{b}]")
+        compare(to64(lse[b]), rl, LSE_MAX, LSE_MEAN, what=f"lse[{b}]", out_bf16=False)
     assert int(cache.err.item()) == 0
+
+
+def _sample_sequences(ctx_len, n, seed):
+    """n sequences drawn by a seeded generator, always with the longest and the shortest
+    context among them."""
+    lens = ctx_len.numpy()
+    rng = np.random.default_rng(seed)
+    pick = set(rng.choice(len(lens), size=n, replace=False).tolist())
+    pick |= {int(np.argmax(lens)), int(np.argmin(lens))}
+    return sorted(pick)
 
 
 def test_decode_batched_config_sampled():
     """128 sequences with context lengths uniform in [8192, 131072], one query each,
-    64 heads, head_dim 512, paged cache + last 128 raw tokens, N(0,1)."""
+    64 heads, head_dim 512, paged cache + last 128 raw tokens, N(0,1). 24 seeded-random
+    sequences plus the longest and the shortest against the oracle."""
     x, cache, desc = _setup(128, 8192, 131072, seed=0)
-    O, _ = _run(x, cache, desc)
-    for b in list(range(0, 128, 9)) + [127]:
-        ref, _ = _oracle(x, b)
+    O, lse = _run(x, cache, desc)
+    for b in _sample_sequences(x.ctx_len, 24, seed=5):
+        ref, rl = _oracle(x, b)
         compare(to64(O[b]), ref, BF16_MAX, BF16_MEAN, what=f"O[{b}]")
+        compare(to64(lse[b]), rl, LSE_MAX, LSE_MEAN, what=f"lse[{b}]", out_bf16=False)
 
 
 @pytest.mark.parametrize("splits", [1, 2, 3, 7, 40, 0])
@@ -118,6 +130,8 @@ def test_decode_equals_prefill_row():
         ctx = torch.tensor([t + 1], dtype=torch.int32, device=dev)
         Od, _ = ops.decode(desc, Q[:, t].contiguous(), ctx, r["cache"], rk, rv)
         torch.cuda.synchronize()
+        # two bf16-rounded results of the same float32 value may land one bf16 ulp apart
+        # (1.6e-2 for |O| in [2, 4))
         compare(to64(Od[0]), to64(r["O"][0, t]), 1.6e-2, 1e-3, what=f"t={t}")
 
 
@@ -143,19 +157,14 @@ def test_decode_ctx_len_out_of_range_is_clamped_and_flagged(dtype, hq):
 def test_decode_running_max_grows_across_chunks():
     """Keys whose scale grows tile by tile: the row max rises by far more than the lazy
     rescale threshold at every 256-key chunk of a split, so O is rescaled in tensor memory
-    between chunks. The softmax is nearly one-hot, so the error bound is the bf16 P
-    rounding bound on the spread of the visible values."""
+    between chunks. The softmax is nearly one-hot: the bf16 tolerance holds because P
+    enters P.V as a bf16 pair (hi + lo), not as one bf16 value."""
     x, cache, desc = _setup(2, 100000, 110000, seed=8, splits=1, k_ramp=1.8)
     O, lse = _run(x, cache, desc)
     for b in range(2):
         ref, rl = _oracle(x, b)
-        t = int(x.ctx_len[b]) - 1
-        nc = max(0, (t + 1 - 128) // 128)
-        ring = [x.ring_v[b, u % 128, 0] for u in range(max(0, t - 127), t + 1)]
-        vals = torch.cat([x.entries_v[b][:nc, 0], torch.stack(ring)]).double()
-        spread = (vals.max(0).values - vals.min(0).values).numpy()[None, :]
-        compare_peaked(to64(O[b]), ref, np.broadcast_to(spread, ref.shape), what=f"O[{b}]")
-        compare(to64(lse[b]), rl, 2e-2, what=f"lse[{b}]", out_bf16=False)
+        compare(to64(O[b]), ref, BF16_MAX, BF16_MEAN, what=f"O[{b}]")
+        compare(to64(lse[b]), rl, LSE_MAX, LSE_MEAN, what=f"lse[{b}]", out_bf16=False)
     assert int(cache.err.item()) == 0
 
 
@@ -168,7 +177,7 @@ def test_decode_bf16_odd_head_counts(nseq, hq, gate):
     for b in range(nseq):
         ref, rl = _oracle(x, b)
         compare(to64(O[b]), ref, BF16_MAX, BF16_MEAN, what=f"O[{b}]")
-        compare(to64(lse[b]), rl, 2e-2, what=f"lse[{b}]", out_bf16=False)
+        compare(to64(lse[b]), rl, LSE_MAX, LSE_MEAN, what=f"lse[{b}]", out_bf16=False)
     assert int(cache.err.item()) == 0
 
 
@@ -180,16 +189,16 @@ def test_decode_more_splits_than_tiles():
     for b in range(3):
         ref, rl = _oracle(x, b)
         compare(to64(O[b]), ref, BF16_MAX, BF16_MEAN, what=f"O[{b}]")
-        compare(to64(lse[b]), rl, 2e-2, what=f"lse[{b}]", out_bf16=False)
+        compare(to64(lse[b]), rl, LSE_MAX, LSE_MEAN, what=f"lse[{b}]", out_bf16=False)
 
 
 def test_decode_1m_config_four_steps_sampled():
     """Long-context decode: 16 sequences at context 1,048,576 (8191 entries + 128 raw
     tokens), 64 heads, head_dim 512, gate on, 4 decode steps; the first step's token
     completes block 8191, whose entry hca_compress writes from the ring. The entry is
-    checked against the block mean, and sequences 0, 7 and 15 against the oracle at every
-    step (the new entry stays invisible to these queries: it is visible from position
-    1,048,703 on)."""
+    checked against the block mean, and 5 seeded-random sequences (a new draw per step)
+    against the oracle at every step (the new entry stays invisible to these queries: it is
+    visible from position 1,048,703 on)."""
     dev = torch.device("cuda")
     nseq, ctx0, W, blk, steps = 16, 1048576, 128, 128, 4
     n_ent = (ctx0 - W) // blk  # 8191 visible entries
@@ -221,7 +230,7 @@ def test_decode_1m_config_four_steps_sampled():
         ops.decode(desc, q.to(dev), ctx, cache, rk, rv, O=O)
         torch.cuda.synchronize()
         assert int(cache.err.item()) == 0
-        for b in (0, 7, 15):
+        for b in sorted(np.random.default_rng(100 + s).choice(nseq, 5, replace=False)):
             ref, _ = orc.hca_decode(to64(q[b]), to64(x.entries_k[b, :n_ent]),
                                     to64(x.entries_v[b, :n_ent]), to64(rk_h[b]), to64(rv_h[b]),
                                     p + 1, blk, W, default_scale(512), gate=to64(tok.G[s][b]))
@@ -233,4 +242,4 @@ def test_decode_1m_config_four_steps_sampled():
             got = to64(cache.kc.view(-1, 1, 512)[row])
             want = orc.compress_blocks(to64(rk_h[0]), blk)[0]
             # one bf16 rounding of a float32 mean (sum of 128 bf16 values / 128): <= 1 ulp
-            compare(got, want, 0.0, what="entry 8191 (K)", out_bf16=True)
+            assert (np.abs(got - want) <= bf16_ulp(want)).all(), "entry 8191 (K)"

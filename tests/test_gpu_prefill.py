@@ -7,8 +7,8 @@ import torch
 from compressed_long_context_hca_b200 import binding as B
 from compressed_long_context_hca_b200 import inputs
 from oracle import hca_oracle as orc
-from tests.gpu_helpers import (BF16_MAX, BF16_MEAN, F32_MAX, compare, compare_peaked,
-                               default_scale, p_rounding_bound, run_prefill, to64)
+from tests.gpu_helpers import (BF16_MAX, BF16_MEAN, F32_MAX, LSE_MAX, LSE_MEAN, compare,
+                               default_scale, run_prefill, to64)
 
 pytestmark = pytest.mark.gpu
 
@@ -70,11 +70,8 @@ def test_bf16_prefill(T, hq, gate, hetero):
     r = run_prefill(x, want_lse=True, want_mask=True)
     assert int(r["cache"].err.item()) == 0
     ref, lse = _oracle(x, 0, None)
-    if hetero:
-        compare_peaked(to64(r["O"][0]), ref, p_rounding_bound(x, 0, range(T)), what="O")
-    else:
-        compare(to64(r["O"][0]), ref, BF16_MAX, BF16_MEAN, what="O")
-    compare(to64(r["lse"][0]), lse, 2e-2, 2e-3, what="lse", out_bf16=False)
+    compare(to64(r["O"][0]), ref, BF16_MAX, BF16_MEAN, what="O")
+    compare(to64(r["lse"][0]), lse, LSE_MAX, LSE_MEAN, what="lse", out_bf16=False)
     assert np.array_equal(r["dbg"][0].cpu().numpy(), orc.mask_table(T, 128, 128))
     assert int(r["cache"].err.item()) == 0
 
@@ -94,7 +91,7 @@ def test_bf16_block_window_shapes(b, T, hq, block, window, gate):
     for bi in range(b):
         ref, lse = _oracle(x, bi, None, block, window)
         compare(to64(r["O"][bi]), ref, BF16_MAX, BF16_MEAN, what=f"O[{bi}]")
-        compare(to64(r["lse"][bi]), lse, 2e-2, 2e-3, what=f"lse[{bi}]", out_bf16=False)
+        compare(to64(r["lse"][bi]), lse, LSE_MAX, LSE_MEAN, what=f"lse[{bi}]", out_bf16=False)
         assert np.array_equal(r["dbg"][bi].cpu().numpy(), orc.mask_table(T, block, window))
 
 
@@ -130,8 +127,7 @@ def test_bf16_two_sequences_many_compressed_tiles():
                       T - 2, T - 1] + rng.integers(0, T, 40).tolist()))
     for bi in range(2):
         ref, _ = _oracle(x, bi, pos)
-        compare_peaked(to64(r["O"][bi, pos]), ref, p_rounding_bound(x, bi, pos),
-                       what=f"O[{bi}]")
+        compare(to64(r["O"][bi, pos]), ref, BF16_MAX, BF16_MEAN, what=f"O[{bi}]")
 
 
 def test_bf16_full_32k_config_sampled():
@@ -211,7 +207,7 @@ def test_bf16_training_context_config_sampled():
     head, head_dim 512, block 128, window 128; every 4th 128-token block scaled x4; fused
     gate G = sigmoid(N(0,1)). Inputs drawn on the GPU (Q alone is 17 GB); sampled
     positions of both sequences against the oracle (first, block edges, the middle, the
-    end, random), with the bf16 P-rounding bound of the peaked softmax."""
+    end, random) at the bf16 tolerance."""
     T = 131072
     x = inputs.prefill_inputs(2, T, 64, 1, 512, "bf16", seed=0, hetero_blocks=True,
                               gate=True, device="cuda")
@@ -222,7 +218,6 @@ def test_bf16_training_context_config_sampled():
     for bi in range(2):
         ref, _ = orc.hca_prefill(_Rows(x.Q[bi], pos), to64(x.K[bi]), to64(x.V[bi]), 128, 128,
                                  default_scale(512), gate=_Rows(x.G[bi], pos), positions=pos)
-        compare_peaked(to64(r["O"][bi, pos]), ref, p_rounding_bound(x, bi, pos),
-                       what=f"O[{bi}]")
+        compare(to64(r["O"][bi, pos]), ref, BF16_MAX, BF16_MEAN, what=f"O[{bi}]")
     assert int(r["cache"].err.item()) == 0
     assert torch.isfinite(r["O"].float()).all()

@@ -327,3 +327,67 @@ def test_planted_mistakes_are_caught(name, monkeypatch):
         except (AssertionError, ValueError, IndexError):
             failed.append(pin.__name__)
     assert failed, f"planted mistake {name!r} passed every pin"
+
+
+# ------------------------------------------------------------------ visible pair counts
+def _pairs_by_enumeration(T, block, window):
+    """Count (t, key) pairs straight from the visibility rule, with no helper of the
+    oracle: entry j is visible to t iff (j + 1) * block <= t + 1 - window; raw token u
+    iff t - window < u <= t."""
+    c = sum(1 for t in range(T) for j in range(T) if (j + 1) * block <= t + 1 - window)
+    w = sum(1 for t in range(T) for u in range(T) if t - window < u <= t)
+    return c, w
+
+
+@pytest.mark.parametrize("T,block,window", [(10, 4, 3), (1, 4, 3), (37, 5, 7), (64, 1, 5),
+                                            (50, 8, 64), (200, 16, 40)])
+def test_visible_pairs_by_enumeration(T, block, window):
+    assert ORC.visible_pairs(T, block, window) == _pairs_by_enumeration(T, block, window)
+
+
+def test_visible_pairs_hand_table():
+    # the T=10, block=4, window=3 table: n_c = 1 at t = 6..9, windows of 1, 2, then 3 keys
+    assert ORC.visible_pairs(10, 4, 3) == (4, 1 + 2 + 3 * 8)
+
+
+def test_bench_pair_count_matches_oracle():
+    """bench.py reports FLOPs from its own closed-form pair count; it must agree with the
+    oracle's count (pinned above) at the workload shapes' block and window."""
+    import bench
+    for T in (1, 127, 128, 129, 255, 256, 1000, 4097):
+        assert bench.visible_pairs(T) == ORC.visible_pairs(T, 128, 128)
+
+
+# ------------------------------------------------------------------ softmax over key parts
+@pytest.mark.parametrize("cuts", [[0, 40], [0, 13, 40], [0, 1, 2, 39, 40], [0, 0, 20, 20, 40]])
+def test_merge_of_parts_is_one_softmax(cuts):
+    """Cutting the keys into parts (empty parts included) and merging the per-part sums
+    gives scipy's softmax over all keys applied to the values, and scipy's logsumexp."""
+    from scipy.special import softmax
+    rng = np.random.default_rng(5)
+    q = rng.standard_normal((6, 16))
+    keys = 3.0 * rng.standard_normal((40, 16))
+    vals = rng.standard_normal((40, 9))
+    scale = 0.25
+    parts = [ORC.attend_part(q, keys[a:b], vals[a:b], scale) for a, b in zip(cuts, cuts[1:])]
+    O, lse = ORC.merge_parts(*zip(*parts))
+    s = (q @ keys.T) * scale
+    assert np.allclose(O, softmax(s, axis=1) @ vals, rtol=0, atol=1e-12)
+    assert np.allclose(lse, logsumexp(s, axis=1), rtol=0, atol=1e-12)
+
+
+def test_single_part_matches_attend_position():
+    """One part holding a position's whole key set reproduces attend_position."""
+    rng = np.random.default_rng(6)
+    T, B, W, D = 300, 16, 40, 8
+    K = rng.standard_normal((T, 1, D))
+    V = rng.standard_normal((T, 1, D))
+    q = rng.standard_normal((3, D))
+    Kc, Vc = ORC.compress_blocks(K, B), ORC.compress_blocks(V, B)
+    t = 250
+    nc = ORC.visible_compressed_count(t, B, W)
+    keys = np.concatenate([Kc[:nc, 0], K[t - W + 1:t + 1, 0]])
+    vals = np.concatenate([Vc[:nc, 0], V[t - W + 1:t + 1, 0]])
+    O, lse = ORC.merge_parts(*zip(ORC.attend_part(q, keys, vals, 0.3)))
+    ref, rl = ORC.attend_position(q, Kc, Vc, K, V, t, B, W, 0.3)
+    assert np.allclose(O, ref, atol=1e-12) and np.allclose(lse, rl, atol=1e-12)
