@@ -18,8 +18,10 @@ Extra results in the same JSON line:
   roofline        prefill kernel vs the measured bf16 dense peak (and HBM)
   cpu_baseline    the float64 oracle on a bounded sample of the same workload
 
-Multi-GPU (torchrun): every rank runs its own replica of the workload (independent
-sequences, no data-path collective); the time is the max over ranks.
+Multi-GPU (torchrun): the same workloads cut over the ranks (compressed_long_context_hca_b200.
+parallel): prefill by query rows (entry all-gather + window-1 halo), batched decode by
+sequences, 1M decode by compressed-entry ranges (all-gather of (m, l, O) partials + merge).
+Total work is fixed as N grows ("scaling": "strong"); the time is the max over ranks.
 ``--impl reference`` times the float64 oracle (rank 0 only) on bounded samples.
 """
 
@@ -70,6 +72,13 @@ def visible_pairs(T: int, block: int = BLOCK, W: int = WIN):
 def prefill_flops(T: int, batch: int = 1) -> float:
     c, w = visible_pairs(T)
     return 4.0 * D * HQ * (c + w) * batch
+
+
+def prefill_flops_rows(T: int, t0: int, t1: int, batch: int = 1) -> float:
+    """Algorithmic FLOPs of query positions [t0, t1) of a T-token sequence."""
+    c1, w1 = visible_pairs(t1)
+    c0, w0 = visible_pairs(t0)
+    return 4.0 * D * HQ * ((c1 - c0) + (w1 - w0)) * batch
 
 
 # ------------------------------------------------------------------ clocks sampler
@@ -198,26 +207,32 @@ def gpu_main(args, rank, world, local_rank):
     barrier, max_over_ranks = rank_tools(world, dev)
 
     # ---------------------------------------------------------------- main: 32K prefill
+    # One sequence; with N ranks its query rows are cut into N ranges of whole blocks
+    # (parallel.prefill_rows: own-block compress, entry all-gather, halo, range prefill).
+    # Every rank draws the whole sequence from the same seed and keeps its rows.
+    from compressed_long_context_hca_b200 import parallel as P
     T = args.seqlen
+    t0, t1 = P.row_range(T, world, rank, BLOCK)
     g = torch.Generator(device=dev)
-    g.manual_seed(1000 + rank)
-    Q = torch.randn((1, T, HQ, D), generator=g, device=dev).to(torch.bfloat16)
-    K = torch.randn((1, T, 1, D), generator=g, device=dev).to(torch.bfloat16)
-    V = torch.randn((1, T, 1, D), generator=g, device=dev).to(torch.bfloat16)
-    O = torch.empty_like(Q)
-    desc = ops.desc_for_prefill(Q, K)
-    cache = B.PagedCache(1, -(-T // BLOCK), 1, D, torch.bfloat16, 128, device=dev)
+    g.manual_seed(1000)
+    Qf = torch.randn((1, T, HQ, D), generator=g, device=dev).to(torch.bfloat16)
+    Q = Qf[:, t0:t1].contiguous()
+    del Qf
+    Kf = torch.randn((1, T, 1, D), generator=g, device=dev).to(torch.bfloat16)
+    Vf = torch.randn((1, T, 1, D), generator=g, device=dev).to(torch.bfloat16)
+    K, V = Kf[:, t0:t1].contiguous(), Vf[:, t0:t1].contiguous()
+    del Kf, Vf
+    group = None
+    be = P.GpuBackend()
 
     def step():
-        ops.compress(desc, K, V, cache)
-        ops.prefill(desc, Q, K, V, cache, O=O)
+        return P.prefill_rows(be, group, Q, K, V, T, BLOCK, WIN)
 
     for _ in range(args.warmup):
-        step()
+        O = step()
     torch.cuda.synchronize()
     flops = prefill_flops(T)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
+    be.kernel_events = []
     clocks = Clocks(local_rank)
     clocks.start()
     time.sleep(0.1)
@@ -227,25 +242,29 @@ def gpu_main(args, rank, world, local_rank):
     e_end = torch.cuda.Event(enable_timing=True)
     e_start.record(stream)
     for i in range(args.steps):
-        ops.compress(desc, K, V, cache)
-        ev[i][0].record(stream)
-        ops.prefill(desc, Q, K, V, cache, O=O)
-        ev[i][1].record(stream)
+        O = step()
     e_end.record(stream)
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
     total_ms = max_over_ranks(e_start.elapsed_time(e_end))
     ms_step = total_ms / args.steps
-    prefill_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    ev = be.kernel_events
+    be.kernel_events = None
+    prefill_ms = sum(a.elapsed_time(b) for a, b in ev) / len(ev)
+    # ours per step: compress and prefill (the entry copies into the range call's cache are
+    # torch copies; at N > 1 the entry and halo gathers are NCCL kernels)
     launches = 2 * args.steps
-    assert int(cache.err.item()) == 0, "kernel raised an error bit"
+    for c in be._caches.values():
+        assert int(c.err.item()) == 0, "kernel raised an error bit"
 
-    value = world * flops / (ms_step * 1e-3) / 1e12
-    achieved = flops / (prefill_ms * 1e-3) / 1e12
+    value = flops / (ms_step * 1e-3) / 1e12
+    # this rank's share of the algorithmic work, over its kernel's time
+    my_flops = prefill_flops_rows(T, t0, t1)
+    achieved = my_flops / (prefill_ms * 1e-3) / 1e12
     bytes_prefill = (2 * Q.numel() + 2 * K.numel() + 2 * V.numel()) * 2  # Q,O + K,V
     traffic = args.traffic
-    if traffic is None and T == 32768:
+    if traffic is None and T == 32768 and world == 1:
         import hashlib
         src = os.path.join(ROOT, "compressed_long_context_hca_b200", "csrc", PREFILL_KERNEL_SRC)
         with open(src, "rb") as f:
@@ -261,13 +280,15 @@ def gpu_main(args, rank, world, local_rank):
         "warmup": args.warmup,
         "ms_per_step": round(ms_step, 4),
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "strong",
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic N(0,1) rounded to bf16, seeded",
         "config": {"workload": "HCA prefill bf16: batch 1, T=32768, 64 query heads, 1 KV head, "
                                "head_dim 512, block 128, window 128, gate off",
-                   "global_batch": world, "seq_len": T, "parallelism": f"replicas x{world}",
+                   "global_batch": 1, "seq_len": T,
+                   "parallelism": f"query rows x{world} (whole blocks; entry all-gather + "
+                                  f"window-1 halo)" if world > 1 else "single GPU",
                    "l2": "inputs larger than L2 (Q 2.1 GB), no flush"},
         "gpu_launches": launches,
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1),
@@ -282,19 +303,20 @@ def gpu_main(args, rank, world, local_rank):
     }
 
     # ---------------------------------------------------------------- e2e (host buffers)
-    # Every step copies its inputs from pinned host memory, runs compress + prefill and
-    # copies its output back. Steps are pipelined over three streams with two device
-    # buffer sets: the upload of step i + 1 and the download of step i - 1 run while step i
-    # computes (PCIe is full duplex). The timed region runs from the first upload to the
-    # last download.
+    # Every step copies this rank's input rows from pinned host memory, runs the same
+    # partitioned compress + prefill and copies its output rows back. Steps are pipelined
+    # over three streams with two device buffer sets: the upload of step i + 1 and the
+    # download of step i - 1 run while step i computes (PCIe is full duplex). The timed
+    # region runs from the first upload to the last download.
     if not args.no_e2e:
         hQ = Q.cpu().pin_memory()
         hK = K.cpu().pin_memory()
         hV = V.cpu().pin_memory()
         hO = torch.empty(O.shape, dtype=O.dtype).pin_memory()
         e2e_steps = max(2, min(args.steps, args.e2e_steps))
-        bufs = [(Q, K, V, O), (torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V),
-                               torch.empty_like(O))]
+        bufs = [(Q, K, V, torch.empty_like(Q)),
+                (torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V),
+                 torch.empty_like(Q))]
         up, comp, down = torch.cuda.Stream(), stream, torch.cuda.Stream()
         ev = lambda: torch.cuda.Event()  # noqa: E731
         inputs_free = [ev(), ev()]   # compute of the buffer set's last step is done
@@ -317,8 +339,7 @@ def gpu_main(args, rank, world, local_rank):
                 if i >= 2:
                     comp.wait_event(out_free[x])
                 with torch.cuda.stream(comp):
-                    ops.compress(desc, k_, v_, cache)
-                    ops.prefill(desc, q_, k_, v_, cache, O=o_)
+                    P.prefill_rows(be, group, q_, k_, v_, T, BLOCK, WIN, out=o_)
                 computed[x].record(comp)
                 inputs_free[x].record(comp)
                 with torch.cuda.stream(down):
@@ -338,7 +359,7 @@ def gpu_main(args, rank, world, local_rank):
         b.record(comp)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks(a.elapsed_time(b)) / e2e_steps
-        result["e2e"] = {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3),
+        result["e2e"] = {"value": round(flops / (e2e_ms * 1e-3) / 1e12, 3),
                          "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 3),
                          "h2d_bytes_per_step": (hQ.numel() + hK.numel() + hV.numel()) * 2,
                          "d2h_bytes_per_step": hO.numel() * 2,
@@ -346,7 +367,7 @@ def gpu_main(args, rank, world, local_rank):
                                     "three streams, two device buffer sets"}
         del hQ, hK, hV, hO, bufs
 
-    del Q, K, V, O, cache
+    del Q, K, V, O, be
     torch.cuda.empty_cache()
 
     # ---------------------------------------------------------------- decode workloads
@@ -409,14 +430,21 @@ def _time_loop(fn, steps, warmup, barrier, max_over_ranks, stream):
 
 
 def bench_decode_batched(args, dev, rank, world, barrier, max_over_ranks, peaks):
+    """128 sequences, context lengths U[8192, 131072]; with N ranks each serves a
+    contiguous range of the sequences (no exchange)."""
     import torch
     from compressed_long_context_hca_b200 import binding as B
     from compressed_long_context_hca_b200 import ops
-    nseq, lo, hi = 128, 8192, 131072
+    from compressed_long_context_hca_b200 import parallel as P
+    nseq_all, lo, hi = 128, 8192, 131072
     g = torch.Generator(device=dev)
-    g.manual_seed(2000 + rank)
-    ctx = torch.randint(lo, hi + 1, (nseq,), generator=g, device=dev, dtype=torch.int64)
-    ctx = ctx.to(torch.int32)
+    g.manual_seed(2000)
+    ctx_all = torch.randint(lo, hi + 1, (nseq_all,), generator=g, device=dev,
+                            dtype=torch.int64).to(torch.int32)
+    s0, s1 = P.seq_range(nseq_all, world, rank)
+    nseq = s1 - s0
+    ctx = ctx_all[s0:s1].contiguous()
+    g.manual_seed(2001 + rank)
     max_ent = (hi - WIN) // BLOCK + 1
     cache = B.PagedCache(nseq, max_ent, 1, D, torch.bfloat16, 128, device=dev)
     cache.kc.normal_(generator=g)
@@ -434,34 +462,61 @@ def bench_decode_batched(args, dev, rank, world, barrier, max_over_ranks, peaks)
     clocks.start()
     ms = _time_graph(fn, args.decode_steps, 3, barrier, max_over_ranks, stream)
     clk = clocks.stop()
-    ctx_h = ctx.cpu().tolist()
+    ctx_h = ctx_all.cpu().tolist()
     keys = sum((c - WIN) // BLOCK + min(WIN, c) for c in ctx_h)
-    byts = keys * D * 2 * 2 + nseq * HQ * D * 2 * 2
+    byts = keys * D * 2 * 2 + nseq_all * HQ * D * 2 * 2
     nsplit = B.hca_decode_workspace_bytes(desc) // (nseq * HQ * (D + 2) * 4)
-    return {"value": round(world * nseq / (ms * 1e-3), 1), "unit": "tokens/s",
+    gbs = byts / (ms * 1e-3) / 1e9 / world  # per GPU
+    return {"value": round(nseq_all / (ms * 1e-3), 1), "unit": "tokens/s",
             "ms_per_step": round(ms, 4),
             "workload": "128 sequences, context U[8192,131072], 1 query each, 64 heads, "
                         "head_dim 512, paged cache + 128-token ring, N(0,1) bf16",
+            "parallelism": f"sequences x{world}" if world > 1 else "single GPU",
+            "timing": "CUDA graph replay of one step",
             "gpu_launches_per_step": 2, "splits": int(nsplit),
-            "roofline": {"bound": "hbm", "achieved": round(byts / (ms * 1e-3) / 1e9, 1),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1),
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": round(byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                         "frac": round(gbs / peaks["hbm_gbs"], 4),
                          "bytes_per_step": byts},
             "clocks": clk}
 
 
+def _shard_cache(nseq, e0, e1, n_total, dev, g):
+    """A paged cache holding only entries [e0, min(e1, n_total)) of every sequence, at
+    their absolute entry indices (pages outside the shard map to page 0 and are never
+    read), filled with N(0,1) values."""
+    import torch
+    from compressed_long_context_hca_b200 import binding as B
+    p0 = e0 // 128
+    p1 = -(-min(e1, n_total) // 128)
+    shard_pages = max(1, p1 - p0)
+    cache = B.PagedCache(nseq, shard_pages * 128, 1, D, torch.bfloat16, 128, device=dev)
+    cache.kc.normal_(generator=g)
+    cache.vc.normal_(generator=g)
+    total_pages = -(-n_total // 128)
+    pt = torch.zeros((nseq, total_pages), dtype=torch.int32)
+    for b in range(nseq):
+        for p in range(p0, min(p1, total_pages)):
+            pt[b, p] = b * shard_pages + (p - p0)
+    cache.page_table = pt.to(dev)
+    cache.c.page_table = cache.page_table.data_ptr()
+    cache.c.max_pages = total_pages
+    return cache
+
+
 def bench_decode_1m(args, dev, rank, world, barrier, max_over_ranks, peaks):
+    """16 sequences at 1,048,576 context, 4 decode steps each with the compress of the block
+    the first step completes. With N ranks the compressed entries of every sequence are cut
+    into N ranges of whole 128-entry tiles (rank r holds only its range), the last rank also
+    holds the ring; every step all-gathers the (m, l, O) partials and merges them."""
     import torch
     from compressed_long_context_hca_b200 import binding as B
     from compressed_long_context_hca_b200 import ops
+    from compressed_long_context_hca_b200 import parallel as P
     nseq, ctx0, steps_per = 16, 1048576, 4
     n_ent = (ctx0 - WIN) // BLOCK  # 8191 visible entries at the first step
     g = torch.Generator(device=dev)
-    g.manual_seed(3000 + rank)
-    cache = B.PagedCache(nseq, n_ent + 2, 1, D, torch.bfloat16, 128, device=dev)
-    cache.kc.normal_(generator=g)
-    cache.vc.normal_(generator=g)
-    cache.n_entries.fill_(n_ent)
+    g.manual_seed(3000)
     q = torch.randn((steps_per, nseq, HQ, D), generator=g, device=dev).to(torch.bfloat16)
     G = torch.sigmoid(torch.randn((steps_per, nseq, HQ, D), generator=g, device=dev))
     G = G.to(torch.bfloat16)
@@ -469,62 +524,84 @@ def bench_decode_1m(args, dev, rank, world, barrier, max_over_ranks, peaks):
     new_v = torch.randn((steps_per, nseq, 1, 1, D), generator=g, device=dev).to(torch.bfloat16)
     rk = torch.randn((nseq, WIN, 1, D), generator=g, device=dev).to(torch.bfloat16)
     rv = torch.randn((nseq, WIN, 1, D), generator=g, device=dev).to(torch.bfloat16)
+    g.manual_seed(3001 + rank)
+    e0, e1 = P.entry_range(n_ent, world, rank) if world > 1 else (0, 1 << 30)
+    last = rank == world - 1
+    cache = _shard_cache(nseq, e0, e1, n_ent + 2, dev, g)
+    cache.n_entries.fill_(n_ent)
     ctx = [torch.full((nseq,), ctx0 + s, dtype=torch.int32, device=dev) for s in range(steps_per)]
     descs = []
     for s in range(steps_per):
         d = B.make_desc(nseq, ctx0 + steps_per, HQ, 1, D)
         ops.attach_gate(d, G[s])
         descs.append(d)
-    ws = ops.decode_workspace(descs[0], dev)
     cdesc = B.make_desc(nseq, ctx0, HQ, 1, D)  # compress of the block ending at ctx0 - 1
-    O = torch.empty((nseq, HQ, D), dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream()
+    be = P.GpuBackend()
+    group = None
 
     def four_steps():
         for s in range(steps_per):
             p = ctx0 - 1 + s                 # position of the new token
-            slot = p % WIN
-            rk[:, slot].copy_(new_k[s, :, 0])
-            rv[:, slot].copy_(new_v[s, :, 0])
-            if (p + 1) % BLOCK == 0:         # token completes block p // BLOCK
-                B.check(B.hca_compress(cdesc, rk.data_ptr(), rv.data_ptr(), WIN, p // BLOCK,
-                                       1, cache.c, torch.cuda.current_stream().cuda_stream),
-                        "hca_compress")
-            ops.decode(descs[s], q[s], ctx[s], cache, rk, rv, O=O, workspace=ws)
+            if last:
+                slot = p % WIN
+                rk[:, slot].copy_(new_k[s, :, 0])
+                rv[:, slot].copy_(new_v[s, :, 0])
+                if (p + 1) % BLOCK == 0:     # token completes block p // BLOCK
+                    B.check(B.hca_compress(cdesc, rk.data_ptr(), rv.data_ptr(), WIN,
+                                           p // BLOCK, 1, cache.c,
+                                           torch.cuda.current_stream().cuda_stream),
+                            "hca_compress")
+            P.decode_split_entries(be, group, q[s], ctx[s], cache, rk, rv, n_ent, descs[s])
 
     clocks = Clocks(dev.index)
     clocks.start()
-    ms = _time_graph(four_steps, args.decode_steps, 3, barrier, max_over_ranks, stream)
+    if world == 1:
+        ms = _time_graph(four_steps, args.decode_steps, 3, barrier, max_over_ranks, stream)
+        timing = "CUDA graph replay of the 4 steps"
+    else:
+        ms = _time_loop(four_steps, args.decode_steps, 3, barrier, max_over_ranks, stream)
+        timing = "launch loop (the steps hold NCCL all-gathers)"
     clk = clocks.stop()
+    assert int(cache.err.item()) == 0, "kernel raised an error bit"
     keys = n_ent + WIN
     byts_step = nseq * (keys * D * 2 * 2 + 3 * HQ * D * 2)
     byts = steps_per * byts_step + nseq * BLOCK * D * 2 * 2
+    gbs = byts / (ms * 1e-3) / 1e9 / world  # per GPU
     nsplit = B.hca_decode_workspace_bytes(descs[0]) // (nseq * HQ * (D + 2) * 4)
-    return {"value": round(world * nseq * steps_per / (ms * 1e-3), 1), "unit": "tokens/s",
+    launches = (4 * 2 + 1) if world == 1 else (4 * 3 + (1 if last else 0))
+    return {"value": round(nseq * steps_per / (ms * 1e-3), 1), "unit": "tokens/s",
             "ms_per_step": round(ms, 4), "ms_per_decode_step": round(ms / steps_per, 4),
             "workload": "16 sequences at context 1,048,576 (8191 entries + 128 raw), 64 heads, "
                         "head_dim 512, 4 decode steps each incl. one hca_compress, gate on",
-            "gpu_launches_per_step": 4 * 2 + 1, "splits": int(nsplit),
-            "roofline": {"bound": "hbm", "achieved": round(byts / (ms * 1e-3) / 1e9, 1),
+            "parallelism": (f"compressed entries x{world} (128-entry tiles; all-gather of "
+                            f"(m, l, O) partials + merge)") if world > 1 else "single GPU",
+            "timing": timing,
+            "gpu_launches_per_step": launches, "splits": int(nsplit),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1),
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": round(byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                         "frac": round(gbs / peaks["hbm_gbs"], 4),
                          "bytes_per_step": byts},
             "clocks": clk}
 
 
 def bench_compress_2x128k(args, dev, rank, world, barrier, max_over_ranks, peaks):
     """hca_compress alone on the K and V of the training-context prefill workload
-    (2 x 131072 tokens, 2048 entries per sequence): read K + V once, write the entries."""
+    (2 x 131072 tokens, 2048 entries per sequence): read K + V once, write the entries.
+    With N ranks each compresses the blocks of its query-row range."""
     import torch
     from compressed_long_context_hca_b200 import binding as B
     from compressed_long_context_hca_b200 import ops
+    from compressed_long_context_hca_b200 import parallel as P
     b, T = 2, 131072
+    t0, t1 = P.row_range(T, world, rank, BLOCK)
+    n = t1 - t0
     g = torch.Generator(device=dev)
     g.manual_seed(5000 + rank)
-    K = torch.randn((b, T, 1, D), generator=g, device=dev).to(torch.bfloat16)
-    V = torch.randn((b, T, 1, D), generator=g, device=dev).to(torch.bfloat16)
+    K = torch.randn((b, n, 1, D), generator=g, device=dev).to(torch.bfloat16)
+    V = torch.randn((b, n, 1, D), generator=g, device=dev).to(torch.bfloat16)
     desc = ops.desc_for_prefill(K, K)
-    cache = B.PagedCache(b, T // BLOCK, 1, D, torch.bfloat16, 128, device=dev)
+    cache = B.PagedCache(b, -(-n // BLOCK), 1, D, torch.bfloat16, 128, device=dev)
     stream = torch.cuda.current_stream()
     clocks = Clocks(dev.index)
     clocks.start()
@@ -532,54 +609,58 @@ def bench_compress_2x128k(args, dev, rank, world, barrier, max_over_ranks, peaks
                     max_over_ranks, stream)
     clk = clocks.stop()
     assert int(cache.err.item()) == 0, "kernel raised an error bit"
-    byts = (K.numel() + V.numel()) * 2 + 2 * b * (T // BLOCK) * D * 2
+    byts = 2 * b * T * D * 2 + 2 * b * (T // BLOCK) * D * 2
     gbs = byts / (ms * 1e-3) / 1e9
-    return {"value": round(world * gbs, 1), "unit": "GB/s", "ms_per_step": round(ms, 4),
+    return {"value": round(gbs, 1), "unit": "GB/s", "ms_per_step": round(ms, 4),
             "workload": "hca_compress of K and V, batch 2 x 131072 tokens, head_dim 512, bf16 "
                         "(536 MB read, larger than L2)",
+            "parallelism": f"query rows x{world}" if world > 1 else "single GPU",
             "gpu_launches_per_step": 1,
-            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
-                         "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+            "roofline": {"bound": "hbm", "achieved": round(gbs / world, 1),
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / world / peaks["hbm_gbs"], 4),
                          "bytes_per_step": byts},
             "clocks": clk}
 
 
 def bench_prefill_128k(args, dev, rank, world, barrier, max_over_ranks, peaks):
+    """2 x 131072 tokens, every 4th block x4, fused gate; with N ranks the query rows of
+    both sequences are cut into N ranges of whole blocks (parallel.prefill_rows)."""
     import torch
-    from compressed_long_context_hca_b200 import binding as B
-    from compressed_long_context_hca_b200 import ops
+    from compressed_long_context_hca_b200 import parallel as P
     b, T = 2, 131072
+    t0, t1 = P.row_range(T, world, rank, BLOCK)
+    n = t1 - t0
     g = torch.Generator(device=dev)
     g.manual_seed(4000 + rank)
-    blk = ((torch.arange(T, device=dev) // BLOCK) % 4 == 3)
+    blk = ((torch.arange(t0, t1, device=dev) // BLOCK) % 4 == 3)
 
     def draw(h):
-        x = torch.randn((b, T, h, D), generator=g, device=dev)
+        x = torch.randn((b, n, h, D), generator=g, device=dev)
         x[:, blk] *= 4.0
         return x.to(torch.bfloat16)
 
     Q, K, V = draw(HQ), draw(1), draw(1)
-    G = torch.sigmoid(torch.randn((b, T, HQ, D), generator=g, device=dev)).to(torch.bfloat16)
-    O = torch.empty_like(Q)
-    desc = ops.desc_for_prefill(Q, K)
-    ops.attach_gate(desc, G)
-    cache = B.PagedCache(b, T // BLOCK, 1, D, torch.bfloat16, 128, device=dev)
+    G = torch.sigmoid(torch.randn((b, n, HQ, D), generator=g, device=dev)).to(torch.bfloat16)
+    be = P.GpuBackend()
     stream = torch.cuda.current_stream()
 
     def step():
-        ops.compress(desc, K, V, cache)
-        ops.prefill(desc, Q, K, V, cache, O=O)
+        P.prefill_rows(be, None, Q, K, V, T, BLOCK, WIN, G=G)
 
     clocks = Clocks(dev.index)
     clocks.start()
     ms = _time_loop(step, args.steps_128k, 3, barrier, max_over_ranks, stream)
     clk = clocks.stop()
+    for c in be._caches.values():
+        assert int(c.err.item()) == 0, "kernel raised an error bit"
     flops = prefill_flops(T, b)
-    tf = world * flops / (ms * 1e-3) / 1e12
+    tf = flops / (ms * 1e-3) / 1e12
     per_gpu = tf / world
     return {"value": round(tf, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 3),
             "workload": "batch 2 x 131072, 64 heads, 1 KV head, head_dim 512, every 4th block "
                         "x4, fused gate",
+            "parallelism": f"query rows x{world}" if world > 1 else "single GPU",
             "gpu_launches_per_step": 2,
             "roofline": {"bound": "tensor", "achieved": round(per_gpu, 1),
                          "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
