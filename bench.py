@@ -12,6 +12,8 @@ Extra results in the same JSON line:
   decode_1m       16 sequences at 1,048,576 context, 4 decode steps each, gate on, with
                   the compress call of the block the first step completes: tokens/s
   prefill_128k    batch 2 x 131072, heterogeneous blocks, fused gate: TFLOP/s
+  backward_32k    the prefill backward of the 32K workload (dQ, dK, dV): TFLOP/s
+  gate_from_latent  G = sigmoid(q_lat . W_g) for 32768 tokens: TFLOP/s
   compress_2x128k hca_compress of the K and V of 2 x 131072 tokens alone: GB/s vs HBM
   e2e             the main metric with host-resident inputs and output (pinned host
                   memory, H2D + D2H inside the timed region)
@@ -382,6 +384,12 @@ def gpu_main(args, rank, world, local_rank):
         result["prefill_128k"] = bench_prefill_128k(args, dev, rank, world, barrier,
                                                     max_over_ranks, peaks)
 
+    if not args.no_backward and world == 1:
+        result["backward_32k"] = bench_backward_32k(args, dev, rank, world, barrier,
+                                                    max_over_ranks, peaks)
+        result["gate_from_latent"] = bench_gate_from_latent(args, dev, rank, world, barrier,
+                                                            max_over_ranks, peaks)
+
     # ---------------------------------------------------------------- CPU baseline
     if rank == 0 and world == 1 and not args.no_cpu:
         tf, n, wall, threads = oracle_sample_prefill(args.cpu_seconds, T)
@@ -670,6 +678,80 @@ def bench_prefill_128k(args, dev, rank, world, barrier, max_over_ranks, peaks):
             "clocks": clk}
 
 
+def bench_backward_32k(args, dev, rank, world, barrier, max_over_ranks, peaks):
+    """The prefill backward (hca_attn_prefill_backward) of the 32K workload (1 x 32768,
+    64 heads, head_dim 512, N(0,1) bf16, gate off) for an N(0,1) output gradient. The
+    forward (compress + prefill with lse) runs once, untimed; every step is one backward
+    call. Algorithmic work: 5 products per visible query-key pair (S, dP, dQ, dK, dV),
+    10 * head_dim * heads FLOPs per pair. Single GPU (the backward is not partitioned)."""
+    import torch
+    from compressed_long_context_hca_b200 import binding as B
+    from compressed_long_context_hca_b200 import ops
+    T = 32768
+    g = torch.Generator(device=dev)
+    g.manual_seed(6000 + rank)
+    Q = torch.randn((1, T, HQ, D), generator=g, device=dev).to(torch.bfloat16)
+    K = torch.randn((1, T, 1, D), generator=g, device=dev).to(torch.bfloat16)
+    V = torch.randn((1, T, 1, D), generator=g, device=dev).to(torch.bfloat16)
+    dO = torch.randn((1, T, HQ, D), generator=g, device=dev).to(torch.bfloat16)
+    desc = ops.desc_for_prefill(Q, K)
+    cache = B.PagedCache(1, T // BLOCK, 1, D, torch.bfloat16, 128, device=dev)
+    ops.compress(desc, K, V, cache)
+    _, lse, _ = ops.prefill(desc, Q, K, V, cache, want_lse=True)
+    n = B.hca_prefill_backward_workspace_bytes(desc)
+    ws = torch.empty(n, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    fn = lambda: ops.prefill_backward(desc, Q, K, V, cache, lse, dO, workspace=ws)  # noqa: E731
+    clocks = Clocks(dev.index)
+    clocks.start()
+    ms = _time_loop(fn, args.steps_bwd, 1, barrier, max_over_ranks, stream)
+    clk = clocks.stop()
+    assert int(cache.err.item()) == 0, "kernel raised an error bit"
+    c, w = visible_pairs(T)
+    flops = 10.0 * D * HQ * (c + w)
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"value": round(tf, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 3),
+            "workload": "prefill backward, batch 1 x 32768, 64 heads, 1 KV head, head_dim 512, "
+                        "N(0,1) bf16, gate off; dQ, dK, dV",
+            "workspace_bytes": n,
+            "roofline": {"bound": "tensor", "achieved": round(tf, 1),
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": round(tf / peaks["bf16_tflops"], 4),
+                         "peak_source": "measured bf16 dense burst",
+                         "note": "algorithmic FLOPs (5 products per visible pair); the "
+                                 "kernels run the window as 256-key bands and every P / dS "
+                                 "product twice (bf16 hi + lo)"},
+            "clocks": clk}
+
+
+def bench_gate_from_latent(args, dev, rank, world, barrier, max_over_ranks, peaks):
+    """The gate from the query latent for the 32K workload: G [32768, 64, 512] =
+    sigmoid(q_lat [32768, 1024] . W_g [1024, 32768]) (hca_gate_from_latent, one GEMM)."""
+    import torch
+    from compressed_long_context_hca_b200 import ops
+    rows, L = 32768, 1024
+    g = torch.Generator(device=dev)
+    g.manual_seed(7000 + rank)
+    q = torch.randn((rows, L), generator=g, device=dev).to(torch.bfloat16)
+    W = (torch.randn((L, HQ * D), generator=g, device=dev) / 32).to(torch.bfloat16)
+    G = torch.empty((rows, HQ, D), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+    clocks = Clocks(dev.index)
+    clocks.start()
+    ms = _time_loop(lambda: ops.gate_from_latent(q, W, HQ, D, G=G), args.decode_steps, 3,
+                    barrier, max_over_ranks, stream)
+    clk = clocks.stop()
+    tf = 2.0 * rows * L * HQ * D / (ms * 1e-3) / 1e12
+    return {"value": round(tf, 1), "unit": "TFLOP/s", "ms_per_step": round(ms, 4),
+            "workload": "G = sigmoid(q_lat . W_g): 32768 x 1024 latent, 1024 x 32768 weights, "
+                        "bf16 gate [32768, 64, 512] out",
+            "roofline": {"bound": "tensor", "achieved": round(tf, 1),
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": round(tf / peaks["bf16_tflops"], 4),
+                         "peak_source": "measured bf16 dense burst"},
+            "clocks": clk}
+
+
 # ------------------------------------------------------------------ reference arm
 def reference_main(args, rank, world):
     if rank != 0:
@@ -763,6 +845,8 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=50)
     ap.add_argument("--steps-128k", type=int, default=10)
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--steps-bwd", type=int, default=5)
+    ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-seconds", type=float, default=10.0)
     ap.add_argument("--traffic", type=float, default=None,

@@ -34,7 +34,9 @@ ABI_VERSION = 1
 EXPORTED = ("hca_abi_version", "hca_status_string", "hca_set_gate", "hca_compress",
             "hca_attn_prefill", "hca_attn_prefill_range", "hca_decode_workspace_bytes",
             "hca_attn_decode", "hca_decode_partial_bytes", "hca_attn_decode_partial",
-            "hca_decode_merge", "hca_attn_decode_noalloc")
+            "hca_decode_merge", "hca_prefill_backward_workspace_bytes",
+            "hca_attn_prefill_backward", "hca_gate_from_latent", "hca_vha_gate",
+            "hca_attn_decode_noalloc")
 HCA_DECODE_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
@@ -95,6 +97,19 @@ def lib() -> ctypes.CDLL:
     L.hca_decode_merge.restype = c_int32
     L.hca_decode_merge.argtypes = [POINTER(HcaDesc), c_void_p, c_int32, c_int64, c_void_p,
                                    c_void_p, c_void_p]
+    L.hca_prefill_backward_workspace_bytes.restype = c_size_t
+    L.hca_prefill_backward_workspace_bytes.argtypes = [POINTER(HcaDesc)]
+    L.hca_attn_prefill_backward.restype = c_int32
+    L.hca_attn_prefill_backward.argtypes = [POINTER(HcaDesc), c_void_p, c_void_p, c_void_p,
+                                            POINTER(HcaCache), c_void_p, c_void_p, c_void_p,
+                                            c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                                            c_void_p]
+    L.hca_gate_from_latent.restype = c_int32
+    L.hca_gate_from_latent.argtypes = [POINTER(HcaDesc), c_void_p, c_void_p, c_int32, c_void_p,
+                                       c_void_p]
+    L.hca_vha_gate.restype = c_int32
+    L.hca_vha_gate.argtypes = [POINTER(HcaDesc), c_void_p, c_void_p, c_void_p, c_int32,
+                               c_void_p, c_void_p]
     L.hca_decode_workspace_bytes.restype = c_size_t
     L.hca_decode_workspace_bytes.argtypes = [POINTER(HcaDesc)]
     L.hca_attn_decode.restype = c_int32
@@ -175,6 +190,32 @@ def hca_decode_merge(desc: HcaDesc, parts: int, n_parts: int, part_stride: int, 
                      lse: int = 0, stream: int = 0) -> int:
     return lib().hca_decode_merge(ctypes.byref(desc), parts or None, n_parts, part_stride,
                                   O or None, lse or None, stream or None)
+
+
+def hca_prefill_backward_workspace_bytes(desc: HcaDesc) -> int:
+    return lib().hca_prefill_backward_workspace_bytes(ctypes.byref(desc))
+
+
+def hca_attn_prefill_backward(desc: HcaDesc, Q: int, K: int, V: int, cache: HcaCache,
+                              lse: int, dO: int, dQ: int, dK: int, dV: int, dG: int,
+                              workspace: int, workspace_bytes: int, stream: int = 0) -> int:
+    return lib().hca_attn_prefill_backward(ctypes.byref(desc), Q or None, K or None, V or None,
+                                           ctypes.byref(cache), lse or None,
+                                           dO or None, dQ or None, dK or None, dV or None,
+                                           dG or None, workspace or None, workspace_bytes,
+                                           stream or None)
+
+
+def hca_gate_from_latent(desc: HcaDesc, q_lat: int, W_g: int, latent: int, G: int,
+                         stream: int = 0) -> int:
+    return lib().hca_gate_from_latent(ctypes.byref(desc), q_lat or None, W_g or None, latent,
+                                      G or None, stream or None)
+
+
+def hca_vha_gate(desc: HcaDesc, O: int, A: int, B: int, rank: int, out: int,
+                 stream: int = 0) -> int:
+    return lib().hca_vha_gate(ctypes.byref(desc), O or None, A or None, B or None, rank,
+                              out or None, stream or None)
 
 
 def hca_decode_workspace_bytes(desc: HcaDesc) -> int:

@@ -10,6 +10,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include "gemm_tc.h"
 #include "hca_internal.h"
 #include "tmap.h"
 
@@ -67,6 +68,21 @@ cudaError_t encode_bf16_rows(CUtensorMap* map, const void* base, uint64_t rows, 
   if (rows == 0) rows = 1;  // a map needs a non-empty extent; nothing reads past the data
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                           uint64_t ld, uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  if (rows == 0) rows = 1;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * 2};
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
@@ -209,6 +225,80 @@ int32_t hca_attn_prefill(const hca_desc* d, const void* Q, const void* K, const 
                          hca_stream_t stream) {
   if (!d) return HCA_EINVAL;
   return hca_attn_prefill_range(d, 0, 0, d->seqlen, Q, K, V, cache, O, lse, dbg_mask, stream);
+}
+
+size_t hca_prefill_backward_workspace_bytes(const hca_desc* d) {
+  if (check_desc(d) != HCA_OK) return 0;
+  return backward_tc_supported(*d) ? backward_tc_workspace_bytes(*d)
+                                   : backward_simt_workspace_bytes(*d);
+}
+
+int32_t hca_attn_prefill_backward(const hca_desc* d, const void* Q, const void* K,
+                                  const void* V, const hca_cache* cache,
+                                  const float* lse, const void* dO, void* dQ, void* dK,
+                                  void* dV, void* dG, void* workspace, size_t workspace_bytes,
+                                  hca_stream_t stream) {
+  int32_t st = check_desc(d);
+  if (st != HCA_OK) return st;
+  if ((st = check_cache(cache)) != HCA_OK) return st;
+  if (d->batch == 0 || d->seqlen == 0) return HCA_OK;
+  if (!Q || !K || !V || !lse || !dO || !dQ || !dK || !dV) return HCA_EINVAL;
+  if ((d->gate != nullptr) != (dG != nullptr)) return HCA_EINVAL;
+  if (d->gate && (d->gate_strides[0] < 0 || d->gate_strides[1] < 0 || d->gate_strides[2] < 0))
+    return HCA_EINVAL;
+  if (d->head_dim % 32 != 0 || d->head_dim > 512) return HCA_EUNSUPPORTED;
+  if ((int64_t)d->batch * d->seqlen * d->hq >= (int64_t(1) << 31)) return HCA_EUNSUPPORTED;
+  const bool tc = backward_tc_supported(*d);
+  const size_t need = tc ? backward_tc_workspace_bytes(*d) : backward_simt_workspace_bytes(*d);
+  if (!workspace || workspace_bytes < need) return HCA_ENOSPACE;
+  if (!aligned16(workspace)) return HCA_EINVAL;
+  const BackwardTensors x{Q, K, V, lse, dO, dQ, dK, dV, dG};
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (tc) {
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(dO) || !aligned16(dQ) ||
+        !aligned16(dK) || !aligned16(dV) || (dG && !aligned16(dG)) ||
+        !aligned16(cache->kc_pool) || !aligned16(cache->vc_pool))
+      return HCA_EINVAL;
+    if (d->gate && (reinterpret_cast<uintptr_t>(d->gate) % 4 || d->gate_strides[2] % 2 ||
+                    d->gate_strides[1] % 2 || d->gate_strides[0] % 2))
+      return HCA_EINVAL;
+    return from_cuda(launch_backward_tc(*d, x, *cache, workspace, s));
+  }
+  return from_cuda(launch_backward_simt(*d, x, *cache, workspace, s));
+}
+
+int32_t hca_gate_from_latent(const hca_desc* d, const void* q_lat, const void* W_g,
+                             int32_t latent, void* G, hca_stream_t stream) {
+  int32_t st = check_desc(d);
+  if (st != HCA_OK) return st;
+  if (latent < 1) return HCA_EINVAL;
+  const int64_t rows = (int64_t)d->batch * d->seqlen;
+  if (rows == 0) return HCA_OK;
+  if (!q_lat || !W_g || !G) return HCA_EINVAL;
+  const int64_t n = (int64_t)d->hq * d->head_dim;
+  if (d->dtype != HCA_BF16) return HCA_EUNSUPPORTED;
+  if (latent % 8 != 0 || n % 8 != 0 || rows >= (int64_t(1) << 31) || n >= (int64_t(1) << 31))
+    return HCA_EUNSUPPORTED;
+  if (!aligned16(q_lat) || !aligned16(W_g) || !aligned16(G)) return HCA_EINVAL;
+  // G [rows, n] = sigmoid(q_lat [rows, latent] . W_g [latent, n]): A K-major, B MN-major
+  const GemmOperand A{q_lat, rows, latent, latent, false, 0, 0};
+  const GemmOperand B{W_g, latent, n, n, true, 0, 0};
+  GemmOutput C{static_cast<float*>(G), n, 0, 0, (int32_t)rows, 1, false, true};
+  return from_cuda(gemm_tc(A, B, C, (int)rows, (int)n, latent, 1, 1.f, 0.f, nullptr,
+                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int32_t hca_vha_gate(const hca_desc* d, const void* O, const float* A, const float* B,
+                     int32_t rank, void* out, hca_stream_t stream) {
+  int32_t st = check_desc(d);
+  if (st != HCA_OK) return st;
+  if (rank < 0 || rank > 16 || d->hq > 128) return HCA_EUNSUPPORTED;
+  if ((int64_t)d->batch * d->seqlen == 0) return HCA_OK;
+  if (!O || !out || (rank > 0 && (!A || !B))) return HCA_EINVAL;
+  if (d->head_dim % 4 != 0 || d->head_dim > 512) return HCA_EUNSUPPORTED;
+  if (d->gate && (d->gate_strides[0] < 0 || d->gate_strides[1] < 0 || d->gate_strides[2] < 0))
+    return HCA_EINVAL;
+  return from_cuda(launch_vha_gate(*d, O, A, B, rank, out, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 size_t hca_decode_workspace_bytes(const hca_desc* d) {

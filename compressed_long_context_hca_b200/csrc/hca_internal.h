@@ -67,6 +67,34 @@ cudaError_t launch_prefill_pair(const hca_desc& d, const void* Q, const void* K,
                                 const hca_cache& c, void* O, float* lse, int32_t* dbg_mask,
                                 const PrefillRange& r, cudaStream_t s);
 
+// Tensors of a prefill backward call (device pointers; dtype of the descriptor, lse f32).
+struct BackwardTensors {
+  const void* Q;
+  const void* K;
+  const void* V;
+  const float* lse;
+  const void* dO;
+  void* dQ;
+  void* dK;
+  void* dV;
+  void* dG;
+};
+
+// CUDA cores, float32 arithmetic, float32 or bf16 tensors (head_dim % 32 == 0, <= 512)
+size_t backward_simt_workspace_bytes(const hca_desc& d);
+cudaError_t launch_backward_simt(const hca_desc& d, const BackwardTensors& x, const hca_cache& c,
+                                 void* ws, cudaStream_t s);
+
+// bf16 on tcgen05 GEMMs (head_dim 512, hkv 1, window <= 128)
+bool backward_tc_supported(const hca_desc& d);
+size_t backward_tc_workspace_bytes(const hca_desc& d);
+cudaError_t launch_backward_tc(const hca_desc& d, const BackwardTensors& x, const hca_cache& c,
+                               void* ws, cudaStream_t s);
+
+// VHA mixing + gate over [batch * seqlen positions, hq, head_dim] (vha.cu)
+cudaError_t launch_vha_gate(const hca_desc& d, const void* O, const float* A, const float* B,
+                            int rank, void* out, cudaStream_t s);
+
 // The key part of a decode call: visible compressed entries [e0, e1) (e0 a multiple of 128)
 // and the raw window if with_ring. out_partial == nullptr: the call writes the final output;
 // else it writes an unnormalised float32 partial result there (decode_partial_bytes).

@@ -20,4 +20,10 @@ cudaError_t encode_bf16_rows(CUtensorMap* map, const void* base, uint64_t rows, 
 cudaError_t encode_bf16_chunks(CUtensorMap* map, const void* base, uint64_t rows,
                                uint32_t box_rows, uint32_t box_chunks);
 
+// 2-D bf16 map over a row-major [rows, cols] array with a row stride of ld elements
+// (ld * 2 a multiple of 16), 128-byte swizzle, box [box_rows, box_cols] (box_cols * 2 must
+// be 128). Loads that fall outside the array are zero-filled.
+cudaError_t encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                           uint64_t ld, uint32_t box_cols, uint32_t box_rows);
+
 }  // namespace hca

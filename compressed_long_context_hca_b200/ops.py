@@ -145,3 +145,53 @@ def decode_merge(desc: B.HcaDesc, parts: torch.Tensor, O: torch.Tensor,
                             O.data_ptr(), _ptr(lse), _stream(stream))
     B.check(st, "hca_decode_merge")
     return O
+
+
+def prefill_backward(desc: B.HcaDesc, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
+                     cache: B.PagedCache, lse: torch.Tensor, dO: torch.Tensor,
+                     workspace: Optional[torch.Tensor] = None, stream=None):
+    """Gradients (dQ, dK, dV, dG or None) of hca_attn_prefill for the output gradient dO."""
+    dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
+    dG = torch.empty_like(Q) if desc.gate else None
+    if workspace is None:
+        n = B.hca_prefill_backward_workspace_bytes(desc)
+        workspace = torch.empty(max(16, n), dtype=torch.uint8, device=Q.device)
+    st = B.hca_attn_prefill_backward(desc, Q.data_ptr(), K.data_ptr(), V.data_ptr(), cache.c,
+                                     lse.data_ptr(), dO.data_ptr(), dQ.data_ptr(),
+                                     dK.data_ptr(), dV.data_ptr(), _ptr(dG),
+                                     workspace.data_ptr(), workspace.numel(), _stream(stream))
+    B.check(st, "hca_attn_prefill_backward")
+    return dQ, dK, dV, dG
+
+
+def gate_from_latent(q_lat: torch.Tensor, W_g: torch.Tensor, hq: int, head_dim: int,
+                     G: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """G [rows, hq, head_dim] = sigmoid(q_lat [rows, latent] . W_g [latent, hq * head_dim])."""
+    rows, latent = q_lat.shape
+    if G is None:
+        G = torch.empty((rows, hq, head_dim), dtype=q_lat.dtype, device=q_lat.device)
+    desc = B.make_desc(1, rows, hq, 1, head_dim, dtype=B.dtype_code(q_lat))
+    st = B.hca_gate_from_latent(desc, q_lat.data_ptr(), W_g.data_ptr(), latent, G.data_ptr(),
+                                _stream(stream))
+    B.check(st, "hca_gate_from_latent")
+    return G
+
+
+def vha_gate(O: torch.Tensor, A: Optional[torch.Tensor], Bm: Optional[torch.Tensor],
+             G: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+             stream=None) -> torch.Tensor:
+    """(O + A (B^T O) across heads) * G for O [b, T, hq, D] (or [nseq, hq, D])."""
+    O4 = O if O.dim() == 4 else O.unsqueeze(1)
+    b, T, hq, D = O4.shape
+    desc = B.make_desc(b, T, hq, 1, D, dtype=B.dtype_code(O))
+    if G is not None:
+        G4 = G if G.dim() == 4 else G.unsqueeze(1)
+        st = G4.stride()
+        B.check(B.hca_set_gate(desc, G4.data_ptr(), (st[0], st[1], st[2])), "hca_set_gate")
+    if out is None:
+        out = torch.empty_like(O)
+    rank = 0 if A is None else A.shape[1]
+    st = B.hca_vha_gate(desc, O.data_ptr(), _ptr(A), _ptr(Bm), rank, out.data_ptr(),
+                        _stream(stream))
+    B.check(st, "hca_vha_gate")
+    return out

@@ -169,6 +169,69 @@ int32_t hca_attn_prefill_range(const hca_desc* d, int32_t q_pos0, int32_t kv_pos
                                const hca_cache* cache, void* O, float* lse, int32_t* dbg_mask,
                                hca_stream_t stream);
 
+/* Bytes of device workspace hca_attn_prefill_backward needs for d (0 if d is invalid). */
+size_t hca_prefill_backward_workspace_bytes(const hca_desc* d);
+
+/* Gradients of hca_attn_prefill for the training context of the pages ([analysis infra 3]:
+ * the communeify.com page, section "33.5T 預訓練資料工程與分散式訓練基礎設施" item 3, quotes
+ * the backward kernel of this operator; the pages print no formulas, so these are the exact
+ * derivatives of the forward definition above). Given the forward's inputs, its lse and
+ * the output gradient dO, per row (b, t, h) with visible keys k_i and values v_i,
+ * p_i = exp(scale q.k_i - lse) and the ungated output O_pre = sum_i p_i v_i:
+ *   dG  = dO * O_pre                          (the gate's gradient; gate attached only)
+ *   dO' = dO * G (dO without a gate),  Delta = dO' . O_pre,  dp_i = dO' . v_i
+ *   ds_i = p_i (dp_i - Delta),  dq = scale sum_i ds_i k_i
+ *   dk_i += scale ds_i q,  dv_i += p_i dO'     (summed over every row that sees key i)
+ * and each token of block j receives 1/count_j of the gradient of entry j (the entry is the
+ * mean of its block's count_j tokens), on top of its window gradient.
+ *   Q, dO, dQ, dG  [batch, seqlen, hq, head_dim];  K, V, dK, dV [batch, seqlen, hkv, head_dim]
+ *   lse [batch, seqlen, hq] float32 (natural log, as hca_attn_prefill writes it)
+ *   cache: the compressed entries the forward used (hca_compress of K, V)
+ *   dG must be non-NULL exactly when d->gate is attached (G > 0, as a sigmoid is).
+ * O_pre is recomputed in float32 from Q, K, V and lse rather than read from the stored
+ * output: a bf16 output carries 2^-9 of |O| of rounding, which Delta (a sum over head_dim
+ * of dO' * O_pre) and dG would inherit.
+ * dQ, dK, dV, dG are written (not accumulated), in d->dtype. workspace: device memory of
+ * hca_prefill_backward_workspace_bytes(d) bytes, 16-byte aligned, contents ignored.
+ * Kernels: bf16 with head_dim 512, hkv 1, window <= 128, hq <= 128 -> the contractions on
+ * tcgen05 tensor cores (groups of 1024 query positions: the scores, dP, P and dS of a group
+ * are held in the workspace, P, dS and dO * G enter the products as bf16 pairs hi + lo);
+ * otherwise (float32, other shapes) CUDA cores with float32 arithmetic (head_dim % 32 == 0,
+ * head_dim <= 512). batch * seqlen * hq below 2^31. The bf16 path's 16-byte alignment rule
+ * applies to its tensors.
+ * Errors: HCA_EINVAL, HCA_EUNSUPPORTED, HCA_ENOSPACE, HCA_ECUDA. */
+int32_t hca_attn_prefill_backward(const hca_desc* d, const void* Q, const void* K,
+                                  const void* V, const hca_cache* cache,
+                                  const float* lse, const void* dO, void* dQ, void* dK,
+                                  void* dV, void* dG, void* workspace, size_t workspace_bytes,
+                                  hca_stream_t stream);
+
+/* The output gate from the attention layer's low-rank query latent ([news 二.1] and
+ * [analysis 1], "Low-Rank Gated Attention": the gate is computed from the query latent, a
+ * quarter of the hidden width, instead of the hidden state). Reading: one gate value per
+ * output element,
+ *   G[r, h, e] = sigmoid(sum_i q_lat[r, i] W_g[i, h * head_dim + e]),
+ * for the d->batch * d->seqlen rows r of q_lat [rows, latent] (bf16) and W_g
+ * [latent, hq * head_dim] (bf16); G [rows, hq, head_dim] bf16 -- the layout hca_set_gate
+ * expects. Runs as one tcgen05 GEMM with the sigmoid in its epilogue.
+ * Errors: HCA_EINVAL, HCA_EUNSUPPORTED (f32; latent or hq * head_dim not a multiple of 8),
+ * HCA_ECUDA. */
+int32_t hca_gate_from_latent(const hca_desc* d, const void* q_lat, const void* W_g,
+                             int32_t latent, void* G, hca_stream_t stream);
+
+/* The layer's attention output with Virtual Head Attention ([news 二.1] and [analysis 1],
+ * "Virtual Head Attention": after the attention computation, a light cross-head low-rank
+ * mixing with an identity skip), then the gate of d if attached. Reading, per position p
+ * (d->batch * d->seqlen positions) and column e:
+ *   z_r = sum_g B[g, r] O[p, g, e],   out[p, h, e] = (O[p, h, e] + sum_r A[h, r] z_r) * G[p, h, e]
+ *   O, out  [batch, seqlen, hq, head_dim] in d->dtype: O the heads' ungated attention outputs
+ *           (hca_attn_prefill / hca_attn_decode run with no gate attached)
+ *   A, B    [hq, rank] float32 device arrays, 0 <= rank <= 16 (rank 0: the gate alone)
+ * Errors: HCA_EINVAL, HCA_EUNSUPPORTED (rank > 16, hq > 128, head_dim % 4 or > 512),
+ * HCA_ECUDA. */
+int32_t hca_vha_gate(const hca_desc* d, const void* O, const float* A, const float* B,
+                     int32_t rank, void* out, hca_stream_t stream);
+
 /* Bytes of device workspace hca_attn_decode needs for `d` (split partials of O, max and
  * sum). 0 if d is invalid. */
 size_t hca_decode_workspace_bytes(const hca_desc* d);

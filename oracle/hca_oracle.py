@@ -391,6 +391,59 @@ def hca_prefill_backward(Q: np.ndarray, K: np.ndarray, V: np.ndarray, dO: np.nda
     return dQ, dK, dV, dG
 
 
+# ---------------------------------------------------------------------------
+# Gate from the low-rank query latent, and the cross-head mixing (VHA)
+# ---------------------------------------------------------------------------
+#
+# [news 二.1], "Low-Rank Gated Attention" paragraph, and [analysis 1], its second bullet:
+# the output gate is computed from the attention layer's own low-rank query latent, a
+# quarter of the hidden width (4096 / 4 = 1024), instead of from the hidden state; the
+# attention output is multiplied by it.  Reading: G = sigmoid(q_lat . W_g), one gate value
+# per output element, W_g of shape [latent, heads * head_dim].
+# Same paragraphs, "Virtual Head Attention": after the attention computation a light
+# cross-head low-rank mixing with an identity skip lets the heads exchange information.
+# Reading: per position and output column d, the vector of the heads' outputs o_.d becomes
+# o_.d + A (B^T o_.d), A and B of shape [heads, rank]; then the gate multiplies.
+
+def sigmoid(x: np.ndarray) -> np.ndarray:
+    """1 / (1 + exp(-x)), float64 (the branch keeps exp from overflowing)."""
+    x = np.asarray(x, dtype=np.float64)
+    out = np.empty_like(x)
+    pos = x >= 0
+    out[pos] = 1.0 / (1.0 + np.exp(-x[pos]))
+    e = np.exp(x[~pos])
+    out[~pos] = e / (1.0 + e)
+    return out
+
+
+def gate_from_latent(q_lat: np.ndarray, W_g: np.ndarray, hq: int, D: int) -> np.ndarray:
+    """G = sigmoid(q_lat . W_g) as [T, hq, D]; q_lat [T, L], W_g [L, hq * D]."""
+    z = np.asarray(q_lat, np.float64) @ np.asarray(W_g, np.float64)
+    return sigmoid(z).reshape(z.shape[0], hq, D)
+
+
+def vha_mix(O: np.ndarray, A: np.ndarray, B: np.ndarray) -> np.ndarray:
+    """Cross-head low-rank mixing with an identity skip: O [T, hq, D], A and B [hq, r];
+    out[t, h] = O[t, h] + sum_r A[h, r] sum_g B[g, r] O[t, g]."""
+    O = np.asarray(O, np.float64)
+    A = np.asarray(A, np.float64)
+    B = np.asarray(B, np.float64)
+    Z = np.einsum("gr,tgd->trd", B, O)          # the rank-r "virtual heads"
+    return O + np.einsum("hr,trd->thd", A, Z)
+
+
+def attention_output(O_attn: np.ndarray, G: Optional[np.ndarray] = None,
+                     A: Optional[np.ndarray] = None, B: Optional[np.ndarray] = None):
+    """The layer's attention output from the heads' attention outputs O_attn [T, hq, D]:
+    the VHA mixing (if A, B are given), then the gate (if G is given)."""
+    out = np.asarray(O_attn, np.float64)
+    if A is not None:
+        out = vha_mix(out, A, B)
+    if G is not None:
+        out = out * np.asarray(G, np.float64)
+    return out
+
+
 def visible_pairs(T: int, block: int, window: int) -> Tuple[int, int]:
     """(compressed, raw) query-key pairs per head for a sequence of T tokens."""
     c = 0

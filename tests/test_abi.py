@@ -195,3 +195,24 @@ def test_range_partial_and_merge_validation(L):
     assert B.hca_decode_merge(dd, 16, 2, pb + 8, 16) == B.HCA_EINVAL
     assert B.hca_decode_merge(dd, 0, 2, pb, 16) == B.HCA_EINVAL
     assert B.hca_decode_merge(d32, 16, 2, pb, 16) == B.HCA_EUNSUPPORTED
+
+
+def test_backward_validation(L):
+    d32 = B.make_desc(1, 256, 4, 1, 512, dtype=B.HCA_F32)
+    # CUDA-core path: Delta (padded to 4 floats) + dKc and dVc of 2 entries
+    assert B.hca_prefill_backward_workspace_bytes(d32) == ((256 * 4 + 3) // 4 * 4 +
+                                                           2 * 2 * 512) * 4
+    d = B.make_desc(1, 256, 64, 1, 512)
+    c = _cache()
+    ws = B.hca_prefill_backward_workspace_bytes(d)
+    # tensor-core path: at least the float32 window rows of dK, dV and the group's dQ rows
+    assert ws >= (2 * 256 * 512 + 256 * 64 * 512) * 4
+    q, k, v, lse, do, dq, dk, dv = [16] * 8
+    call = lambda desc, dg, w, wb: B.hca_attn_prefill_backward(  # noqa: E731
+        desc, q, k, v, c, lse, do, dq, dk, dv, dg, w, wb)
+    assert B.hca_attn_prefill_backward(d, q, k, v, c, 0, do, dq, dk, dv, 0, 16,
+                                       ws) == B.HCA_EINVAL          # no lse
+    assert call(d, 16, 16, ws) == B.HCA_EINVAL                      # dG without a gate
+    assert call(d, 0, 16, ws - 16) == B.HCA_ENOSPACE
+    assert call(d, 0, 8, ws) == B.HCA_EINVAL                        # misaligned workspace
+    assert call(B.make_desc(1, 256, 64, 1, 520), 0, 16, 1 << 30) == B.HCA_EUNSUPPORTED

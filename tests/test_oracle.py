@@ -391,3 +391,63 @@ def test_single_part_matches_attend_position():
     O, lse = ORC.merge_parts(*zip(ORC.attend_part(q, keys, vals, 0.3)))
     ref, rl = ORC.attend_position(q, Kc, Vc, K, V, t, B, W, 0.3)
     assert np.allclose(O, ref, atol=1e-12) and np.allclose(lse, rl, atol=1e-12)
+
+
+# ------------------------------------------------------------------ gate from latent, VHA
+def test_sigmoid_values_and_symmetry():
+    x = np.array([-800.0, -3.0, 0.0, 2.5, 800.0])
+    s = ORC.sigmoid(x)
+    assert s[2] == 0.5 and s[0] == 0.0 and s[-1] == 1.0
+    assert abs(s[1] - 1.0 / (1.0 + math.e ** 3.0)) < 1e-15
+    y = np.linspace(-30, 30, 121)
+    assert np.allclose(ORC.sigmoid(y) + ORC.sigmoid(-y), 1.0, atol=1e-15)
+
+
+def test_gate_from_latent_by_loops():
+    """Each gate value is sigmoid of one dot product of the latent with a column of W_g,
+    laid out head-major: G[t, h, d] uses column h * D + d."""
+    rng = np.random.default_rng(11)
+    T, L, hq, D = 3, 5, 2, 4
+    q = rng.standard_normal((T, L))
+    W = rng.standard_normal((L, hq * D))
+    G = ORC.gate_from_latent(q, W, hq, D)
+    for t in range(T):
+        for h in range(hq):
+            for d in range(D):
+                z = sum(q[t, i] * W[i, h * D + d] for i in range(L))
+                assert abs(G[t, h, d] - 1.0 / (1.0 + math.exp(-z))) < 1e-14
+    assert np.all(ORC.gate_from_latent(q, np.zeros_like(W), hq, D) == 0.5)
+
+
+def test_vha_mix_special_cases():
+    rng = np.random.default_rng(12)
+    T, hq, D, r = 4, 5, 3, 2
+    O = rng.standard_normal((T, hq, D))
+    # no mixing: the identity skip alone
+    assert np.array_equal(ORC.vha_mix(O, np.zeros((hq, r)), rng.standard_normal((hq, r))), O)
+    # rank one, A = e_i, B = e_j: head i gains head j's output, the others are unchanged
+    A = np.zeros((hq, 1)); A[1, 0] = 1.0
+    B = np.zeros((hq, 1)); B[3, 0] = 1.0
+    out = ORC.vha_mix(O, A, B)
+    want = O.copy(); want[:, 1] += O[:, 3]
+    assert np.allclose(out, want, atol=1e-15)
+    # equals the explicit [hq, hq] matrix I + A B^T applied across heads, by loops
+    A, B = rng.standard_normal((hq, r)), rng.standard_normal((hq, r))
+    out = ORC.vha_mix(O, A, B)
+    M = [[(1.0 if h == g else 0.0) + sum(A[h, k] * B[g, k] for k in range(r))
+          for g in range(hq)] for h in range(hq)]
+    for t in range(T):
+        for h in range(hq):
+            for d in range(D):
+                assert abs(out[t, h, d] - sum(M[h][g] * O[t, g, d] for g in range(hq))) < 1e-12
+
+
+def test_attention_output_order():
+    """The mixing runs on the ungated outputs and the gate multiplies after it."""
+    rng = np.random.default_rng(13)
+    O = rng.standard_normal((2, 3, 4))
+    G = rng.uniform(0.1, 0.9, (2, 3, 4))
+    A, B = rng.standard_normal((3, 2)), rng.standard_normal((3, 2))
+    out = ORC.attention_output(O, G, A, B)
+    assert np.allclose(out, ORC.vha_mix(O, A, B) * G, atol=1e-15)
+    assert not np.allclose(out, ORC.vha_mix(O * G, A, B))
