@@ -665,6 +665,129 @@ def bench_prefill_128k(args, dev, rank, world, barrier, max_over_ranks, peaks):
     flops = prefill_flops(T, b)
     tf = flops / (ms * 1e-3) / 1e12
     per_gpu = tf / world
+    e2e = None
+    if not args.no_e2e and world == 1:
+        e2e = _e2e_prefill_128k(args, dev, Q, K, V, G, flops, barrier, max_over_ranks)
+    del Q, K, V, G, be
+    torch.cuda.empty_cache()
+    out = _prefill_128k_result(tf, ms, per_gpu, world, peaks, clk)
+    if e2e is not None:
+        out["e2e"] = e2e
+    return out
+
+
+def _e2e_prefill_128k(args, dev, Q, K, V, G, flops, barrier, max_over_ranks):
+    """The 2 x 128K gated prefill end to end through the C ABI from pinned host memory:
+    per step, K and V of both sequences are uploaded and compressed, then every chunk of
+    8192 query positions uploads its Q and G rows, runs hca_attn_prefill_range (K/V rows from
+    127 positions before the chunk) and downloads its O rows. Uploads, compute and downloads
+    of consecutive chunks overlap on three streams with two device buffer sets."""
+    import torch
+    from compressed_long_context_hca_b200 import binding as B
+    from compressed_long_context_hca_b200 import ops
+    b, T = Q.shape[0], Q.shape[1]
+    C = 8192
+    hQ = torch.empty(Q.shape, dtype=Q.dtype, pin_memory=True)
+    hG = torch.empty(G.shape, dtype=G.dtype, pin_memory=True)
+    hO = torch.empty(Q.shape, dtype=Q.dtype, pin_memory=True)
+    hQ.copy_(Q)
+    hG.copy_(G)
+    hK = K.cpu().pin_memory()
+    hV = V.cpu().pin_memory()
+    dK, dV = torch.empty_like(K), torch.empty_like(V)
+    desc_all = B.make_desc(b, T, HQ, 1, D)
+    cache = B.PagedCache(b, T // BLOCK, 1, D, torch.bfloat16, 128, device=dev)
+    bufs = [(torch.empty((1, C, HQ, D), dtype=Q.dtype, device=dev),
+             torch.empty((1, C, HQ, D), dtype=Q.dtype, device=dev),
+             torch.empty((1, C, HQ, D), dtype=Q.dtype, device=dev)) for _ in range(2)]
+    up, comp, down = torch.cuda.Stream(), torch.cuda.current_stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    in_free, out_free, uploaded, computed = [ev(), ev()], [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    kv_up = ev()
+    chunks = [(bi, q0) for bi in range(b) for q0 in range(0, T, C)]
+    # one descriptor per chunk position: the gate rows of the chunk buffer, K/V rows of the
+    # sequence from kv0 = q0 - 127 (the cache holds every block's entry)
+    descs = {}
+    for bi, q0 in chunks:
+        d = B.make_desc(1, C, HQ, 1, D)
+        descs[(bi, q0)] = d
+
+    def run():
+        up.wait_stream(comp)  # the previous step's range calls have read dK, dV and buffers
+        with torch.cuda.stream(up):
+            dK.copy_(hK, non_blocking=True)
+            dV.copy_(hV, non_blocking=True)
+            kv_up.record(up)
+        comp.wait_event(kv_up)
+        with torch.cuda.stream(comp):
+            ops.compress(desc_all, dK, dV, cache)
+        for i, (bi, q0) in enumerate(chunks):
+            x = i % 2
+            q_, g_, o_ = bufs[x]
+            with torch.cuda.stream(up):
+                if i >= 2:
+                    up.wait_event(in_free[x])
+                q_.copy_(hQ[bi:bi + 1, q0:q0 + C], non_blocking=True)
+                g_.copy_(hG[bi:bi + 1, q0:q0 + C], non_blocking=True)
+                uploaded[x].record(up)
+            comp.wait_event(uploaded[x])
+            if i >= 2:
+                comp.wait_event(out_free[x])
+            with torch.cuda.stream(comp):
+                d = descs[(bi, q0)]
+                ops.attach_gate(d, g_)
+                kv0 = max(0, q0 - WIN + 1)
+                ops.prefill_range(d, q0, kv0, q_, dK[bi:bi + 1, kv0:q0 + C],
+                                  dV[bi:bi + 1, kv0:q0 + C], _SeqCache(cache, bi), O=o_)
+                computed[x].record(comp)
+                in_free[x].record(comp)
+            with torch.cuda.stream(down):
+                down.wait_event(computed[x])
+                hO[bi:bi + 1, q0:q0 + C].copy_(o_, non_blocking=True)
+                out_free[x].record(down)
+        comp.wait_stream(down)
+
+    run()
+    torch.cuda.synchronize()
+    steps = max(1, min(2, args.e2e_steps))
+    barrier()
+    a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(comp)
+    up.wait_stream(comp)
+    down.wait_stream(comp)
+    for _ in range(steps):
+        run()
+    e.record(comp)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(e)) / steps
+    assert int(cache.err.item()) == 0, "kernel raised an error bit"
+    out = {"value": round(flops / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+           "ms_per_step": round(ms, 2),
+           "h2d_bytes_per_step": (hQ.numel() + hG.numel() + hK.numel() + hV.numel()) * 2,
+           "d2h_bytes_per_step": hO.numel() * 2,
+           "overlap": "8192-position chunks through hca_attn_prefill_range; uploads / compute / "
+                      "downloads of consecutive chunks on three streams"}
+    del hQ, hG, hO, hK, hV, bufs, dK, dV
+    return out
+
+
+class _SeqCache:
+    """The cache of one sequence of a batch, as a one-sequence cache (its page-table row and
+    entry count), so a per-sequence range call reads that sequence's entries."""
+
+    def __init__(self, cache, b):
+        from compressed_long_context_hca_b200 import binding as B
+        c = B.HcaCache()
+        c.kc_pool, c.vc_pool = cache.c.kc_pool, cache.c.vc_pool
+        c.page_table = cache.page_table[b].data_ptr()
+        c.n_entries = cache.n_entries[b:b + 1].data_ptr()
+        c.page_entries, c.max_pages, c.num_pages = (cache.c.page_entries, cache.c.max_pages,
+                                                    cache.c.num_pages)
+        c.err_word = cache.c.err_word
+        self.c = c
+
+
+def _prefill_128k_result(tf, ms, per_gpu, world, peaks, clk):
     return {"value": round(tf, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 3),
             "workload": "batch 2 x 131072, 64 heads, 1 KV head, head_dim 512, every 4th block "
                         "x4, fused gate",

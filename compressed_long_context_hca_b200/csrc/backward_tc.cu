@@ -323,31 +323,23 @@ cudaError_t launch_backward_tc(const hca_desc& d, const BackwardTensors& x, cons
       const GemmOperand Qg = kmajor(x.Q, rowsQ, kD, kD, (int32_t)r0);
       const GemmOperand Qg_mn = mnmajor(x.Q, rowsQ, kD, kD, (int32_t)r0);
       // ---- scores and dP: compressed part [R, E], window bands [R, 256]
+      const GemmOperand* dop_lo_p = gated ? &dop_lo : nullptr;
       if (E > 0) {
-        HCA_TRY(gemm_tc(Qg, kmajor(H(pl.kc), pl.NE, kD, kD), out_rows(F(pl.sc), pl.Ep, R), R, E,
-                        kD, 1, 1.f, 0.f, err, s));
-        HCA_TRY(gemm_tc(dop_hi, kmajor(H(pl.vc), pl.NE, kD, kD), out_rows(F(pl.dpc), pl.Ep, R), R,
-                        E, kD, 1, 1.f, 0.f, err, s));
-        if (gated)
-          HCA_TRY(gemm_tc(dop_lo, kmajor(H(pl.vc), pl.NE, kD, kD), out_rows(F(pl.dpc), pl.Ep, R),
-                          R, E, kD, 1, 1.f, 1.f, err, s));
+        HCA_TRY(gemm_tc(Qg, nullptr, kmajor(H(pl.kc), pl.NE, kD, kD), out_rows(F(pl.sc), pl.Ep, R),
+                        R, E, kD, 1, 1.f, 0.f, err, s));
+        HCA_TRY(gemm_tc(dop_hi, dop_lo_p, kmajor(H(pl.vc), pl.NE, kD, kD),
+                        out_rows(F(pl.dpc), pl.Ep, R), R, E, kD, 1, 1.f, 0.f, err, s));
       }
       const GemmOperand Qb = kmajor(x.Q, rowsQ, kD, kD, (int32_t)r0, Mw);
       const GemmOperand Kband = kmajor(x.K, rowsK, kD, kD, kv_row0, kSub);
       const GemmOperand Vband = kmajor(x.V, rowsK, kD, kD, kv_row0, kSub);
-      HCA_TRY(gemm_tc(Qb, Kband, out_rows(F(pl.sw), kBand, R, 0, Mw), Mw, kBand, kD, nsub, 1.f,
-                      0.f, err, s));
+      HCA_TRY(gemm_tc(Qb, nullptr, Kband, out_rows(F(pl.sw), kBand, R, 0, Mw), Mw, kBand, kD,
+                      nsub, 1.f, 0.f, err, s));
       {
-        GemmOperand a = dop_hi;
-        a.bstride = Mw;
-        HCA_TRY(gemm_tc(a, Vband, out_rows(F(pl.dpw), kBand, R, 0, Mw), Mw, kBand, kD, nsub, 1.f,
-                        0.f, err, s));
-        if (gated) {
-          GemmOperand al = dop_lo;
-          al.bstride = Mw;
-          HCA_TRY(gemm_tc(al, Vband, out_rows(F(pl.dpw), kBand, R, 0, Mw), Mw, kBand, kD, nsub,
-                          1.f, 1.f, err, s));
-        }
+        GemmOperand a = dop_hi, al = dop_lo;
+        a.bstride = al.bstride = Mw;
+        HCA_TRY(gemm_tc(a, gated ? &al : nullptr, Vband, out_rows(F(pl.dpw), kBand, R, 0, Mw), Mw,
+                        kBand, kD, nsub, 1.f, 0.f, err, s));
       }
       // ---- P, Delta, dS
       SoftmaxArgs sa;
@@ -375,7 +367,7 @@ cudaError_t launch_backward_tc(const hca_desc& d, const BackwardTensors& x, cons
       sa.scale = d.scale;
       softmax_bwd_kernel<<<(R + 3) / 4, 128, 0, s>>>(sa);
       HCA_TRY(cudaGetLastError());
-      // ---- products with a bf16 pair operand X = hi + lo: out (+)= X . B or X^T . B
+      // ---- products with a bf16 pair operand X = hi + lo (one pass of gemm_tc each)
       auto pair = [&](size_t hi, size_t lo, int64_t rows, int64_t cols, bool mn, int32_t bst) {
         return std::make_pair(GemmOperand{H(hi), rows, cols, cols, mn, 0, bst},
                               GemmOperand{H(lo), rows, cols, cols, mn, 0, bst});
@@ -386,16 +378,14 @@ cudaError_t launch_backward_tc(const hca_desc& d, const BackwardTensors& x, cons
         if (E > 0) {
           auto ds = pair(pl.dsch, pl.dscl, R, pl.Ep, false, 0);
           const GemmOperand kc_mn = mnmajor(H(pl.kc), pl.NE, kD, kD);
-          HCA_TRY(gemm_tc(ds.first, kc_mn, out_rows(F(pl.dq), kD, R), R, kD, E, 1, 1.f, 0.f, err, s));
-          HCA_TRY(gemm_tc(ds.second, kc_mn, out_rows(F(pl.dq), kD, R), R, kD, E, 1, 1.f, 1.f, err, s));
+          HCA_TRY(gemm_tc(ds.first, &ds.second, kc_mn, out_rows(F(pl.dq), kD, R), R, kD, E, 1,
+                          1.f, 0.f, err, s));
           first = false;
         }
         auto dsw = pair(pl.dswh, pl.dswl, R, kBand, false, Mw);
         const GemmOperand kb_mn = mnmajor(x.K, rowsK, kD, kD, kv_row0, kSub);
-        HCA_TRY(gemm_tc(dsw.first, kb_mn, out_rows(F(pl.dq), kD, R, 0, Mw), Mw, kD, kBand, nsub,
-                        1.f, first ? 0.f : 1.f, err, s));
-        HCA_TRY(gemm_tc(dsw.second, kb_mn, out_rows(F(pl.dq), kD, R, 0, Mw), Mw, kD, kBand, nsub,
-                        1.f, 1.f, err, s));
+        HCA_TRY(gemm_tc(dsw.first, &dsw.second, kb_mn, out_rows(F(pl.dq), kD, R, 0, Mw), Mw, kD,
+                        kBand, nsub, 1.f, first ? 0.f : 1.f, err, s));
         const int64_t n = (int64_t)R * kD;
         rows_to_bf16_kernel<<<1184, 256, 0, s>>>(F(pl.dq), nullptr, n,
                                                  static_cast<__nv_bfloat16*>(x.dQ) + r0 * kD);
@@ -407,17 +397,15 @@ cudaError_t launch_backward_tc(const hca_desc& d, const BackwardTensors& x, cons
         if (E > 0) {
           auto pc = pair(pl.pch, pl.pcl, R, pl.Ep, false, 0);
           const GemmOperand vc_mn = mnmajor(H(pl.vc), pl.NE, kD, kD);
-          HCA_TRY(gemm_tc(pc.first, vc_mn, out_rows(F(pl.opre), kD, R), R, kD, E, 1, 1.f, 0.f, err, s));
-          HCA_TRY(gemm_tc(pc.second, vc_mn, out_rows(F(pl.opre), kD, R), R, kD, E, 1, 1.f, 1.f, err, s));
+          HCA_TRY(gemm_tc(pc.first, &pc.second, vc_mn, out_rows(F(pl.opre), kD, R), R, kD, E, 1,
+                          1.f, 0.f, err, s));
           first = false;
         }
         auto pw = pair(pl.pwh, pl.pwl, R, kBand, false, Mw);
         const GemmOperand vb_mn = mnmajor(x.V, rowsK, kD, kD, kv_row0, kSub);
-        HCA_TRY(gemm_tc(pw.first, vb_mn, out_rows(F(pl.opre), kD, R, 0, Mw), Mw, kD, kBand, nsub,
-                        1.f, first ? 0.f : 1.f, err, s));
-        HCA_TRY(gemm_tc(pw.second, vb_mn, out_rows(F(pl.opre), kD, R, 0, Mw), Mw, kD, kBand, nsub,
-                        1.f, 1.f, err, s));
-        // dG rows of the group: dO * O_pre (the gate's stride layout is dense [b, T, hq, D])
+        HCA_TRY(gemm_tc(pw.first, &pw.second, vb_mn, out_rows(F(pl.opre), kD, R, 0, Mw), Mw, kD,
+                        kBand, nsub, 1.f, first ? 0.f : 1.f, err, s));
+        // dG rows of the group: dO * O_pre (dG is dense [b, T, hq, D])
         rows_to_bf16_kernel<<<1184, 256, 0, s>>>(F(pl.opre),
                                                  static_cast<const __nv_bfloat16*>(x.dO) + r0 * kD,
                                                  (int64_t)R * kD,
@@ -436,11 +424,9 @@ cudaError_t launch_backward_tc(const hca_desc& d, const BackwardTensors& x, cons
         dh.bstride = dl.bstride = ksplit;
         const GemmOutput okc = out_rows(F(pl.dkc), kD, pl.NE, 0, 0, 1, true);
         const GemmOutput ovc = out_rows(F(pl.dvc), kD, pl.NE, 0, 0, 1, true);
-        HCA_TRY(gemm_tc(dsT.first, q, okc, E, kD, ksplit, nspl, 1.f, 0.f, err, s));
-        HCA_TRY(gemm_tc(dsT.second, q, okc, E, kD, ksplit, nspl, 1.f, 0.f, err, s));
-        HCA_TRY(gemm_tc(pT.first, dh, ovc, E, kD, ksplit, nspl, 1.f, 0.f, err, s));
-        HCA_TRY(gemm_tc(pT.second, dh, ovc, E, kD, ksplit, nspl, 1.f, 0.f, err, s));
-        if (gated) HCA_TRY(gemm_tc(pT.first, dl, ovc, E, kD, ksplit, nspl, 1.f, 0.f, err, s));
+        HCA_TRY(gemm_tc(dsT.first, &dsT.second, q, okc, E, kD, ksplit, nspl, 1.f, 0.f, err, s));
+        HCA_TRY(gemm_tc(pT.first, &pT.second, dh, ovc, E, kD, ksplit, nspl, 1.f, 0.f, err, s));
+        if (gated) HCA_TRY(gemm_tc(pT.first, nullptr, dl, ovc, E, kD, ksplit, nspl, 1.f, 0.f, err, s));
       }
       // dK_band += dSw^T Q_band, dV_band += Pw^T dO'_band  (K = 128 hq rows per band,
       // split in 4; bands of neighbouring sub-chunks overlap: atomics)
@@ -456,11 +442,9 @@ cudaError_t launch_backward_tc(const hca_desc& d, const BackwardTensors& x, cons
         const GemmOutput ok = out_rows(F(pl.dkw), kD, T, p0 - kSub, kSub, sp, true);
         const GemmOutput ov = out_rows(F(pl.dvw), kD, T, p0 - kSub, kSub, sp, true);
         const int nb = nsub * sp;
-        HCA_TRY(gemm_tc(dsT.first, q, ok, kBand, kD, kb, nb, 1.f, 0.f, err, s));
-        HCA_TRY(gemm_tc(dsT.second, q, ok, kBand, kD, kb, nb, 1.f, 0.f, err, s));
-        HCA_TRY(gemm_tc(pT.first, dh, ov, kBand, kD, kb, nb, 1.f, 0.f, err, s));
-        HCA_TRY(gemm_tc(pT.second, dh, ov, kBand, kD, kb, nb, 1.f, 0.f, err, s));
-        if (gated) HCA_TRY(gemm_tc(pT.first, dl, ov, kBand, kD, kb, nb, 1.f, 0.f, err, s));
+        HCA_TRY(gemm_tc(dsT.first, &dsT.second, q, ok, kBand, kD, kb, nb, 1.f, 0.f, err, s));
+        HCA_TRY(gemm_tc(pT.first, &pT.second, dh, ov, kBand, kD, kb, nb, 1.f, 0.f, err, s));
+        if (gated) HCA_TRY(gemm_tc(pT.first, nullptr, dl, ov, kBand, kD, kb, nb, 1.f, 0.f, err, s));
       }
     }
     finalize_kv_kernel<<<T, 128, 0, s>>>(F(pl.dkw), F(pl.dvw), F(pl.dkc), F(pl.dvc), T, d.block,

@@ -32,9 +32,11 @@ struct GemmOutput {
   bool sigmoid_bf16;
 };
 
-// C = alpha * A . B^T + beta * C for `batch` products of M x N over K (bf16 in, f32 out).
-cudaError_t gemm_tc(const GemmOperand& A, const GemmOperand& B, const GemmOutput& C, int M,
-                    int N, int K, int batch, float alpha, float beta, int32_t* err_word,
-                    cudaStream_t s);
+// C = alpha * (A + A_lo) . B^T + beta * C for `batch` products of M x N over K (bf16 in,
+// f32 out). A_lo (optional, may be nullptr): the low part of a bf16 pair, laid out as A
+// (same rows, cols, major, shift, bstride); its product accumulates with A's in one pass.
+cudaError_t gemm_tc(const GemmOperand& A, const GemmOperand* A_lo, const GemmOperand& B,
+                    const GemmOutput& C, int M, int N, int K, int batch, float alpha, float beta,
+                    int32_t* err_word, cudaStream_t s);
 
 }  // namespace hca

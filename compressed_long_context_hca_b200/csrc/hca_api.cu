@@ -284,7 +284,7 @@ int32_t hca_gate_from_latent(const hca_desc* d, const void* q_lat, const void* W
   const GemmOperand A{q_lat, rows, latent, latent, false, 0, 0};
   const GemmOperand B{W_g, latent, n, n, true, 0, 0};
   GemmOutput C{static_cast<float*>(G), n, 0, 0, (int32_t)rows, 1, false, true};
-  return from_cuda(gemm_tc(A, B, C, (int)rows, (int)n, latent, 1, 1.f, 0.f, nullptr,
+  return from_cuda(gemm_tc(A, nullptr, B, C, (int)rows, (int)n, latent, 1, 1.f, 0.f, nullptr,
                            reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -179,7 +179,7 @@ __device__ __forceinline__ int k_slots(const Tile& t) { return t.kind == kRaw16 
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffRing = kQBytes;
 constexpr uint32_t kOffBar = kOffRing + kStages * kSlotBytes;
-constexpr uint32_t kOffL = kOffBar + 256;
+constexpr uint32_t kOffL = kOffBar + 512;
 constexpr uint32_t kSmemBytes = kOffL + 2 * kBM * 4 + 1024;
 
 struct Bars {
@@ -189,15 +189,15 @@ struct Bars {
   uint64_t o_done[2];  // P.V of tiles of even / odd index
   uint64_t o_free, o_final, drain;
   uint64_t l_full[2];
+  // leader only: where each load stream stopped issuing (see drain_loads), 4 K/V producers
+  // (rank * 2 + parity) and 2 Q producers (rank), and the barrier they arrive on
+  uint64_t stops_full;
+  int32_t kv_stop[4];
+  int32_t q_stop[2];
   uint32_t tmem_base;
   int abort;
 };
-static_assert(sizeof(Bars) <= 256, "barrier block too large");
-
-__device__ __forceinline__ void raise_timeout(const Params& p, Bars* bars, int role) {
-  bars->abort = 1;
-  if (p.err_word) atomicOr(p.err_word, kErrTimeout | (1 << (8 + role)));
-}
+static_assert(sizeof(Bars) <= 512, "barrier block too large");
 
 // ------------------------------------------------------------------------ cluster PTX
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -229,6 +229,33 @@ __device__ __forceinline__ void cluster_sync_all() {
 // and fence::after_thread_sync after the wait, as for a local hand-off.
 __device__ __forceinline__ void mbar_arrive_cl(uint32_t bar_cl) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cl) : "memory");
+}
+
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr_cl, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr_cl), "r"(v) : "memory");
+}
+// arrive with release at cluster scope: a store to the other CTA's shared memory made
+// before it is visible to whoever observes the phase
+__device__ __forceinline__ void mbar_arrive_release_cl(uint32_t bar_cl) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cl)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_complete_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.complete_tx.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+// A role gave up waiting: every role of both CTAs stops at its next wait.
+__device__ __forceinline__ void raise_timeout(const Params& p, Bars* bars, int role) {
+  bars->abort = 1;
+  st_cluster_u32(map_rank(&bars->abort, cluster_rank() ^ 1u), 1u);
+  if (p.err_word) atomicOr(p.err_word, kErrTimeout | (1 << (8 + role)));
+}
+
+// A load stream publishes, in the leader CTA, the first sequence number it did not issue.
+__device__ __forceinline__ void publish_stop(Bars* bars, int32_t* slot, int32_t stop) {
+  st_cluster_u32(map_rank(slot, 0), (uint32_t)stop);
+  mbar_arrive_release_cl(map_rank(&bars->stops_full, 0));
 }
 
 // ------------------------------------------------------------------------ 2-SM tcgen05
@@ -324,6 +351,83 @@ __device__ __forceinline__ void st_stream_hint32(void* ptr, const uint32_t* v, u
       : "memory");
 }
 
+// Per-CTA bytes of K/V load n of cluster c: the producers' load sequence walked again (K of
+// tile j of an item, then V of the tile before it, possibly of the previous item; the V of
+// the very last tile closes the sequence). Returns 0 past the end.
+__device__ uint32_t kv_load_bytes(const Params& p, int G, int c, int32_t n) {
+  int32_t cnt = 0;
+  Item pit;
+  int pj = -1;
+  auto v_bytes = [&](const Item& it, int j) { return tile_of(it, j).kind == kRaw16 ? kV16Box : kVBox; };
+  for (int r = 0;; ++r) {
+    const int k = cluster_item(r, G, c);
+    if (k >= p.n_items) break;
+    const Item it = make_item(p, k);
+    for (int j = 0; j < it.ntiles; ++j) {
+      const Tile t = tile_of(it, j);
+      const int nk = k_slots(t);
+      if (n < cnt + nk) return t.kind == kRaw16 ? kK8Box : kKBox;
+      cnt += nk;
+      if (pj >= 0) {
+        if (n == cnt) return v_bytes(pit, pj);
+        ++cnt;
+      }
+      pit = it;
+      pj = j;
+    }
+  }
+  if (pj >= 0 && n == cnt) return v_bytes(pit, pj);
+  return 0;
+}
+
+// After a time-out (leader, one thread): wait, bounded, until every bulk load either CTA
+// has issued has landed, so that neither CTA's shared memory goes away under a copy.
+// The peer's loads complete on the leader's barriers, which the peer cannot wait on; each
+// load stream published the first sequence number it did not issue (kv_stop, q_stop).
+// A stream issues load n of a ring slot only after the slot's previous phase completed, so
+// on each barrier at most its last issued load can be outstanding: n* = the largest issued
+// sequence number on the slot, and no load after it exists, which keeps the parity wait
+// exact. The leader armed 2 x the bytes of every load it issued: a half the peer never
+// issued is completed by hand; a load only the peer issued is armed now.
+__device__ void drain_loads(const Params& p, Bars* bars, int G, int c) {
+  volatile int no_abort = 0;
+  if (!mbar_wait(&bars->stops_full, 0, &no_abort, 3000000000ull)) return;
+  // every stop is now visible (release arrives, acquire here)
+  asm volatile("fence.acq_rel.cluster;" ::: "memory");
+  const volatile int32_t* kv = bars->kv_stop;
+  for (int s = 0; s < kStages; ++s) {
+    int32_t nstar = -1;
+    for (int cm = 0; cm < 4; ++cm) {  // stream (rank cm / 2, parity cm % 2)
+      for (int32_t n = kv[cm] - 1; n >= 0 && n >= kv[cm] - 6; --n)
+        if ((n & 1) == (cm & 1) && n % kStages == s) {
+          nstar = max(nstar, n);
+          break;
+        }
+    }
+    if (nstar < 0) continue;
+    const bool L = nstar < kv[0 * 2 + (nstar & 1)];
+    const bool P = nstar < kv[1 * 2 + (nstar & 1)];
+    const uint32_t b = kv_load_bytes(p, G, c, nstar);
+    if (L && !P) mbar_complete_tx(&bars->ring_full[s], b);
+    if (!L && P) mbar_expect_tx(&bars->ring_full[s], b);
+    mbar_wait(&bars->ring_full[s], (uint32_t)(nstar / kStages) & 1, &no_abort, 100000000ull);
+  }
+  // Q: box q of walked item r is sequence number 4 r + q; only even items load (odd ones
+  // reuse the tile and only the leader arrives, without bytes)
+  const volatile int32_t* qs = bars->q_stop;
+  for (int q = 0; q < kQPairs; ++q) {
+    int r0 = -1, r1 = -1;
+    if (qs[0] > q) r0 = (qs[0] - 1 - q) / kQPairs;
+    if (qs[1] > q) r1 = (qs[1] - 1 - q) / kQPairs;
+    const int rstar = max(r0, r1);
+    if (rstar < 0 || (rstar & 1)) continue;
+    const bool L = rstar <= r0, P = rstar <= r1;
+    if (L && !P) mbar_complete_tx(&bars->q_full[q], kSlotBytes);
+    if (!L && P) mbar_expect_tx(&bars->q_full[q], kSlotBytes);
+    mbar_wait(&bars->q_full[q], (uint32_t)rstar & 1, &no_abort, 100000000ull);
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_pair_kernel(const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -360,6 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars->l_full[0], 4);
     mbar_init(&bars->l_full[1], 4);
     mbar_init(&bars->drain, 1);
+    mbar_init(&bars->stops_full, 6);  // 4 K/V producers and 2 Q producers of the pair
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -475,22 +580,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (ok && pj >= 0) ok = load_tile(pit, pj, true);
-      if (!ok) {
-        raise_timeout(p, bars, 1);
-        // let this producer's loads in flight land before shared memory goes away: the
-        // leader sees them on its own barriers; the peer's complete on the leader's, so it
-        // gives them a fixed millisecond
-        volatile int no_abort = 0;
-        if (leader) {
-          const uint32_t first = cnt > kStages ? cnt - kStages : 0;
-          for (uint32_t q = first; q < cnt; ++q)
-            if ((q & 1u) == mine)
-              mbar_wait(&bars->ring_full[q % kStages], (q / kStages) & 1, &no_abort, 100000000ull);
-        } else {
-          const uint64_t t0 = globaltimer_ns();
-          while (globaltimer_ns() - t0 < 1000000ull) __nanosleep(1000);
-        }
-      }
+      if (!ok) raise_timeout(p, bars, 1);
+      // every sequence number of this producer's parity below the stop was issued; the one
+      // whose slot wait failed (cnt - 1) was not. The leader waits for what is in flight
+      // (drain_loads) before either CTA leaves.
+      publish_stop(bars, &bars->kv_stop[rank * 2 + mine], (int32_t)(ok ? cnt : cnt - 1));
     }
   } else if (warp == 11) {
     // ------------------------------------------------------------------ Q TMA producer
@@ -503,6 +597,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int q = 0; q < kQPairs; ++q) qfull_cl[q] = map_rank(&bars->q_full[q], 0);
       int nitem = 0;
+      int32_t qstop = 0;  // boxes walked (item-major, 4 per item), then the first not issued
       bool ok = true;
       for (int r = 0; ok; ++r) {
         const int k = cluster_item(r, G, c);
@@ -512,6 +607,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool reuse = (r & 1) != 0;
         for (int q = 0; q < kQPairs && ok; ++q) {
           if (nitem > 0 && !(ok = mbar_wait(&bars->q_empty[q], (nitem - 1) & 1, abort))) break;
+          ++qstop;
           if (reuse) {
             if (leader) mbar_arrive(&bars->q_full[q]);
           } else {
@@ -521,17 +617,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ++nitem;
       }
-      if (!ok) {
-        raise_timeout(p, bars, 2);
-        volatile int no_abort = 0;
-        if (leader) {
-          for (int q = 0; q < kQPairs; ++q)
-            mbar_wait(&bars->q_full[q], (nitem - 1) & 1, &no_abort, 100000000ull);
-        } else {
-          const uint64_t t0 = globaltimer_ns();
-          while (globaltimer_ns() - t0 < 1000000ull) __nanosleep(1000);
-        }
-      }
+      if (!ok) raise_timeout(p, bars, 2);
+      publish_stop(bars, &bars->q_stop[rank], qstop);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ UMMA issuer
@@ -932,9 +1019,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // both CTAs leave together: the leader's UMMAs (which read the peer's shared memory and
-  // write its TMEM) have drained before either CTA passes this point
+  // write its TMEM) have drained before either CTA passes this point. After a time-out the
+  // leader first waits for the loads still in flight into either CTA (drain_loads); the
+  // peer cannot pass the cluster barrier before the leader arrives.
   tc_fence_before();
-  __syncwarp();
+  __syncthreads();
+  if (leader && threadIdx.x == 0 && *abort) drain_loads(p, bars, G, c);
+  __syncthreads();
   cluster_sync_all();
   if (warp == 1) {
     __syncwarp();
