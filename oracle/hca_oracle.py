@@ -453,3 +453,85 @@ def visible_pairs(T: int, block: int, window: int) -> Tuple[int, int]:
         lo, hi = window_bounds(t, window)
         w += hi - lo + 1
     return c, w
+
+
+# ---------------------------------------------------------------------------
+# 8-bit compressed cache
+# ---------------------------------------------------------------------------
+#
+# The communeify.com page, section "本地部署與推論實戰指南", item 3, serves the model through
+# vLLM with an 8-bit KV cache (`--kv-cache-dtype fp8`) -- cited below as [serve fp8].  The
+# pages give no format details.  Readings:
+#   * element format: e4m3 as in the OCP 8-bit floating-point specification (the default
+#     8-bit cache format of that engine): 1 sign bit, 4 exponent bits with bias 7, 3
+#     fraction bits, subnormals when the exponent field is 0, no infinities, and the one
+#     pattern with all exponent and fraction bits set is NaN, so the largest finite
+#     magnitude is 448;
+#   * what is stored in 8 bits: the compressed pools Kc and Vc (the cache that grows with
+#     the context); the raw window stays in the model's dtype;
+#   * scale granularity: one float32 scale per pool (per tensor), stored value =
+#     e4m3(entry / scale), read back as value(code) * scale;
+#   * quantisation: the block mean as a float32 (the value the 16-bit cache would round
+#     from), divided by the scale in float32, rounded to the nearest e4m3 value with ties
+#     to the even code, magnitudes of 448 and above stored as 448 (saturation).
+
+_E4M3_MAX = 448.0
+
+
+def e4m3_value(codes) -> np.ndarray:
+    """Value of each 8-bit e4m3 code (uint8 array), float64; NaN for the NaN codes.
+
+    Field layout from the format definition: bit 7 sign, bits 3-6 exponent e (bias 7),
+    bits 0-2 fraction m.  e = 0: m/8 * 2^-6 (subnormal, or zero); e = 15 with m = 7: NaN;
+    otherwise (1 + m/8) * 2^(e - 7).
+    """
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    mag = np.where((e == 15) & (m == 7), np.nan, mag)
+    return sign * mag
+
+
+def _e4m3_positive_table() -> np.ndarray:
+    """Values of the non-negative finite codes 0..126, ascending with the code."""
+    return e4m3_value(np.arange(127, dtype=np.uint8))
+
+
+def e4m3_quantize(x) -> np.ndarray:
+    """Nearest e4m3 code of each float32 value (ties to the even code), saturating
+    magnitudes >= 448 to 448; NaN inputs give the NaN code.  Returns uint8."""
+    x = np.asarray(x, dtype=np.float32).astype(np.float64)
+    table = _e4m3_positive_table()
+    a = np.abs(x)
+    neg = np.signbit(x)
+    hi = np.clip(np.searchsorted(table, a, side="left"), 1, 126)   # table[hi-1] < a <= table[hi]
+    lo = hi - 1
+    d_lo = a - table[lo]
+    d_hi = table[hi] - a
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo)
+    code = np.where(a == 0.0, 0, code)
+    code = np.where(a >= _E4M3_MAX, 126, code)
+    code = code | np.where(neg, 0x80, 0)
+    code = np.where(np.isnan(x), 0x7F, code)
+    return code.astype(np.uint8)
+
+
+def e4m3_dequantize(codes, scale: float) -> np.ndarray:
+    """Stored value of each code of a pool with per-tensor ``scale``: value(code) * scale,
+    float64 ([serve fp8], readings above)."""
+    return e4m3_value(codes) * np.float64(np.float32(scale))
+
+
+def compress_blocks_e4m3(X: np.ndarray, block: int, scale: float) -> np.ndarray:
+    """Compressed entries of ``compress_blocks`` stored in 8 bits ([serve fp8]).
+
+    The mean of each block, taken as the float32 nearest to its float64 value, divided
+    by ``scale`` in float32, rounded to e4m3 (readings above).  Returns uint8 codes of
+    shape [ceil(T/block), H, D].
+    """
+    mean32 = compress_blocks(X, block).astype(np.float32)
+    y = (mean32 / np.float32(scale)).astype(np.float32)
+    return e4m3_quantize(y)
