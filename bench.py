@@ -378,6 +378,11 @@ def gpu_main(args, rank, world, local_rank):
                                                         max_over_ranks, peaks)
         result["decode_1m"] = bench_decode_1m(args, dev, rank, world, barrier, max_over_ranks,
                                               peaks)
+        if not args.no_e4m3:
+            result["decode_batched_e4m3"] = bench_decode_batched(
+                args, dev, rank, world, barrier, max_over_ranks, peaks, e4m3=True)
+            result["decode_1m_e4m3"] = bench_decode_1m(args, dev, rank, world, barrier,
+                                                       max_over_ranks, peaks, e4m3=True)
     if args.with_128k:
         result["compress_2x128k"] = bench_compress_2x128k(args, dev, rank, world, barrier,
                                                           max_over_ranks, peaks)
@@ -437,9 +442,22 @@ def _time_loop(fn, steps, warmup, barrier, max_over_ranks, stream):
     return max_over_ranks(a.elapsed_time(b)) / steps
 
 
-def bench_decode_batched(args, dev, rank, world, barrier, max_over_ranks, peaks):
+E4M3_SCALES = (1.0 / 16, 1.0 / 16)
+
+
+def _fill_e4m3(t, g):
+    """Random e4m3 codes in place: a random sign over a magnitude code uniform in
+    0..0x5F (the recipe of inputs.e4m3_codes, drawn on the device)."""
+    import torch
+    t.random_(0, 0x60, generator=g)
+    sign = torch.randint(0, 2, t.shape, generator=g, device=t.device, dtype=torch.uint8)
+    t.bitwise_or_(sign << 7)
+
+
+def bench_decode_batched(args, dev, rank, world, barrier, max_over_ranks, peaks, e4m3=False):
     """128 sequences, context lengths U[8192, 131072]; with N ranks each serves a
-    contiguous range of the sequences (no exchange)."""
+    contiguous range of the sequences (no exchange). e4m3: the compressed cache holds
+    8-bit codes (per-pool scales 1/16); the window ring stays bf16."""
     import torch
     from compressed_long_context_hca_b200 import binding as B
     from compressed_long_context_hca_b200 import ops
@@ -454,9 +472,14 @@ def bench_decode_batched(args, dev, rank, world, barrier, max_over_ranks, peaks)
     ctx = ctx_all[s0:s1].contiguous()
     g.manual_seed(2001 + rank)
     max_ent = (hi - WIN) // BLOCK + 1
-    cache = B.PagedCache(nseq, max_ent, 1, D, torch.bfloat16, 128, device=dev)
-    cache.kc.normal_(generator=g)
-    cache.vc.normal_(generator=g)
+    cache = B.PagedCache(nseq, max_ent, 1, D, torch.bfloat16, 128, device=dev,
+                         e4m3_scales=E4M3_SCALES if e4m3 else None)
+    if e4m3:
+        _fill_e4m3(cache.kc, g)
+        _fill_e4m3(cache.vc, g)
+    else:
+        cache.kc.normal_(generator=g)
+        cache.vc.normal_(generator=g)
     cache.n_entries.fill_(max_ent)
     q = torch.randn((nseq, HQ, D), generator=g, device=dev).to(torch.bfloat16)
     rk = torch.randn((nseq, WIN, 1, D), generator=g, device=dev).to(torch.bfloat16)
@@ -471,14 +494,19 @@ def bench_decode_batched(args, dev, rank, world, barrier, max_over_ranks, peaks)
     ms = _time_graph(fn, args.decode_steps, 3, barrier, max_over_ranks, stream)
     clk = clocks.stop()
     ctx_h = ctx_all.cpu().tolist()
-    keys = sum((c - WIN) // BLOCK + min(WIN, c) for c in ctx_h)
-    byts = keys * D * 2 * 2 + nseq_all * HQ * D * 2 * 2
+    entries = sum(max(0, c - WIN) // BLOCK for c in ctx_h)
+    raw = sum(min(WIN, c) for c in ctx_h)
+    # K and V of every visible key (1 byte per element for e4m3 entries), Q in, O out
+    byts = (entries * D * 2 * (1 if e4m3 else 2) + raw * D * 2 * 2 +
+            nseq_all * HQ * D * 2 * 2)
     nsplit = B.hca_decode_workspace_bytes(desc) // (nseq * HQ * (D + 2) * 4)
     gbs = byts / (ms * 1e-3) / 1e9 / world  # per GPU
+    cache_txt = ("e4m3 compressed cache (scales 1/16) + bf16 128-token ring" if e4m3 else
+                 "paged cache + 128-token ring, N(0,1) bf16")
     return {"value": round(nseq_all / (ms * 1e-3), 1), "unit": "tokens/s",
             "ms_per_step": round(ms, 4),
             "workload": "128 sequences, context U[8192,131072], 1 query each, 64 heads, "
-                        "head_dim 512, paged cache + 128-token ring, N(0,1) bf16",
+                        "head_dim 512, " + cache_txt,
             "parallelism": f"sequences x{world}" if world > 1 else "single GPU",
             "timing": "CUDA graph replay of one step",
             "gpu_launches_per_step": 2, "splits": int(nsplit),
@@ -489,18 +517,23 @@ def bench_decode_batched(args, dev, rank, world, barrier, max_over_ranks, peaks)
             "clocks": clk}
 
 
-def _shard_cache(nseq, e0, e1, n_total, dev, g):
+def _shard_cache(nseq, e0, e1, n_total, dev, g, e4m3=False):
     """A paged cache holding only entries [e0, min(e1, n_total)) of every sequence, at
     their absolute entry indices (pages outside the shard map to page 0 and are never
-    read), filled with N(0,1) values."""
+    read), filled with N(0,1) values (or random e4m3 codes)."""
     import torch
     from compressed_long_context_hca_b200 import binding as B
     p0 = e0 // 128
     p1 = -(-min(e1, n_total) // 128)
     shard_pages = max(1, p1 - p0)
-    cache = B.PagedCache(nseq, shard_pages * 128, 1, D, torch.bfloat16, 128, device=dev)
-    cache.kc.normal_(generator=g)
-    cache.vc.normal_(generator=g)
+    cache = B.PagedCache(nseq, shard_pages * 128, 1, D, torch.bfloat16, 128, device=dev,
+                         e4m3_scales=E4M3_SCALES if e4m3 else None)
+    if e4m3:
+        _fill_e4m3(cache.kc, g)
+        _fill_e4m3(cache.vc, g)
+    else:
+        cache.kc.normal_(generator=g)
+        cache.vc.normal_(generator=g)
     total_pages = -(-n_total // 128)
     pt = torch.zeros((nseq, total_pages), dtype=torch.int32)
     for b in range(nseq):
@@ -512,7 +545,7 @@ def _shard_cache(nseq, e0, e1, n_total, dev, g):
     return cache
 
 
-def bench_decode_1m(args, dev, rank, world, barrier, max_over_ranks, peaks):
+def bench_decode_1m(args, dev, rank, world, barrier, max_over_ranks, peaks, e4m3=False):
     """16 sequences at 1,048,576 context, 4 decode steps each with the compress of the block
     the first step completes. With N ranks the compressed entries of every sequence are cut
     into N ranges of whole 128-entry tiles (rank r holds only its range), the last rank also
@@ -535,7 +568,7 @@ def bench_decode_1m(args, dev, rank, world, barrier, max_over_ranks, peaks):
     g.manual_seed(3001 + rank)
     e0, e1 = P.entry_range(n_ent, world, rank) if world > 1 else (0, 1 << 30)
     last = rank == world - 1
-    cache = _shard_cache(nseq, e0, e1, n_ent + 2, dev, g)
+    cache = _shard_cache(nseq, e0, e1, n_ent + 2, dev, g, e4m3)
     cache.n_entries.fill_(n_ent)
     ctx = [torch.full((nseq,), ctx0 + s, dtype=torch.int32, device=dev) for s in range(steps_per)]
     descs = []
@@ -572,16 +605,18 @@ def bench_decode_1m(args, dev, rank, world, barrier, max_over_ranks, peaks):
         timing = "launch loop (the steps hold NCCL all-gathers)"
     clk = clocks.stop()
     assert int(cache.err.item()) == 0, "kernel raised an error bit"
-    keys = n_ent + WIN
-    byts_step = nseq * (keys * D * 2 * 2 + 3 * HQ * D * 2)
-    byts = steps_per * byts_step + nseq * BLOCK * D * 2 * 2
+    eb = 1 if e4m3 else 2  # bytes per compressed element
+    byts_step = nseq * (n_ent * D * 2 * eb + WIN * D * 2 * 2 + 3 * HQ * D * 2)
+    # the compress reads the ring's K and V once and writes one entry each
+    byts = steps_per * byts_step + nseq * (BLOCK * D * 2 * 2 + D * 2 * eb)
     gbs = byts / (ms * 1e-3) / 1e9 / world  # per GPU
     nsplit = B.hca_decode_workspace_bytes(descs[0]) // (nseq * HQ * (D + 2) * 4)
     launches = (4 * 2 + 1) if world == 1 else (4 * 3 + (1 if last else 0))
     return {"value": round(nseq * steps_per / (ms * 1e-3), 1), "unit": "tokens/s",
             "ms_per_step": round(ms, 4), "ms_per_decode_step": round(ms / steps_per, 4),
             "workload": "16 sequences at context 1,048,576 (8191 entries + 128 raw), 64 heads, "
-                        "head_dim 512, 4 decode steps each incl. one hca_compress, gate on",
+                        "head_dim 512, 4 decode steps each incl. one hca_compress, gate on" +
+                        (", e4m3 compressed cache (scales 1/16), bf16 ring" if e4m3 else ""),
             "parallelism": (f"compressed entries x{world} (128-entry tiles; all-gather of "
                             f"(m, l, O) partials + merge)") if world > 1 else "single GPU",
             "timing": timing,
@@ -927,23 +962,51 @@ def profile_case(args):
         cache = B.PagedCache(2, -(-T // BLOCK), 1, D, torch.bfloat16, 128, device=dev)
         for _ in range(2):
             ops.compress(desc, K, V, cache)
-    elif args.profile == "prefill":
+    elif args.profile in ("prefill", "prefill_gate"):
+        # prefill_gate: the 2 x 128K leg's features (every 4th block x4, fused gate)
         T = args.seqlen
-        Q = torch.randn((1, T, HQ, D), generator=g, device=dev).to(torch.bfloat16)
-        K = torch.randn((1, T, 1, D), generator=g, device=dev).to(torch.bfloat16)
-        V = torch.randn((1, T, 1, D), generator=g, device=dev).to(torch.bfloat16)
+        blk = ((torch.arange(T, device=dev) // BLOCK) % 4 == 3)
+
+        def draw(h):
+            x = torch.randn((1, T, h, D), generator=g, device=dev)
+            if args.profile == "prefill_gate":
+                x[:, blk] *= 4.0
+            return x.to(torch.bfloat16)
+
+        Q, K, V = draw(HQ), draw(1), draw(1)
         desc = ops.desc_for_prefill(Q, K)
+        if args.profile == "prefill_gate":
+            G = torch.sigmoid(torch.randn((1, T, HQ, D), generator=g, device=dev))
+            ops.attach_gate(desc, G.to(torch.bfloat16))
         cache = B.PagedCache(1, -(-T // BLOCK), 1, D, torch.bfloat16, 128, device=dev)
         O = torch.empty_like(Q)
         ops.compress(desc, K, V, cache)
         for _ in range(2):
             ops.prefill(desc, Q, K, V, cache, O=O)
+    elif args.profile == "backward":
+        T = args.seqlen
+        Q = torch.randn((1, T, HQ, D), generator=g, device=dev).to(torch.bfloat16)
+        K = torch.randn((1, T, 1, D), generator=g, device=dev).to(torch.bfloat16)
+        V = torch.randn((1, T, 1, D), generator=g, device=dev).to(torch.bfloat16)
+        dO = torch.randn((1, T, HQ, D), generator=g, device=dev).to(torch.bfloat16)
+        desc = ops.desc_for_prefill(Q, K)
+        cache = B.PagedCache(1, -(-T // BLOCK), 1, D, torch.bfloat16, 128, device=dev)
+        ops.compress(desc, K, V, cache)
+        _, lse, _ = ops.prefill(desc, Q, K, V, cache, want_lse=True)
+        for _ in range(2):
+            ops.prefill_backward(desc, Q, K, V, cache, lse, dO)
     else:
         nseq, ctx = args.nseq, args.ctx
         nent = (ctx - WIN) // BLOCK + 1
-        cache = B.PagedCache(nseq, nent, 1, D, torch.bfloat16, 128, device=dev)
-        cache.kc.normal_(generator=g)
-        cache.vc.normal_(generator=g)
+        e4m3 = args.profile == "decode_e4m3"
+        cache = B.PagedCache(nseq, nent, 1, D, torch.bfloat16, 128, device=dev,
+                             e4m3_scales=E4M3_SCALES if e4m3 else None)
+        if e4m3:
+            _fill_e4m3(cache.kc, g)
+            _fill_e4m3(cache.vc, g)
+        else:
+            cache.kc.normal_(generator=g)
+            cache.vc.normal_(generator=g)
         cache.n_entries.fill_(nent)
         q = torch.randn((nseq, HQ, D), generator=g, device=dev).to(torch.bfloat16)
         rk = torch.randn((nseq, WIN, 1, D), generator=g, device=dev).to(torch.bfloat16)
@@ -977,9 +1040,11 @@ def main():
     ap.add_argument("--with-128k", action="store_true", default=True)
     ap.add_argument("--no-128k", dest="with_128k", action="store_false")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e4m3", action="store_true", help="skip the 8-bit cache decode legs")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--profile", choices=["prefill", "decode", "compress"], default=None,
+    ap.add_argument("--profile", choices=["prefill", "prefill_gate", "decode", "decode_e4m3",
+                                          "compress", "backward"], default=None,
                     help="run a small fixed case for ncu and exit")
     ap.add_argument("--nseq", type=int, default=16)
     ap.add_argument("--ctx", type=int, default=1048576)

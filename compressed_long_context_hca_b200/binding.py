@@ -25,11 +25,13 @@ HCA_ENOSPACE = -3
 HCA_ECUDA = -4
 HCA_BF16 = 0
 HCA_F32 = 1
+HCA_POOL_NATIVE = 0
+HCA_POOL_E4M3 = 1
 HCA_ERR_PAGE_RANGE = 1
 HCA_ERR_CACHE_SHORT = 2
 HCA_ERR_TIMEOUT = 4
 HCA_ERR_CTX_RANGE = 8
-ABI_VERSION = 1
+ABI_VERSION = 2
 
 EXPORTED = ("hca_abi_version", "hca_status_string", "hca_set_gate", "hca_compress",
             "hca_attn_prefill", "hca_attn_prefill_range", "hca_decode_workspace_bytes",
@@ -50,7 +52,8 @@ class HcaDesc(ctypes.Structure):
 class HcaCache(ctypes.Structure):
     _fields_ = [("kc_pool", c_void_p), ("vc_pool", c_void_p), ("page_table", c_void_p),
                 ("n_entries", c_void_p), ("page_entries", c_int32), ("max_pages", c_int32),
-                ("num_pages", c_int32), ("err_word", c_void_p)]
+                ("num_pages", c_int32), ("err_word", c_void_p), ("pool_format", c_int32),
+                ("k_scale", c_float), ("v_scale", c_float)]
 
 
 class HcaError(RuntimeError):
@@ -272,17 +275,20 @@ class PagedCache:
     """Device memory for a paged compressed cache, allocated through torch.
 
     ``page_table`` is a [batch, max_pages] int32 tensor of page ids (any order).
+    ``e4m3_scales=(k_scale, v_scale)`` makes the pools 8-bit (uint8 tensors of e4m3 codes,
+    HCA_POOL_E4M3) with those per-pool scales.
     """
 
     def __init__(self, batch: int, max_entries: int, hkv: int, head_dim: int, dtype,
-                 page_entries: int = 128, page_table=None, device="cuda"):
+                 page_entries: int = 128, page_table=None, device="cuda", e4m3_scales=None):
         import torch
         self.page_entries = page_entries
         self.max_pages = max(1, -(-max_entries // page_entries))
         self.num_pages = batch * self.max_pages
         shape = (self.num_pages, page_entries, hkv, head_dim)
-        self.kc = torch.zeros(shape, dtype=dtype, device=device)
-        self.vc = torch.zeros(shape, dtype=dtype, device=device)
+        pool_dtype = torch.uint8 if e4m3_scales is not None else dtype
+        self.kc = torch.zeros(shape, dtype=pool_dtype, device=device)
+        self.vc = torch.zeros(shape, dtype=pool_dtype, device=device)
         if page_table is None:
             page_table = torch.arange(self.num_pages, dtype=torch.int32).view(batch, -1)
         self.page_table = page_table.to(device=device, dtype=torch.int32).contiguous()
@@ -297,6 +303,10 @@ class PagedCache:
         c.max_pages = self.max_pages
         c.num_pages = self.num_pages
         c.err_word = self.err.data_ptr()
+        if e4m3_scales is not None:
+            c.pool_format = HCA_POOL_E4M3
+            c.k_scale, c.v_scale = float(e4m3_scales[0]), float(e4m3_scales[1])
+        self.e4m3_scales = e4m3_scales
         self.c = c
 
     def entry_rows(self, b: int, n: int):

@@ -8,8 +8,10 @@
 // threads split the row into 16-byte vectors and the block's tokens into `groups`
 // interleaved row sets; partial float32 sums meet in shared memory. Accumulation is
 // float32, the mean is an IEEE division by the token count, rounded once to the storage
-// type.
+// type. An 8-bit cache ([serve fp8] in include/hca.h) stores e4m3(mean / scale): an IEEE
+// float32 division by the pool's scale, then round-to-nearest-even with saturation at 448.
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include "hca_internal.h"
@@ -77,7 +79,28 @@ struct CompressArgs {
   int32_t groups;             // row groups per CTA
   int32_t seqlen, block, first_block, n_blocks;
   int32_t page_entries, max_pages, num_pages;
+  int32_t e4m3;               // pools hold e4m3 codes (one byte per element)
+  float scale[2];             // e4m3: K, V pool scales
 };
+
+// N float32 means -> N e4m3 codes of mean / scale (N = 8 or 4), stored at byte offset
+// `elem` of the pool (8 or 4 bytes, aligned: rows are a multiple of 8 bytes)
+template <int N>
+__device__ __forceinline__ void store_e4m3(uint8_t* pool, int64_t elem, const float* x,
+                                           float scale) {
+  uint32_t w[2] = {0u, 0u};
+#pragma unroll
+  for (int i = 0; i < N; i += 2) {
+    const __nv_fp8x2_storage_t c = __nv_cvt_float2_to_fp8x2(
+        make_float2(__fdiv_rn(x[i], scale), __fdiv_rn(x[i + 1], scale)), __NV_SATFINITE,
+        __NV_E4M3);
+    w[i >> 2] |= (uint32_t)c << (8 * (i & 3));
+  }
+  if (N == 8)
+    *reinterpret_cast<uint2*>(pool + elem) = make_uint2(w[0], w[1]);
+  else
+    *reinterpret_cast<uint32_t*>(pool + elem) = w[0];
+}
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads) compress_kernel(CompressArgs a) {
@@ -142,8 +165,13 @@ __global__ void __launch_bounds__(kThreads) compress_kernel(CompressArgs a) {
         if (a.err_word) atomicOr(a.err_word, kErrPageRange);
       } else {
         const int64_t row = (int64_t)page * a.page_entries + j % a.page_entries;
-        uint4* dst = reinterpret_cast<uint4*>(a.pool[which]) + row * a.row_vecs + vofs + v;
-        *dst = V16::pack(sum);
+        if (a.e4m3) {
+          store_e4m3<N>(static_cast<uint8_t*>(a.pool[which]),
+                        (row * a.row_vecs + vofs + v) * N, sum, a.scale[which]);
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(a.pool[which]) + row * a.row_vecs + vofs + v;
+          *dst = V16::pack(sum);
+        }
       }
     }
     __syncthreads();
@@ -175,6 +203,9 @@ cudaError_t launch_compress(const hca_desc& d, const void* K, const void* V,
   a.page_entries = c.page_entries;
   a.max_pages = c.max_pages;
   a.num_pages = c.num_pages;
+  a.e4m3 = c.pool_format == HCA_POOL_E4M3 ? 1 : 0;
+  a.scale[0] = c.k_scale;
+  a.scale[1] = c.v_scale;
   // Few blocks (a decode step completing one block per sequence): split each row's columns
   // over up to 8 CTAs until there are about two CTAs per SM, so that enough loads are in
   // flight; each CTA then walks the block's rows over fewer columns.

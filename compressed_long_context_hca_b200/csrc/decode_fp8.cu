@@ -1,0 +1,826 @@
+// decode_fp8.cu -- one HCA decode step over an 8-bit (e4m3) compressed cache, on tcgen05
+// tensor cores, followed (with several splits) by the merge of the 16-bit decode.
+//
+// Operation ([news 二.1] / [analysis 1] / [gate] / [serve fp8] in include/hca.h): the newest
+// token t = ctx_len - 1 attends with one softmax to the compressed entries j < n_c(t),
+// stored as e4m3 codes with one float32 scale per pool (value = value(code) * scale), and
+// to the last `window` raw tokens, which stay bf16 in a ring of `window` slots.
+//
+// Design for sm_100a (HBM-bound; a compressed tile of 128 entries is 64 KB of keys and
+// 64 KB of values, half of the 16-bit cache):
+//  * Scores of a compressed tile run on kind::f8f6f4 UMMAs straight from the stored codes
+//    (K-major, as TMA lands them). The query is carried exactly as two e4m3 parts: with
+//    r_h a power of two per head that puts the head's largest |q| in [128, 256),
+//    q / r_h = Q1 + Q2 / 16, Q1 = e4m3(q / r_h), Q2 = e4m3(16 (q / r_h - Q1)). A bf16 q has
+//    8 significant bits; Q1 takes the top 4 and the remainder has at most 4, so both parts
+//    are exact for every element within 2^13 of the head's largest (below that the part
+//    error is under 2^-21 of the largest |q|). S1 = Q1 K and S2 = Q2 K go to two TMEM
+//    accumulators; the softmax forms s = (S1 + S2 / 16) * r_h * k_scale * scale.
+//  * P.V runs on kind::f16 with f16 operands. Converter warps widen each 16-key group of
+//    e4m3 values to f16 (exact: every e4m3 value is an f16 value) into a 4-deep ring of
+//    MN-major 128-byte-swizzled buffers, with the global loads of the next four groups in
+//    flight in registers. P is split into f16 hi + lo parts (two UMMAs) and pre-scaled by
+//    2^7, so that small P stay clear of the f16 subnormal range while the largest (2^15
+//    between lazy rescales) stays finite. O accumulates in units of the V codes; v_scale
+//    multiplies it once at the end.
+//  * The ring tile (the raw window, bf16) is the last tile of the last split and runs the
+//    16-bit way inside the same CTA: once the last e4m3 score MMA has completed, the bf16
+//    query replaces Q1/Q2 in shared memory, its scores accumulate in S1 (kind::f16 bf16),
+//    its P goes to bf16 hi + lo parts divided by v_scale (O stays in code units), and its
+//    values land in the same V buffers by TMA.
+//  * Roles: warp 0 issues the K loads (TMA boxes of 128 rows x 128 bytes, a 4-slot ring)
+//    and the bf16 query of the ring tile; warp 1 issues the UMMAs; warps 2-5 run the
+//    softmax (lazy rescale, as the 16-bit kernel) and the epilogue; warps 6-9 prepare
+//    Q1/Q2 and widen V.
+//  * TMEM: O (64 x 512 f32, M = 64 layout) in lanes 0-15 of each 32-lane subpartition;
+//    two score buffers of S1 | S2 (128 columns each) in lanes 16-31.
+//  * All mbarrier waits are bounded (HCA_ERR_TIMEOUT on give-up); on give-up every issuing
+//    thread waits (bounded) for its own copies still in flight before the CTA leaves.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <string.h>
+
+#include "decode_keys.cuh"
+#include "hca_internal.h"
+#include "sm100.cuh"
+#include "tmap.h"
+
+namespace hca {
+namespace {
+
+using namespace dkeys;
+
+constexpr int kM = 64;    // head rows
+constexpr int kD = 512;
+constexpr int kThreads = 320;  // TMA warp, UMMA warp, 4 softmax warps, 4 converter warps
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kLaneS = 16u << 16;   // lane offset of the score accumulators
+
+constexpr uint32_t kQChunkBytes = kM * 128;     // 8 KB: 64 rows x 128 bytes (either type)
+constexpr uint32_t kQPartBytes = 4 * kQChunkBytes;  // 32 KB: one e4m3 part of the query
+constexpr uint32_t kQ16Bytes = 8 * kQChunkBytes;    // 64 KB: the bf16 query
+constexpr uint32_t kPChunkBytes = kM * 128;     // 8 KB: 64 rows x 64 keys (16-bit)
+constexpr uint32_t kPBytes = 2 * kPChunkBytes;  // 16 KB: one part of P (128 keys)
+constexpr int kKStages = 4;
+constexpr uint32_t kKSlot = 128 * 128;          // 16 KB: 128 key rows x one 128-byte chunk
+constexpr int kVStages = 4;
+constexpr uint32_t kVChunkBytes = 16 * 128;     // 2 KB: 16 keys x 64 values (16-bit)
+constexpr uint32_t kVSlot = 8 * kVChunkBytes;   // 16 KB: 16 keys x 512 values
+
+constexpr uint32_t kOffQ = 0;                           // Q1 | Q2, later the bf16 query
+constexpr uint32_t kOffP = kQ16Bytes;                   // P hi | P lo
+constexpr uint32_t kOffK = kOffP + 2 * kPBytes;
+constexpr uint32_t kOffV = kOffK + kKStages * kKSlot;
+constexpr uint32_t kOffBar = kOffV + kVStages * kVSlot;
+constexpr uint32_t kOffRowScale = kOffBar + 256;        // 64 floats
+constexpr uint32_t kSmemBytes = kOffRowScale + 256 + 1024;
+static_assert(2 * kQPartBytes == kQ16Bytes, "Q1 | Q2 and the bf16 query share one region");
+
+constexpr float kRescaleThreshold = 8.0f;  // log2 units, as the 16-bit kernel
+constexpr float kPShift = 7.0f;            // P = 2^(s - max + 7) <= 2^15 between rescales
+// End of a CTA: O is staged row-major in the P + K + V region (free once the last PV is
+// done) with a padded row stride, then written out coalesced.
+constexpr int kORow = kD + 4;
+constexpr uint32_t kOffStage = kOffP;
+static_assert(kM * kORow * 4 + 3 * kM * 4 <= kOffBar - kOffStage, "staging space");
+
+struct Params8 {
+  CUtensorMap tmK8;  // e4m3 Kc pool {128 bytes, rows, 4 chunks}, box {128, 128, 1}
+  CUtensorMap tmQb;  // bf16 Q {64, batch*hq, 8}, box {64, 64, 4}
+  CUtensorMap tmRk;  // bf16 ring K {64, batch*W, 8}, box {64, 128, 1}
+  CUtensorMap tmRv;  // bf16 ring V {64, batch*W, 8}, box {64, 16, 8}
+  const __nv_bfloat16* Q;  // [batch, hq, 512]
+  const uint8_t* vc8;      // e4m3 Vc pool [rows, 512]
+  const int32_t* ctx_len;
+  const int32_t* page_table;
+  const int32_t* n_entries;
+  int32_t* err_word;
+  float* ws_ml;  // [nseq, nsplit, hq, 2]
+  float* ws_o;   // [nseq, nsplit, hq, 512]
+  __nv_bfloat16* O;  // nsplit == 1 && !partial: the final output
+  float* lse;
+  const __nv_bfloat16* gate;
+  int64_t gs0, gs2;
+  int32_t nseq, seqlen, hq, W, block, PE, max_pages, num_pages, nsplit;
+  int32_t e0, e1, with_ring, partial;
+  float scale_log2, k_scale, v_scale;
+};
+
+struct Bars8 {
+  uint64_t q_ready;   // Q1, Q2 and the row scales written (converters)
+  uint64_t qb_full;   // bf16 query of the ring tile landed (TMA)
+  uint64_t q8_free;   // the last e4m3 score MMA completed: the query region may be reused
+  uint64_t k_full[kKStages], k_empty[kKStages];
+  uint64_t v_full[kVStages], v_empty[kVStages];
+  uint64_t s_full[2], p_full[2], o_done[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(Bars8) <= 256, "barrier block too large");
+
+__device__ __forceinline__ uint4 ld_stream16(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// two e4m3 codes (low byte first) -> f16x2 (exact)
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)two_codes, __NV_E4M3);
+  return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+
+// f16 pair split: hi = RNE f16 of each value, lo = RNE f16 of the remainder (exact in f32)
+__device__ __forceinline__ void split_f16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  const __half2 h = __floats2half2_rn(a, b);
+  const float2 hf = __half22float2(h);
+  const __half2 l = __floats2half2_rn(a - hf.x, b - hf.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+__device__ __forceinline__ void named_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// Named barrier that also returns the AND of `pred` over the participating threads, so
+// that a loop's continue/stop decision is the same in every warp that takes part.
+__device__ __forceinline__ bool named_sync_and(int id, int threads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.cta.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(threads)
+      : "memory");
+  return r != 0;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_constant__ Params8 p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sQ = smem + kOffQ;
+  uint8_t* sP = smem + kOffP;
+  uint8_t* sK = smem + kOffK;
+  uint8_t* sV = smem + kOffV;
+  Bars8* bars = reinterpret_cast<Bars8*>(smem + kOffBar);
+  float* sRS = reinterpret_cast<float*>(smem + kOffRowScale);
+  volatile int* abort = &bars->abort;
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const int b = blockIdx.y;
+  const int split = blockIdx.x;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_ready, 1);
+    mbar_init(&bars->qb_full, 1);
+    mbar_init(&bars->q8_free, 1);
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&bars->s_full[x], 1);
+      mbar_init(&bars->p_full[x], 4);
+      mbar_init(&bars->o_done[x], 1);
+    }
+    mbar_init(&bars->drain, 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  pdl_wait();
+  pdl_trigger();
+  const Seq sq = make_seq(p, b, split);
+  const int ntiles = sq.j1 - sq.j0;
+  const bool has_ring = ntiles > 0 && tile_of(p, sq, sq.j1 - 1).kind == kRing;
+  const int nct = ntiles - (has_ring ? 1 : 0);  // compressed (e4m3) tiles of this split
+
+  if (ntiles <= 0) {
+    // empty split: an all-zero partial that the merge skips
+    for (int h = threadIdx.x; h < p.hq; h += blockDim.x) {
+      float* ml = p.ws_ml + (((int64_t)b * p.nsplit + split) * p.hq + h) * 2;
+      ml[0] = -INFINITY;
+      ml[1] = 0.f;
+    }
+  } else if (warp == 0) {
+    // ------------------------------------------------------------------ K producer
+    if (elect_one()) {
+      const uint64_t pol = policy_evict_first();  // every cache row is read once
+      if (split == 0 && p.err_word) {
+        const int ctx = p.ctx_len[b];
+        if (ctx < 1 || ctx > p.seqlen) atomicOr(p.err_word, kErrCtxRange);
+        const int x = sq.t + 1 - p.W;
+        if ((x < 0 ? 0 : x / p.block) > p.n_entries[b]) atomicOr(p.err_word, kErrCacheShort);
+      }
+      uint32_t cnt = 0;  // loads issued
+      bool ok = true, q_issued = false;
+      auto load = [&](const CUtensorMap* map, int row, int chunk) -> bool {
+        const uint32_t s = cnt % kKStages;
+        if (cnt >= (uint32_t)kKStages &&
+            !mbar_wait(&bars->k_empty[s], ((cnt / kKStages) - 1) & 1, abort))
+          return false;
+        mbar_expect_tx(&bars->k_full[s], kKSlot);
+        tma_load_3d(sK + s * kKSlot, map, &bars->k_full[s], 0, row, chunk, pol);
+        ++cnt;
+        return true;
+      };
+      for (int j = sq.j0; j < sq.j1 && ok; ++j) {
+        const Tile t = tile_of(p, sq, j);
+        if (t.kind == kCompressed) {
+          int page = p.page_table[(int64_t)b * p.max_pages + t.key0 / p.PE];
+          if (page < 0 || page >= p.num_pages) {
+            if (p.err_word) atomicOr(p.err_word, kErrPageRange);
+            page = 0;
+          }
+          const int row = page * p.PE + t.key0 % p.PE;
+          for (int q = 0; q < 4 && ok; ++q) ok = load(&p.tmK8, row, q);
+        } else {
+          // the bf16 query replaces Q1/Q2 once the last e4m3 score MMA has completed
+          if (!(ok = mbar_wait(&bars->q8_free, 0, abort))) break;
+          mbar_expect_tx(&bars->qb_full, kQ16Bytes);
+          for (int h = 0; h < 2; ++h)
+            tma_load_3d(sQ + h * (kQ16Bytes / 2), &p.tmQb, &bars->qb_full, 0, b * p.hq, 4 * h,
+                        pol);
+          q_issued = true;
+          for (int q = 0; q < 8 && ok; ++q) ok = load(&p.tmRk, b * p.W, q);
+        }
+      }
+      if (!ok) {
+        bars->abort = 1;
+        if (p.err_word) atomicOr(p.err_word, kErrTimeout | (1 << 9));
+        // load n could only be issued once load n - 4 had been consumed: at most the last
+        // four are in flight, plus the bf16 query
+        volatile int no_abort = 0;
+        const uint32_t first = cnt > (uint32_t)kKStages ? cnt - kKStages : 0;
+        for (uint32_t n = first; n < cnt; ++n)
+          mbar_wait(&bars->k_full[n % kKStages], (n / kKStages) & 1, &no_abort, 100000000ull);
+        if (q_issued) mbar_wait(&bars->qb_full, 0, &no_abort, 100000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ UMMA issuer
+    // Order: S(0), then per step c >= 1: S(c) (if any), PV(c - 1), as the 16-bit kernel.
+    if (elect_one()) {
+      bool ok = mbar_wait(&bars->q_ready, 0, abort);
+      tc_fence_after();
+      uint32_t ck = 0, cv = 0;  // K slots, V groups consumed
+      bool q8_released = false;
+      const uint32_t qbase = smem_u32(sQ);
+      const uint32_t pbase = smem_u32(sP);
+      const uint32_t kbase = smem_u32(sK);
+      const uint32_t vbase = smem_u32(sV);
+      for (int c = 0; c <= ntiles && ok; ++c) {
+        if (c < ntiles) {
+          const Tile t = tile_of(p, sq, sq.j0 + c);
+          const uint32_t sb = tmem + kLaneS + (c & 1) * 256;  // S1 at sb, S2 at sb + 128
+          if (t.kind == kCompressed) {
+            const uint32_t idesc = idesc_e4m3_f32(kM, t.n);
+            for (int q = 0; q < 4 && ok; ++q) {
+              const uint32_t s = ck % kKStages;
+              if (!(ok = mbar_wait(&bars->k_full[s], (ck / kKStages) & 1, abort))) break;
+              tc_fence_after();
+              const uint32_t kaddr = kbase + s * kKSlot;
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {  // K = 32 codes per UMMA
+                const uint64_t kd = sdesc_sw128(kaddr + kk * 32, 16, 1024);
+                const uint32_t acc = (q | kk) != 0;
+                const uint32_t qa = qbase + q * kQChunkBytes + kk * 32;
+                umma_ss_f8(sb, sdesc_sw128(qa, 16, 1024), kd, idesc, acc);
+                umma_ss_f8(sb + 128, sdesc_sw128(qa + kQPartBytes, 16, 1024), kd, idesc, acc);
+              }
+              umma_commit(&bars->k_empty[s]);
+              ++ck;
+            }
+          } else {
+            if (!q8_released) {  // a split whose only tile is the ring tile
+              umma_commit(&bars->q8_free);
+              q8_released = true;
+            }
+            if (!(ok = mbar_wait(&bars->qb_full, 0, abort))) break;
+            tc_fence_after();
+            const uint32_t idesc = idesc_bf16_f32(kM, t.n, false);
+            for (int q = 0; q < 8 && ok; ++q) {
+              const uint32_t s = ck % kKStages;
+              if (!(ok = mbar_wait(&bars->k_full[s], (ck / kKStages) & 1, abort))) break;
+              tc_fence_after();
+              const uint32_t kaddr = kbase + s * kKSlot;
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)  // K = 16 bf16 per UMMA
+                umma_ss(sb, sdesc_sw128(qbase + q * kQChunkBytes + kk * 32, 16, 1024),
+                        sdesc_sw128(kaddr + kk * 32, 16, 1024), idesc, (q | kk) != 0);
+              umma_commit(&bars->k_empty[s]);
+              ++ck;
+            }
+          }
+          if (ok) umma_commit(&bars->s_full[c & 1]);
+          // after the last e4m3 score MMAs of a split that ends with the ring tile, the
+          // bf16 query may replace Q1/Q2 as soon as they complete
+          if (ok && has_ring && c + 1 == nct && !q8_released) {
+            umma_commit(&bars->q8_free);
+            q8_released = true;
+          }
+        }
+        if (c >= 1 && ok) {
+          const int pc = c - 1;
+          if (!(ok = mbar_wait(&bars->p_full[pc & 1], (pc >> 1) & 1, abort))) break;
+          tc_fence_after();
+          const Tile t = tile_of(p, sq, sq.j0 + pc);
+          const uint32_t idesc = t.kind == kCompressed ? idesc_f16_f32(kM, 256, true)
+                                                       : idesc_bf16_f32(kM, 256, true);
+          // O[:, 256 h .. 256 h + 255] += P(group) V(group, columns of half h): one N = 256
+          // UMMA per half and part of P
+          for (int g = 0; g < t.n / 16 && ok; ++g) {
+            const uint32_t s = cv % kVStages;
+            if (!(ok = mbar_wait(&bars->v_full[s], (cv / kVStages) & 1, abort))) break;
+            tc_fence_after();
+            const uint32_t vaddr = vbase + s * kVSlot;
+            const uint32_t paddr = pbase + (g >> 2) * kPChunkBytes + (g & 3) * 32;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint64_t vd = sdesc_sw128(vaddr + h * 4 * kVChunkBytes, kVChunkBytes, 1024);
+              umma_ss(tmem + h * 256, sdesc_sw128(paddr, 16, 1024), vd, idesc,
+                      (pc > 0 || g > 0));
+              umma_ss(tmem + h * 256, sdesc_sw128(paddr + kPBytes, 16, 1024), vd, idesc, 1u);
+            }
+            umma_commit(&bars->v_empty[s]);
+            ++cv;
+          }
+          if (ok) umma_commit(&bars->o_done[pc & 1]);
+        }
+      }
+      if (!ok) {
+        bars->abort = 1;
+        if (p.err_word) atomicOr(p.err_word, kErrTimeout | (1 << 11));
+      }
+      volatile int no_abort = 0;
+      umma_commit(&bars->drain);
+      mbar_wait(&bars->drain, 0, &no_abort, 100000000ull);
+    }
+  } else if (warp >= 2 && warp < 6) {
+    // ------------------------------------------------------------------ softmax + partials
+    // Lane l + 16 of a warp holds score row quad * 16 + l; lane l (< 16) holds the O row of
+    // the same head. The protocol is that of the 16-bit kernel: per chunk c (one tile):
+    // wait S(c); row max; wait PV(c - 1); lazy rescale of O; P(c); arrive p_full.
+    const int quad = warp & 3;
+    const bool s_lane = lane >= 16;
+    const int hrow = quad * 16 + (lane & 15);
+    const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+    bool ok = __all_sync(0xffffffffu, mbar_wait(&bars->q_ready, 0, abort));
+    const float rs8 = sRS[hrow];            // r_h * k_scale * scale * log2(e)
+    const float inv_vs = 1.f / p.v_scale;   // ring values enter O in V-code units
+    float base = -INFINITY, l = 0.f;
+    for (int c = 0; c < ntiles && ok; ++c) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[c & 1], (c >> 1) & 1, abort));
+      if (!ok) break;
+      tc_fence_after();
+      const Tile tl = tile_of(p, sq, sq.j0 + c);
+      const bool f8 = tl.kind == kCompressed;
+      const uint32_t sbuf = tmem + lane_addr + (c & 1) * 256;
+      // visible columns: a prefix of a compressed tile, or ring slots 0..min(W,t+1)-1
+      const int vhi = f8 ? min(tl.n, sq.e1 - tl.key0) : min(p.W, sq.t + 1);
+      const uint32_t vlen = vhi > 0 ? (uint32_t)vhi : 0u;
+      const float rs = f8 ? rs8 : p.scale_log2;
+      // 32 raw scores of columns q*32 .. q*32+31: S1 + S2 / 16 (e4m3 tile) or S1 (ring)
+      auto load_scores = [&](int q, uint32_t (&v)[32]) {
+        tmem_ld32(sbuf + q * 32, v);
+        if (f8) {
+          uint32_t w[32];
+          tmem_ld32(sbuf + 128 + q * 32, w);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            v[e] = __float_as_uint(fmaf(__uint_as_float(w[e]), 0.0625f, __uint_as_float(v[e])));
+        } else {
+          tmem_wait_ld();
+        }
+      };
+      // pass 1: row max over the visible keys (branch-free selects)
+      float mx[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
+      for (int q = 0; q < kTN / 32; ++q) {
+        if (q * 32 >= tl.n) break;
+        uint32_t v[32];
+        load_scores(q, v);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const bool in = (uint32_t)(q * 32 + e) < vlen;
+          mx[e & 7] = fmaxf(mx[e & 7], in ? __uint_as_float(v[e]) : -INFINITY);
+        }
+      }
+      const float cmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) *
+                         rs;
+      const bool grow = s_lane && (c == 0 || cmax > base + kRescaleThreshold);
+      float factor = 1.f;
+      if (grow) {
+        factor = c == 0 ? 1.f : fast_exp2(base - cmax);
+        l *= factor;
+        base = cmax;
+      }
+      if (c > 0) {
+        // PV(c - 1) done: the P buffer is free and O holds every earlier chunk
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait(&bars->o_done[(c - 1) & 1], ((c - 1) >> 1) & 1, abort));
+        if (!ok) break;
+      }
+      if (c > 0 && __any_sync(0xffffffffu, grow)) {
+        // the 32-lane read-modify-write also rewrites the score lanes (unchanged): no UMMA
+        // may be in flight, so S(c + 1) (if issued) must have completed. PV(c) waits for
+        // our p_full.
+        if (c + 1 < ntiles)
+          ok = mbar_wait(&bars->s_full[(c + 1) & 1], ((c + 1) >> 1) & 1, abort);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        const float f_o = __shfl_sync(0xffffffffu, factor, (lane & 15) + 16);
+        const float f = s_lane ? 1.f : f_o;
+#pragma unroll 1
+        for (int q = 0; q < kD / 32; ++q) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_addr + q * 32, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
+          tmem_st32(tmem + lane_addr + q * 32, v);
+        }
+        tmem_wait_st();
+      }
+      // pass 2: P = 2^(s - base + 7) -> hi + lo parts in two K-major 128B-swizzled buffers:
+      // f16 for an e4m3 tile; bf16 times 1/v_scale for the ring tile
+      const float bb = base == -INFINITY ? 0.f : base - kPShift;
+      float ps[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int q = 0; q < kTN / 32; ++q) {
+        if (q * 32 >= tl.n) break;
+        uint32_t v[32];
+        load_scores(q, v);
+        if (s_lane) {
+          uint32_t pk[16], pl[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int c0 = q * 32 + 2 * e;
+            const float p0 = (uint32_t)c0 < vlen
+                                 ? fast_exp2(fmaf(__uint_as_float(v[2 * e]), rs, -bb))
+                                 : 0.f;
+            const float p1 = (uint32_t)(c0 + 1) < vlen
+                                 ? fast_exp2(fmaf(__uint_as_float(v[2 * e + 1]), rs, -bb))
+                                 : 0.f;
+            if (f8)
+              split_f16x2(p0, p1, pk[e], pl[e]);
+            else
+              split_bf16x2(p0 * inv_vs, p1 * inv_vs, pk[e], pl[e]);
+            ps[e & 3] += p0 + p1;
+          }
+          // keys q*32 .. -> 64-key P chunk q/2, 16-byte units (q&1)*4 + w
+          uint8_t* rowp = sP + (q >> 1) * kPChunkBytes + hrow * 128;
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const int u = (q & 1) * 4 + w;
+            const int us = u ^ (hrow & 7);
+            *reinterpret_cast<uint4*>(rowp + us * 16) =
+                make_uint4(pk[4 * w], pk[4 * w + 1], pk[4 * w + 2], pk[4 * w + 3]);
+            *reinterpret_cast<uint4*>(rowp + kPBytes + us * 16) =
+                make_uint4(pl[4 * w], pl[4 * w + 1], pl[4 * w + 2], pl[4 * w + 3]);
+          }
+        }
+      }
+      l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->p_full[c & 1]);
+    }
+    // the last PV's commit covers every earlier UMMA of this CTA
+    if (ok) ok = mbar_wait(&bars->o_done[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, abort);
+    ok = __all_sync(0xffffffffu, ok);
+    float* sO = reinterpret_cast<float*>(smem + kOffStage);  // [64][kORow]
+    float* sM = sO + kM * kORow;                               // reference max (log2 units)
+    float* sL = sM + kM;                                       // row sum
+    float* sInv = sL + kM;                                     // v_scale / row sum
+    if (ok) {
+      tc_fence_after();
+      if (s_lane) {
+        sM[hrow] = base - kPShift;  // l and O carry the 2^7 of P
+        sL[hrow] = l;
+        sInv[hrow] = 1.f / l;
+      }
+      const float vs = p.v_scale;
+      float* orow = sO + hrow * kORow;
+#pragma unroll 1
+      for (int q = 0; q < kD / 32; ++q) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_addr + q * 32, v);
+        tmem_wait_ld();
+        if (!s_lane) {
+          float4* o4 = reinterpret_cast<float4*>(orow + q * 32);
+#pragma unroll
+          for (int w = 0; w < 8; ++w)
+            o4[w] = make_float4(__uint_as_float(v[4 * w]) * vs, __uint_as_float(v[4 * w + 1]) * vs,
+                                __uint_as_float(v[4 * w + 2]) * vs,
+                                __uint_as_float(v[4 * w + 3]) * vs);
+        }
+      }
+    } else {
+      bars->abort = 1;
+      if (p.err_word) atomicOr(p.err_word, kErrTimeout | (1 << 12));
+    }
+    named_sync(1, 128);
+    const int tid = threadIdx.x - 64;  // 0..127 over the four softmax warps
+    if (p.nsplit == 1 && !p.partial) {
+      // final output: O / l, gate, bf16 in 16-byte units; lse in natural log
+      __nv_bfloat16* ob = p.O + (int64_t)b * p.hq * kD;
+#pragma unroll 4
+      for (int i = tid; i < p.hq * (kD / 8); i += 128) {
+        const int h = i / (kD / 8);
+        const int c = 8 * (i % (kD / 8));
+        const float4 x0 = *reinterpret_cast<const float4*>(sO + h * kORow + c);
+        const float4 x1 = *reinterpret_cast<const float4*>(sO + h * kORow + c + 4);
+        const float inv = sInv[h];
+        float o[8] = {x0.x * inv, x0.y * inv, x0.z * inv, x0.w * inv,
+                      x1.x * inv, x1.y * inv, x1.z * inv, x1.w * inv};
+        if (p.gate) {
+          const __nv_bfloat162* gp = reinterpret_cast<const __nv_bfloat162*>(
+              p.gate + (int64_t)b * p.gs0 + (int64_t)h * p.gs2 + c);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 g = __bfloat1622float2(gp[k]);
+            o[2 * k] *= g.x;
+            o[2 * k + 1] *= g.y;
+          }
+        }
+        *reinterpret_cast<uint4*>(ob + (int64_t)h * kD + c) =
+            make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
+                       pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
+      }
+      if (p.lse)
+        for (int h = tid; h < p.hq; h += 128)
+          p.lse[(int64_t)b * p.hq + h] = (sM[h] + __log2f(sL[h])) * 0.69314718055994531f;
+    } else {
+      // split partial: unnormalised O (value units), (reference max, sum) per head
+      const int64_t slot0 = ((int64_t)b * p.nsplit + split) * p.hq;
+      float* ob = p.ws_o + slot0 * kD;
+      for (int i = tid; i < p.hq * (kD / 4); i += 128) {
+        const int h = i / (kD / 4);
+        const int c = 4 * (i % (kD / 4));
+        *reinterpret_cast<float4*>(ob + (int64_t)h * kD + c) =
+            *reinterpret_cast<const float4*>(sO + h * kORow + c);
+      }
+      for (int h = tid; h < p.hq; h += 128) {
+        p.ws_ml[(slot0 + h) * 2] = sM[h];
+        p.ws_ml[(slot0 + h) * 2 + 1] = sL[h];
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ converters
+    const int ct = threadIdx.x - 192;  // 0..127
+    const int cw = ct >> 5;
+    // (1) Q1, Q2 and the per-head scale: two threads per head row, 256 elements each
+    {
+      const int h = ct >> 1, half = ct & 1;
+      const bool live = h < p.hq;
+      const __nv_bfloat16* qrow = p.Q + ((int64_t)b * p.hq + (live ? h : 0)) * kD + half * 256;
+      float amax = 0.f;
+      if (live)
+        for (int i = 0; i < 32; ++i) {
+          const uint4 x = *reinterpret_cast<const uint4*>(qrow + 8 * i);
+          const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&x);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 f = __bfloat1622float2(x2[k]);
+            amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+          }
+        }
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      // r_h = 2^e puts the head's largest |q| / r_h in [128, 256)
+      const int e = amax > 0.f ? ilogbf(amax) - 7 : 0;
+      for (int u = 0; u < 16; ++u) {  // 16-element units
+        uint32_t w1[4] = {0u, 0u, 0u, 0u}, w2[4] = {0u, 0u, 0u, 0u};
+        if (live) {
+#pragma unroll
+          for (int hv = 0; hv < 2; ++hv) {
+            const uint4 x = *reinterpret_cast<const uint4*>(qrow + 16 * u + 8 * hv);
+            const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&x);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const float2 f = __bfloat1622float2(x2[k]);
+              const float a0 = ldexpf(f.x, -e), a1 = ldexpf(f.y, -e);
+              const __nv_fp8x2_storage_t q1 =
+                  __nv_cvt_float2_to_fp8x2(make_float2(a0, a1), __NV_SATFINITE, __NV_E4M3);
+              const __half2_raw h1 = __nv_cvt_fp8x2_to_halfraw2(q1, __NV_E4M3);
+              const float2 v1 = __half22float2(__half2(h1));
+              const __nv_fp8x2_storage_t q2 = __nv_cvt_float2_to_fp8x2(
+                  make_float2(16.f * (a0 - v1.x), 16.f * (a1 - v1.y)), __NV_SATFINITE, __NV_E4M3);
+              const int pos = hv * 8 + 2 * k;  // code index within the 16-byte unit
+              w1[pos >> 2] |= (uint32_t)q1 << (8 * (pos & 3));
+              w2[pos >> 2] |= (uint32_t)q2 << (8 * (pos & 3));
+            }
+          }
+        }
+        const int elem = half * 256 + 16 * u;
+        const uint32_t off = (elem >> 7) * kQChunkBytes + h * 128 +
+                             ((((elem & 127) >> 4) ^ (h & 7)) << 4);
+        *reinterpret_cast<uint4*>(sQ + off) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+        *reinterpret_cast<uint4*>(sQ + kQPartBytes + off) = make_uint4(w2[0], w2[1], w2[2], w2[3]);
+      }
+      if (half == 0) sRS[h] = ldexpf(p.scale_log2 * p.k_scale, e);
+    }
+    fence_proxy_async_smem();
+    named_sync(2, 128);
+    if (ct == 0) mbar_arrive(&bars->q_ready);
+
+    // (2) V groups of 16 keys in key order: e4m3 tiles widened here, the ring tile by TMA.
+    // Thread (cw, lane) handles keys kr and kr + 8 of a group at values 32*c32 .. +31.
+    const int kr = lane & 7;
+    const int c32 = cw * 4 + (lane >> 3);
+    const int gc = nct > 0 ? (nct - 1) * 8 + tile_of(p, sq, sq.j0 + nct - 1).n / 16 : 0;
+    // global source of group n (n < gc) for this thread's two keys; invalid keys read as 0
+    auto fetch = [&](int n, uint4 (&r)[4]) {
+      if (n >= gc) return;
+      const Tile t = tile_of(p, sq, sq.j0 + (n >> 3));
+      int page = p.page_table[(int64_t)b * p.max_pages + t.key0 / p.PE];
+      if (page < 0 || page >= p.num_pages) page = 0;  // flagged by the K producer
+      const int vlen = min(t.n, sq.e1 - t.key0);
+      const int k0 = (n & 7) * 16 + kr;
+      const uint8_t* src =
+          p.vc8 + ((int64_t)page * p.PE + t.key0 % p.PE + k0) * kD + c32 * 32;
+#pragma unroll
+      for (int it = 0; it < 2; ++it) {
+        if (k0 + 8 * it < vlen) {
+          r[2 * it] = ld_stream16(src + it * 8 * kD);
+          r[2 * it + 1] = ld_stream16(src + it * 8 * kD + 16);
+        } else {
+          r[2 * it] = make_uint4(0, 0, 0, 0);
+          r[2 * it + 1] = make_uint4(0, 0, 0, 0);
+        }
+      }
+    };
+    bool ok = true;
+    uint4 buf[4][4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) fetch(u, buf[u]);
+    for (int n0 = 0; n0 < gc && ok; n0 += 4) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int n = n0 + u;  // group n uses V slot u = n % 4
+        if (n < gc && ok) {
+          bool w_ok = true;
+          if (n >= kVStages)
+            w_ok = __all_sync(0xffffffffu,
+                              mbar_wait(&bars->v_empty[u], ((n / kVStages) - 1) & 1, abort));
+          if (w_ok) {
+            uint8_t* slot = sV + u * kVSlot;
+#pragma unroll
+            for (int it = 0; it < 2; ++it) {
+              const int k = kr + 8 * it;
+              uint8_t* rowp = slot + (c32 >> 1) * kVChunkBytes + it * 1024 + kr * 128;
+              const uint4 lo = buf[u][2 * it], hi = buf[u][2 * it + 1];
+              const uint32_t cw8[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+              for (int w = 0; w < 4; ++w) {
+                const uint32_t a = cw8[2 * w], bq = cw8[2 * w + 1];
+                const int unit = ((c32 & 1) << 2) + w;
+                *reinterpret_cast<uint4*>(rowp + ((unit ^ (k & 7)) << 4)) =
+                    make_uint4(e4m3x2_to_f16x2(a & 0xffffu), e4m3x2_to_f16x2(a >> 16),
+                               e4m3x2_to_f16x2(bq & 0xffffu), e4m3x2_to_f16x2(bq >> 16));
+              }
+            }
+            fence_proxy_async_smem();
+          }
+          // every converter thread arrives here once per group; the barrier's AND makes
+          // the stop decision (a give-up in any warp, or an abort raised by another role)
+          // the same in all four warps, so none is left waiting at the next barrier
+          ok = named_sync_and(2, 128, w_ok && !*abort);
+          if (ok && ct == 0) mbar_arrive(&bars->v_full[u]);
+          if (ok) fetch(n + 4, buf[u]);
+        }
+      }
+    }
+    if (has_ring && ok && ct == 0) {
+      // the raw window's values, bf16, one TMA box of 16 rows x 512 values per group
+      const uint64_t pol = policy_evict_first();
+      const int ng = round16(p.W) / 16;
+      uint32_t issued = 0;
+      for (int g = 0; g < ng && ok; ++g) {
+        const uint32_t n = (uint32_t)(gc + g);
+        const uint32_t s = n % kVStages;
+        if (n >= (uint32_t)kVStages &&
+            !(ok = mbar_wait(&bars->v_empty[s], ((n / kVStages) - 1) & 1, abort)))
+          break;
+        mbar_expect_tx(&bars->v_full[s], kVSlot);
+        tma_load_3d(sV + s * kVSlot, &p.tmRv, &bars->v_full[s], 0, b * p.W + 16 * g, 0, pol);
+        ++issued;
+      }
+      if (!ok) {
+        bars->abort = 1;
+        if (p.err_word) atomicOr(p.err_word, kErrTimeout | (1 << 13));
+        volatile int no_abort = 0;
+        const uint32_t end = (uint32_t)gc + issued;
+        const uint32_t first = issued > (uint32_t)kVStages ? end - kVStages : (uint32_t)gc;
+        for (uint32_t n = first; n < end; ++n)
+          mbar_wait(&bars->v_full[n % kVStages], (n / kVStages) & 1, &no_abort, 100000000ull);
+      }
+    }
+    if (!ok && ct == 0) {
+      bars->abort = 1;
+      if (p.err_word) atomicOr(p.err_word, kErrTimeout | (1 << 13));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_decode_fp8(const hca_desc& d, const void* Q, const int32_t* ctx_len,
+                              const hca_cache& c, const void* ring_k, const void* ring_v,
+                              const DecodePart& part, void* O, float* lse, void* ws,
+                              cudaStream_t s) {
+  Params8 p;
+  memset(&p, 0, sizeof(p));
+  const int nsplit = part_num_splits(d, part);
+  cudaError_t e;
+  const uint64_t rowsC = (uint64_t)c.num_pages * c.page_entries;
+  const uint64_t rowsR = (uint64_t)d.batch * d.window;
+  if ((e = encode_u8_chunks(&p.tmK8, c.kc_pool, rowsC, kTN, 1)) != cudaSuccess) return e;
+  if ((e = encode_bf16_chunks(&p.tmQb, Q, (uint64_t)d.batch * d.hq, kM, 4)) != cudaSuccess)
+    return e;
+  if ((e = encode_bf16_chunks(&p.tmRk, ring_k, rowsR, kTN, 1)) != cudaSuccess) return e;
+  if ((e = encode_bf16_chunks(&p.tmRv, ring_v, rowsR, 16, 8)) != cudaSuccess) return e;
+  float* pml = static_cast<float*>(part.out_partial);
+  float* po = pml ? pml + ml_floats(d, 1) : nullptr;
+  p.Q = static_cast<const __nv_bfloat16*>(Q);
+  p.vc8 = static_cast<const uint8_t*>(c.vc_pool);
+  p.ctx_len = ctx_len;
+  p.page_table = c.page_table;
+  p.n_entries = c.n_entries;
+  p.err_word = c.err_word;
+  if (pml && nsplit == 1) {
+    p.ws_ml = pml;
+    p.ws_o = po;
+  } else {
+    p.ws_ml = static_cast<float*>(ws);
+    p.ws_o = p.ws_ml + ml_floats(d, nsplit);
+  }
+  p.nseq = d.batch;
+  p.seqlen = d.seqlen;
+  p.hq = d.hq;
+  p.W = d.window;
+  p.block = d.block;
+  p.PE = c.page_entries;
+  p.max_pages = c.max_pages;
+  p.num_pages = c.num_pages;
+  p.nsplit = nsplit;
+  p.e0 = part.e0;
+  p.e1 = part.e1;
+  p.with_ring = part.with_ring ? 1 : 0;
+  p.partial = pml ? 1 : 0;
+  p.scale_log2 = d.scale * 1.4426950408889634f;
+  p.k_scale = c.k_scale;
+  p.v_scale = c.v_scale;
+  p.O = static_cast<__nv_bfloat16*>(O);
+  p.lse = lse;
+  p.gate = static_cast<const __nv_bfloat16*>(d.gate);
+  p.gs0 = d.gate_strides[0];
+  p.gs2 = d.gate_strides[2];
+  static PerDevice<int> smem_limit_set;
+  if ((e = set_smem_limit_once(smem_limit_set, (const void*)decode_fp8_kernel,
+                               (int)kSmemBytes)) != cudaSuccess)
+    return e;
+  cudaLaunchAttribute pdl[1];
+  cudaLaunchConfig_t cfg = pdl_config(pdl, s);
+  cfg.gridDim = dim3(nsplit, d.batch);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  if ((e = cudaLaunchKernelEx(&cfg, decode_fp8_kernel, p)) != cudaSuccess) return e;
+  if (nsplit == 1) return cudaSuccess;
+  return launch_split_merge(d, p.ws_ml, p.ws_o, nsplit, pml, po, O, lse, s);
+}
+
+}  // namespace hca

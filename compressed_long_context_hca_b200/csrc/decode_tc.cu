@@ -31,16 +31,18 @@
 
 #include "hca_internal.h"
 #include "sm100.cuh"
+#include "decode_keys.cuh"
 #include "tmap.h"
 
 namespace hca {
 namespace {
 
+using namespace dkeys;
+
 constexpr int kM = 64;                    // head rows
 constexpr int kD = 512;
 constexpr int kKC = 64;                   // elements per 128-byte swizzle row ("chunk")
 constexpr int kNCh = kD / kKC;            // 8
-constexpr int kTN = 128;                  // keys per tile (compressed or ring)
 constexpr uint32_t kChunk128 = 128 * kKC * 2;           // 16 KB: 128 rows x one chunk
 constexpr uint32_t kSlotBytes = 2 * kChunk128;          // 32 KB: one 3-D box, 2 chunks
 constexpr int kSlotsPerTile = kNCh / 2;                 // 4 for K, 4 for V
@@ -67,8 +69,6 @@ constexpr int kORow = kD + 4;  // floats per staged row: rows r and r + 8 share 
 constexpr uint32_t kOffStage = kOffP;
 static_assert(kOffRing == kOffP + 2 * kPBytes, "P and ring must be adjacent");
 static_assert(kM * kORow * 4 + 3 * kM * 4 <= 2 * kPBytes + kStages * kSlotBytes, "staging space");
-
-enum { kCompressed = 0, kRing = 1 };
 
 struct Params {
   // 3-D maps {64 elements, rows, 8 chunks}
@@ -101,67 +101,6 @@ struct Bars {
   int abort;
 };
 static_assert(sizeof(Bars) <= 256, "barrier block too large");
-
-struct Seq {
-  int t, nc;      // query position, visible compressed entries
-  int e0, e1;     // compressed entries of the call's part, [e0, e1)
-  int nct, total, j0, j1;  // tiles [j0, j1) belong to this split
-};
-
-struct Tile {
-  int kind, key0, n;
-};
-
-__device__ __forceinline__ int round16(int x) { return (x + 15) & ~15; }
-
-__device__ __forceinline__ Seq make_seq(const Params& p, int b, int split) {
-  Seq s;
-  // ctx_len is clamped into [1, seqlen]: the host sized the splits (and with them the TMEM
-  // columns a split's scores take) for seqlen
-  const int ctx = p.ctx_len[b];
-  s.t = min(max(ctx, 1), p.seqlen) - 1;
-  int x = s.t + 1 - p.W;
-  int nc = x < 0 ? 0 : x / p.block;
-  s.nc = min(nc, min(p.n_entries[b], p.max_pages * p.PE));
-  s.e0 = min(p.e0, s.nc);
-  s.e1 = max(s.e0, min(p.e1, s.nc));
-  s.nct = (s.e1 - s.e0 + kTN - 1) / kTN;
-  s.total = s.nct + (p.with_ring ? 1 : 0);
-  const int tps = (s.total + p.nsplit - 1) / p.nsplit;
-  s.j0 = min(s.total, split * tps);
-  s.j1 = min(s.total, s.j0 + tps);
-  return s;
-}
-
-__device__ __forceinline__ Tile tile_of(const Params& p, const Seq& s, int j) {
-  Tile t;
-  if (j < s.nct) {
-    t.kind = kCompressed;
-    t.key0 = s.e0 + j * kTN;
-    t.n = min(kTN, round16(s.e1 - t.key0));
-  } else {
-    t.kind = kRing;
-    t.key0 = 0;
-    t.n = round16(p.W);
-  }
-  return t;
-}
-
-__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
-                                            int32_t row, int32_t chunk, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      ".L2::cache_hint [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(0), "r"(row), "r"(chunk),
-      "l"(policy)
-      : "memory");
-}
-
-__device__ __forceinline__ uint64_t policy_evict_first() {
-  uint64_t pol;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-  return pol;
-}
 
 __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -236,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         }
         mbar_expect_tx(&bars->q_full, kQBytes);
         for (int h = 0; h < 2; ++h)
-          tma_load_3d(sQ + h * (kQBytes / 2), &p.tmQ, &bars->q_full, b * p.hq, 4 * h, pol);
+          tma_load_3d(sQ + h * (kQBytes / 2), &p.tmQ, &bars->q_full, 0, b * p.hq, 4 * h, pol);
       }
       uint32_t cnt = 0;
       auto load_tile = [&](int j, bool is_v) -> bool {
@@ -261,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           const uint32_t round = n / kStages;
           if (round > 0 && !mbar_wait(&bars->ring_empty[s], (round - 1) & 1, abort)) return false;
           mbar_expect_tx(&bars->ring_full[s], kSlotBytes);
-          tma_load_3d(sRing + s * kSlotBytes, map, &bars->ring_full[s], row, 2 * q, pol);
+          tma_load_3d(sRing + s * kSlotBytes, map, &bars->ring_full[s], 0, row, 2 * q, pol);
         }
         return true;
       };
@@ -767,7 +706,7 @@ int decode_num_splits(const hca_desc& d) {
 
 // Split count of a call over the key part: at most that of the whole key list, so the
 // workspace of hca_decode_workspace_bytes(d) always suffices.
-static int part_num_splits(const hca_desc& d, const DecodePart& part) {
+int part_num_splits(const hca_desc& d, const DecodePart& part) {
   const int64_t nc = max_visible_entries(d);
   const int64_t e1 = part.e1 < nc ? part.e1 : nc;
   const int64_t n = e1 > part.e0 ? e1 - part.e0 : 0;
@@ -780,7 +719,7 @@ static int part_num_splits(const hca_desc& d, const DecodePart& part) {
 // Workspace layout: ws_ml [batch, nsplit, hq, 2] float, padded to a multiple of 4 floats so
 // that ws_o [batch, nsplit, hq, 512] float (read and written as float4) starts 16-byte
 // aligned whatever batch * nsplit * hq is. A partial result is this layout with nsplit 1.
-static size_t ml_floats(const hca_desc& d, int nsplit) {
+size_t ml_floats(const hca_desc& d, int nsplit) {
   const size_t n = (size_t)d.batch * nsplit * d.hq * 2;
   return (n + 3) & ~size_t(3);
 }
@@ -800,7 +739,7 @@ size_t decode_part_workspace_bytes(const hca_desc& d, const DecodePart& part) {
   return (ml_floats(d, ns) + (size_t)d.batch * ns * d.hq * kD) * sizeof(float);
 }
 
-static cudaLaunchConfig_t pdl_config(cudaLaunchAttribute* pdl, cudaStream_t s) {
+cudaLaunchConfig_t pdl_config(cudaLaunchAttribute* pdl, cudaStream_t s) {
   // programmatic dependent of the grid before it on the stream (each kernel waits for it
   // with griddepcontrol.wait before touching memory)
   pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -816,6 +755,8 @@ cudaError_t launch_decode_part(const hca_desc& d, const void* Q, const int32_t* 
                                const hca_cache& c, const void* ring_k, const void* ring_v,
                                const DecodePart& part, void* O, float* lse, void* ws,
                                cudaStream_t s) {
+  if (c.pool_format == HCA_POOL_E4M3)
+    return launch_decode_fp8(d, Q, ctx_len, c, ring_k, ring_v, part, O, lse, ws, s);
   Params p;
   memset(&p, 0, sizeof(p));
   const int nsplit = part_num_splits(d, part);
@@ -874,10 +815,16 @@ cudaError_t launch_decode_part(const hca_desc& d, const void* Q, const int32_t* 
   cfg.dynamicSmemBytes = kSmemBytes;
   if ((e = cudaLaunchKernelEx(&cfg, decode_tc_kernel, p)) != cudaSuccess) return e;
   if (nsplit == 1) return cudaSuccess;  // the decode CTAs wrote their result themselves
+  return launch_split_merge(d, p.ws_ml, p.ws_o, nsplit, pml, po, O, lse, s);
+}
+
+cudaError_t launch_split_merge(const hca_desc& d, const float* ws_ml, const float* ws_o,
+                               int nsplit, float* pml, float* po, void* O, float* lse,
+                               cudaStream_t s) {
   MergeArgs m;
   memset(&m, 0, sizeof(m));
-  m.ml = p.ws_ml;
-  m.o = p.ws_o;
+  m.ml = ws_ml;
+  m.o = ws_o;
   m.ml_ss = (int64_t)d.hq * 2;
   m.ml_bs = (int64_t)nsplit * d.hq * 2;
   m.o_ss = (int64_t)d.hq * kD;
@@ -891,6 +838,7 @@ cudaError_t launch_decode_part(const hca_desc& d, const void* Q, const int32_t* 
   m.lse = lse;
   m.pml = pml;
   m.po = po;
+  cudaLaunchAttribute pdl[1];
   cudaLaunchConfig_t mcfg = pdl_config(pdl, s);
   mcfg.gridDim = dim3(d.hq, d.batch);
   mcfg.blockDim = dim3(kMergeThreads);

@@ -106,6 +106,21 @@ cudaError_t encode_bf16_chunks(CUtensorMap* map, const void* base, uint64_t rows
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+cudaError_t encode_u8_chunks(CUtensorMap* map, const void* base, uint64_t rows,
+                             uint32_t box_rows, uint32_t box_chunks) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  if (rows == 0) rows = 1;
+  cuuint64_t dims[3] = {128, rows, 4};
+  cuuint64_t strides[2] = {512, 128};
+  cuuint32_t box[3] = {128, box_rows, box_chunks};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 }  // namespace hca
 
 using namespace hca;
@@ -132,11 +147,19 @@ int32_t check_desc(const hca_desc* d) {
   return HCA_OK;
 }
 
+bool finite_positive(float x) { return x > 0.f && x <= 3.4028234663852886e38f; }
+
 int32_t check_cache(const hca_cache* c) {
   if (!c || !c->kc_pool || !c->vc_pool || !c->page_table || !c->n_entries) return HCA_EINVAL;
   if (c->page_entries < 1 || c->max_pages < 1 || c->num_pages < 1) return HCA_EINVAL;
+  if (c->pool_format != HCA_POOL_NATIVE && c->pool_format != HCA_POOL_E4M3) return HCA_EINVAL;
+  if (c->pool_format == HCA_POOL_E4M3 && (!finite_positive(c->k_scale) ||
+                                          !finite_positive(c->v_scale)))
+    return HCA_EINVAL;
   return HCA_OK;
 }
+
+bool e4m3_cache(const hca_cache* c) { return c->pool_format == HCA_POOL_E4M3; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -195,6 +218,7 @@ int32_t hca_attn_prefill_range(const hca_desc* d, int32_t q_pos0, int32_t kv_pos
   if (st != HCA_OK) return st;
   if ((st = check_cache(cache)) != HCA_OK) return st;
   if (q_pos0 < 0 || kv_pos0 < 0 || kv_len < 0) return HCA_EINVAL;
+  if (e4m3_cache(cache)) return HCA_EUNSUPPORTED;
   if (d->batch == 0 || d->seqlen == 0) return HCA_OK;
   if (!Q || !K || !V || !O) return HCA_EINVAL;
   if ((int64_t)q_pos0 + d->seqlen > INT32_MAX) return HCA_EINVAL;
@@ -241,6 +265,7 @@ int32_t hca_attn_prefill_backward(const hca_desc* d, const void* Q, const void* 
   int32_t st = check_desc(d);
   if (st != HCA_OK) return st;
   if ((st = check_cache(cache)) != HCA_OK) return st;
+  if (e4m3_cache(cache)) return HCA_EUNSUPPORTED;
   if (d->batch == 0 || d->seqlen == 0) return HCA_OK;
   if (!Q || !K || !V || !lse || !dO || !dQ || !dK || !dV) return HCA_EINVAL;
   if ((d->gate != nullptr) != (dG != nullptr)) return HCA_EINVAL;
@@ -319,7 +344,8 @@ int32_t hca_attn_decode(const hca_desc* d, const void* Q, const int32_t* ctx_len
   if (d->seqlen < 1) return HCA_EINVAL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (d->dtype == HCA_F32) {
-    if (d->head_dim % 32 != 0 || d->head_dim > 512) return HCA_EUNSUPPORTED;
+    if (d->head_dim % 32 != 0 || d->head_dim > 512 || e4m3_cache(cache))
+      return HCA_EUNSUPPORTED;
     return from_cuda(launch_decode_simt(*d, Q, ctx_len, *cache, ring_k, ring_v, O, lse, s));
   }
   if (!decode_tc_supported(*d, *cache)) return HCA_EUNSUPPORTED;

@@ -117,6 +117,22 @@ size_t decode_tc_workspace_bytes(const hca_desc& d);
 cudaError_t launch_decode_tc(const hca_desc& d, const void* Q, const int32_t* ctx_len,
                              const hca_cache& c, const void* ring_k, const void* ring_v,
                              void* O, float* lse, void* ws, cudaStream_t s);
+// Shared by the 16-bit and 8-bit decode launches (decode_tc.cu): the split count of a part,
+// the float count of the (m, l) block of a workspace of nsplit splits, the PDL launch
+// attribute, and the merge of nsplit split partials (ws_ml, ws_o) into the final output or,
+// when pml != nullptr, into one partial (pml, po).
+int part_num_splits(const hca_desc& d, const DecodePart& part);
+size_t ml_floats(const hca_desc& d, int nsplit);
+cudaLaunchConfig_t pdl_config(cudaLaunchAttribute* pdl, cudaStream_t s);
+cudaError_t launch_split_merge(const hca_desc& d, const float* ws_ml, const float* ws_o,
+                               int nsplit, float* pml, float* po, void* O, float* lse,
+                               cudaStream_t s);
+// 8-bit compressed pools (hca_cache.pool_format == HCA_POOL_E4M3; decode_fp8.cu): same
+// arguments, workspace layout and split rule as launch_decode_part.
+cudaError_t launch_decode_fp8(const hca_desc& d, const void* Q, const int32_t* ctx_len,
+                              const hca_cache& c, const void* ring_k, const void* ring_v,
+                              const DecodePart& part, void* O, float* lse, void* ws,
+                              cudaStream_t s);
 cudaError_t launch_decode_tc_noalloc(const hca_desc& d, const void* Q, const int32_t* ctx_len,
                                      const hca_cache& c, const void* ring_k,
                                      const void* ring_v, void* O, float* lse, cudaStream_t s);

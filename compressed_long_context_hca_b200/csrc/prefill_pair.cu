@@ -636,12 +636,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t sb = gg & 1;
         const uint32_t d_tmem = tmem + kTmS0 + sb * 128;
         const uint32_t idesc = idesc_bf16_f32(2 * kBM, t.n, false);
-        if (j == 0) {
-          for (int q = 0; q < kQPairs; ++q)
-            if (!mbar_wait(&bars->q_full[q], ni & 1, abort)) return false;
-        }
         const int nsl = k_slots(t);
         for (int q = 0; q < nsl; ++q) {
+          // an item's first tile waits for its Q boxes slot by slot: a 64-key K slot reads Q
+          // pairs 2q and 2q+1 only (the 16-key slot reads all four), so the first slot's MMAs
+          // start while the later boxes of a new Q tile are still landing
+          if (j == 0) {
+            const int q0 = t.kind == kRaw16 ? 0 : 2 * q;
+            const int q1 = t.kind == kRaw16 ? kQPairs : 2 * q + 2;
+            for (int qq = q0; qq < q1; ++qq)
+              if (!mbar_wait(&bars->q_full[qq], ni & 1, abort)) return false;
+          }
           const uint32_t s = cnt % kStages;
           if (!mbar_wait(&bars->ring_full[s], (cnt / kStages) & 1, abort)) return false;
           tc_fence_after();

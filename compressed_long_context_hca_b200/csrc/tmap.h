@@ -26,4 +26,11 @@ cudaError_t encode_bf16_chunks(CUtensorMap* map, const void* base, uint64_t rows
 cudaError_t encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                            uint64_t ld, uint32_t box_cols, uint32_t box_rows);
 
+// 3-D map over a row-major [rows, 512] array of bytes (e4m3 codes) seen as
+// {128 bytes, rows, 4 chunks} (row stride 512 B, chunk stride 128 B), 128-byte swizzle.
+// One box = box_rows rows x box_chunks consecutive 128-byte chunks, chunk-major in shared
+// memory like encode_bf16_chunks.
+cudaError_t encode_u8_chunks(CUtensorMap* map, const void* base, uint64_t rows,
+                             uint32_t box_rows, uint32_t box_chunks);
+
 }  // namespace hca

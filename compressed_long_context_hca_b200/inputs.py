@@ -15,7 +15,9 @@ heads, head_dim 512, 128K training and 1M inference context):
 * decode: context lengths are uniform integers in [lo, hi] from the same
   generator; cache entries and ring tokens are N(0, 1);
 * pages of the compressed cache are handed out in a seeded random order so
-  that no test relies on pages being contiguous.
+  that no test relies on pages being contiguous;
+* 8-bit decode workloads: the cache entries are e4m3 codes, a random sign bit over a
+  magnitude code uniform in 0..0x5F (drawn as bytes, not computed from values).
 """
 
 from __future__ import annotations
@@ -111,6 +113,40 @@ def decode_inputs(nseq: int, hq: int, hkv: int, D: int, W: int, block: int,
     if gate:
         G = torch.sigmoid(torch.randn((nseq, hq, D), generator=g,
                                       device=device)).to(dt)
+    return DecodeInputs(q, ctx, ek, ev, rk, rv, G)
+
+
+def e4m3_codes(shape, generator: torch.Generator, max_magnitude_code: int = 0x5F,
+               device: str = "cpu") -> torch.Tensor:
+    """Random 8-bit e4m3 codes (uint8): a random sign bit over a magnitude code drawn
+    uniformly from 0 .. max_magnitude_code (0x5F: exponent fields 0..11, values up to 30,
+    spread evenly over the binades). No NaN code is drawn."""
+    mag = torch.randint(0, max_magnitude_code + 1, shape, generator=generator, device=device,
+                        dtype=torch.int32)
+    sign = torch.randint(0, 2, shape, generator=generator, device=device, dtype=torch.int32)
+    return (mag | (sign << 7)).to(torch.uint8)
+
+
+def decode_inputs_e4m3(nseq: int, hq: int, hkv: int, D: int, W: int, block: int,
+                       ctx_lo: int, ctx_hi: int, max_entries: int, seed: int = 0,
+                       gate: bool = False, device: str = "cpu") -> DecodeInputs:
+    """One decode step over an 8-bit compressed cache: as decode_inputs (bf16 query, ring
+    and gate from the same generator order), but the cache entries are e4m3 codes drawn by
+    e4m3_codes (the workload states the stored bytes; with a pool scale of 1/16 their
+    values lie within +-1.875)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    dt = torch.bfloat16
+    ctx = torch.randint(ctx_lo, ctx_hi + 1, (nseq,), generator=g, device=device,
+                        dtype=torch.int64).to(torch.int32)
+    q = torch.randn((nseq, hq, D), generator=g, device=device).to(dt)
+    ek = e4m3_codes((nseq, max_entries, hkv, D), g, device=device)
+    ev = e4m3_codes((nseq, max_entries, hkv, D), g, device=device)
+    rk = torch.randn((nseq, W, hkv, D), generator=g, device=device).to(dt)
+    rv = torch.randn((nseq, W, hkv, D), generator=g, device=device).to(dt)
+    G = None
+    if gate:
+        G = torch.sigmoid(torch.randn((nseq, hq, D), generator=g, device=device)).to(dt)
     return DecodeInputs(q, ctx, ek, ev, rk, rv, G)
 
 

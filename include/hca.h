@@ -87,6 +87,20 @@ typedef struct {
                               decode [sequence, unused, head]; head_dim is contiguous */
 } hca_desc;
 
+/* Element format of the compressed pools (hca_cache.pool_format). */
+typedef enum {
+  HCA_POOL_NATIVE = 0,  /* the pools hold desc->dtype elements */
+  HCA_POOL_E4M3 = 1     /* 8-bit cache of [serve fp8]: one e4m3 code per element */
+} hca_pool_format;
+
+/* [serve fp8]: the communeify.com page ("百度 ERNIE 5.5 Flash Base 完整解析"), section
+ * "本地部署與推論實戰指南" item 3, serves the model with an 8-bit KV cache
+ * (`--kv-cache-dtype fp8`). Readings where it is silent: the compressed pools are what is
+ * stored in 8 bits (the raw window ring stays in desc->dtype); the element format is e4m3
+ * of the OCP 8-bit floating-point specification (bias 7, subnormals, no infinities, largest
+ * finite 448); one float32 scale per pool: stored code = e4m3(entry / scale), value read
+ * back = value(code) * scale. */
+
 /* Paged compressed-KV cache. Entry j of sequence b lives in pool row
  *   page_table[b * max_pages + j / page_entries] * page_entries + j % page_entries. */
 typedef struct {
@@ -98,10 +112,13 @@ typedef struct {
   int32_t max_pages;          /* columns of page_table */
   int32_t num_pages;          /* pages in each pool */
   int32_t* err_word;          /* optional device int32 error bits (HCA_ERR_*), may be NULL */
+  int32_t pool_format;        /* hca_pool_format; 0 (native) for a zero-initialised struct */
+  float k_scale;              /* HCA_POOL_E4M3: Kc value = value(code) * k_scale (finite, > 0) */
+  float v_scale;              /* HCA_POOL_E4M3: Vc value = value(code) * v_scale (finite, > 0) */
 } hca_cache;
 
 /* ABI version of this header (bumped on any layout change of the structs above). */
-#define HCA_ABI_VERSION 1
+#define HCA_ABI_VERSION 2
 int32_t hca_abi_version(void);
 
 /* Human-readable name of a status code. Static string, never NULL. */
@@ -118,13 +135,19 @@ int32_t hca_set_gate(hca_desc* d, const void* gate, const int64_t* strides);
  *   Kc[j] = mean of K rows of tokens [j*block, min((j+1)*block, d->seqlen)), same for V,
  * accumulated in float32 and rounded once to d->dtype, stored into the cache pools at the
  * row the page table gives; then n_entries[b] = first_block + n_blocks.
+ * An HCA_POOL_E4M3 cache ([serve fp8]) stores instead the code e4m3(mean / scale): the
+ * float32 mean divided by k_scale (Kc) or v_scale (Vc) in float32, rounded to the nearest
+ * e4m3 value (ties to even) with magnitudes of 448 and more stored as 448. Pool rows are
+ * then hkv * head_dim bytes.
  * K, V point at the first token of block `first_block` of sequence 0; the token rows of
  * sequence b start `b * batch_stride_tokens` token rows later (prefill: batch_stride_tokens
  * = seqlen with K advanced by first_block*block rows; a decode ring of `block` slots:
  * batch_stride_tokens = block).
  * Errors: HCA_EINVAL (NULL pointer, n_blocks < 0, first_block < 0, a block starting at or
  * past seqlen), HCA_ENOSPACE (first_block + n_blocks > max_pages * page_entries),
- * HCA_EUNSUPPORTED (head_dim not a multiple of 8), HCA_ECUDA. */
+ * HCA_EUNSUPPORTED (head_dim not a multiple of 8), HCA_ECUDA. An HCA_POOL_E4M3 cache also
+ * gives HCA_EINVAL for a scale that is not finite and positive, and an unknown pool_format
+ * gives HCA_EINVAL on every entry point. */
 int32_t hca_compress(const hca_desc* d, const void* K, const void* V,
                      int64_t batch_stride_tokens, int32_t first_block, int32_t n_blocks,
                      const hca_cache* cache, hca_stream_t stream);
@@ -137,7 +160,9 @@ int32_t hca_compress(const hca_desc* d, const void* K, const void* V,
  *   O[b,t,h] *= G[b,t,h] when a gate is attached
  *   lse[b,t,h] = natural log of the softmax denominator incl. the max (if lse != NULL)
  *   dbg_mask[(b*seqlen+t)*3 + {0,1,2}] = (n_c(t), window lo, window hi) (if non-NULL)
- * Compressed entries are read from `cache` (hca_compress must have written them).
+ * Compressed entries are read from `cache` (hca_compress must have written them); an
+ * HCA_POOL_E4M3 cache gives HCA_EUNSUPPORTED here and in the backward (the 8-bit cache
+ * serves decode).
  * Kernels: bf16 -> tcgen05/TMEM tensor-core kernels (need head_dim 512, hkv 1, hq in
  * {8,16,32,64,128}, window <= 128, page_entries % 128 == 0, batch*seqlen*hq and
  * num_pages*page_entries below 2^31). hq >= 16 runs on clusters of two CTAs sharing the
@@ -249,6 +274,13 @@ size_t hca_decode_workspace_bytes(const hca_desc* d);
  * `workspace`, and a merge kernel combines them, applies the gate and casts.
  * Kernels: bf16 -> tcgen05/TMEM kernel (head_dim 512, hkv 1, hq <= 64, window <= 128,
  * page_entries % 128 == 0, num_pages*page_entries below 2^31); f32 -> CUDA-core kernel.
+ * An HCA_POOL_E4M3 cache ([serve fp8]; bf16 only, same shape limits) runs the 8-bit
+ * kernel: the compressed keys enter q.k as e4m3 codes (the query is carried exactly as two
+ * e4m3 parts per element with a power-of-two scale per head), the compressed values are
+ * widened to f16 (exact), the scales apply in float32, and the raw window runs in bf16 as
+ * above; the result is that of the decode above over the dequantised entries
+ * value(code) * scale. The same holds for hca_attn_decode_partial and
+ * hca_attn_decode_noalloc.
  * Errors: HCA_EINVAL, HCA_EUNSUPPORTED, HCA_ENOSPACE (workspace_bytes too small),
  * HCA_ECUDA. */
 int32_t hca_attn_decode(const hca_desc* d, const void* Q, const int32_t* ctx_len,

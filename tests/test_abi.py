@@ -54,8 +54,35 @@ def test_struct_layouts_match_header():
     assert ctypes.sizeof(B.HcaDesc) == 72
     assert B.HcaDesc.gate.offset == 40
     assert B.HcaDesc.gate_strides.offset == 48
-    assert ctypes.sizeof(B.HcaCache) == 56
+    assert ctypes.sizeof(B.HcaCache) == 72
     assert B.HcaCache.err_word.offset == 48
+    assert B.HcaCache.pool_format.offset == 56
+    assert B.HcaCache.k_scale.offset == 60 and B.HcaCache.v_scale.offset == 64
+
+
+def test_struct_layouts_match_c_compiler(tmp_path):
+    # the C compiler's own offsets for the header, against the ctypes mirror
+    src = tmp_path / "layout.c"
+    src.write_text(
+        '#include <stddef.h>\n#include <stdio.h>\n#include "hca.h"\n'
+        "int main(void) {\n"
+        '  printf("%zu %zu %zu %zu\\n", sizeof(hca_desc), offsetof(hca_desc, gate),\n'
+        "         offsetof(hca_desc, gate_strides), offsetof(hca_desc, decode_splits));\n"
+        '  printf("%zu %zu %zu %zu %zu\\n", sizeof(hca_cache), offsetof(hca_cache, err_word),\n'
+        "         offsetof(hca_cache, pool_format), offsetof(hca_cache, k_scale),\n"
+        "         offsetof(hca_cache, v_scale));\n"
+        "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    rc = os.system(f"gcc -I {os.path.join(ROOT, 'include')} -o {exe} {src}")
+    assert rc == 0
+    lines = os.popen(str(exe)).read().split("\n")
+    d = [int(x) for x in lines[0].split()]
+    c = [int(x) for x in lines[1].split()]
+    assert d == [ctypes.sizeof(B.HcaDesc), B.HcaDesc.gate.offset, B.HcaDesc.gate_strides.offset,
+                 B.HcaDesc.decode_splits.offset]
+    assert c == [ctypes.sizeof(B.HcaCache), B.HcaCache.err_word.offset,
+                 B.HcaCache.pool_format.offset, B.HcaCache.k_scale.offset,
+                 B.HcaCache.v_scale.offset]
 
 
 def _cache():
@@ -141,6 +168,28 @@ def test_decode_workspace_and_space(L):
     c = _cache()
     st = B.hca_attn_decode(d, 16, 16, c, 16, 16, 16, 0, 16, n - 1)
     assert st == B.HCA_ENOSPACE
+
+
+def test_e4m3_cache_validation(L):
+    d = B.make_desc(1, 1000, 64, 1, 512)
+    c = _cache()
+    c.pool_format = B.HCA_POOL_E4M3
+    # scales must be finite and positive
+    for ks, vs in ((0.0, 1.0), (1.0, -1.0), (float("inf"), 1.0), (1.0, float("nan"))):
+        c.k_scale, c.v_scale = ks, vs
+        assert B.hca_compress(d, 16, 16, 1000, 0, 1, c) == B.HCA_EINVAL
+        assert B.hca_attn_decode(d, 16, 16, c, 16, 16, 16, 0, 16, 1 << 30) == B.HCA_EINVAL
+    c.k_scale, c.v_scale = 0.01, 0.02
+    # the 8-bit cache serves decode: prefill and its backward have no kernel for it
+    assert B.hca_attn_prefill(d, 16, 16, 16, c, 16) == B.HCA_EUNSUPPORTED
+    assert B.hca_attn_prefill_backward(d, 16, 16, 16, c, 16, 16, 16, 16, 16, 0, 16,
+                                  1 << 30) == B.HCA_EUNSUPPORTED
+    # nor does the float32 decode
+    df = B.make_desc(1, 1000, 4, 1, 512, dtype=B.HCA_F32)
+    assert B.hca_attn_decode(df, 16, 16, c, 16, 16, 16, 0, 16, 1 << 30) == B.HCA_EUNSUPPORTED
+    # an unknown pool format
+    c.pool_format = 5
+    assert B.hca_attn_decode(d, 16, 16, c, 16, 16, 16, 0, 16, 1 << 30) == B.HCA_EINVAL
 
 
 def test_set_gate(L):
