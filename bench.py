@@ -43,12 +43,14 @@ if ROOT not in sys.path:
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM bytes (read + write) of one prefill launch of the 32K workload, from an ncu capture
-# of the 8K case scaled by query positions (x4; Q and O dominate, K/V stay in L2). Keyed by
-# the SHA-1 prefix of the kernel source the capture was made on: any change to the kernel
-# makes the figure null.
+# DRAM bytes (read + write) of one prefill launch, from ncu captures of 8K cases scaled by
+# query positions (Q, O and the gate dominate and scale with them; K/V stay in L2): the
+# 32K workload is x4 of the 8K case; the gated 2 x 128K workload is x32 of the gated 8K
+# case with every 4th block x4. Keyed by the SHA-1 prefix of the kernel source the
+# captures were made on: any change to the kernel makes the figures null.
 PREFILL_KERNEL_SRC = "prefill_pair.cu"
-PREFILL_TRAFFIC = {"d217f8017f04": 4.150e9}  # 1.0376 GB at 8K, x 4
+PREFILL_TRAFFIC = {"569d220a1c08": 4 * 1.037858e9}         # 1.0379 GB at 8K
+PREFILL_128K_TRAFFIC = {"569d220a1c08": 32 * 1.584315e9}   # 1.5843 GB at 8K, gated
 D, HQ, BLOCK, WIN = 512, 64, 128, 128
 
 
@@ -267,10 +269,7 @@ def gpu_main(args, rank, world, local_rank):
     bytes_prefill = (2 * Q.numel() + 2 * K.numel() + 2 * V.numel()) * 2  # Q,O + K,V
     traffic = args.traffic
     if traffic is None and T == 32768 and world == 1:
-        import hashlib
-        src = os.path.join(ROOT, "compressed_long_context_hca_b200", "csrc", PREFILL_KERNEL_SRC)
-        with open(src, "rb") as f:
-            traffic = PREFILL_TRAFFIC.get(hashlib.sha1(f.read()).hexdigest()[:12])
+        traffic = PREFILL_TRAFFIC.get(_prefill_kernel_sha())
     hbm_achieved = bytes_prefill / (prefill_ms * 1e-3) / 1e9
     result = {
         "metric": "HCA prefill TFLOP/s at d=512 (32K bf16, compress+prefill step); "
@@ -822,7 +821,15 @@ class _SeqCache:
         self.c = c
 
 
+def _prefill_kernel_sha():
+    import hashlib
+    src = os.path.join(ROOT, "compressed_long_context_hca_b200", "csrc", PREFILL_KERNEL_SRC)
+    with open(src, "rb") as f:
+        return hashlib.sha1(f.read()).hexdigest()[:12]
+
+
 def _prefill_128k_result(tf, ms, per_gpu, world, peaks, clk):
+    traffic = PREFILL_128K_TRAFFIC.get(_prefill_kernel_sha()) if world == 1 else None
     return {"value": round(tf, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 3),
             "workload": "batch 2 x 131072, 64 heads, 1 KV head, head_dim 512, every 4th block "
                         "x4, fused gate",
@@ -831,6 +838,7 @@ def _prefill_128k_result(tf, ms, per_gpu, world, peaks, clk):
             "roofline": {"bound": "tensor", "achieved": round(per_gpu, 1),
                          "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
                          "frac": round(per_gpu / peaks["bf16_tflops_sustained"], 4),
+                         "traffic": traffic, "kernel": "prefill_pair_kernel",
                          "peak_source": "measured bf16 dense sustained (a 53 ms step under "
                                         "the power cap)"},
             "clocks": clk}

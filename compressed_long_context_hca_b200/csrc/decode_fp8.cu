@@ -16,10 +16,11 @@
 //    are exact for every element within 2^13 of the head's largest (below that the part
 //    error is under 2^-21 of the largest |q|). S1 = Q1 K and S2 = Q2 K go to two TMEM
 //    accumulators; the softmax forms s = (S1 + S2 / 16) * r_h * k_scale * scale.
-//  * P.V runs on kind::f16 with f16 operands. Converter warps widen each 16-key group of
-//    e4m3 values to f16 (exact: every e4m3 value is an f16 value) into a 4-deep ring of
-//    MN-major 128-byte-swizzled buffers, with the global loads of the next four groups in
-//    flight in registers. P is split into f16 hi + lo parts (two UMMAs) and pre-scaled by
+//  * P.V runs on kind::f16 with f16 operands. The e4m3 values arrive by TMA in the same ring
+//    as the keys (one 16 KB box = 32 keys x 512 codes), loaded a tile ahead; converter warps
+//    widen each 16-key group to f16 (exact: every e4m3 value is an f16 value) into a 2-deep
+//    ring of MN-major 128-byte-swizzled buffers and release a box as soon as its two groups
+//    are widened. P is split into f16 hi + lo parts (two UMMAs) and pre-scaled by
 //    2^7, so that small P stay clear of the f16 subnormal range while the largest (2^15
 //    between lazy rescales) stays finite. O accumulates in units of the V codes; v_scale
 //    multiplies it once at the end.
@@ -28,10 +29,11 @@
 //    query replaces Q1/Q2 in shared memory, its scores accumulate in S1 (kind::f16 bf16),
 //    its P goes to bf16 hi + lo parts divided by v_scale (O stays in code units), and its
 //    values land in the same V buffers by TMA.
-//  * Roles: warp 0 issues the K loads (TMA boxes of 128 rows x 128 bytes, a 4-slot ring)
-//    and the bf16 query of the ring tile; warp 1 issues the UMMAs; warps 2-5 run the
-//    softmax (lazy rescale, as the 16-bit kernel) and the epilogue; warps 6-9 prepare
-//    Q1/Q2 and widen V.
+//  * Roles: warp 0 issues the loads into a 6-slot ring of 16 KB boxes in the order K(0),
+//    then per step c >= 1: K(c), V(c - 1) (K: 128 keys x one 128-byte column chunk; V: 32
+//    keys x 512 codes; the window tile's bf16 K in 64-column chunks), and the bf16 query of
+//    the window tile; warp 1 issues the UMMAs; warps 2-5 run the softmax (lazy rescale, as
+//    the 16-bit kernel) and the epilogue; warps 6-9 prepare Q1/Q2 and widen V.
 //  * TMEM: O (64 x 512 f32, M = 64 layout) in lanes 0-15 of each 32-lane subpartition;
 //    two score buffers of S1 | S2 (128 columns each) in lanes 16-31.
 //  * All mbarrier waits are bounded (HCA_ERR_TIMEOUT on give-up); on give-up every issuing
@@ -64,18 +66,20 @@ constexpr uint32_t kQPartBytes = 4 * kQChunkBytes;  // 32 KB: one e4m3 part of t
 constexpr uint32_t kQ16Bytes = 8 * kQChunkBytes;    // 64 KB: the bf16 query
 constexpr uint32_t kPChunkBytes = kM * 128;     // 8 KB: 64 rows x 64 keys (16-bit)
 constexpr uint32_t kPBytes = 2 * kPChunkBytes;  // 16 KB: one part of P (128 keys)
-constexpr int kKStages = 4;
-constexpr uint32_t kKSlot = 128 * 128;          // 16 KB: 128 key rows x one 128-byte chunk
-constexpr int kVStages = 4;
+constexpr int kStages = 6;
+constexpr uint32_t kSlot = 16384;               // 16 KB ring slot
+constexpr int kVRows = 32;                      // keys of one e4m3 V box (4 chunks x 4 KB)
+constexpr uint32_t kV8Chunk = kVRows * 128;     // 4 KB: 32 keys x 128 codes
+constexpr int kVStages = 2;
 constexpr uint32_t kVChunkBytes = 16 * 128;     // 2 KB: 16 keys x 64 values (16-bit)
 constexpr uint32_t kVSlot = 8 * kVChunkBytes;   // 16 KB: 16 keys x 512 values
 
 constexpr uint32_t kOffQ = 0;                           // Q1 | Q2, later the bf16 query
 constexpr uint32_t kOffP = kQ16Bytes;                   // P hi | P lo
-constexpr uint32_t kOffK = kOffP + 2 * kPBytes;
-constexpr uint32_t kOffV = kOffK + kKStages * kKSlot;
+constexpr uint32_t kOffRing = kOffP + 2 * kPBytes;
+constexpr uint32_t kOffV = kOffRing + kStages * kSlot;
 constexpr uint32_t kOffBar = kOffV + kVStages * kVSlot;
-constexpr uint32_t kOffRowScale = kOffBar + 256;        // 64 floats
+constexpr uint32_t kOffRowScale = kOffBar + 512;        // 64 floats
 constexpr uint32_t kSmemBytes = kOffRowScale + 256 + 1024;
 static_assert(2 * kQPartBytes == kQ16Bytes, "Q1 | Q2 and the bf16 query share one region");
 
@@ -89,11 +93,11 @@ static_assert(kM * kORow * 4 + 3 * kM * 4 <= kOffBar - kOffStage, "staging space
 
 struct Params8 {
   CUtensorMap tmK8;  // e4m3 Kc pool {128 bytes, rows, 4 chunks}, box {128, 128, 1}
+  CUtensorMap tmV8;  // e4m3 Vc pool {128 bytes, rows, 4 chunks}, box {128, 32, 4}
   CUtensorMap tmQb;  // bf16 Q {64, batch*hq, 8}, box {64, 64, 4}
   CUtensorMap tmRk;  // bf16 ring K {64, batch*W, 8}, box {64, 128, 1}
   CUtensorMap tmRv;  // bf16 ring V {64, batch*W, 8}, box {64, 16, 8}
   const __nv_bfloat16* Q;  // [batch, hq, 512]
-  const uint8_t* vc8;      // e4m3 Vc pool [rows, 512]
   const int32_t* ctx_len;
   const int32_t* page_table;
   const int32_t* n_entries;
@@ -113,22 +117,17 @@ struct Bars8 {
   uint64_t q_ready;   // Q1, Q2 and the row scales written (converters)
   uint64_t qb_full;   // bf16 query of the ring tile landed (TMA)
   uint64_t q8_free;   // the last e4m3 score MMA completed: the query region may be reused
-  uint64_t k_full[kKStages], k_empty[kKStages];
+  // A ring slot holds a K box or a V box; each kind completes on its own barrier, so that
+  // each consumer (UMMA warp: K; converter warps: V) waits only on phases of its own boxes,
+  // in order, and a parity wait can never match a phase that belongs to the other kind.
+  uint64_t k_full[kStages], v8_full[kStages], ring_empty[kStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[2], p_full[2], o_done[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
 };
-static_assert(sizeof(Bars8) <= 256, "barrier block too large");
-
-__device__ __forceinline__ uint4 ld_stream16(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
+static_assert(sizeof(Bars8) <= 512, "barrier block too large");
 
 // two e4m3 codes (low byte first) -> f16x2 (exact)
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
@@ -170,23 +169,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
                                              ~uintptr_t(1023));
   uint8_t* sQ = smem + kOffQ;
   uint8_t* sP = smem + kOffP;
-  uint8_t* sK = smem + kOffK;
+  uint8_t* sRing = smem + kOffRing;
   uint8_t* sV = smem + kOffV;
   Bars8* bars = reinterpret_cast<Bars8*>(smem + kOffBar);
   float* sRS = reinterpret_cast<float*>(smem + kOffRowScale);
   volatile int* abort = &bars->abort;
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const int b = blockIdx.y;
-  const int split = blockIdx.x;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_ready, 1);
     mbar_init(&bars->qb_full, 1);
     mbar_init(&bars->q8_free, 1);
-    for (int s = 0; s < kKStages; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars->k_full[s], 1);
-      mbar_init(&bars->k_empty[s], 1);
+      mbar_init(&bars->v8_full[s], 1);
+      mbar_init(&bars->ring_empty[s], 1);
     }
     for (int s = 0; s < kVStages; ++s) {
       mbar_init(&bars->v_full[s], 1);
@@ -211,6 +209,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
   const uint32_t tmem = bars->tmem_base;
   pdl_wait();
   pdl_trigger();
+  const int b = blockIdx.y;
+  const int split = blockIdx.x;
+  // where a partial result goes: [b, split] of the workspace (with one split and a partial
+  // call, the workspace is the call's partial output)
+  float* dst_ml = p.ws_ml + ((int64_t)b * p.nsplit + split) * p.hq * 2;
+  float* dst_o = p.ws_o + ((int64_t)b * p.nsplit + split) * p.hq * kD;
   const Seq sq = make_seq(p, b, split);
   const int ntiles = sq.j1 - sq.j0;
   const bool has_ring = ntiles > 0 && tile_of(p, sq, sq.j1 - 1).kind == kRing;
@@ -219,12 +223,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
   if (ntiles <= 0) {
     // empty split: an all-zero partial that the merge skips
     for (int h = threadIdx.x; h < p.hq; h += blockDim.x) {
-      float* ml = p.ws_ml + (((int64_t)b * p.nsplit + split) * p.hq + h) * 2;
-      ml[0] = -INFINITY;
-      ml[1] = 0.f;
+      dst_ml[2 * h] = -INFINITY;
+      dst_ml[2 * h + 1] = 0.f;
     }
   } else if (warp == 0) {
-    // ------------------------------------------------------------------ K producer
+    // ------------------------------------------------------------------ loads
+    // One ring of 16 KB boxes, in the order K(0), then per step c >= 1: K(c), V(c - 1).
+    // The UMMA warp consumes (and releases) the K boxes, the converter warps the V boxes.
     if (elect_one()) {
       const uint64_t pol = policy_evict_first();  // every cache row is read once
       if (split == 0 && p.err_word) {
@@ -234,61 +239,91 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
         if ((x < 0 ? 0 : x / p.block) > p.n_entries[b]) atomicOr(p.err_word, kErrCacheShort);
       }
       uint32_t cnt = 0;  // loads issued
+      uint32_t kph = 0, vph = 0;  // per slot: parity of the next K / V phase
+      uint32_t last_v = 0;        // per slot: the latest box was a V box
       bool ok = true, q_issued = false;
-      auto load = [&](const CUtensorMap* map, int row, int chunk) -> bool {
-        const uint32_t s = cnt % kKStages;
-        if (cnt >= (uint32_t)kKStages &&
-            !mbar_wait(&bars->k_empty[s], ((cnt / kKStages) - 1) & 1, abort))
+      auto load = [&](const CUtensorMap* map, int row, int chunk, bool is_v) -> bool {
+        const uint32_t s = cnt % kStages;
+        if (cnt >= (uint32_t)kStages &&
+            !mbar_wait(&bars->ring_empty[s], ((cnt / kStages) - 1) & 1, abort))
           return false;
-        mbar_expect_tx(&bars->k_full[s], kKSlot);
-        tma_load_3d(sK + s * kKSlot, map, &bars->k_full[s], 0, row, chunk, pol);
+        uint64_t* full = is_v ? &bars->v8_full[s] : &bars->k_full[s];
+        mbar_expect_tx(full, kSlot);
+        tma_load_3d(sRing + s * kSlot, map, full, 0, row, chunk, pol);
+        if (is_v) {
+          vph ^= 1u << s;
+          last_v |= 1u << s;
+        } else {
+          kph ^= 1u << s;
+          last_v &= ~(1u << s);
+        }
         ++cnt;
         return true;
       };
-      for (int j = sq.j0; j < sq.j1 && ok; ++j) {
+      auto load_tile = [&](int j, bool is_v) -> bool {
         const Tile t = tile_of(p, sq, j);
         if (t.kind == kCompressed) {
           int page = p.page_table[(int64_t)b * p.max_pages + t.key0 / p.PE];
           if (page < 0 || page >= p.num_pages) {
-            if (p.err_word) atomicOr(p.err_word, kErrPageRange);
+            if (p.err_word && !is_v) atomicOr(p.err_word, kErrPageRange);
             page = 0;
           }
           const int row = page * p.PE + t.key0 % p.PE;
-          for (int q = 0; q < 4 && ok; ++q) ok = load(&p.tmK8, row, q);
-        } else {
-          // the bf16 query replaces Q1/Q2 once the last e4m3 score MMA has completed
-          if (!(ok = mbar_wait(&bars->q8_free, 0, abort))) break;
+          if (is_v) {
+            for (int q = 0; q < (t.n + kVRows - 1) / kVRows; ++q)
+              if (!load(&p.tmV8, row + q * kVRows, 0, true)) return false;
+          } else {
+            for (int q = 0; q < 4; ++q)
+              if (!load(&p.tmK8, row, q, false)) return false;
+          }
+        } else if (!is_v) {
+          // the bf16 query replaces Q1/Q2 once the last e4m3 score MMA has completed; the
+          // window's values go to the V buffers directly (converter warps)
+          if (!mbar_wait(&bars->q8_free, 0, abort)) return false;
           mbar_expect_tx(&bars->qb_full, kQ16Bytes);
           for (int h = 0; h < 2; ++h)
             tma_load_3d(sQ + h * (kQ16Bytes / 2), &p.tmQb, &bars->qb_full, 0, b * p.hq, 4 * h,
                         pol);
           q_issued = true;
-          for (int q = 0; q < 8 && ok; ++q) ok = load(&p.tmRk, b * p.W, q);
+          for (int q = 0; q < 8; ++q)
+            if (!load(&p.tmRk, b * p.W, q, false)) return false;
         }
+        return true;
+      };
+      for (int c = 0; c <= ntiles && ok; ++c) {
+        if (c < ntiles) ok = load_tile(sq.j0 + c, false);
+        if (c >= 1 && ok) ok = load_tile(sq.j0 + c - 1, true);
       }
       if (!ok) {
         bars->abort = 1;
         if (p.err_word) atomicOr(p.err_word, kErrTimeout | (1 << 9));
-        // load n could only be issued once load n - 4 had been consumed: at most the last
-        // four are in flight, plus the bf16 query
+        // load n could only be issued once load n - kStages had been released: at most the
+        // latest box of each slot is in flight, plus the bf16 query. The latest box of slot
+        // s completes the phase of parity (kph or vph, bit s) ^ 1 of its kind's barrier.
         volatile int no_abort = 0;
-        const uint32_t first = cnt > (uint32_t)kKStages ? cnt - kKStages : 0;
-        for (uint32_t n = first; n < cnt; ++n)
-          mbar_wait(&bars->k_full[n % kKStages], (n / kKStages) & 1, &no_abort, 100000000ull);
+        const uint32_t used = cnt < (uint32_t)kStages ? cnt : (uint32_t)kStages;
+        for (uint32_t s = 0; s < used; ++s) {
+          if ((last_v >> s) & 1u)
+            mbar_wait(&bars->v8_full[s], ((vph >> s) & 1u) ^ 1u, &no_abort, 100000000ull);
+          else
+            mbar_wait(&bars->k_full[s], ((kph >> s) & 1u) ^ 1u, &no_abort, 100000000ull);
+        }
         if (q_issued) mbar_wait(&bars->qb_full, 0, &no_abort, 100000000ull);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ UMMA issuer
-    // Order: S(0), then per step c >= 1: S(c) (if any), PV(c - 1), as the 16-bit kernel.
+    // Order: S(0), then per step c >= 1: S(c) (if any), PV(c - 1), as the 16-bit kernel;
+    // it walks the load order and steps over the V boxes (the converters' share).
     if (elect_one()) {
       bool ok = mbar_wait(&bars->q_ready, 0, abort);
       tc_fence_after();
-      uint32_t ck = 0, cv = 0;  // K slots, V groups consumed
+      uint32_t n = 0, cv = 0;  // ring position, V groups consumed
+      uint32_t kph = 0;        // per slot: parity of the next K phase
       bool q8_released = false;
       const uint32_t qbase = smem_u32(sQ);
       const uint32_t pbase = smem_u32(sP);
-      const uint32_t kbase = smem_u32(sK);
+      const uint32_t rbase = smem_u32(sRing);
       const uint32_t vbase = smem_u32(sV);
       for (int c = 0; c <= ntiles && ok; ++c) {
         if (c < ntiles) {
@@ -297,10 +332,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
           if (t.kind == kCompressed) {
             const uint32_t idesc = idesc_e4m3_f32(kM, t.n);
             for (int q = 0; q < 4 && ok; ++q) {
-              const uint32_t s = ck % kKStages;
-              if (!(ok = mbar_wait(&bars->k_full[s], (ck / kKStages) & 1, abort))) break;
+              const uint32_t s = n % kStages;
+              if (!(ok = mbar_wait(&bars->k_full[s], (kph >> s) & 1u, abort))) break;
+              kph ^= 1u << s;
               tc_fence_after();
-              const uint32_t kaddr = kbase + s * kKSlot;
+              const uint32_t kaddr = rbase + s * kSlot;
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {  // K = 32 codes per UMMA
                 const uint64_t kd = sdesc_sw128(kaddr + kk * 32, 16, 1024);
@@ -309,8 +345,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
                 umma_ss_f8(sb, sdesc_sw128(qa, 16, 1024), kd, idesc, acc);
                 umma_ss_f8(sb + 128, sdesc_sw128(qa + kQPartBytes, 16, 1024), kd, idesc, acc);
               }
-              umma_commit(&bars->k_empty[s]);
-              ++ck;
+              umma_commit(&bars->ring_empty[s]);
+              ++n;
             }
           } else {
             if (!q8_released) {  // a split whose only tile is the ring tile
@@ -321,16 +357,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
             tc_fence_after();
             const uint32_t idesc = idesc_bf16_f32(kM, t.n, false);
             for (int q = 0; q < 8 && ok; ++q) {
-              const uint32_t s = ck % kKStages;
-              if (!(ok = mbar_wait(&bars->k_full[s], (ck / kKStages) & 1, abort))) break;
+              const uint32_t s = n % kStages;
+              if (!(ok = mbar_wait(&bars->k_full[s], (kph >> s) & 1u, abort))) break;
+              kph ^= 1u << s;
               tc_fence_after();
-              const uint32_t kaddr = kbase + s * kKSlot;
+              const uint32_t kaddr = rbase + s * kSlot;
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)  // K = 16 bf16 per UMMA
                 umma_ss(sb, sdesc_sw128(qbase + q * kQChunkBytes + kk * 32, 16, 1024),
                         sdesc_sw128(kaddr + kk * 32, 16, 1024), idesc, (q | kk) != 0);
-              umma_commit(&bars->k_empty[s]);
-              ++ck;
+              umma_commit(&bars->ring_empty[s]);
+              ++n;
             }
           }
           if (ok) umma_commit(&bars->s_full[c & 1]);
@@ -343,9 +380,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
         }
         if (c >= 1 && ok) {
           const int pc = c - 1;
+          const Tile t = tile_of(p, sq, sq.j0 + pc);
+          if (t.kind == kCompressed) n += (t.n + kVRows - 1) / kVRows;  // V(pc): converters
           if (!(ok = mbar_wait(&bars->p_full[pc & 1], (pc >> 1) & 1, abort))) break;
           tc_fence_after();
-          const Tile t = tile_of(p, sq, sq.j0 + pc);
           const uint32_t idesc = t.kind == kCompressed ? idesc_f16_f32(kM, 256, true)
                                                        : idesc_bf16_f32(kM, 256, true);
           // O[:, 256 h .. 256 h + 255] += P(group) V(group, columns of half h): one N = 256
@@ -578,17 +616,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
           p.lse[(int64_t)b * p.hq + h] = (sM[h] + __log2f(sL[h])) * 0.69314718055994531f;
     } else {
       // split partial: unnormalised O (value units), (reference max, sum) per head
-      const int64_t slot0 = ((int64_t)b * p.nsplit + split) * p.hq;
-      float* ob = p.ws_o + slot0 * kD;
       for (int i = tid; i < p.hq * (kD / 4); i += 128) {
         const int h = i / (kD / 4);
         const int c = 4 * (i % (kD / 4));
-        *reinterpret_cast<float4*>(ob + (int64_t)h * kD + c) =
+        *reinterpret_cast<float4*>(dst_o + (int64_t)h * kD + c) =
             *reinterpret_cast<const float4*>(sO + h * kORow + c);
       }
       for (int h = tid; h < p.hq; h += 128) {
-        p.ws_ml[(slot0 + h) * 2] = sM[h];
-        p.ws_ml[(slot0 + h) * 2 + 1] = sL[h];
+        dst_ml[h * 2] = sM[h];
+        dst_ml[h * 2 + 1] = sL[h];
       }
     }
   } else {
@@ -649,96 +685,97 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
     named_sync(2, 128);
     if (ct == 0) mbar_arrive(&bars->q_ready);
 
-    // (2) V groups of 16 keys in key order: e4m3 tiles widened here, the ring tile by TMA.
-    // Thread (cw, lane) handles keys kr and kr + 8 of a group at values 32*c32 .. +31.
+    // (2) V groups of 16 keys in key order into the 2-deep V buffer ring: e4m3 boxes of the
+    // load ring widened to f16, the window tile's bf16 values by TMA. Thread (cw, lane)
+    // widens keys kr and kr + 8 of a group at values 32*c32 .. 32*c32 + 31.
     const int kr = lane & 7;
     const int c32 = cw * 4 + (lane >> 3);
-    const int gc = nct > 0 ? (nct - 1) * 8 + tile_of(p, sq, sq.j0 + nct - 1).n / 16 : 0;
-    // global source of group n (n < gc) for this thread's two keys; invalid keys read as 0
-    auto fetch = [&](int n, uint4 (&r)[4]) {
-      if (n >= gc) return;
-      const Tile t = tile_of(p, sq, sq.j0 + (n >> 3));
-      int page = p.page_table[(int64_t)b * p.max_pages + t.key0 / p.PE];
-      if (page < 0 || page >= p.num_pages) page = 0;  // flagged by the K producer
-      const int vlen = min(t.n, sq.e1 - t.key0);
-      const int k0 = (n & 7) * 16 + kr;
-      const uint8_t* src =
-          p.vc8 + ((int64_t)page * p.PE + t.key0 % p.PE + k0) * kD + c32 * 32;
-#pragma unroll
-      for (int it = 0; it < 2; ++it) {
-        if (k0 + 8 * it < vlen) {
-          r[2 * it] = ld_stream16(src + it * 8 * kD);
-          r[2 * it + 1] = ld_stream16(src + it * 8 * kD + 16);
-        } else {
-          r[2 * it] = make_uint4(0, 0, 0, 0);
-          r[2 * it + 1] = make_uint4(0, 0, 0, 0);
-        }
-      }
-    };
     bool ok = true;
-    uint4 buf[4][4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) fetch(u, buf[u]);
-    for (int n0 = 0; n0 < gc && ok; n0 += 4) {
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int n = n0 + u;  // group n uses V slot u = n % 4
-        if (n < gc && ok) {
+    uint32_t n = 0, cv = 0;  // ring position, V groups produced
+    uint32_t vph = 0;        // per slot: parity of the next V phase
+    for (int c = 0; c <= ntiles && ok; ++c) {
+      if (c < ntiles) n += tile_of(p, sq, sq.j0 + c).kind == kCompressed ? 4 : 8;  // K(c)
+      if (c == 0) continue;
+      const Tile t = tile_of(p, sq, sq.j0 + c - 1);
+      const int ng = t.n / 16;
+      if (t.kind == kCompressed) {
+        // keys at or past the visible end of the tile are written as 0 (their P is 0, and
+        // the pool rows behind them may hold anything)
+        const int vlen = min(t.n, sq.e1 - t.key0);
+        for (int g = 0; g < ng && ok; ++g, ++cv) {
+          const uint32_t sidx = n + (g >> 1);
+          const uint32_t rs = sidx % kStages;
           bool w_ok = true;
-          if (n >= kVStages)
+          if ((g & 1) == 0) {
+            w_ok = __all_sync(0xffffffffu, mbar_wait(&bars->v8_full[rs], (vph >> rs) & 1u, abort));
+            vph ^= 1u << rs;
+          }
+          const uint32_t vs = cv % kVStages;
+          if (w_ok && cv >= (uint32_t)kVStages)
             w_ok = __all_sync(0xffffffffu,
-                              mbar_wait(&bars->v_empty[u], ((n / kVStages) - 1) & 1, abort));
+                              mbar_wait(&bars->v_empty[vs], ((cv / kVStages) - 1) & 1, abort));
           if (w_ok) {
-            uint8_t* slot = sV + u * kVSlot;
+            const uint8_t* box = sRing + rs * kSlot + (c32 >> 2) * kV8Chunk;
+            uint8_t* dst = sV + vs * kVSlot + (c32 >> 1) * kVChunkBytes;
 #pragma unroll
             for (int it = 0; it < 2; ++it) {
-              const int k = kr + 8 * it;
-              uint8_t* rowp = slot + (c32 >> 1) * kVChunkBytes + it * 1024 + kr * 128;
-              const uint4 lo = buf[u][2 * it], hi = buf[u][2 * it + 1];
+              const int k = kr + 8 * it;              // key within the group
+              const int r = 16 * (g & 1) + k;         // row within the box
+              uint4 lo = make_uint4(0, 0, 0, 0), hi = make_uint4(0, 0, 0, 0);
+              if (16 * g + k < vlen) {
+                const uint8_t* rowp = box + r * 128;
+                const int u0 = 2 * (c32 & 3);
+                lo = *reinterpret_cast<const uint4*>(rowp + ((u0 ^ (r & 7)) << 4));
+                hi = *reinterpret_cast<const uint4*>(rowp + (((u0 + 1) ^ (r & 7)) << 4));
+              }
               const uint32_t cw8[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+              uint8_t* rowd = dst + it * 1024 + kr * 128;
 #pragma unroll
               for (int w = 0; w < 4; ++w) {
                 const uint32_t a = cw8[2 * w], bq = cw8[2 * w + 1];
                 const int unit = ((c32 & 1) << 2) + w;
-                *reinterpret_cast<uint4*>(rowp + ((unit ^ (k & 7)) << 4)) =
+                *reinterpret_cast<uint4*>(rowd + ((unit ^ (k & 7)) << 4)) =
                     make_uint4(e4m3x2_to_f16x2(a & 0xffffu), e4m3x2_to_f16x2(a >> 16),
                                e4m3x2_to_f16x2(bq & 0xffffu), e4m3x2_to_f16x2(bq >> 16));
               }
             }
             fence_proxy_async_smem();
           }
-          // every converter thread arrives here once per group; the barrier's AND makes
-          // the stop decision (a give-up in any warp, or an abort raised by another role)
-          // the same in all four warps, so none is left waiting at the next barrier
+          // every converter thread arrives here once per group; the barrier's AND makes the
+          // stop decision (a give-up in any warp, or an abort raised by another role) the
+          // same in all four warps, so none is left waiting at the next barrier
           ok = named_sync_and(2, 128, w_ok && !*abort);
-          if (ok && ct == 0) mbar_arrive(&bars->v_full[u]);
-          if (ok) fetch(n + 4, buf[u]);
+          if (ok && ct == 0) {
+            mbar_arrive(&bars->v_full[vs]);
+            // the box is free once both of its groups (or the tile's last) are widened
+            if ((g & 1) == 1 || g == ng - 1) mbar_arrive(&bars->ring_empty[rs]);
+          }
         }
-      }
-    }
-    if (has_ring && ok && ct == 0) {
-      // the raw window's values, bf16, one TMA box of 16 rows x 512 values per group
-      const uint64_t pol = policy_evict_first();
-      const int ng = round16(p.W) / 16;
-      uint32_t issued = 0;
-      for (int g = 0; g < ng && ok; ++g) {
-        const uint32_t n = (uint32_t)(gc + g);
-        const uint32_t s = n % kVStages;
-        if (n >= (uint32_t)kVStages &&
-            !(ok = mbar_wait(&bars->v_empty[s], ((n / kVStages) - 1) & 1, abort)))
-          break;
-        mbar_expect_tx(&bars->v_full[s], kVSlot);
-        tma_load_3d(sV + s * kVSlot, &p.tmRv, &bars->v_full[s], 0, b * p.W + 16 * g, 0, pol);
-        ++issued;
-      }
-      if (!ok) {
-        bars->abort = 1;
-        if (p.err_word) atomicOr(p.err_word, kErrTimeout | (1 << 13));
-        volatile int no_abort = 0;
-        const uint32_t end = (uint32_t)gc + issued;
-        const uint32_t first = issued > (uint32_t)kVStages ? end - kVStages : (uint32_t)gc;
-        for (uint32_t n = first; n < end; ++n)
-          mbar_wait(&bars->v_full[n % kVStages], (n / kVStages) & 1, &no_abort, 100000000ull);
+        n += (t.n + kVRows - 1) / kVRows;
+      } else if (ct == 0) {
+        // the window's values, bf16, one TMA box of 16 rows x 512 values per group
+        const uint64_t pol = policy_evict_first();
+        uint32_t issued = 0;
+        const uint32_t cv0 = cv;
+        for (int g = 0; g < ng && ok; ++g) {
+          const uint32_t vs = (cv0 + g) % kVStages;
+          if (cv0 + g >= (uint32_t)kVStages &&
+              !(ok = mbar_wait(&bars->v_empty[vs], (((cv0 + g) / kVStages) - 1) & 1, abort)))
+            break;
+          mbar_expect_tx(&bars->v_full[vs], kVSlot);
+          tma_load_3d(sV + vs * kVSlot, &p.tmRv, &bars->v_full[vs], 0, b * p.W + 16 * g, 0,
+                      pol);
+          ++issued;
+        }
+        if (!ok) {
+          volatile int no_abort = 0;
+          const uint32_t end = cv0 + issued;
+          const uint32_t first = issued > (uint32_t)kVStages ? end - kVStages : cv0;
+          for (uint32_t m = first; m < end; ++m)
+            mbar_wait(&bars->v_full[m % kVStages], (m / kVStages) & 1, &no_abort,
+                      100000000ull);
+        }
+        cv += ng;
       }
     }
     if (!ok && ct == 0) {
@@ -769,6 +806,7 @@ cudaError_t launch_decode_fp8(const hca_desc& d, const void* Q, const int32_t* c
   const uint64_t rowsC = (uint64_t)c.num_pages * c.page_entries;
   const uint64_t rowsR = (uint64_t)d.batch * d.window;
   if ((e = encode_u8_chunks(&p.tmK8, c.kc_pool, rowsC, kTN, 1)) != cudaSuccess) return e;
+  if ((e = encode_u8_chunks(&p.tmV8, c.vc_pool, rowsC, kVRows, 4)) != cudaSuccess) return e;
   if ((e = encode_bf16_chunks(&p.tmQb, Q, (uint64_t)d.batch * d.hq, kM, 4)) != cudaSuccess)
     return e;
   if ((e = encode_bf16_chunks(&p.tmRk, ring_k, rowsR, kTN, 1)) != cudaSuccess) return e;
@@ -776,12 +814,11 @@ cudaError_t launch_decode_fp8(const hca_desc& d, const void* Q, const int32_t* c
   float* pml = static_cast<float*>(part.out_partial);
   float* po = pml ? pml + ml_floats(d, 1) : nullptr;
   p.Q = static_cast<const __nv_bfloat16*>(Q);
-  p.vc8 = static_cast<const uint8_t*>(c.vc_pool);
   p.ctx_len = ctx_len;
   p.page_table = c.page_table;
   p.n_entries = c.n_entries;
   p.err_word = c.err_word;
-  if (pml && nsplit == 1) {
+  if (pml && nsplit == 1) {  // the decode CTAs write the partial result themselves
     p.ws_ml = pml;
     p.ws_o = po;
   } else {

@@ -32,10 +32,10 @@ struct Tile {
 
 __device__ __forceinline__ int round16(int x) { return (x + 15) & ~15; }
 
-// P: any parameter block with ctx_len, n_entries, seqlen, W, block, PE, max_pages, nsplit,
-// e0, e1 and with_ring.
+// P: any parameter block with ctx_len, n_entries, seqlen, W, block, PE, max_pages, e0, e1
+// and with_ring; the sequence's key list is cut into nsplit splits.
 template <typename P>
-__device__ __forceinline__ Seq make_seq(const P& p, int b, int split) {
+__device__ __forceinline__ Seq make_seq_n(const P& p, int b, int split, int nsplit) {
   Seq s;
   // ctx_len is clamped into [1, seqlen]: the host sized the splits (and with them the TMEM
   // columns a split's scores take) for seqlen
@@ -48,10 +48,15 @@ __device__ __forceinline__ Seq make_seq(const P& p, int b, int split) {
   s.e1 = max(s.e0, min(p.e1, s.nc));
   s.nct = (s.e1 - s.e0 + kTN - 1) / kTN;
   s.total = s.nct + (p.with_ring ? 1 : 0);
-  const int tps = (s.total + p.nsplit - 1) / p.nsplit;
+  const int tps = (s.total + nsplit - 1) / nsplit;
   s.j0 = min(s.total, split * tps);
   s.j1 = min(s.total, s.j0 + tps);
   return s;
+}
+
+template <typename P>
+__device__ __forceinline__ Seq make_seq(const P& p, int b, int split) {
+  return make_seq_n(p, b, split, p.nsplit);
 }
 
 template <typename P>
