@@ -18,22 +18,25 @@
 //    accumulators; the softmax forms s = (S1 + S2 / 16) * r_h * k_scale * scale.
 //  * P.V runs on kind::f16 with f16 operands. The e4m3 values arrive by TMA in the same ring
 //    as the keys (one 16 KB box = 32 keys x 512 codes), loaded a tile ahead; converter warps
-//    widen each 16-key group to f16 (exact: every e4m3 value is an f16 value) into a 2-deep
-//    ring of MN-major 128-byte-swizzled buffers and release a box as soon as its two groups
-//    are widened. P is split into f16 hi + lo parts (two UMMAs) and pre-scaled by
-//    2^7, so that small P stay clear of the f16 subnormal range while the largest (2^15
-//    between lazy rescales) stays finite. O accumulates in units of the V codes; v_scale
-//    multiplies it once at the end.
+//    widen each 16-key group to f16 values times 2^-8 (exact, by moving the code's bits) into
+//    a 3-deep ring of MN-major 128-byte-swizzled buffers (each warp hands its part of a
+//    group over on its own; the UMMA warp releases a box once both of its groups are in).
+//    P enters as one f16 value (11 significant bits: its rounding moves the output by at
+//    most 2^-12 of the value spread, a quarter of the bf16 output's own rounding),
+//    pre-scaled by 2^7 so that small P stay clear of the f16 subnormal range while the
+//    largest (2^15 between lazy rescales) stays finite. O accumulates in units of the
+//    widened values; v_scale * 2^8 multiplies it once at the end.
 //  * The ring tile (the raw window, bf16) is the last tile of the last split and runs the
 //    16-bit way inside the same CTA: once the last e4m3 score MMA has completed, the bf16
 //    query replaces Q1/Q2 in shared memory, its scores accumulate in S1 (kind::f16 bf16),
-//    its P goes to bf16 hi + lo parts divided by v_scale (O stays in code units), and its
+//    its P goes to bf16 hi + lo parts divided by v_scale * 2^8 (O keeps its units), and its
 //    values land in the same V buffers by TMA.
-//  * Roles: warp 0 issues the loads into a 6-slot ring of 16 KB boxes in the order K(0),
+//  * Roles: warp 0 issues the loads into a 5-slot ring of 16 KB boxes in the order K(0),
 //    then per step c >= 1: K(c), V(c - 1) (K: 128 keys x one 128-byte column chunk; V: 32
-//    keys x 512 codes; the window tile's bf16 K in 64-column chunks), and the bf16 query of
-//    the window tile; warp 1 issues the UMMAs; warps 2-5 run the softmax (lazy rescale, as
-//    the 16-bit kernel) and the epilogue; warps 6-9 prepare Q1/Q2 and widen V.
+//    keys x 512 codes; the window tile's bf16 K in 64-column chunks), the bf16 query (staged
+//    for the converters at the start, and again for the window tile); warp 1 issues the
+//    UMMAs; warps 2-5 run the softmax (lazy rescale, as the 16-bit kernel) and the
+//    epilogue; warps 6-9 prepare Q1/Q2 and widen V.
 //  * TMEM: O (64 x 512 f32, M = 64 layout) in lanes 0-15 of each 32-lane subpartition;
 //    two score buffers of S1 | S2 (128 columns each) in lanes 16-31.
 //  * All mbarrier waits are bounded (HCA_ERR_TIMEOUT on give-up); on give-up every issuing
@@ -66,11 +69,11 @@ constexpr uint32_t kQPartBytes = 4 * kQChunkBytes;  // 32 KB: one e4m3 part of t
 constexpr uint32_t kQ16Bytes = 8 * kQChunkBytes;    // 64 KB: the bf16 query
 constexpr uint32_t kPChunkBytes = kM * 128;     // 8 KB: 64 rows x 64 keys (16-bit)
 constexpr uint32_t kPBytes = 2 * kPChunkBytes;  // 16 KB: one part of P (128 keys)
-constexpr int kStages = 6;
+constexpr int kStages = 5;
 constexpr uint32_t kSlot = 16384;               // 16 KB ring slot
 constexpr int kVRows = 32;                      // keys of one e4m3 V box (4 chunks x 4 KB)
 constexpr uint32_t kV8Chunk = kVRows * 128;     // 4 KB: 32 keys x 128 codes
-constexpr int kVStages = 2;
+constexpr int kVStages = 3;
 constexpr uint32_t kVChunkBytes = 16 * 128;     // 2 KB: 16 keys x 64 values (16-bit)
 constexpr uint32_t kVSlot = 8 * kVChunkBytes;   // 16 KB: 16 keys x 512 values
 
@@ -97,7 +100,6 @@ struct Params8 {
   CUtensorMap tmQb;  // bf16 Q {64, batch*hq, 8}, box {64, 64, 4}
   CUtensorMap tmRk;  // bf16 ring K {64, batch*W, 8}, box {64, 128, 1}
   CUtensorMap tmRv;  // bf16 ring V {64, batch*W, 8}, box {64, 16, 8}
-  const __nv_bfloat16* Q;  // [batch, hq, 512]
   const int32_t* ctx_len;
   const int32_t* page_table;
   const int32_t* n_entries;
@@ -114,6 +116,7 @@ struct Params8 {
 };
 
 struct Bars8 {
+  uint64_t qs_full;   // the bf16 query staged for the converters landed (TMA)
   uint64_t q_ready;   // Q1, Q2 and the row scales written (converters)
   uint64_t qb_full;   // bf16 query of the ring tile landed (TMA)
   uint64_t q8_free;   // the last e4m3 score MMA completed: the query region may be reused
@@ -129,38 +132,31 @@ struct Bars8 {
 };
 static_assert(sizeof(Bars8) <= 512, "barrier block too large");
 
-// two e4m3 codes (low byte first) -> f16x2 (exact)
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
-  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)two_codes, __NV_E4M3);
-  return (uint32_t)h.x | ((uint32_t)h.y << 16);
+// Two e4m3 codes of a word (bytes 0-1 for sel 0, 2-3 for sel 1; the lower byte to the lower
+// half) -> f16x2 of their values times 2^-8, exactly, by moving bits: the code's exponent and
+// fraction fields (bits 0-6) become the f16 exponent and fraction fields shifted left by 7
+// (same exponent field, biases 7 and 15: the value is 2^-8 times the code's; the subnormal
+// codes land on f16 subnormals), the sign bit goes to bit 15.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2_s8(uint32_t w, int sel) {
+  const uint32_t y = __byte_perm(w, 0u, sel ? 0x3424u : 0x1404u);  // codes in bytes 1 and 3
+  return (y & 0x80008000u) | ((y >> 1) & 0x3f803f80u);
+}
+constexpr float kV16Scale = 256.f;  // the widened values are the codes' values times 2^-8
+
+// two floats -> f16x2 (round to nearest even), `a` in the low half
+__device__ __forceinline__ uint32_t pack_f16x2(float a, float b) {
+  const __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// f16 pair split: hi = RNE f16 of each value, lo = RNE f16 of the remainder (exact in f32)
-__device__ __forceinline__ void split_f16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
-  const __half2 h = __floats2half2_rn(a, b);
-  const float2 hf = __half22float2(h);
-  const __half2 l = __floats2half2_rn(a - hf.x, b - hf.y);
-  hi = *reinterpret_cast<const uint32_t*>(&h);
-  lo = *reinterpret_cast<const uint32_t*>(&l);
+// 2^k as a float for k in [-126, 127] (exact; the exponent field built directly)
+__device__ __forceinline__ float exp2i(int k) {
+  k = k < -126 ? -126 : (k > 127 ? 127 : k);
+  return __int_as_float((k + 127) << 23);
 }
 
 __device__ __forceinline__ void named_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
-}
-
-// Named barrier that also returns the AND of `pred` over the participating threads, so
-// that a loop's continue/stop decision is the same in every warp that takes part.
-__device__ __forceinline__ bool named_sync_and(int id, int threads, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "barrier.cta.red.and.pred q, %2, %3, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)pred), "r"(id), "r"(threads)
-      : "memory");
-  return r != 0;
 }
 
 __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_constant__ Params8 p) {
@@ -178,6 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
   const int lane = threadIdx.x % 32;
 
   if (threadIdx.x == 0) {
+    mbar_init(&bars->qs_full, 1);
     mbar_init(&bars->q_ready, 1);
     mbar_init(&bars->qb_full, 1);
     mbar_init(&bars->q8_free, 1);
@@ -187,7 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
       mbar_init(&bars->ring_empty[s], 1);
     }
     for (int s = 0; s < kVStages; ++s) {
-      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->v_full[s], 4);  // one arrival per converter warp
       mbar_init(&bars->v_empty[s], 1);
     }
     for (int x = 0; x < 2; ++x) {
@@ -238,6 +235,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
         const int x = sq.t + 1 - p.W;
         if ((x < 0 ? 0 : x / p.block) > p.n_entries[b]) atomicOr(p.err_word, kErrCacheShort);
       }
+      // the bf16 query, staged for the converter warps in the P buffer (box of chunks 0-3)
+      // and the V buffers (chunks 4-7): both are free until Q1/Q2 are ready
+      mbar_expect_tx(&bars->qs_full, kQ16Bytes);
+      tma_load_3d(sP, &p.tmQb, &bars->qs_full, 0, b * p.hq, 0, pol);
+      tma_load_3d(sV, &p.tmQb, &bars->qs_full, 0, b * p.hq, 4, pol);
       uint32_t cnt = 0;  // loads issued
       uint32_t kph = 0, vph = 0;  // per slot: parity of the next K / V phase
       uint32_t last_v = 0;        // per slot: the latest box was a V box
@@ -309,6 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
             mbar_wait(&bars->k_full[s], ((kph >> s) & 1u) ^ 1u, &no_abort, 100000000ull);
         }
         if (q_issued) mbar_wait(&bars->qb_full, 0, &no_abort, 100000000ull);
+        mbar_wait(&bars->qs_full, 0, &no_abort, 100000000ull);
       }
     }
   } else if (warp == 1) {
@@ -381,6 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
         if (c >= 1 && ok) {
           const int pc = c - 1;
           const Tile t = tile_of(p, sq, sq.j0 + pc);
+          const uint32_t vstart = n;  // ring position of V(pc)'s first box
           if (t.kind == kCompressed) n += (t.n + kVRows - 1) / kVRows;  // V(pc): converters
           if (!(ok = mbar_wait(&bars->p_full[pc & 1], (pc >> 1) & 1, abort))) break;
           tc_fence_after();
@@ -388,9 +392,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
                                                        : idesc_bf16_f32(kM, 256, true);
           // O[:, 256 h .. 256 h + 255] += P(group) V(group, columns of half h): one N = 256
           // UMMA per half and part of P
-          for (int g = 0; g < t.n / 16 && ok; ++g) {
+          const bool f8 = t.kind == kCompressed;
+          const int ng = t.n / 16;
+          for (int g = 0; g < ng && ok; ++g) {
             const uint32_t s = cv % kVStages;
             if (!(ok = mbar_wait(&bars->v_full[s], (cv / kVStages) & 1, abort))) break;
+            // every converter warp has widened this group: an e4m3 box is free once both of
+            // its groups (or the tile's last) are in
+            if (f8 && ((g & 1) == 1 || g == ng - 1))
+              mbar_arrive(&bars->ring_empty[(vstart + (g >> 1)) % kStages]);
             tc_fence_after();
             const uint32_t vaddr = vbase + s * kVSlot;
             const uint32_t paddr = pbase + (g >> 2) * kPChunkBytes + (g & 3) * 32;
@@ -399,7 +409,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
               const uint64_t vd = sdesc_sw128(vaddr + h * 4 * kVChunkBytes, kVChunkBytes, 1024);
               umma_ss(tmem + h * 256, sdesc_sw128(paddr, 16, 1024), vd, idesc,
                       (pc > 0 || g > 0));
-              umma_ss(tmem + h * 256, sdesc_sw128(paddr + kPBytes, 16, 1024), vd, idesc, 1u);
+              if (!f8)
+                umma_ss(tmem + h * 256, sdesc_sw128(paddr + kPBytes, 16, 1024), vd, idesc, 1u);
             }
             umma_commit(&bars->v_empty[s]);
             ++cv;
@@ -426,7 +437,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
     bool ok = __all_sync(0xffffffffu, mbar_wait(&bars->q_ready, 0, abort));
     const float rs8 = sRS[hrow];            // r_h * k_scale * scale * log2(e)
-    const float inv_vs = 1.f / p.v_scale;   // ring values enter O in V-code units
+    // ring values enter O in the units of the widened e4m3 values (value / (v_scale * 2^8))
+    const float inv_vs = 1.f / (p.v_scale * kV16Scale);
     float base = -INFINITY, l = 0.f;
     for (int c = 0; c < ntiles && ok; ++c) {
       ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[c & 1], (c >> 1) & 1, abort));
@@ -505,8 +517,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
         }
         tmem_wait_st();
       }
-      // pass 2: P = 2^(s - base + 7) -> hi + lo parts in two K-major 128B-swizzled buffers:
-      // f16 for an e4m3 tile; bf16 times 1/v_scale for the ring tile
+      // pass 2: P = 2^(s - base + 7) into the K-major 128B-swizzled P buffer: one f16 value
+      // for an e4m3 tile; hi + lo bf16 parts (two buffers) times 1/v_scale for the ring tile
       const float bb = base == -INFINITY ? 0.f : base - kPShift;
       float ps[4] = {0.f, 0.f, 0.f, 0.f};
       for (int q = 0; q < kTN / 32; ++q) {
@@ -525,7 +537,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
                                  ? fast_exp2(fmaf(__uint_as_float(v[2 * e + 1]), rs, -bb))
                                  : 0.f;
             if (f8)
-              split_f16x2(p0, p1, pk[e], pl[e]);
+              pk[e] = pack_f16x2(p0, p1);
             else
               split_bf16x2(p0 * inv_vs, p1 * inv_vs, pk[e], pl[e]);
             ps[e & 3] += p0 + p1;
@@ -538,8 +550,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
             const int us = u ^ (hrow & 7);
             *reinterpret_cast<uint4*>(rowp + us * 16) =
                 make_uint4(pk[4 * w], pk[4 * w + 1], pk[4 * w + 2], pk[4 * w + 3]);
-            *reinterpret_cast<uint4*>(rowp + kPBytes + us * 16) =
-                make_uint4(pl[4 * w], pl[4 * w + 1], pl[4 * w + 2], pl[4 * w + 3]);
+            if (!f8)
+              *reinterpret_cast<uint4*>(rowp + kPBytes + us * 16) =
+                  make_uint4(pl[4 * w], pl[4 * w + 1], pl[4 * w + 2], pl[4 * w + 3]);
           }
         }
       }
@@ -563,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
         sL[hrow] = l;
         sInv[hrow] = 1.f / l;
       }
-      const float vs = p.v_scale;
+      const float vs = p.v_scale * kV16Scale;
       float* orow = sO + hrow * kORow;
 #pragma unroll 1
       for (int q = 0; q < kD / 32; ++q) {
@@ -631,15 +644,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
     // ------------------------------------------------------------------ converters
     const int ct = threadIdx.x - 192;  // 0..127
     const int cw = ct >> 5;
-    // (1) Q1, Q2 and the per-head scale: two threads per head row, 256 elements each
+    // (1) Q1, Q2 and the per-head scale: two threads per head row, 256 elements each, from
+    // the staged bf16 query (chunk c of row h at stage(c) + (c % 4) * 8 KB + h * 128, its
+    // 16-byte units swizzled by h % 8)
+    bool q_ok = __all_sync(0xffffffffu, mbar_wait(&bars->qs_full, 0, abort));
     {
       const int h = ct >> 1, half = ct & 1;
-      const bool live = h < p.hq;
-      const __nv_bfloat16* qrow = p.Q + ((int64_t)b * p.hq + (live ? h : 0)) * kD + half * 256;
+      const bool live = h < p.hq && q_ok;
+      const uint8_t* stage = half == 0 ? sP : sV;  // chunks 4 * half .. 4 * half + 3
+      auto unit = [&](int i) {  // 16-byte unit i (8 elements) of this thread's 256
+        const uint8_t* rowp = stage + (i >> 3) * kQChunkBytes + h * 128;
+        return *reinterpret_cast<const uint4*>(rowp + (((i & 7) ^ (h & 7)) << 4));
+      };
       float amax = 0.f;
       if (live)
         for (int i = 0; i < 32; ++i) {
-          const uint4 x = *reinterpret_cast<const uint4*>(qrow + 8 * i);
+          const uint4 x = unit(i);
           const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&x);
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
@@ -649,18 +669,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
         }
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
       // r_h = 2^e puts the head's largest |q| / r_h in [128, 256)
-      const int e = amax > 0.f ? ilogbf(amax) - 7 : 0;
-      for (int u = 0; u < 16; ++u) {  // 16-element units
+      // (the exponent field of amax; e is kept in [-126, 126] so that r_h and 1 / r_h are
+      // both normal floats: a row whose largest |q| is below 2^-119 keeps a smaller range)
+      const int ebits = (__float_as_int(amax) >> 23) & 0xff;
+      int e = amax > 0.f ? (ebits > 0 ? ebits - 127 : -126) - 7 : 0;
+      e = e < -126 ? -126 : (e > 126 ? 126 : e);
+      const float rinv = exp2i(-e);  // 1 / r_h, exact
+      for (int u = 0; u < 16; ++u) {  // 16-element units of the e4m3 parts
         uint32_t w1[4] = {0u, 0u, 0u, 0u}, w2[4] = {0u, 0u, 0u, 0u};
         if (live) {
 #pragma unroll
           for (int hv = 0; hv < 2; ++hv) {
-            const uint4 x = *reinterpret_cast<const uint4*>(qrow + 16 * u + 8 * hv);
+            const uint4 x = unit(2 * u + hv);
             const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&x);
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               const float2 f = __bfloat1622float2(x2[k]);
-              const float a0 = ldexpf(f.x, -e), a1 = ldexpf(f.y, -e);
+              const float a0 = f.x * rinv, a1 = f.y * rinv;
               const __nv_fp8x2_storage_t q1 =
                   __nv_cvt_float2_to_fp8x2(make_float2(a0, a1), __NV_SATFINITE, __NV_E4M3);
               const __half2_raw h1 = __nv_cvt_fp8x2_to_halfraw2(q1, __NV_E4M3);
@@ -679,18 +704,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
         *reinterpret_cast<uint4*>(sQ + off) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
         *reinterpret_cast<uint4*>(sQ + kQPartBytes + off) = make_uint4(w2[0], w2[1], w2[2], w2[3]);
       }
-      if (half == 0) sRS[h] = ldexpf(p.scale_log2 * p.k_scale, e);
+      if (half == 0) sRS[h] = p.scale_log2 * p.k_scale * exp2i(e);
     }
     fence_proxy_async_smem();
     named_sync(2, 128);
     if (ct == 0) mbar_arrive(&bars->q_ready);
 
-    // (2) V groups of 16 keys in key order into the 2-deep V buffer ring: e4m3 boxes of the
+    // (2) V groups of 16 keys in key order into the 3-deep V buffer ring: e4m3 boxes of the
     // load ring widened to f16, the window tile's bf16 values by TMA. Thread (cw, lane)
     // widens keys kr and kr + 8 of a group at values 32*c32 .. 32*c32 + 31.
     const int kr = lane & 7;
     const int c32 = cw * 4 + (lane >> 3);
-    bool ok = true;
+    bool ok = q_ok;
     uint32_t n = 0, cv = 0;  // ring position, V groups produced
     uint32_t vph = 0;        // per slot: parity of the next V phase
     for (int c = 0; c <= ntiles && ok; ++c) {
@@ -735,21 +760,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
                 const uint32_t a = cw8[2 * w], bq = cw8[2 * w + 1];
                 const int unit = ((c32 & 1) << 2) + w;
                 *reinterpret_cast<uint4*>(rowd + ((unit ^ (k & 7)) << 4)) =
-                    make_uint4(e4m3x2_to_f16x2(a & 0xffffu), e4m3x2_to_f16x2(a >> 16),
-                               e4m3x2_to_f16x2(bq & 0xffffu), e4m3x2_to_f16x2(bq >> 16));
+                    make_uint4(e4m3x2_to_f16x2_s8(a, 0), e4m3x2_to_f16x2_s8(a, 1),
+                               e4m3x2_to_f16x2_s8(bq, 0), e4m3x2_to_f16x2_s8(bq, 1));
               }
             }
             fence_proxy_async_smem();
           }
-          // every converter thread arrives here once per group; the barrier's AND makes the
-          // stop decision (a give-up in any warp, or an abort raised by another role) the
-          // same in all four warps, so none is left waiting at the next barrier
-          ok = named_sync_and(2, 128, w_ok && !*abort);
-          if (ok && ct == 0) {
-            mbar_arrive(&bars->v_full[vs]);
-            // the box is free once both of its groups (or the tile's last) are widened
-            if ((g & 1) == 1 || g == ng - 1) mbar_arrive(&bars->ring_empty[rs]);
-          }
+          // each warp hands its quarter of the group over on its own (v_full counts four
+          // arrivals); a warp that gave up stops, and the others' bounded waits end on the
+          // abort flag
+          ok = w_ok;
+          __syncwarp();
+          if (ok && lane == 0) mbar_arrive(&bars->v_full[vs]);
         }
         n += (t.n + kVRows - 1) / kVRows;
       } else if (ct == 0) {
@@ -762,7 +784,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
           if (cv0 + g >= (uint32_t)kVStages &&
               !(ok = mbar_wait(&bars->v_empty[vs], (((cv0 + g) / kVStages) - 1) & 1, abort)))
             break;
+          // the four arrivals of a converted group: this one with the bytes, three plain
           mbar_expect_tx(&bars->v_full[vs], kVSlot);
+          mbar_arrive(&bars->v_full[vs]);
+          mbar_arrive(&bars->v_full[vs]);
+          mbar_arrive(&bars->v_full[vs]);
           tma_load_3d(sV + vs * kVSlot, &p.tmRv, &bars->v_full[vs], 0, b * p.W + 16 * g, 0,
                       pol);
           ++issued;
@@ -778,7 +804,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
         cv += ng;
       }
     }
-    if (!ok && ct == 0) {
+    if (!ok && lane == 0) {
       bars->abort = 1;
       if (p.err_word) atomicOr(p.err_word, kErrTimeout | (1 << 13));
     }
@@ -813,7 +839,6 @@ cudaError_t launch_decode_fp8(const hca_desc& d, const void* Q, const int32_t* c
   if ((e = encode_bf16_chunks(&p.tmRv, ring_v, rowsR, 16, 8)) != cudaSuccess) return e;
   float* pml = static_cast<float*>(part.out_partial);
   float* po = pml ? pml + ml_floats(d, 1) : nullptr;
-  p.Q = static_cast<const __nv_bfloat16*>(Q);
   p.ctx_len = ctx_len;
   p.page_table = c.page_table;
   p.n_entries = c.n_entries;

@@ -7,13 +7,14 @@ returns as soon as the phase count's parity differs from P (so a wait on a phase
 ahead of the current one returns at once: the aliasing the kernel must avoid).
 
 The roles, restated from the kernel: the load warp issues, in order, K(0), then per step
-c >= 1: K(c), V(c - 1), into a ring of 6 slots (waiting for the slot's previous box to be
+c >= 1: K(c), V(c - 1), into a ring of 5 slots (waiting for the slot's previous box to be
 released); a compressed tile is 4 K boxes and ceil(n / 32) V boxes, the window tile 8 K
 boxes (and its bf16 query, after the last e4m3 score MMA); the UMMA warp consumes the K
-boxes in order (and the V groups from a 2-slot buffer ring after the softmax of the tile);
+boxes in order (and the V groups from a 3-slot buffer ring after the softmax of the tile);
 the converter warps consume the V boxes in order, two 16-key groups per box, into the
-buffer ring; the softmax of tile c waits for its scores and for P.V(c - 1). Asynchronous
-completions (TMA landings, MMA commits) happen at random later times.
+buffer ring, and the UMMA warp releases a V box once it has both of its groups; the
+softmax of tile c waits for its scores and for P.V(c - 1). Asynchronous completions (TMA
+landings, MMA commits) happen at random later times.
 
 Checked, over many random schedules and tile lists (one compressed tile and the window,
 several partial tiles, window only, no window): no role waits forever, and every box a
@@ -25,8 +26,8 @@ compressed tile and the window tile.
 
 import random
 
-STAGES = 6
-VSTAGES = 2
+STAGES = 5    # load ring slots of the kernel
+VSTAGES = 3   # V buffer slots
 
 
 class Bar:
@@ -159,13 +160,19 @@ def run(tiles, typed, rng):
             if c >= 1:
                 pc = c - 1
                 t = tiles[pc]
+                vstart = n
                 n += vboxes(t)
                 yield ("wait", ("p_full", pc & 1), (pc >> 1) & 1)
-                for g in range(t[1] // 16):
+                ng = t[1] // 16
+                for g in range(ng):
                     s = cv % VSTAGES
                     yield ("wait", ("v_full", s), (cv // VSTAGES) & 1)
                     if vbuf[s] != (pc, g):
                         fail.append(f"PV read {vbuf[s]} for group {(pc, g)}")
+                    # the converters have read the e4m3 box of this group: released once both
+                    # of its groups (or the tile's last) are in
+                    if t[0] == "c" and (g % 2 == 1 or g == ng - 1):
+                        B[("ring_empty", (vstart + g // 2) % STAGES)].arrive()
                     commit(("v_empty", s))
                     cv += 1
                 commit(("o_done", pc & 1))
@@ -207,8 +214,6 @@ def run(tiles, typed, rng):
                         fail.append(f"converter read {slot_box[rs]} for V{(c - 1, g >> 1)}")
                     vbuf[vs] = (c - 1, g)
                     B[("v_full", vs)].arrive()
-                    if g % 2 == 1 or g == ng - 1:
-                        B[("ring_empty", rs)].arrive()
                     cv += 1
                 n += vboxes(t)
             else:

@@ -251,3 +251,36 @@ def test_decode_e4m3_1m_config_sampled():
     rng = np.random.default_rng(56)
     _check(x, O, lse, sorted(rng.choice(16, 5, replace=False)))
     assert int(cache.err.item()) == 0
+
+
+def test_decode_e4m3_subnormal_values():
+    """Values whose codes are all e4m3 subnormals (exponent field 0) with a large scale:
+    the widened values are f16 subnormals on their way through P.V, and must count. Keys
+    all zero, so every visible key gets the same weight and O is the mean value."""
+    ensure_built()
+    dev = torch.device("cuda")
+    nseq, ctx, W, D = 3, 20000, 128, 512
+    n_ent = (ctx - W) // 128
+    g = torch.Generator()
+    g.manual_seed(57)
+    ek = torch.zeros((nseq, n_ent, 1, D), dtype=torch.uint8)
+    ev = torch.randint(1, 8, (nseq, n_ent, 1, D), generator=g).to(torch.uint8)
+    q = torch.randn((nseq, 64, D), generator=g).to(torch.bfloat16)
+    rk = torch.zeros((nseq, W, 1, D), dtype=torch.bfloat16)
+    rv = torch.zeros((nseq, W, 1, D), dtype=torch.bfloat16)
+    vs = 64.0  # values m / 8 (m = 1..7): outputs near 0.5, where bf16 rounds finely
+    cache = B.PagedCache(nseq, n_ent, 1, D, torch.bfloat16, 128,
+                         page_table=inputs.page_table(nseq, -(-n_ent // 128)), device=dev,
+                         e4m3_scales=(1.0, vs))
+    for b in range(nseq):
+        cache.fill(b, ek[b].to(dev), ev[b].to(dev))
+    desc = B.make_desc(nseq, ctx, 64, 1, D, 128, W, None, B.HCA_BF16, 0)
+    ctxl = torch.full((nseq,), ctx, dtype=torch.int32)
+    O, _ = ops.decode(desc, q.to(dev), ctxl.to(dev), cache, rk.to(dev), rv.to(dev))
+    torch.cuda.synchronize()
+    for b in range(nseq):
+        ref, _ = orc.hca_decode(to64(q[b]), orc.e4m3_dequantize(ek[b].numpy(), 1.0),
+                                orc.e4m3_dequantize(ev[b].numpy(), vs), to64(rk[b]),
+                                to64(rv[b]), ctx, 128, W, default_scale(D))
+        assert ref.mean() > 0.25  # the subnormal values carry the output (0 if flushed)
+        compare(to64(O[b]), ref, BF16_MAX, BF16_MEAN, what=f"O[{b}]")
