@@ -49,6 +49,7 @@
 #include <string.h>
 
 #include "decode_keys.cuh"
+#include "decode_softmax.cuh"
 #include "hca_internal.h"
 #include "sm100.cuh"
 #include "tmap.h"
@@ -57,6 +58,7 @@ namespace hca {
 namespace {
 
 using namespace dkeys;
+using namespace dsoft;
 
 constexpr int kM = 64;    // head rows
 constexpr int kD = 512;
@@ -142,12 +144,6 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2_s8(uint32_t w, int sel) {
   return (y & 0x80008000u) | ((y >> 1) & 0x3f803f80u);
 }
 constexpr float kV16Scale = 256.f;  // the widened values are the codes' values times 2^-8
-
-// two floats -> f16x2 (round to nearest even), `a` in the low half
-__device__ __forceinline__ uint32_t pack_f16x2(float a, float b) {
-  const __half2 h = __floats2half2_rn(a, b);
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
 
 // 2^k as a float for k in [-126, 127] (exact; the exponent field built directly)
 __device__ __forceinline__ float exp2i(int k) {
@@ -403,7 +399,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
               mbar_arrive(&bars->ring_empty[(vstart + (g >> 1)) % kStages]);
             tc_fence_after();
             const uint32_t vaddr = vbase + s * kVSlot;
-            const uint32_t paddr = pbase + (g >> 2) * kPChunkBytes + (g & 3) * 32;
+            const uint32_t paddr =
+                pbase + (f8 ? (pc & 1) * kPBytes : 0u) + (g >> 2) * kPChunkBytes + (g & 3) * 32;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               const uint64_t vd = sdesc_sw128(vaddr + h * 4 * kVChunkBytes, kVChunkBytes, 1024);
@@ -465,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
           tmem_wait_ld();
         }
       };
-      // pass 1: row max over the visible keys (branch-free selects)
+      // pass 1: row max over the visible keys
       float mx[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
@@ -473,10 +470,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
         if (q * 32 >= tl.n) break;
         uint32_t v[32];
         load_scores(q, v);
+        if ((uint32_t)(q * 32 + 32) <= vlen) {  // a fully visible piece: no masks
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const bool in = (uint32_t)(q * 32 + e) < vlen;
-          mx[e & 7] = fmaxf(mx[e & 7], in ? __uint_as_float(v[e]) : -INFINITY);
+          for (int e = 0; e < 32; ++e) mx[e & 7] = fmaxf(mx[e & 7], __uint_as_float(v[e]));
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const bool in = (uint32_t)(q * 32 + e) < vlen;
+            mx[e & 7] = fmaxf(mx[e & 7], in ? __uint_as_float(v[e]) : -INFINITY);
+          }
         }
       }
       const float cmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
@@ -489,13 +491,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
         l *= factor;
         base = cmax;
       }
-      if (c > 0) {
-        // PV(c - 1) done: the P buffer is free and O holds every earlier chunk
+      // The P of an e4m3 tile goes to buffer c & 1, free once PV(c - 2) is done, so that
+      // this pass overlaps PV(c - 1); the window tile's hi and lo parts take both buffers,
+      // and rescaling O needs every earlier PV done: both wait for PV(c - 1).
+      const bool rescale = c > 0 && __any_sync(0xffffffffu, grow);
+      const int pv_wait = (rescale || !f8) ? c - 1 : c - 2;
+      if (pv_wait >= 0) {
         ok = __all_sync(0xffffffffu,
-                        mbar_wait(&bars->o_done[(c - 1) & 1], ((c - 1) >> 1) & 1, abort));
+                        mbar_wait(&bars->o_done[pv_wait & 1], (pv_wait >> 1) & 1, abort));
         if (!ok) break;
       }
-      if (c > 0 && __any_sync(0xffffffffu, grow)) {
+      if (rescale) {
         // the 32-lane read-modify-write also rewrites the score lanes (unchanged): no UMMA
         // may be in flight, so S(c + 1) (if issued) must have completed. PV(c) waits for
         // our p_full.
@@ -518,45 +524,44 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
         tmem_wait_st();
       }
       // pass 2: P = 2^(s - base + 7) into the K-major 128B-swizzled P buffer: one f16 value
-      // for an e4m3 tile; hi + lo bf16 parts (two buffers) times 1/v_scale for the ring tile
-      const float bb = base == -INFINITY ? 0.f : base - kPShift;
-      float ps[4] = {0.f, 0.f, 0.f, 0.f};
+      // for an e4m3 tile; hi + lo bf16 parts (two buffers) times 1/v_scale for the ring tile.
+      // All 32 lanes work: of each 32-column piece of row hrow, lane l + 16 takes columns
+      // 0..15 and lane l columns 16..31, handed over by a shuffle.
+      const float b_own = base == -INFINITY ? 0.f : base - kPShift;
+      const float b_pair = __shfl_xor_sync(0xffffffffu, b_own, 16);
+      const float bb = s_lane ? b_own : b_pair;
+      const int half = s_lane ? 0 : 16;
+      uint8_t* pbuf = sP + (f8 ? (c & 1) * kPBytes : 0u);
+      float ps = 0.f;
       for (int q = 0; q < kTN / 32; ++q) {
         if (q * 32 >= tl.n) break;
         uint32_t v[32];
         load_scores(q, v);
-        if (s_lane) {
-          uint32_t pk[16], pl[16];
+        float x[16];
+        pair_split(v, s_lane, x);
+        const int col0 = q * 32 + half;
+        uint32_t pk[8], pl[8];
+        const bool visible = (uint32_t)(q * 32 + 32) <= vlen;  // the whole piece: no masks
+        if (f8)
+          ps += visible ? p_piece<false, kPF16>(x, rs, bb, col0, vlen, inv_vs, pk, pl)
+                        : p_piece<true, kPF16>(x, rs, bb, col0, vlen, inv_vs, pk, pl);
+        else
+          ps += visible ? p_piece<false, kPBf16PairScaled>(x, rs, bb, col0, vlen, inv_vs, pk, pl)
+                        : p_piece<true, kPBf16PairScaled>(x, rs, bb, col0, vlen, inv_vs, pk, pl);
+        // keys col0 .. col0 + 15 -> 64-key P chunk q/2, 16-byte units (q&1)*4 + half/8 + w
+        uint8_t* rowp = pbuf + (q >> 1) * kPChunkBytes + hrow * 128;
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int c0 = q * 32 + 2 * e;
-            const float p0 = (uint32_t)c0 < vlen
-                                 ? fast_exp2(fmaf(__uint_as_float(v[2 * e]), rs, -bb))
-                                 : 0.f;
-            const float p1 = (uint32_t)(c0 + 1) < vlen
-                                 ? fast_exp2(fmaf(__uint_as_float(v[2 * e + 1]), rs, -bb))
-                                 : 0.f;
-            if (f8)
-              pk[e] = pack_f16x2(p0, p1);
-            else
-              split_bf16x2(p0 * inv_vs, p1 * inv_vs, pk[e], pl[e]);
-            ps[e & 3] += p0 + p1;
-          }
-          // keys q*32 .. -> 64-key P chunk q/2, 16-byte units (q&1)*4 + w
-          uint8_t* rowp = sP + (q >> 1) * kPChunkBytes + hrow * 128;
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            const int u = (q & 1) * 4 + w;
-            const int us = u ^ (hrow & 7);
-            *reinterpret_cast<uint4*>(rowp + us * 16) =
-                make_uint4(pk[4 * w], pk[4 * w + 1], pk[4 * w + 2], pk[4 * w + 3]);
-            if (!f8)
-              *reinterpret_cast<uint4*>(rowp + kPBytes + us * 16) =
-                  make_uint4(pl[4 * w], pl[4 * w + 1], pl[4 * w + 2], pl[4 * w + 3]);
-          }
+        for (int w = 0; w < 2; ++w) {
+          const int u = (q & 1) * 4 + (half >> 3) + w;
+          const int us = u ^ (hrow & 7);
+          *reinterpret_cast<uint4*>(rowp + us * 16) =
+              make_uint4(pk[4 * w], pk[4 * w + 1], pk[4 * w + 2], pk[4 * w + 3]);
+          if (!f8)
+            *reinterpret_cast<uint4*>(rowp + kPBytes + us * 16) =
+                make_uint4(pl[4 * w], pl[4 * w + 1], pl[4 * w + 2], pl[4 * w + 3]);
         }
       }
-      l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+      l += ps + __shfl_xor_sync(0xffffffffu, ps, 16);
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();

@@ -32,12 +32,14 @@
 #include "hca_internal.h"
 #include "sm100.cuh"
 #include "decode_keys.cuh"
+#include "decode_softmax.cuh"
 #include "tmap.h"
 
 namespace hca {
 namespace {
 
 using namespace dkeys;
+using namespace dsoft;
 
 constexpr int kM = 64;                    // head rows
 constexpr int kD = 512;
@@ -339,10 +341,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           uint32_t v[32];
           tmem_ld32(sbuf + col0 + q * 32, v);
           tmem_wait_ld();
+          if ((uint32_t)(q * 32 + 32) <= vlen) {  // a fully visible piece: no masks
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const bool in = (uint32_t)(q * 32 + e) < vlen;
-            mx[e & 7] = fmaxf(mx[e & 7], in ? __uint_as_float(v[e]) : -INFINITY);
+            for (int e = 0; e < 32; ++e) mx[e & 7] = fmaxf(mx[e & 7], __uint_as_float(v[e]));
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const bool in = (uint32_t)(q * 32 + e) < vlen;
+              mx[e & 7] = fmaxf(mx[e & 7], in ? __uint_as_float(v[e]) : -INFINITY);
+            }
           }
         }
       }
@@ -386,10 +393,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         tmem_wait_st();
       }
       // pass 2: P = exp2(s * scale - base) -> bf16 parts P_hi = bf16(P), P_lo = bf16(P - P_hi)
-      // in two K-major 128B-swizzled buffers; O += P_hi V + P_lo V keeps ~16 bits of P
+      // in two K-major 128B-swizzled buffers; O += P_hi V + P_lo V keeps ~16 bits of P.
+      // All 32 lanes work: of each 32-column piece of row hrow, lane l + 16 takes columns
+      // 0..15 and lane l columns 16..31.
       uint8_t* pbuf = sP;
-      const float bb = base == -INFINITY ? 0.f : base;
-      float ps[4] = {0.f, 0.f, 0.f, 0.f};
+      const float b_own = base == -INFINITY ? 0.f : base;
+      const float b_pair = __shfl_xor_sync(0xffffffffu, b_own, 16);
+      const float bb = s_lane ? b_own : b_pair;
+      const int half = s_lane ? 0 : 16;
+      float ps = 0.f;
       for (int j = chunk_t0(c); j < chunk_t1(c); ++j) {
         const Tile tl = tile_of(p, sq, j);
         const int vhi = tl.kind == kCompressed ? min(tl.n, sq.e1 - tl.key0) : min(W, t + 1);
@@ -400,35 +412,28 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           uint32_t v[32];
           tmem_ld32(sbuf + jt * kTN + q * 32, v);
           tmem_wait_ld();
-          if (s_lane) {
-            uint32_t pk[16], pl[16];
+          float x[16];
+          pair_split(v, s_lane, x);
+          const int col0 = q * 32 + half;
+          uint32_t pk[8], pl[8];
+          const bool visible = (uint32_t)(q * 32 + 32) <= vlen;  // the whole piece: no masks
+          ps += visible ? p_piece<false, kPBf16Pair>(x, p.scale_log2, bb, col0, vlen, 1.f, pk, pl)
+                        : p_piece<true, kPBf16Pair>(x, p.scale_log2, bb, col0, vlen, 1.f, pk, pl);
+          // chunk keys jt*128 + col0 .. -> 64-key P chunk (jt*2 + q/2), 16-byte units
+          // (q&1)*4 + half/8 + w
+          uint8_t* rowp = pbuf + (jt * 2 + (q >> 1)) * kPChunkBytes + hrow * 128;
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int c0 = q * 32 + 2 * e;
-              const float p0 = (uint32_t)c0 < vlen
-                                   ? fast_exp2(fmaf(__uint_as_float(v[2 * e]), p.scale_log2, -bb))
-                                   : 0.f;
-              const float p1 = (uint32_t)(c0 + 1) < vlen
-                                   ? fast_exp2(fmaf(__uint_as_float(v[2 * e + 1]), p.scale_log2, -bb))
-                                   : 0.f;
-              split_bf16x2(p0, p1, pk[e], pl[e]);
-              ps[e & 3] += p0 + p1;
-            }
-            // chunk keys jt*128 + q*32 .. -> 64-key P chunk (jt*2 + q/2), units (q&1)*4 + w
-            uint8_t* rowp = pbuf + (jt * 2 + (q >> 1)) * kPChunkBytes + hrow * 128;
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-              const int u = (q & 1) * 4 + w;
-              const int us = u ^ (hrow & 7);
-              *reinterpret_cast<uint4*>(rowp + us * 16) =
-                  make_uint4(pk[4 * w], pk[4 * w + 1], pk[4 * w + 2], pk[4 * w + 3]);
-              *reinterpret_cast<uint4*>(rowp + kPBytes + us * 16) =
-                  make_uint4(pl[4 * w], pl[4 * w + 1], pl[4 * w + 2], pl[4 * w + 3]);
-            }
+          for (int w = 0; w < 2; ++w) {
+            const int u = (q & 1) * 4 + (half >> 3) + w;
+            const int us = u ^ (hrow & 7);
+            *reinterpret_cast<uint4*>(rowp + us * 16) =
+                make_uint4(pk[4 * w], pk[4 * w + 1], pk[4 * w + 2], pk[4 * w + 3]);
+            *reinterpret_cast<uint4*>(rowp + kPBytes + us * 16) =
+                make_uint4(pl[4 * w], pl[4 * w + 1], pl[4 * w + 2], pl[4 * w + 3]);
           }
         }
       }
-      l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+      l += ps + __shfl_xor_sync(0xffffffffu, ps, 16);
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();

@@ -13,12 +13,15 @@ boxes (and its bf16 query, after the last e4m3 score MMA); the UMMA warp consume
 boxes in order (and the V groups from a 3-slot buffer ring after the softmax of the tile);
 the converter warps consume the V boxes in order, two 16-key groups per box, into the
 buffer ring, and the UMMA warp releases a V box once it has both of its groups; the
-softmax of tile c waits for its scores and for P.V(c - 1). Asynchronous completions (TMA
-landings, MMA commits) happen at random later times.
+softmax of tile c waits for its scores and for the P buffer it writes: an e4m3 tile's P
+alternates between two buffers (free once P.V(c - 2) is done), the window tile's two
+parts take both (free once P.V(c - 1) is done). Asynchronous completions (TMA landings,
+MMA commits) happen at random later times.
 
 Checked, over many random schedules and tile lists (one compressed tile and the window,
-several partial tiles, window only, no window): no role waits forever, and every box a
-consumer reads is the box it expects (it has landed and has not been replaced). The same
+several partial tiles, window only, no window): no role waits forever, every box a
+consumer reads is the box it expects (it has landed and has not been replaced), and no P
+buffer is rewritten while a P.V product that reads it is in flight. The same
 model with one shared full barrier per slot (the consumers waiting on parities of the
 slot's position in the load order) must fail the second check for a split made of one
 compressed tile and the window tile.
@@ -55,9 +58,16 @@ class Bar:
         return (self.phase & 1) != parity
 
 
-def run(tiles, typed, rng):
+def run(tiles, typed, rng, nbuf=2):
     """tiles: list of (kind, n) with kind 'c' (e4m3 tile of n keys) or 'r' (window tile).
-    Returns None when every role finished with valid reads, else a failure string."""
+    nbuf: P buffers an e4m3 tile's P alternates over (1 models writing a single buffer
+    under the same waits). Returns None when every role finished with valid reads, else a
+    failure string."""
+
+    def p_bufs(c):
+        if tiles[c][0] == "r":
+            return [0, 1]
+        return [c % nbuf]
     B = {}
     for s in range(STAGES):
         B[("k_full", s)] = Bar(1)
@@ -74,6 +84,8 @@ def run(tiles, typed, rng):
         B[(name,)] = Bar(1)
     slot_box = [None] * STAGES   # box id currently in the slot (after it landed)
     vbuf = [None] * VSTAGES
+    pbuf = [None, None]          # tile whose P each buffer holds
+    p_reading = set()            # buffers read by P.V products not yet completed
     pending = []                 # async events: (callable)
     fail = []
     ntiles = len(tiles)
@@ -163,6 +175,11 @@ def run(tiles, typed, rng):
                 vstart = n
                 n += vboxes(t)
                 yield ("wait", ("p_full", pc & 1), (pc >> 1) & 1)
+                bufs = p_bufs(pc)
+                for x in bufs:
+                    if pbuf[x] != pc:
+                        fail.append(f"PV({pc}) read P buffer {x} holding {pbuf[x]}")
+                    p_reading.add(x)
                 ng = t[1] // 16
                 for g in range(ng):
                     s = cv % VSTAGES
@@ -175,14 +192,23 @@ def run(tiles, typed, rng):
                         B[("ring_empty", (vstart + g // 2) % STAGES)].arrive()
                     commit(("v_empty", s))
                     cv += 1
-                commit(("o_done", pc & 1))
+                def pv_done(pc=pc, bufs=tuple(bufs)):
+                    for x in bufs:
+                        p_reading.discard(x)
+                    B[("o_done", pc & 1)].arrive()
+                pending.append(pv_done)
 
     def softmax():
         yield ("wait", ("q_ready",), 0)
         for c in range(ntiles):
             yield ("wait", ("s_full", c & 1), (c >> 1) & 1)
-            if c > 0:
-                yield ("wait", ("o_done", (c - 1) & 1), ((c - 1) >> 1) & 1)
+            pv = c - 1 if tiles[c][0] == "r" else c - 2
+            if pv >= 0:
+                yield ("wait", ("o_done", pv & 1), (pv >> 1) & 1)
+            for x in p_bufs(c):
+                if x in p_reading:
+                    fail.append(f"softmax({c}) rewrote P buffer {x} under a P.V product")
+                pbuf[x] = c
             B[("p_full", c & 1)].arrive()
 
     def converter():
@@ -284,3 +310,11 @@ def test_shared_parity_ring_aliases():
     rng = random.Random(11)
     failures = [run([("c", 80), ("r", 128)], False, rng) for _ in range(200)]
     assert any(f is not None and "read" in f for f in failures)
+
+
+def test_one_p_buffer_with_the_same_waits_races():
+    # writing every e4m3 tile's P to one buffer while waiting only for P.V(c - 2) rewrites
+    # the buffer that P.V(c - 1) may still be reading
+    rng = random.Random(5)
+    failures = [run([("c", 128)] * 4 + [("r", 128)], True, rng, nbuf=1) for _ in range(200)]
+    assert any(f is not None and "rewrote" in f for f in failures)

@@ -71,6 +71,28 @@ def test_decode_bf16(nseq, lo, hi, gate):
     assert int(cache.err.item()) == 0
 
 
+# the last compressed tile holds 16 * odd entries, all visible: its last 32-column score
+# piece runs 16 columns past the tile, and those columns (stale tensor memory, scores of an
+# earlier tile) must enter neither P nor the row sum
+MID_PIECE_CASES = [
+    (128 * 80 + 5, 0),            # one compressed tile of 80 entries
+    (128 * (256 + 48) + 100, 0),  # last tile of 48 entries
+    (128 * (384 + 16) + 127, 2),  # last tile of 16, two splits
+    (128 * (128 + 112) + 64, 1),  # last tile of 112, one split
+]
+
+
+@pytest.mark.parametrize("ctx,splits", MID_PIECE_CASES)
+def test_decode_tile_ends_mid_piece(ctx, splits):
+    x, cache, desc = _setup(2, ctx, ctx, seed=60 + splits, splits=splits)
+    O, lse = _run(x, cache, desc)
+    for b in range(2):
+        ref, rl = _oracle(x, b)
+        compare(to64(O[b]), ref, BF16_MAX, BF16_MEAN, what=f"ctx={ctx} O[{b}]")
+        compare(to64(lse[b]), rl, LSE_MAX, LSE_MEAN, what=f"ctx={ctx} lse[{b}]", out_bf16=False)
+    assert int(cache.err.item()) == 0
+
+
 def _sample_sequences(ctx_len, n, seed):
     """n sequences drawn by a seeded generator, always with the longest and the shortest
     context among them."""

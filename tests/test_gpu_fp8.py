@@ -181,6 +181,21 @@ def test_decode_e4m3(nseq, lo, hi, gate, hq, W):
     assert int(cache.err.item()) == 0
 
 
+@pytest.mark.parametrize("ctx,splits", [
+    (128 * 80 + 5, 0),            # one compressed tile of 80 entries
+    (128 * (256 + 48) + 100, 0),  # last tile of 48 entries
+    (128 * (384 + 16) + 127, 2),  # last tile of 16, two splits
+    (128 * (128 + 112) + 64, 1),  # last tile of 112, one split
+])
+def test_decode_e4m3_tile_ends_mid_piece(ctx, splits):
+    """The last compressed tile holds 16 * odd entries, all visible: the columns of its
+    last 32-column score piece past the tile must enter neither P nor the row sum."""
+    x, cache, desc = _setup8(2, ctx, ctx, seed=70 + splits, splits=splits)
+    O, lse = _run(x, cache, desc)
+    _check(x, O, lse, range(2), what=f"ctx={ctx}")
+    assert int(cache.err.item()) == 0
+
+
 def _sample_sequences(ctx_len, n, seed):
     lens = ctx_len.numpy()
     rng = np.random.default_rng(seed)
