@@ -308,7 +308,8 @@ def gpu_main(args, rank, world, local_rank):
     # partitioned compress + prefill and copies its output rows back. Steps are pipelined
     # over three streams with two device buffer sets: the upload of step i + 1 and the
     # download of step i - 1 run while step i computes (PCIe is full duplex). The timed
-    # region runs from the first upload to the last download.
+    # region runs from the first upload to the last download, so the first upload and the
+    # last download (one step's worth of each) are spread over the timed steps.
     if not args.no_e2e:
         hQ = Q.cpu().pin_memory()
         hK = K.cpu().pin_memory()
@@ -1038,7 +1039,8 @@ def main():
     ap.add_argument("--seqlen", type=int, default=32768)
     ap.add_argument("--decode-steps", type=int, default=50)
     ap.add_argument("--steps-128k", type=int, default=10)
-    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=12,
+                    help="steps of the 32K e2e pipeline (fill and drain amortised over them)")
     ap.add_argument("--steps-bwd", type=int, default=5)
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

@@ -62,7 +62,9 @@ using namespace dsoft;
 
 constexpr int kM = 64;    // head rows
 constexpr int kD = 512;
-constexpr int kThreads = 320;  // TMA warp, UMMA warp, 4 softmax warps, 4 converter warps
+// TMA warp, score-MMA warp, 4 softmax warps, 4 converter warps, P.V-MMA warp
+constexpr int kThreads = 352;
+constexpr int kPvWarp = 10;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kLaneS = 16u << 16;   // lane offset of the score accumulators
 
@@ -128,7 +130,7 @@ struct Bars8 {
   uint64_t k_full[kStages], v8_full[kStages], ring_empty[kStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[2], p_full[2], o_done[2];
-  uint64_t drain;
+  uint64_t drain, drain_pv;  // each UMMA issuer's MMAs complete (end of the CTA)
   uint32_t tmem_base;
   int abort;
 };
@@ -189,6 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
       mbar_init(&bars->o_done[x], 1);
     }
     mbar_init(&bars->drain, 1);
+    mbar_init(&bars->drain_pv, 1);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -310,22 +313,38 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
         mbar_wait(&bars->qs_full, 0, &no_abort, 100000000ull);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------ UMMA issuer
-    // Order: S(0), then per step c >= 1: S(c) (if any), PV(c - 1), as the 16-bit kernel;
-    // it walks the load order and steps over the V boxes (the converters' share).
+  } else if (warp == 1 || warp == kPvWarp) {
+    // ------------------------------------------------------------------ UMMA issuers
+    // Warp 1 issues the score MMAs S(c) in tile order, warp kPvWarp the P.V MMAs PV(c):
+    // S(c + 1) goes out as soon as its K boxes have landed and the softmax has released
+    // score buffer (c + 1) & 1, not behind PV(c - 1), which is paced by the widening of V;
+    // its K slots then free early and the load warp streams V(c) behind them. The two
+    // streams touch different TMEM columns and shared memory; each warp's commits track its
+    // own MMAs. Both walk the load order K(0), then per step c >= 1: K(c), V(c - 1).
+    auto kboxes = [&](int c) -> uint32_t {
+      return tile_of(p, sq, sq.j0 + c).kind == kCompressed ? 4u : 8u;
+    };
+    auto vboxes = [&](const Tile& t) -> uint32_t {
+      return t.kind == kCompressed ? (uint32_t)((t.n + kVRows - 1) / kVRows) : 0u;
+    };
     if (elect_one()) {
-      bool ok = mbar_wait(&bars->q_ready, 0, abort);
-      tc_fence_after();
-      uint32_t n = 0, cv = 0;  // ring position, V groups consumed
-      uint32_t kph = 0;        // per slot: parity of the next K phase
-      bool q8_released = false;
+      bool ok = true;
       const uint32_t qbase = smem_u32(sQ);
       const uint32_t pbase = smem_u32(sP);
       const uint32_t rbase = smem_u32(sRing);
       const uint32_t vbase = smem_u32(sV);
-      for (int c = 0; c <= ntiles && ok; ++c) {
-        if (c < ntiles) {
+      if (warp == 1) {
+        ok = mbar_wait(&bars->q_ready, 0, abort);
+        tc_fence_after();
+        uint32_t n = 0;    // ring position
+        uint32_t kph = 0;  // per slot: parity of the next K phase
+        bool q8_released = false;
+        for (int c = 0; c < ntiles && ok; ++c) {
+          // K(c) follows V(c - 2) in the load order
+          if (c >= 2) n += vboxes(tile_of(p, sq, sq.j0 + c - 2));
+          // S(c) overwrites score buffer c & 1: the softmax of tile c - 2 is done with it
+          if (c >= 2 && !(ok = mbar_wait(&bars->p_full[c & 1], ((c - 2) >> 1) & 1, abort)))
+            break;
           const Tile t = tile_of(p, sq, sq.j0 + c);
           const uint32_t sb = tmem + kLaneS + (c & 1) * 256;  // S1 at sb, S2 at sb + 128
           if (t.kind == kCompressed) {
@@ -377,11 +396,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
             q8_released = true;
           }
         }
-        if (c >= 1 && ok) {
-          const int pc = c - 1;
+      } else {
+        uint32_t nk = ntiles > 0 ? kboxes(0) : 0u, nv = 0, cv = 0;  // ring counts, V groups
+        for (int pc = 0; pc < ntiles && ok; ++pc) {
           const Tile t = tile_of(p, sq, sq.j0 + pc);
-          const uint32_t vstart = n;  // ring position of V(pc)'s first box
-          if (t.kind == kCompressed) n += (t.n + kVRows - 1) / kVRows;  // V(pc): converters
+          // ring position of V(pc)'s first box: K(0 .. pc + 1) and V(0 .. pc - 1) precede it
+          if (pc + 1 < ntiles) nk += kboxes(pc + 1);
+          const uint32_t vstart = nk + nv;
+          nv += vboxes(t);
           if (!(ok = mbar_wait(&bars->p_full[pc & 1], (pc >> 1) & 1, abort))) break;
           tc_fence_after();
           const uint32_t idesc = t.kind == kCompressed ? idesc_f16_f32(kM, 256, true)
@@ -417,17 +439,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
       }
       if (!ok) {
         bars->abort = 1;
-        if (p.err_word) atomicOr(p.err_word, kErrTimeout | (1 << 11));
+        if (p.err_word) atomicOr(p.err_word, kErrTimeout | (1 << (warp == 1 ? 11 : 14)));
       }
+      // each issuer waits for its own MMAs before the CTA may release TMEM
       volatile int no_abort = 0;
-      umma_commit(&bars->drain);
-      mbar_wait(&bars->drain, 0, &no_abort, 100000000ull);
+      uint64_t* drain = warp == 1 ? &bars->drain : &bars->drain_pv;
+      umma_commit(drain);
+      mbar_wait(drain, 0, &no_abort, 100000000ull);
     }
   } else if (warp >= 2 && warp < 6) {
     // ------------------------------------------------------------------ softmax + partials
     // Lane l + 16 of a warp holds score row quad * 16 + l; lane l (< 16) holds the O row of
-    // the same head. The protocol is that of the 16-bit kernel: per chunk c (one tile):
-    // wait S(c); row max; wait PV(c - 1); lazy rescale of O; P(c); arrive p_full.
+    // the same head. Per tile c: wait S(c); row max; wait for the P buffer (PV(c - 2), or
+    // PV(c - 1) for the window tile or a rescale); lazy rescale of O; P(c); arrive p_full,
+    // which also releases score buffer c & 1 to S(c + 2).
     const int quad = warp & 3;
     const bool s_lane = lane >= 16;
     const int hrow = quad * 16 + (lane & 15);
@@ -567,7 +592,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->p_full[c & 1]);
     }
-    // the last PV's commit covers every earlier UMMA of this CTA
+    // the last PV's commit covers every earlier P.V MMA; every score MMA completed before
+    // its s_full was seen
     if (ok) ok = mbar_wait(&bars->o_done[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1, abort);
     ok = __all_sync(0xffffffffu, ok);
     float* sO = reinterpret_cast<float*>(smem + kOffStage);  // [64][kORow]

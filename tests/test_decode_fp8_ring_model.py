@@ -9,10 +9,12 @@ ahead of the current one returns at once: the aliasing the kernel must avoid).
 The roles, restated from the kernel: the load warp issues, in order, K(0), then per step
 c >= 1: K(c), V(c - 1), into a ring of 5 slots (waiting for the slot's previous box to be
 released); a compressed tile is 4 K boxes and ceil(n / 32) V boxes, the window tile 8 K
-boxes (and its bf16 query, after the last e4m3 score MMA); the UMMA warp consumes the K
-boxes in order (and the V groups from a 3-slot buffer ring after the softmax of the tile);
+boxes (and its bf16 query, after the last e4m3 score MMA); one UMMA warp consumes the K
+boxes in order for the score MMAs, S(c) once the softmax of tile c - 2 has released score
+buffer c & 1, and a second UMMA warp consumes the V groups from a 3-slot buffer ring after
+the softmax of each tile;
 the converter warps consume the V boxes in order, two 16-key groups per box, into the
-buffer ring, and the UMMA warp releases a V box once it has both of its groups; the
+buffer ring, and the P.V warp releases a V box once it has both of its groups; the
 softmax of tile c waits for its scores and for the P buffer it writes: an e4m3 tile's P
 alternates between two buffers (free once P.V(c - 2) is done), the window tile's two
 parts take both (free once P.V(c - 1) is done). Asynchronous completions (TMA landings,
@@ -85,6 +87,7 @@ def run(tiles, typed, rng, nbuf=2):
     slot_box = [None] * STAGES   # box id currently in the slot (after it landed)
     vbuf = [None] * VSTAGES
     pbuf = [None, None]          # tile whose P each buffer holds
+    s_reading = [None, None]     # tile whose scores the softmax is reading, per buffer
     p_reading = set()            # buffers read by P.V products not yet completed
     pending = []                 # async events: (callable)
     fail = []
@@ -140,68 +143,80 @@ def run(tiles, typed, rng, nbuf=2):
         # a tcgen05.commit: arrives once the MMAs issued so far have completed
         pending.append(lambda: B[name].arrive())
 
-    def umma():
+    def umma_s():
         yield ("wait", ("q_ready",), 0)
         n = 0
         kph = [0] * STAGES
-        cv = 0
         released = False
-        for c in range(ntiles + 1):
-            if c < ntiles:
-                t = tiles[c]
-                if t[0] == "r":
-                    if not released:
-                        commit(("q8_free",))
-                        released = True
-                    yield ("wait", ("qb_full",), 0)
-                for q in range(kboxes(t)):
-                    s = n % STAGES
-                    if typed:
-                        yield ("wait", ("k_full", s), kph[s])
-                        kph[s] ^= 1
-                    else:
-                        yield ("wait", ("k_full", s), (n // STAGES) & 1)
-                    if slot_box[s] != ("K", c, q):
-                        fail.append(f"UMMA read {slot_box[s]} for K{(c, q)}")
-                    commit(("ring_empty", s))
-                    n += 1
-                commit(("s_full", c & 1))
-                if has_ring and c + 1 == nct and not released:
+        for c in range(ntiles):
+            if c >= 2:
+                n += vboxes(tiles[c - 2])
+                # score buffer c & 1 is free once the softmax of tile c - 2 is done
+                yield ("wait", ("p_full", c & 1), ((c - 2) >> 1) & 1)
+                if s_reading[c & 1] is not None:
+                    fail.append(f"S({c}) overwrote the scores of tile {s_reading[c & 1]}")
+            t = tiles[c]
+            if t[0] == "r":
+                if not released:
                     commit(("q8_free",))
                     released = True
-            if c >= 1:
-                pc = c - 1
-                t = tiles[pc]
-                vstart = n
-                n += vboxes(t)
-                yield ("wait", ("p_full", pc & 1), (pc >> 1) & 1)
-                bufs = p_bufs(pc)
+                yield ("wait", ("qb_full",), 0)
+            for q in range(kboxes(t)):
+                s = n % STAGES
+                if typed:
+                    yield ("wait", ("k_full", s), kph[s])
+                    kph[s] ^= 1
+                else:
+                    yield ("wait", ("k_full", s), (n // STAGES) & 1)
+                if slot_box[s] != ("K", c, q):
+                    fail.append(f"UMMA read {slot_box[s]} for K{(c, q)}")
+                commit(("ring_empty", s))
+                n += 1
+            commit(("s_full", c & 1))
+            if has_ring and c + 1 == nct and not released:
+                commit(("q8_free",))
+                released = True
+
+    def umma_pv():
+        nk = kboxes(tiles[0]) if ntiles else 0
+        nv = 0
+        cv = 0
+        for pc in range(ntiles):
+            t = tiles[pc]
+            if pc + 1 < ntiles:
+                nk += kboxes(tiles[pc + 1])
+            vstart = nk + nv
+            nv += vboxes(t)
+            yield ("wait", ("p_full", pc & 1), (pc >> 1) & 1)
+            bufs = p_bufs(pc)
+            for x in bufs:
+                if pbuf[x] != pc:
+                    fail.append(f"PV({pc}) read P buffer {x} holding {pbuf[x]}")
+                p_reading.add(x)
+            ng = t[1] // 16
+            for g in range(ng):
+                s = cv % VSTAGES
+                yield ("wait", ("v_full", s), (cv // VSTAGES) & 1)
+                if vbuf[s] != (pc, g):
+                    fail.append(f"PV read {vbuf[s]} for group {(pc, g)}")
+                # the converters have read the e4m3 box of this group: released once both
+                # of its groups (or the tile's last) are in
+                if t[0] == "c" and (g % 2 == 1 or g == ng - 1):
+                    B[("ring_empty", (vstart + g // 2) % STAGES)].arrive()
+                commit(("v_empty", s))
+                cv += 1
+
+            def pv_done(pc=pc, bufs=tuple(bufs)):
                 for x in bufs:
-                    if pbuf[x] != pc:
-                        fail.append(f"PV({pc}) read P buffer {x} holding {pbuf[x]}")
-                    p_reading.add(x)
-                ng = t[1] // 16
-                for g in range(ng):
-                    s = cv % VSTAGES
-                    yield ("wait", ("v_full", s), (cv // VSTAGES) & 1)
-                    if vbuf[s] != (pc, g):
-                        fail.append(f"PV read {vbuf[s]} for group {(pc, g)}")
-                    # the converters have read the e4m3 box of this group: released once both
-                    # of its groups (or the tile's last) are in
-                    if t[0] == "c" and (g % 2 == 1 or g == ng - 1):
-                        B[("ring_empty", (vstart + g // 2) % STAGES)].arrive()
-                    commit(("v_empty", s))
-                    cv += 1
-                def pv_done(pc=pc, bufs=tuple(bufs)):
-                    for x in bufs:
-                        p_reading.discard(x)
-                    B[("o_done", pc & 1)].arrive()
-                pending.append(pv_done)
+                    p_reading.discard(x)
+                B[("o_done", pc & 1)].arrive()
+            pending.append(pv_done)
 
     def softmax():
         yield ("wait", ("q_ready",), 0)
         for c in range(ntiles):
             yield ("wait", ("s_full", c & 1), (c >> 1) & 1)
+            s_reading[c & 1] = c
             pv = c - 1 if tiles[c][0] == "r" else c - 2
             if pv >= 0:
                 yield ("wait", ("o_done", pv & 1), (pv >> 1) & 1)
@@ -209,6 +224,7 @@ def run(tiles, typed, rng, nbuf=2):
                 if x in p_reading:
                     fail.append(f"softmax({c}) rewrote P buffer {x} under a P.V product")
                 pbuf[x] = c
+            s_reading[c & 1] = None
             B[("p_full", c & 1)].arrive()
 
     def converter():
@@ -255,8 +271,8 @@ def run(tiles, typed, rng, nbuf=2):
                     pending.append(landing)
                     cv += 1
 
-    roles = {"producer": producer(), "umma": umma(), "softmax": softmax(),
-             "converter": converter()}
+    roles = {"producer": producer(), "umma_s": umma_s(), "umma_pv": umma_pv(),
+             "softmax": softmax(), "converter": converter()}
     waiting = {name: None for name in roles}
     for _ in range(200000):
         runnable = [r for r in roles if waiting[r] is None or
