@@ -62,9 +62,11 @@ using namespace dsoft;
 
 constexpr int kM = 64;    // head rows
 constexpr int kD = 512;
-// TMA warp, score-MMA warp, 4 softmax warps, 4 converter warps, P.V-MMA warp
-constexpr int kThreads = 352;
+// K load warp, score-MMA warp, 4 softmax warps, 4 converter warps, P.V-MMA warp,
+// V load warp
+constexpr int kThreads = 384;
 constexpr int kPvWarp = 10;
+constexpr int kVLoadWarp = 11;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kLaneS = 16u << 16;   // lane offset of the score accumulators
 
@@ -73,18 +75,20 @@ constexpr uint32_t kQPartBytes = 4 * kQChunkBytes;  // 32 KB: one e4m3 part of t
 constexpr uint32_t kQ16Bytes = 8 * kQChunkBytes;    // 64 KB: the bf16 query
 constexpr uint32_t kPChunkBytes = kM * 128;     // 8 KB: 64 rows x 64 keys (16-bit)
 constexpr uint32_t kPBytes = 2 * kPChunkBytes;  // 16 KB: one part of P (128 keys)
-constexpr int kStages = 5;
+constexpr int kKStages = 3;                     // K ring: 16 KB boxes
+constexpr int kV8Stages = 3;                    // V ring: 16 KB boxes of e4m3 values
 constexpr uint32_t kSlot = 16384;               // 16 KB ring slot
 constexpr int kVRows = 32;                      // keys of one e4m3 V box (4 chunks x 4 KB)
 constexpr uint32_t kV8Chunk = kVRows * 128;     // 4 KB: 32 keys x 128 codes
-constexpr int kVStages = 3;
+constexpr int kVStages = 2;
 constexpr uint32_t kVChunkBytes = 16 * 128;     // 2 KB: 16 keys x 64 values (16-bit)
 constexpr uint32_t kVSlot = 8 * kVChunkBytes;   // 16 KB: 16 keys x 512 values
 
 constexpr uint32_t kOffQ = 0;                           // Q1 | Q2, later the bf16 query
 constexpr uint32_t kOffP = kQ16Bytes;                   // P hi | P lo
-constexpr uint32_t kOffRing = kOffP + 2 * kPBytes;
-constexpr uint32_t kOffV = kOffRing + kStages * kSlot;
+constexpr uint32_t kOffRing = kOffP + 2 * kPBytes;      // K ring
+constexpr uint32_t kOffVRing = kOffRing + kKStages * kSlot;
+constexpr uint32_t kOffV = kOffVRing + kV8Stages * kSlot;
 constexpr uint32_t kOffBar = kOffV + kVStages * kVSlot;
 constexpr uint32_t kOffRowScale = kOffBar + 512;        // 64 floats
 constexpr uint32_t kSmemBytes = kOffRowScale + 256 + 1024;
@@ -124,10 +128,10 @@ struct Bars8 {
   uint64_t q_ready;   // Q1, Q2 and the row scales written (converters)
   uint64_t qb_full;   // bf16 query of the ring tile landed (TMA)
   uint64_t q8_free;   // the last e4m3 score MMA completed: the query region may be reused
-  // A ring slot holds a K box or a V box; each kind completes on its own barrier, so that
-  // each consumer (UMMA warp: K; converter warps: V) waits only on phases of its own boxes,
-  // in order, and a parity wait can never match a phase that belongs to the other kind.
-  uint64_t k_full[kStages], v8_full[kStages], ring_empty[kStages];
+  // K boxes and e4m3 V boxes stream through rings of their own, each filled by its own
+  // load warp, so that V boxes waiting to be widened never hold back the K stream
+  uint64_t k_full[kKStages], k_empty[kKStages];
+  uint64_t v8_full[kV8Stages], v8_empty[kV8Stages];
   uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[2], p_full[2], o_done[2];
   uint64_t drain, drain_pv;  // each UMMA issuer's MMAs complete (end of the CTA)
@@ -164,6 +168,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
   uint8_t* sQ = smem + kOffQ;
   uint8_t* sP = smem + kOffP;
   uint8_t* sRing = smem + kOffRing;
+  uint8_t* sVRing = smem + kOffVRing;
   uint8_t* sV = smem + kOffV;
   Bars8* bars = reinterpret_cast<Bars8*>(smem + kOffBar);
   float* sRS = reinterpret_cast<float*>(smem + kOffRowScale);
@@ -176,10 +181,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
     mbar_init(&bars->q_ready, 1);
     mbar_init(&bars->qb_full, 1);
     mbar_init(&bars->q8_free, 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kKStages; ++s) {
       mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
+    }
+    for (int s = 0; s < kV8Stages; ++s) {
       mbar_init(&bars->v8_full[s], 1);
-      mbar_init(&bars->ring_empty[s], 1);
+      mbar_init(&bars->v8_empty[s], 1);
     }
     for (int s = 0; s < kVStages; ++s) {
       mbar_init(&bars->v_full[s], 4);  // one arrival per converter warp
@@ -222,111 +230,90 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
       dst_ml[2 * h] = -INFINITY;
       dst_ml[2 * h + 1] = 0.f;
     }
-  } else if (warp == 0) {
+  } else if (warp == 0 || warp == kVLoadWarp) {
     // ------------------------------------------------------------------ loads
-    // One ring of 16 KB boxes, in the order K(0), then per step c >= 1: K(c), V(c - 1).
-    // The UMMA warp consumes (and releases) the K boxes, the converter warps the V boxes.
+    // Warp 0 streams the K boxes of the split's tiles into the K ring (and the queries),
+    // warp kVLoadWarp the e4m3 V boxes into the V ring; the window tile's values go to the
+    // f16 V buffers directly (converter warps). Box n of a ring sits in slot n % stages and
+    // completes phase n / stages of that slot's full barrier.
     if (elect_one()) {
       const uint64_t pol = policy_evict_first();  // every cache row is read once
-      if (split == 0 && p.err_word) {
-        const int ctx = p.ctx_len[b];
-        if (ctx < 1 || ctx > p.seqlen) atomicOr(p.err_word, kErrCtxRange);
-        const int x = sq.t + 1 - p.W;
-        if ((x < 0 ? 0 : x / p.block) > p.n_entries[b]) atomicOr(p.err_word, kErrCacheShort);
-      }
-      // the bf16 query, staged for the converter warps in the P buffer (box of chunks 0-3)
-      // and the V buffers (chunks 4-7): both are free until Q1/Q2 are ready
-      mbar_expect_tx(&bars->qs_full, kQ16Bytes);
-      tma_load_3d(sP, &p.tmQb, &bars->qs_full, 0, b * p.hq, 0, pol);
-      tma_load_3d(sV, &p.tmQb, &bars->qs_full, 0, b * p.hq, 4, pol);
-      uint32_t cnt = 0;  // loads issued
-      uint32_t kph = 0, vph = 0;  // per slot: parity of the next K / V phase
-      uint32_t last_v = 0;        // per slot: the latest box was a V box
-      bool ok = true, q_issued = false;
-      auto load = [&](const CUtensorMap* map, int row, int chunk, bool is_v) -> bool {
-        const uint32_t s = cnt % kStages;
-        if (cnt >= (uint32_t)kStages &&
-            !mbar_wait(&bars->ring_empty[s], ((cnt / kStages) - 1) & 1, abort))
-          return false;
-        uint64_t* full = is_v ? &bars->v8_full[s] : &bars->k_full[s];
-        mbar_expect_tx(full, kSlot);
-        tma_load_3d(sRing + s * kSlot, map, full, 0, row, chunk, pol);
-        if (is_v) {
-          vph ^= 1u << s;
-          last_v |= 1u << s;
-        } else {
-          kph ^= 1u << s;
-          last_v &= ~(1u << s);
+      const bool kw = warp == 0;
+      const int stages = kw ? kKStages : kV8Stages;
+      uint64_t* full = kw ? bars->k_full : bars->v8_full;
+      uint64_t* empty = kw ? bars->k_empty : bars->v8_empty;
+      uint8_t* ring = kw ? sRing : sVRing;
+      if (kw) {
+        if (split == 0 && p.err_word) {
+          const int ctx = p.ctx_len[b];
+          if (ctx < 1 || ctx > p.seqlen) atomicOr(p.err_word, kErrCtxRange);
+          const int x = sq.t + 1 - p.W;
+          if ((x < 0 ? 0 : x / p.block) > p.n_entries[b]) atomicOr(p.err_word, kErrCacheShort);
         }
+        // the bf16 query, staged for the converter warps in the P buffer (box of chunks
+        // 0-3) and the V buffers (chunks 4-7): both are free until Q1/Q2 are ready
+        mbar_expect_tx(&bars->qs_full, kQ16Bytes);
+        tma_load_3d(sP, &p.tmQb, &bars->qs_full, 0, b * p.hq, 0, pol);
+        tma_load_3d(sV, &p.tmQb, &bars->qs_full, 0, b * p.hq, 4, pol);
+      }
+      uint32_t cnt = 0;  // boxes issued into this ring
+      bool ok = true, q_issued = false;
+      auto load = [&](const CUtensorMap* map, int row, int chunk) -> bool {
+        const uint32_t s = cnt % stages;
+        if (cnt >= (uint32_t)stages &&
+            !mbar_wait(&empty[s], ((cnt / stages) - 1) & 1, abort))
+          return false;
+        mbar_expect_tx(&full[s], kSlot);
+        tma_load_3d(ring + s * kSlot, map, &full[s], 0, row, chunk, pol);
         ++cnt;
         return true;
       };
-      auto load_tile = [&](int j, bool is_v) -> bool {
-        const Tile t = tile_of(p, sq, j);
+      for (int c = 0; c < ntiles && ok; ++c) {
+        const Tile t = tile_of(p, sq, sq.j0 + c);
         if (t.kind == kCompressed) {
           int page = p.page_table[(int64_t)b * p.max_pages + t.key0 / p.PE];
           if (page < 0 || page >= p.num_pages) {
-            if (p.err_word && !is_v) atomicOr(p.err_word, kErrPageRange);
+            if (p.err_word && kw) atomicOr(p.err_word, kErrPageRange);
             page = 0;
           }
           const int row = page * p.PE + t.key0 % p.PE;
-          if (is_v) {
-            for (int q = 0; q < (t.n + kVRows - 1) / kVRows; ++q)
-              if (!load(&p.tmV8, row + q * kVRows, 0, true)) return false;
+          if (kw) {
+            for (int q = 0; q < 4 && ok; ++q) ok = load(&p.tmK8, row, q);
           } else {
-            for (int q = 0; q < 4; ++q)
-              if (!load(&p.tmK8, row, q, false)) return false;
+            for (int q = 0; q < (t.n + kVRows - 1) / kVRows && ok; ++q)
+              ok = load(&p.tmV8, row + q * kVRows, 0);
           }
-        } else if (!is_v) {
-          // the bf16 query replaces Q1/Q2 once the last e4m3 score MMA has completed; the
-          // window's values go to the V buffers directly (converter warps)
-          if (!mbar_wait(&bars->q8_free, 0, abort)) return false;
+        } else if (kw) {
+          // the bf16 query replaces Q1/Q2 once the last e4m3 score MMA has completed
+          if (!(ok = mbar_wait(&bars->q8_free, 0, abort))) break;
           mbar_expect_tx(&bars->qb_full, kQ16Bytes);
           for (int h = 0; h < 2; ++h)
             tma_load_3d(sQ + h * (kQ16Bytes / 2), &p.tmQb, &bars->qb_full, 0, b * p.hq, 4 * h,
                         pol);
           q_issued = true;
-          for (int q = 0; q < 8; ++q)
-            if (!load(&p.tmRk, b * p.W, q, false)) return false;
+          for (int q = 0; q < 8 && ok; ++q) ok = load(&p.tmRk, b * p.W, q);
         }
-        return true;
-      };
-      for (int c = 0; c <= ntiles && ok; ++c) {
-        if (c < ntiles) ok = load_tile(sq.j0 + c, false);
-        if (c >= 1 && ok) ok = load_tile(sq.j0 + c - 1, true);
       }
       if (!ok) {
         bars->abort = 1;
-        if (p.err_word) atomicOr(p.err_word, kErrTimeout | (1 << 9));
-        // load n could only be issued once load n - kStages had been released: at most the
-        // latest box of each slot is in flight, plus the bf16 query. The latest box of slot
-        // s completes the phase of parity (kph or vph, bit s) ^ 1 of its kind's barrier.
+        if (p.err_word) atomicOr(p.err_word, kErrTimeout | (1 << (kw ? 9 : 15)));
+        // box n could only be issued once box n - stages had been released: at most the
+        // last `stages` boxes are in flight, plus the queries
         volatile int no_abort = 0;
-        const uint32_t used = cnt < (uint32_t)kStages ? cnt : (uint32_t)kStages;
-        for (uint32_t s = 0; s < used; ++s) {
-          if ((last_v >> s) & 1u)
-            mbar_wait(&bars->v8_full[s], ((vph >> s) & 1u) ^ 1u, &no_abort, 100000000ull);
-          else
-            mbar_wait(&bars->k_full[s], ((kph >> s) & 1u) ^ 1u, &no_abort, 100000000ull);
-        }
+        const uint32_t first = cnt > (uint32_t)stages ? cnt - stages : 0u;
+        for (uint32_t n = first; n < cnt; ++n)
+          mbar_wait(&full[n % stages], (n / stages) & 1, &no_abort, 100000000ull);
         if (q_issued) mbar_wait(&bars->qb_full, 0, &no_abort, 100000000ull);
-        mbar_wait(&bars->qs_full, 0, &no_abort, 100000000ull);
+        if (kw) mbar_wait(&bars->qs_full, 0, &no_abort, 100000000ull);
       }
     }
   } else if (warp == 1 || warp == kPvWarp) {
     // ------------------------------------------------------------------ UMMA issuers
     // Warp 1 issues the score MMAs S(c) in tile order, warp kPvWarp the P.V MMAs PV(c):
     // S(c + 1) goes out as soon as its K boxes have landed and the softmax has released
-    // score buffer (c + 1) & 1, not behind PV(c - 1), which is paced by the widening of V;
-    // its K slots then free early and the load warp streams V(c) behind them. The two
-    // streams touch different TMEM columns and shared memory; each warp's commits track its
-    // own MMAs. Both walk the load order K(0), then per step c >= 1: K(c), V(c - 1).
-    auto kboxes = [&](int c) -> uint32_t {
-      return tile_of(p, sq, sq.j0 + c).kind == kCompressed ? 4u : 8u;
-    };
-    auto vboxes = [&](const Tile& t) -> uint32_t {
-      return t.kind == kCompressed ? (uint32_t)((t.n + kVRows - 1) / kVRows) : 0u;
-    };
+    // score buffer (c + 1) & 1, not behind PV(c - 1), which is paced by the widening of V.
+    // The two streams touch different TMEM columns and shared memory; each warp's commits
+    // track its own MMAs.
     if (elect_one()) {
       bool ok = true;
       const uint32_t qbase = smem_u32(sQ);
@@ -336,12 +323,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
       if (warp == 1) {
         ok = mbar_wait(&bars->q_ready, 0, abort);
         tc_fence_after();
-        uint32_t n = 0;    // ring position
-        uint32_t kph = 0;  // per slot: parity of the next K phase
+        uint32_t n = 0;  // K boxes consumed
         bool q8_released = false;
         for (int c = 0; c < ntiles && ok; ++c) {
-          // K(c) follows V(c - 2) in the load order
-          if (c >= 2) n += vboxes(tile_of(p, sq, sq.j0 + c - 2));
           // S(c) overwrites score buffer c & 1: the softmax of tile c - 2 is done with it
           if (c >= 2 && !(ok = mbar_wait(&bars->p_full[c & 1], ((c - 2) >> 1) & 1, abort)))
             break;
@@ -350,9 +334,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
           if (t.kind == kCompressed) {
             const uint32_t idesc = idesc_e4m3_f32(kM, t.n);
             for (int q = 0; q < 4 && ok; ++q) {
-              const uint32_t s = n % kStages;
-              if (!(ok = mbar_wait(&bars->k_full[s], (kph >> s) & 1u, abort))) break;
-              kph ^= 1u << s;
+              const uint32_t s = n % kKStages;
+              if (!(ok = mbar_wait(&bars->k_full[s], (n / kKStages) & 1, abort))) break;
               tc_fence_after();
               const uint32_t kaddr = rbase + s * kSlot;
 #pragma unroll
@@ -363,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
                 umma_ss_f8(sb, sdesc_sw128(qa, 16, 1024), kd, idesc, acc);
                 umma_ss_f8(sb + 128, sdesc_sw128(qa + kQPartBytes, 16, 1024), kd, idesc, acc);
               }
-              umma_commit(&bars->ring_empty[s]);
+              umma_commit(&bars->k_empty[s]);
               ++n;
             }
           } else {
@@ -375,16 +358,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
             tc_fence_after();
             const uint32_t idesc = idesc_bf16_f32(kM, t.n, false);
             for (int q = 0; q < 8 && ok; ++q) {
-              const uint32_t s = n % kStages;
-              if (!(ok = mbar_wait(&bars->k_full[s], (kph >> s) & 1u, abort))) break;
-              kph ^= 1u << s;
+              const uint32_t s = n % kKStages;
+              if (!(ok = mbar_wait(&bars->k_full[s], (n / kKStages) & 1, abort))) break;
               tc_fence_after();
               const uint32_t kaddr = rbase + s * kSlot;
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)  // K = 16 bf16 per UMMA
                 umma_ss(sb, sdesc_sw128(qbase + q * kQChunkBytes + kk * 32, 16, 1024),
                         sdesc_sw128(kaddr + kk * 32, 16, 1024), idesc, (q | kk) != 0);
-              umma_commit(&bars->ring_empty[s]);
+              umma_commit(&bars->k_empty[s]);
               ++n;
             }
           }
@@ -397,13 +379,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
           }
         }
       } else {
-        uint32_t nk = ntiles > 0 ? kboxes(0) : 0u, nv = 0, cv = 0;  // ring counts, V groups
+        uint32_t nv = 0, cv = 0;  // V boxes before the tile, V groups consumed
         for (int pc = 0; pc < ntiles && ok; ++pc) {
           const Tile t = tile_of(p, sq, sq.j0 + pc);
-          // ring position of V(pc)'s first box: K(0 .. pc + 1) and V(0 .. pc - 1) precede it
-          if (pc + 1 < ntiles) nk += kboxes(pc + 1);
-          const uint32_t vstart = nk + nv;
-          nv += vboxes(t);
+          const uint32_t vstart = nv;  // V ring index of the tile's first box
+          if (t.kind == kCompressed) nv += (t.n + kVRows - 1) / kVRows;
           if (!(ok = mbar_wait(&bars->p_full[pc & 1], (pc >> 1) & 1, abort))) break;
           tc_fence_after();
           const uint32_t idesc = t.kind == kCompressed ? idesc_f16_f32(kM, 256, true)
@@ -418,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
             // every converter warp has widened this group: an e4m3 box is free once both of
             // its groups (or the tile's last) are in
             if (f8 && ((g & 1) == 1 || g == ng - 1))
-              mbar_arrive(&bars->ring_empty[(vstart + (g >> 1)) % kStages]);
+              mbar_arrive(&bars->v8_empty[(vstart + (g >> 1)) % kV8Stages]);
             tc_fence_after();
             const uint32_t vaddr = vbase + s * kVSlot;
             const uint32_t paddr =
@@ -741,17 +721,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
     named_sync(2, 128);
     if (ct == 0) mbar_arrive(&bars->q_ready);
 
-    // (2) V groups of 16 keys in key order into the 3-deep V buffer ring: e4m3 boxes of the
-    // load ring widened to f16, the window tile's bf16 values by TMA. Thread (cw, lane)
-    // widens keys kr and kr + 8 of a group at values 32*c32 .. 32*c32 + 31.
+    // (2) V groups of 16 keys in key order into the f16 V buffers: e4m3 boxes of the V
+    // ring widened, the window tile's bf16 values by TMA. Thread (cw, lane) widens keys kr
+    // and kr + 8 of a group at values 32*c32 .. 32*c32 + 31.
     const int kr = lane & 7;
     const int c32 = cw * 4 + (lane >> 3);
     bool ok = q_ok;
-    uint32_t n = 0, cv = 0;  // ring position, V groups produced
-    uint32_t vph = 0;        // per slot: parity of the next V phase
-    for (int c = 0; c <= ntiles && ok; ++c) {
-      if (c < ntiles) n += tile_of(p, sq, sq.j0 + c).kind == kCompressed ? 4 : 8;  // K(c)
-      if (c == 0) continue;
+    uint32_t n = 0, cv = 0;  // V ring boxes before the tile, V groups produced
+    for (int c = 1; c <= ntiles && ok; ++c) {
       const Tile t = tile_of(p, sq, sq.j0 + c - 1);
       const int ng = t.n / 16;
       if (t.kind == kCompressed) {
@@ -760,18 +737,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
         const int vlen = min(t.n, sq.e1 - t.key0);
         for (int g = 0; g < ng && ok; ++g, ++cv) {
           const uint32_t sidx = n + (g >> 1);
-          const uint32_t rs = sidx % kStages;
+          const uint32_t rs = sidx % kV8Stages;
           bool w_ok = true;
-          if ((g & 1) == 0) {
-            w_ok = __all_sync(0xffffffffu, mbar_wait(&bars->v8_full[rs], (vph >> rs) & 1u, abort));
-            vph ^= 1u << rs;
-          }
+          if ((g & 1) == 0)
+            w_ok = __all_sync(0xffffffffu,
+                              mbar_wait(&bars->v8_full[rs], (sidx / kV8Stages) & 1, abort));
           const uint32_t vs = cv % kVStages;
           if (w_ok && cv >= (uint32_t)kVStages)
             w_ok = __all_sync(0xffffffffu,
                               mbar_wait(&bars->v_empty[vs], ((cv / kVStages) - 1) & 1, abort));
           if (w_ok) {
-            const uint8_t* box = sRing + rs * kSlot + (c32 >> 2) * kV8Chunk;
+            const uint8_t* box = sVRing + rs * kSlot + (c32 >> 2) * kV8Chunk;
             uint8_t* dst = sV + vs * kVSlot + (c32 >> 1) * kVChunkBytes;
 #pragma unroll
             for (int it = 0; it < 2; ++it) {
