@@ -16,11 +16,11 @@
 //    are exact for every element within 2^13 of the head's largest (below that the part
 //    error is under 2^-21 of the largest |q|). S1 = Q1 K and S2 = Q2 K go to two TMEM
 //    accumulators; the softmax forms s = (S1 + S2 / 16) * r_h * k_scale * scale.
-//  * P.V runs on kind::f16 with f16 operands. The e4m3 values arrive by TMA in the same ring
-//    as the keys (one 16 KB box = 32 keys x 512 codes), loaded a tile ahead; converter warps
-//    widen each 16-key group to f16 values times 2^-8 (exact, by moving the code's bits) into
-//    a 3-deep ring of MN-major 128-byte-swizzled buffers (each warp hands its part of a
-//    group over on its own; the UMMA warp releases a box once both of its groups are in).
+//  * P.V runs on kind::f16 with f16 operands. The e4m3 values arrive by TMA in a ring of
+//    their own (one 16 KB box = 32 keys x 512 codes); converter warps widen each 16-key
+//    group to f16 values times 2^-8 (exact, by moving the code's bits) into two MN-major
+//    128-byte-swizzled buffers (each warp hands its part of a group over on its own; the
+//    P.V warp releases a box once both of its groups are in).
 //    P enters as one f16 value (11 significant bits: its rounding moves the output by at
 //    most 2^-12 of the value spread, a quarter of the bf16 output's own rounding),
 //    pre-scaled by 2^7 so that small P stay clear of the f16 subnormal range while the
@@ -31,12 +31,12 @@
 //    query replaces Q1/Q2 in shared memory, its scores accumulate in S1 (kind::f16 bf16),
 //    its P goes to bf16 hi + lo parts divided by v_scale * 2^8 (O keeps its units), and its
 //    values land in the same V buffers by TMA.
-//  * Roles: warp 0 issues the loads into a 5-slot ring of 16 KB boxes in the order K(0),
-//    then per step c >= 1: K(c), V(c - 1) (K: 128 keys x one 128-byte column chunk; V: 32
-//    keys x 512 codes; the window tile's bf16 K in 64-column chunks), the bf16 query (staged
-//    for the converters at the start, and again for the window tile); warp 1 issues the
-//    UMMAs; warps 2-5 run the softmax (lazy rescale, as the 16-bit kernel) and the
-//    epilogue; warps 6-9 prepare Q1/Q2 and widen V.
+//  * Roles: warp 0 loads the K boxes into a 3-slot K ring (128 keys x one 128-byte column
+//    chunk; the window tile's bf16 K in 64-column chunks) and the bf16 query (staged for
+//    the converters at the start, and again for the window tile); warp 11 loads the e4m3 V
+//    boxes into a 3-slot V ring; warp 1 issues the score UMMAs, warp 10 the P.V UMMAs;
+//    warps 2-5 run the softmax (lazy rescale, as the 16-bit kernel) and the epilogue;
+//    warps 6-9 prepare Q1/Q2 and widen V.
 //  * TMEM: O (64 x 512 f32, M = 64 layout) in lanes 0-15 of each 32-lane subpartition;
 //    two score buffers of S1 | S2 (128 columns each) in lanes 16-31.
 //  * All mbarrier waits are bounded (HCA_ERR_TIMEOUT on give-up); on give-up every issuing
