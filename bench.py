@@ -591,9 +591,8 @@ def bench_decode_1m(args, dev, rank, world, barrier, max_over_ranks, peaks, e4m3
         for s in range(steps_per):
             p = ctx0 - 1 + s                 # position of the new token
             if last:
-                slot = p % WIN
-                rk[:, slot].copy_(new_k[s, :, 0])
-                rv[:, slot].copy_(new_v[s, :, 0])
+                # the new token into ring slot p % WIN (one launch for K and V)
+                ops.ring_append(descs[s], new_k[s], new_v[s], ctx[s], rk, rv)
                 if (p + 1) % BLOCK == 0:     # token completes block p // BLOCK
                     B.check(B.hca_compress(cdesc, rk.data_ptr(), rv.data_ptr(), WIN,
                                            p // BLOCK, 1, cache.c,
@@ -617,7 +616,8 @@ def bench_decode_1m(args, dev, rank, world, barrier, max_over_ranks, peaks, e4m3
     byts = steps_per * byts_step + nseq * (BLOCK * D * 2 * 2 + D * 2 * eb)
     gbs = byts / (ms * 1e-3) / 1e9 / world  # per GPU
     nsplit = B.hca_decode_workspace_bytes(descs[0]) // (nseq * HQ * (D + 2) * 4)
-    launches = (4 * 2 + 1) if world == 1 else (4 * 3 + (1 if last else 0))
+    # per step: ring update (the rank holding the ring), decode, merge; one compress
+    launches = (4 * 3 + 1) if world == 1 else (4 * 3 + (4 + 1 if last else 0))
     return {"value": round(nseq * steps_per / (ms * 1e-3), 1), "unit": "tokens/s",
             "ms_per_step": round(ms, 4), "ms_per_decode_step": round(ms / steps_per, 4),
             "workload": "16 sequences at context 1,048,576 (8191 entries + 128 raw), 64 heads, "

@@ -15,7 +15,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libhca.so")
-SOURCES = ["hca_api.cu", "compress.cu", "simt.cu", "prefill_tc.cu", "prefill_pair.cu", "decode_tc.cu", "decode_fp8.cu",
+SOURCES = ["hca_api.cu", "compress.cu", "ring.cu", "simt.cu", "prefill_tc.cu", "prefill_pair.cu", "decode_tc.cu", "decode_fp8.cu",
            "backward_simt.cu", "backward_tc.cu", "gemm_tc.cu", "vha.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -210,6 +210,22 @@ int32_t hca_compress(const hca_desc* d, const void* K, const void* V,
                                    reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int32_t hca_ring_append(const hca_desc* d, const void* new_k, const void* new_v,
+                        const int32_t* ctx_len, void* ring_k, void* ring_v,
+                        hca_stream_t stream) {
+  int32_t st = check_desc(d);
+  if (st != HCA_OK) return st;
+  if (d->batch == 0) return HCA_OK;
+  if (!new_k || !new_v || !ctx_len || !ring_k || !ring_v) return HCA_EINVAL;
+  if (d->seqlen < 1) return HCA_EINVAL;
+  const int esize = d->dtype == HCA_BF16 ? 2 : 4;
+  if (((int64_t)d->hkv * d->head_dim * esize) % 16 != 0) return HCA_EUNSUPPORTED;
+  if (!aligned16(new_k) || !aligned16(new_v) || !aligned16(ring_k) || !aligned16(ring_v))
+    return HCA_EINVAL;
+  return from_cuda(launch_ring_append(*d, new_k, new_v, ctx_len, ring_k, ring_v,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int32_t hca_attn_prefill_range(const hca_desc* d, int32_t q_pos0, int32_t kv_pos0,
                                int32_t kv_len, const void* Q, const void* K, const void* V,
                                const hca_cache* cache, void* O, float* lse, int32_t* dbg_mask,

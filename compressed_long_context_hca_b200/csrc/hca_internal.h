@@ -41,6 +41,9 @@ int device_sm_count();
 cudaError_t launch_compress(const hca_desc& d, const void* K, const void* V,
                             int64_t batch_stride_tokens, int32_t first_block,
                             int32_t n_blocks, const hca_cache& c, cudaStream_t s);
+cudaError_t launch_ring_append(const hca_desc& d, const void* new_k, const void* new_v,
+                               const int32_t* ctx_len, void* ring_k, void* ring_v,
+                               cudaStream_t s);
 
 // Query rows of a prefill call: row t of a sequence is position q_pos0 + t; K/V row u is
 // position kv_pos0 + u, kv_len rows per sequence (a whole sequence: 0, 0, seqlen).

@@ -56,6 +56,18 @@ def compress(desc: B.HcaDesc, K: torch.Tensor, V: torch.Tensor, cache: B.PagedCa
     B.check(st, "hca_compress")
 
 
+def ring_append(desc: B.HcaDesc, new_k: torch.Tensor, new_v: torch.Tensor,
+                ctx_len: torch.Tensor, ring_k: torch.Tensor, ring_v: torch.Tensor,
+                stream=None) -> None:
+    """Write the new token's rows new_k/new_v [nseq, hkv, D] into slot (ctx_len - 1) % W of
+    the rings ring_k/ring_v [nseq, W, hkv, D] (one launch)."""
+    for t in (new_k, new_v, ring_k, ring_v):
+        assert t.is_contiguous()
+    st = B.hca_ring_append(desc, new_k.data_ptr(), new_v.data_ptr(), ctx_len.data_ptr(),
+                           ring_k.data_ptr(), ring_v.data_ptr(), _stream(stream))
+    B.check(st, "hca_ring_append")
+
+
 def prefill(desc: B.HcaDesc, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
             cache: B.PagedCache, O: Optional[torch.Tensor] = None, want_lse: bool = False,
             want_mask: bool = False, stream=None):

@@ -152,6 +152,22 @@ int32_t hca_compress(const hca_desc* d, const void* K, const void* V,
                      int64_t batch_stride_tokens, int32_t first_block, int32_t n_blocks,
                      const hca_cache* cache, hca_stream_t stream);
 
+/* Decode-step update of the raw window ([news 二.1]: the last `window` raw tokens are
+ * attended as they are; the decode path keeps them in a ring, token u in slot u % window).
+ * For every sequence b < d->batch the new token, at position t = ctx_len[b] - 1:
+ *   ring_k[b, t % window] = new_k[b],   ring_v[b, t % window] = new_v[b]
+ *   new_k, new_v    [batch, hkv, head_dim]          d->dtype, contiguous
+ *   ring_k, ring_v  [batch, window, hkv, head_dim]  d->dtype, contiguous
+ *   ctx_len         device int32 [batch], as passed to hca_attn_decode (clamped into
+ *                   [1, seqlen] the same way, so both agree on the slot)
+ * One launch for both rows of every sequence; run it before hca_attn_decode of the step
+ * (and before hca_compress of a block the token completes).
+ * Errors: HCA_EINVAL (NULL pointer, a pointer not 16-byte aligned), HCA_EUNSUPPORTED
+ * (hkv * head_dim * element size not a multiple of 16 bytes), HCA_ECUDA. */
+int32_t hca_ring_append(const hca_desc* d, const void* new_k, const void* new_v,
+                        const int32_t* ctx_len, void* ring_k, void* ring_v,
+                        hca_stream_t stream);
+
 /* HCA prefill attention of [news 二.1] / [analysis 1] with the optional gate of [gate].
  * For every sequence b, position t < seqlen and head h:
  *   keys  = compressed entries j < n_c(t) of sequence b, then raw tokens u in

@@ -71,6 +71,36 @@ def test_decode_bf16(nseq, lo, hi, gate):
     assert int(cache.err.item()) == 0
 
 
+@pytest.mark.parametrize("dtype,hkv,D", [("bf16", 1, 512), ("f32", 2, 64)])
+def test_ring_append(dtype, hkv, D):
+    """hca_ring_append writes each sequence's new rows to slot (ctx_len - 1) % W, ctx_len
+    clamped into [1, seqlen] as decode clamps it: compared byte for byte with plain indexing
+    of the same tensors (slots 0 and W - 1, a wrap, a clamp at each end)."""
+    ensure_built()
+    dev = torch.device("cuda")
+    W, seqlen = 128, 5000
+    ctx = [1, 128, 129, 4999, 0, 7000]
+    nseq = len(ctx)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    g = torch.Generator().manual_seed(31)
+    ring_k = torch.randn((nseq, W, hkv, D), generator=g).to(tdt)
+    ring_v = torch.randn((nseq, W, hkv, D), generator=g).to(tdt)
+    new_k = torch.randn((nseq, hkv, D), generator=g).to(tdt)
+    new_v = torch.randn((nseq, hkv, D), generator=g).to(tdt)
+    want_k, want_v = ring_k.clone(), ring_v.clone()
+    for b, c in enumerate(ctx):
+        slot = (min(max(c, 1), seqlen) - 1) % W
+        want_k[b, slot] = new_k[b]
+        want_v[b, slot] = new_v[b]
+    rk, rv = ring_k.to(dev), ring_v.to(dev)
+    desc = B.make_desc(nseq, seqlen, 4 * hkv, hkv, D, 128, W, None,
+                       B.HCA_BF16 if dtype == "bf16" else B.HCA_F32)
+    ops.ring_append(desc, new_k.to(dev), new_v.to(dev),
+                    torch.tensor(ctx, dtype=torch.int32, device=dev), rk, rv)
+    torch.cuda.synchronize()
+    assert torch.equal(rk.cpu(), want_k) and torch.equal(rv.cpu(), want_v)
+
+
 # the last compressed tile holds 16 * odd entries, all visible: its last 32-column score
 # piece runs 16 columns past the tile, and those columns (stale tensor memory, scores of an
 # earlier tile) must enter neither P nor the row sum
@@ -238,17 +268,18 @@ def test_decode_1m_config_four_steps_sampled():
     for s in range(steps):
         p = ctx0 - 1 + s
         q = x.q if s == 0 else tok.q[s]
+        desc = B.make_desc(nseq, ctx0 + steps, 64, 1, 512)
+        ctx = torch.full((nseq,), p + 1, dtype=torch.int32, device=dev)
         if s > 0:
-            rk[:, p % W] = tok.k[s].to(dev)
-            rv[:, p % W] = tok.v[s].to(dev)
+            # the library's ring update on the device, plain indexing for the oracle's copy
+            ops.ring_append(desc, tok.k[s].to(dev).contiguous(), tok.v[s].to(dev).contiguous(),
+                            ctx, rk, rv)
             rk_h[:, p % W] = tok.k[s]
             rv_h[:, p % W] = tok.v[s]
         if (p + 1) % blk == 0:
             B.check(B.hca_compress(cdesc, rk.data_ptr(), rv.data_ptr(), W, p // blk, 1, cache.c,
                                    torch.cuda.current_stream().cuda_stream), "hca_compress")
-        desc = B.make_desc(nseq, ctx0 + steps, 64, 1, 512)
         ops.attach_gate(desc, tok.G[s].to(dev))
-        ctx = torch.full((nseq,), p + 1, dtype=torch.int32, device=dev)
         ops.decode(desc, q.to(dev), ctx, cache, rk, rv, O=O)
         torch.cuda.synchronize()
         assert int(cache.err.item()) == 0
