@@ -11,11 +11,13 @@
 //  * Scores of a compressed tile run on kind::f8f6f4 UMMAs straight from the stored codes
 //    (K-major, as TMA lands them). The query is carried exactly as two e4m3 parts: with
 //    r_h a power of two per head that puts the head's largest |q| in [128, 256),
-//    q / r_h = Q1 + Q2 / 16, Q1 = e4m3(q / r_h), Q2 = e4m3(16 (q / r_h - Q1)). A bf16 q has
-//    8 significant bits; Q1 takes the top 4 and the remainder has at most 4, so both parts
-//    are exact for every element within 2^13 of the head's largest (below that the part
-//    error is under 2^-21 of the largest |q|). S1 = Q1 K and S2 = Q2 K go to two TMEM
-//    accumulators; the softmax forms s = (S1 + S2 / 16) * r_h * k_scale * scale.
+//    q / r_h = Q1 + Q2, Q1 = e4m3(q / r_h), Q2 = e4m3(q / r_h - Q1). A bf16 q has 8
+//    significant bits; Q1 takes the top 4 and the remainder has at most 4, so the two parts
+//    are exact for every element within 2^9 of the head's largest (|q / r_h| >= 1/4, where
+//    the remainder's last bit is still an e4m3 step); below, the part error is at most 2^-10,
+//    i.e. 2^-17 of the largest |q / r_h|. Both parts accumulate into one TMEM accumulator,
+//    S = Q1 K + Q2 K (two UMMAs per 32-code step), and the softmax forms
+//    s = S * r_h * k_scale * scale.
 //  * P.V runs on kind::f16 with f16 operands. The e4m3 values arrive by TMA in a ring of
 //    their own (one 16 KB box = 32 keys x 512 codes); converter warps widen each 16-key
 //    group to f16 values times 2^-8 (exact, by moving the code's bits) into two MN-major
@@ -28,9 +30,9 @@
 //    widened values; v_scale * 2^8 multiplies it once at the end.
 //  * The ring tile (the raw window, bf16) is the last tile of the last split and runs the
 //    16-bit way inside the same CTA: once the last e4m3 score MMA has completed, the bf16
-//    query replaces Q1/Q2 in shared memory, its scores accumulate in S1 (kind::f16 bf16),
-//    its P goes to bf16 hi + lo parts divided by v_scale * 2^8 (O keeps its units), and its
-//    values land in the same V buffers by TMA.
+//    query replaces Q1/Q2 in shared memory, its scores accumulate in the score buffer
+//    (kind::f16 bf16), its P goes to bf16 hi + lo parts divided by v_scale * 2^8 (O keeps
+//    its units), and its values land in the same V buffers by TMA.
 //  * Roles: warp 0 loads the K boxes into a 3-slot K ring (128 keys x one 128-byte column
 //    chunk; the window tile's bf16 K in 64-column chunks) and the bf16 query (staged for
 //    the converters at the start, and again for the window tile); warp 11 loads the e4m3 V
@@ -38,7 +40,7 @@
 //    warps 2-5 run the softmax (lazy rescale, as the 16-bit kernel) and the epilogue;
 //    warps 6-9 prepare Q1/Q2 and widen V.
 //  * TMEM: O (64 x 512 f32, M = 64 layout) in lanes 0-15 of each 32-lane subpartition;
-//    two score buffers of S1 | S2 (128 columns each) in lanes 16-31.
+//    two score buffers (128 columns each) in lanes 16-31.
 //  * All mbarrier waits are bounded (HCA_ERR_TIMEOUT on give-up); on give-up every issuing
 //    thread waits (bounded) for its own copies still in flight before the CTA leaves.
 #include <cuda.h>
@@ -330,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
           if (c >= 2 && !(ok = mbar_wait(&bars->p_full[c & 1], ((c - 2) >> 1) & 1, abort)))
             break;
           const Tile t = tile_of(p, sq, sq.j0 + c);
-          const uint32_t sb = tmem + kLaneS + (c & 1) * 256;  // S1 at sb, S2 at sb + 128
+          const uint32_t sb = tmem + kLaneS + (c & 1) * 128;  // score buffer c & 1
           if (t.kind == kCompressed) {
             const uint32_t idesc = idesc_e4m3_f32(kM, t.n);
             for (int q = 0; q < 4 && ok; ++q) {
@@ -344,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
                 const uint32_t acc = (q | kk) != 0;
                 const uint32_t qa = qbase + q * kQChunkBytes + kk * 32;
                 umma_ss_f8(sb, sdesc_sw128(qa, 16, 1024), kd, idesc, acc);
-                umma_ss_f8(sb + 128, sdesc_sw128(qa + kQPartBytes, 16, 1024), kd, idesc, acc);
+                umma_ss_f8(sb, sdesc_sw128(qa + kQPartBytes, 16, 1024), kd, idesc, 1u);
               }
               umma_commit(&bars->k_empty[s]);
               ++n;
@@ -448,24 +450,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
       tc_fence_after();
       const Tile tl = tile_of(p, sq, sq.j0 + c);
       const bool f8 = tl.kind == kCompressed;
-      const uint32_t sbuf = tmem + lane_addr + (c & 1) * 256;
+      const uint32_t sbuf = tmem + lane_addr + (c & 1) * 128;
       // visible columns: a prefix of a compressed tile, or ring slots 0..min(W,t+1)-1
       const int vhi = f8 ? min(tl.n, sq.e1 - tl.key0) : min(p.W, sq.t + 1);
       const uint32_t vlen = vhi > 0 ? (uint32_t)vhi : 0u;
       const float rs = f8 ? rs8 : p.scale_log2;
-      // 32 raw scores of columns q*32 .. q*32+31: S1 + S2 / 16 (e4m3 tile) or S1 (ring)
+      // 32 raw scores of columns q*32 .. q*32+31
       auto load_scores = [&](int q, uint32_t (&v)[32]) {
         tmem_ld32(sbuf + q * 32, v);
-        if (f8) {
-          uint32_t w[32];
-          tmem_ld32(sbuf + 128 + q * 32, w);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e)
-            v[e] = __float_as_uint(fmaf(__uint_as_float(w[e]), 0.0625f, __uint_as_float(v[e])));
-        } else {
-          tmem_wait_ld();
-        }
+        tmem_wait_ld();
       };
       // pass 1: row max over the visible keys
       float mx[8];
@@ -702,7 +695,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
               const __half2_raw h1 = __nv_cvt_fp8x2_to_halfraw2(q1, __NV_E4M3);
               const float2 v1 = __half22float2(__half2(h1));
               const __nv_fp8x2_storage_t q2 = __nv_cvt_float2_to_fp8x2(
-                  make_float2(16.f * (a0 - v1.x), 16.f * (a1 - v1.y)), __NV_SATFINITE, __NV_E4M3);
+                  make_float2(a0 - v1.x, a1 - v1.y), __NV_SATFINITE, __NV_E4M3);
               const int pos = hv * 8 + 2 * k;  // code index within the 16-byte unit
               w1[pos >> 2] |= (uint32_t)q1 << (8 * (pos & 3));
               w2[pos >> 2] |= (uint32_t)q2 << (8 * (pos & 3));
