@@ -9,7 +9,7 @@
 // Design for sm_100a (HBM-bound; a compressed tile of 128 entries is 64 KB of keys and
 // 64 KB of values, half of the 16-bit cache):
 //  * Scores of a compressed tile run on kind::f8f6f4 UMMAs straight from the stored codes
-//    (K-major, as TMA lands them). The query is carried exactly as two e4m3 parts: with
+//    (K-major, as TMA lands them). The query is carried as two e4m3 parts: with
 //    r_h a power of two per head that puts the head's largest |q| in [128, 256),
 //    q / r_h = Q1 + Q2, Q1 = e4m3(q / r_h), Q2 = e4m3(q / r_h - Q1). A bf16 q has 8
 //    significant bits; Q1 takes the top 4 and the remainder has at most 4, so the two parts
