@@ -226,6 +226,78 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
   const bool has_ring = ntiles > 0 && tile_of(p, sq, sq.j1 - 1).kind == kRing;
   const int nct = ntiles - (has_ring ? 1 : 0);  // compressed (e4m3) tiles of this split
 
+  // Q1, Q2 and the per-head scale r_h of the two-part query, computed by the softmax and
+  // converter warps together (qt = 0..255 over warps 2-9, four threads per head row, 128
+  // elements each) from the bf16 query staged in shared memory (chunk c of row h at
+  // stage(c) + (c % 4) * 8 KB + h * 128, stage(c) the P buffer for c < 4 and the V buffers
+  // after; 16-byte units swizzled by h % 8). Ends with a barrier of the 256 threads; one of
+  // them then announces q_ready to the score-MMA warp. Returns false on a time-out.
+  auto prep_query = [&](int qt) -> bool {
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&bars->qs_full, 0, abort));
+    const int h = qt >> 2, quarter = qt & 3;
+    const bool live = h < p.hq && ok;
+    const uint8_t* stage = quarter < 2 ? sP : sV;
+    auto unit = [&](int i) {  // 16-byte unit i (8 elements) of this thread's 128
+      const int gc = 2 * quarter + (i >> 3);  // chunk of the row
+      const uint8_t* rowp = stage + (gc & 3) * kQChunkBytes + h * 128;
+      return *reinterpret_cast<const uint4*>(rowp + (((i & 7) ^ (h & 7)) << 4));
+    };
+    float amax = 0.f;
+    if (live)
+      for (int i = 0; i < 16; ++i) {
+        const uint4 x = unit(i);
+        const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&x);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 f = __bfloat1622float2(x2[k]);
+          amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+        }
+      }
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    // r_h = 2^e puts the head's largest |q| / r_h in [128, 256)
+    // (the exponent field of amax; e is kept in [-126, 126] so that r_h and 1 / r_h are
+    // both normal floats: a row whose largest |q| is below 2^-119 keeps a smaller range)
+    const int ebits = (__float_as_int(amax) >> 23) & 0xff;
+    int e = amax > 0.f ? (ebits > 0 ? ebits - 127 : -126) - 7 : 0;
+    e = e < -126 ? -126 : (e > 126 ? 126 : e);
+    const float rinv = exp2i(-e);  // 1 / r_h, exact
+    for (int u = 0; u < 8; ++u) {  // 16-element units of the e4m3 parts
+      uint32_t w1[4] = {0u, 0u, 0u, 0u}, w2[4] = {0u, 0u, 0u, 0u};
+      if (live) {
+#pragma unroll
+        for (int hv = 0; hv < 2; ++hv) {
+          const uint4 x = unit(2 * u + hv);
+          const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&x);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 f = __bfloat1622float2(x2[k]);
+            const float a0 = f.x * rinv, a1 = f.y * rinv;
+            const __nv_fp8x2_storage_t q1 =
+                __nv_cvt_float2_to_fp8x2(make_float2(a0, a1), __NV_SATFINITE, __NV_E4M3);
+            const __half2_raw h1 = __nv_cvt_fp8x2_to_halfraw2(q1, __NV_E4M3);
+            const float2 v1 = __half22float2(__half2(h1));
+            const __nv_fp8x2_storage_t q2 = __nv_cvt_float2_to_fp8x2(
+                make_float2(a0 - v1.x, a1 - v1.y), __NV_SATFINITE, __NV_E4M3);
+            const int pos = hv * 8 + 2 * k;  // code index within the 16-byte unit
+            w1[pos >> 2] |= (uint32_t)q1 << (8 * (pos & 3));
+            w2[pos >> 2] |= (uint32_t)q2 << (8 * (pos & 3));
+          }
+        }
+      }
+      const int elem = quarter * 128 + 16 * u;
+      const uint32_t off = (elem >> 7) * kQChunkBytes + h * 128 +
+                           ((((elem & 127) >> 4) ^ (h & 7)) << 4);
+      *reinterpret_cast<uint4*>(sQ + off) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+      *reinterpret_cast<uint4*>(sQ + kQPartBytes + off) = make_uint4(w2[0], w2[1], w2[2], w2[3]);
+    }
+    if (quarter == 0) sRS[h] = p.scale_log2 * p.k_scale * exp2i(e);
+    fence_proxy_async_smem();
+    named_sync(2, 256);
+    if (qt == 0) mbar_arrive(&bars->q_ready);
+    return ok;
+  };
+
   if (ntiles <= 0) {
     // empty split: an all-zero partial that the merge skips
     for (int h = threadIdx.x; h < p.hq; h += blockDim.x) {
@@ -439,7 +511,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
     const bool s_lane = lane >= 16;
     const int hrow = quad * 16 + (lane & 15);
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-    bool ok = __all_sync(0xffffffffu, mbar_wait(&bars->q_ready, 0, abort));
+    // Q1, Q2 and r_h with the converter warps (the barrier at its end orders sRS)
+    bool ok = prep_query(threadIdx.x - 64);
     const float rs8 = sRS[hrow];            // r_h * k_scale * scale * log2(e)
     // ring values enter O in the units of the widened e4m3 values (value / (v_scale * 2^8))
     const float inv_vs = 1.f / (p.v_scale * kV16Scale);
@@ -648,71 +721,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
     // ------------------------------------------------------------------ converters
     const int ct = threadIdx.x - 192;  // 0..127
     const int cw = ct >> 5;
-    // (1) Q1, Q2 and the per-head scale: two threads per head row, 256 elements each, from
-    // the staged bf16 query (chunk c of row h at stage(c) + (c % 4) * 8 KB + h * 128, its
-    // 16-byte units swizzled by h % 8)
-    bool q_ok = __all_sync(0xffffffffu, mbar_wait(&bars->qs_full, 0, abort));
-    {
-      const int h = ct >> 1, half = ct & 1;
-      const bool live = h < p.hq && q_ok;
-      const uint8_t* stage = half == 0 ? sP : sV;  // chunks 4 * half .. 4 * half + 3
-      auto unit = [&](int i) {  // 16-byte unit i (8 elements) of this thread's 256
-        const uint8_t* rowp = stage + (i >> 3) * kQChunkBytes + h * 128;
-        return *reinterpret_cast<const uint4*>(rowp + (((i & 7) ^ (h & 7)) << 4));
-      };
-      float amax = 0.f;
-      if (live)
-        for (int i = 0; i < 32; ++i) {
-          const uint4 x = unit(i);
-          const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&x);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float2 f = __bfloat1622float2(x2[k]);
-            amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
-          }
-        }
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-      // r_h = 2^e puts the head's largest |q| / r_h in [128, 256)
-      // (the exponent field of amax; e is kept in [-126, 126] so that r_h and 1 / r_h are
-      // both normal floats: a row whose largest |q| is below 2^-119 keeps a smaller range)
-      const int ebits = (__float_as_int(amax) >> 23) & 0xff;
-      int e = amax > 0.f ? (ebits > 0 ? ebits - 127 : -126) - 7 : 0;
-      e = e < -126 ? -126 : (e > 126 ? 126 : e);
-      const float rinv = exp2i(-e);  // 1 / r_h, exact
-      for (int u = 0; u < 16; ++u) {  // 16-element units of the e4m3 parts
-        uint32_t w1[4] = {0u, 0u, 0u, 0u}, w2[4] = {0u, 0u, 0u, 0u};
-        if (live) {
-#pragma unroll
-          for (int hv = 0; hv < 2; ++hv) {
-            const uint4 x = unit(2 * u + hv);
-            const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&x);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const float2 f = __bfloat1622float2(x2[k]);
-              const float a0 = f.x * rinv, a1 = f.y * rinv;
-              const __nv_fp8x2_storage_t q1 =
-                  __nv_cvt_float2_to_fp8x2(make_float2(a0, a1), __NV_SATFINITE, __NV_E4M3);
-              const __half2_raw h1 = __nv_cvt_fp8x2_to_halfraw2(q1, __NV_E4M3);
-              const float2 v1 = __half22float2(__half2(h1));
-              const __nv_fp8x2_storage_t q2 = __nv_cvt_float2_to_fp8x2(
-                  make_float2(a0 - v1.x, a1 - v1.y), __NV_SATFINITE, __NV_E4M3);
-              const int pos = hv * 8 + 2 * k;  // code index within the 16-byte unit
-              w1[pos >> 2] |= (uint32_t)q1 << (8 * (pos & 3));
-              w2[pos >> 2] |= (uint32_t)q2 << (8 * (pos & 3));
-            }
-          }
-        }
-        const int elem = half * 256 + 16 * u;
-        const uint32_t off = (elem >> 7) * kQChunkBytes + h * 128 +
-                             ((((elem & 127) >> 4) ^ (h & 7)) << 4);
-        *reinterpret_cast<uint4*>(sQ + off) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
-        *reinterpret_cast<uint4*>(sQ + kQPartBytes + off) = make_uint4(w2[0], w2[1], w2[2], w2[3]);
-      }
-      if (half == 0) sRS[h] = p.scale_log2 * p.k_scale * exp2i(e);
-    }
-    fence_proxy_async_smem();
-    named_sync(2, 128);
-    if (ct == 0) mbar_arrive(&bars->q_ready);
+    // (1) Q1, Q2 and the per-head scale, with the softmax warps
+    const bool q_ok = prep_query(threadIdx.x - 64);
 
     // (2) V groups of 16 keys in key order into the f16 V buffers: e4m3 boxes of the V
     // ring widened, the window tile's bf16 values by TMA. Thread (cw, lane) widens keys kr
