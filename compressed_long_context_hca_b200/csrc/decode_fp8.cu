@@ -242,10 +242,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
       const uint8_t* rowp = stage + (gc & 3) * kQChunkBytes + h * 128;
       return *reinterpret_cast<const uint4*>(rowp + (((i & 7) ^ (h & 7)) << 4));
     };
+    // the four threads of a row walk their units in staggered orders: unit i of every
+    // chunk sits in the same banks, so equal i in the four quarters would conflict
     float amax = 0.f;
     if (live)
-      for (int i = 0; i < 16; ++i) {
-        const uint4 x = unit(i);
+      for (int i0 = 0; i0 < 16; ++i0) {
+        const uint4 x = unit((i0 + 2 * quarter) & 15);
         const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&x);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -262,7 +264,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
     int e = amax > 0.f ? (ebits > 0 ? ebits - 127 : -126) - 7 : 0;
     e = e < -126 ? -126 : (e > 126 ? 126 : e);
     const float rinv = exp2i(-e);  // 1 / r_h, exact
-    for (int u = 0; u < 8; ++u) {  // 16-element units of the e4m3 parts
+    for (int u0 = 0; u0 < 8; ++u0) {  // 16-element units of the e4m3 parts
+      const int u = (u0 + 2 * quarter) & 7;
       uint32_t w1[4] = {0u, 0u, 0u, 0u}, w2[4] = {0u, 0u, 0u, 0u};
       if (live) {
 #pragma unroll
