@@ -192,6 +192,22 @@ def test_e4m3_cache_validation(L):
     assert B.hca_attn_decode(d, 16, 16, c, 16, 16, 16, 0, 16, 1 << 30) == B.HCA_EINVAL
 
 
+def test_ring_append_validation(L):
+    """hca_ring_append rejects what it cannot launch, before any device work."""
+    d = B.make_desc(2, 1000, 64, 1, 512)
+    # NULL pointers
+    assert B.hca_ring_append(d, 0, 16, 16, 16, 16) == B.HCA_EINVAL
+    assert B.hca_ring_append(d, 16, 16, 0, 16, 16) == B.HCA_EINVAL
+    # every row pointer 16-byte aligned
+    assert B.hca_ring_append(d, 16, 16, 16, 24, 16) == B.HCA_EINVAL
+    assert B.hca_ring_append(d, 16, 18, 16, 16, 16) == B.HCA_EINVAL
+    # rows of hkv * head_dim elements whose size is not a multiple of 16 bytes
+    odd = B.make_desc(2, 1000, 4, 1, 12)
+    assert B.hca_ring_append(odd, 16, 16, 16, 16, 16) == B.HCA_EUNSUPPORTED
+    # an empty batch is a no-op
+    assert B.hca_ring_append(B.make_desc(0, 1000, 64, 1, 512), 0, 0, 0, 0, 0) == B.HCA_OK
+
+
 def test_set_gate(L):
     d = B.make_desc(1, 8, 64, 1, 512)
     assert B.hca_set_gate(d, 0x2000, (1, 2, 3)) == B.HCA_OK
