@@ -7,11 +7,14 @@
 // [1, seqlen] exactly as the decode kernels clamp it, so both agree on the slot.
 //
 // Pure data movement (2 x hkv x head_dim elements per sequence): one CTA per sequence
-// copies both rows in 16-byte units.
+// copies both rows in 16-byte units. Launched as a programmatic dependent of the kernel
+// before it (the previous step's merge or decode) and letting the next one (the step's
+// decode) be scheduled early; each waits for its predecessor before touching memory.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
 #include "hca_internal.h"
+#include "sm100.cuh"
 
 namespace hca {
 namespace {
@@ -27,6 +30,8 @@ struct RingArgs {
 };
 
 __global__ void __launch_bounds__(128) ring_append_kernel(const RingArgs a) {
+  pdl_wait();  // the previous step's reads of the ring are complete
+  pdl_trigger();
   const int b = blockIdx.x;
   int ctx = a.ctx_len[b];
   ctx = ctx < 1 ? 1 : (ctx > a.seqlen ? a.seqlen : ctx);
@@ -54,8 +59,11 @@ cudaError_t launch_ring_append(const hca_desc& d, const void* new_k, const void*
   a.row_units = (int32_t)((int64_t)d.hkv * d.head_dim * esize / 16);
   a.window = d.window;
   a.seqlen = d.seqlen;
-  ring_append_kernel<<<d.batch, 128, 0, s>>>(a);
-  return cudaGetLastError();
+  cudaLaunchAttribute pdl[1];
+  cudaLaunchConfig_t cfg = pdl_config(pdl, s);
+  cfg.gridDim = dim3(d.batch);
+  cfg.blockDim = dim3(128);
+  return cudaLaunchKernelEx(&cfg, ring_append_kernel, a);
 }
 
 }  // namespace hca
