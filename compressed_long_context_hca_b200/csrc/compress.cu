@@ -106,6 +106,8 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads) compress_kernel(CompressArgs a) {
   using V16 = Vec16<T>;
   constexpr int N = V16::N;
+  pdl_wait();  // the kernel before this one on the stream (e.g. the ring update) is done
+  pdl_trigger();
   const int jrel = blockIdx.x;
   const int b = blockIdx.y;
   const int which = blockIdx.z & 1;          // 0: K, 1: V
@@ -219,19 +221,23 @@ cudaError_t launch_compress(const hca_desc& d, const void* K, const void* V,
   if (a.groups > d.block) a.groups = d.block;
   const int vec_elems = 16 / esize;
   const size_t smem = (size_t)a.groups * lanes * vec_elems * sizeof(float);
-  dim3 grid(n_blocks, d.batch, 2 * csplit);
+  // a programmatic dependent of the kernel before it on the stream (it waits for it in the
+  // kernel before touching memory), so its launch overlaps that kernel's tail
+  cudaLaunchAttribute pdl[1];
+  cudaLaunchConfig_t cfg = pdl_config(pdl, s);
+  cfg.gridDim = dim3(n_blocks, d.batch, 2 * csplit);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
   if (d.dtype == HCA_BF16) {
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(compress_kernel<__nv_bfloat16>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    compress_kernel<__nv_bfloat16><<<grid, kThreads, smem, s>>>(a);
-  } else {
-    if (smem > 48 * 1024)
-      cudaFuncSetAttribute(compress_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem);
-    compress_kernel<float><<<grid, kThreads, smem, s>>>(a);
+    return cudaLaunchKernelEx(&cfg, compress_kernel<__nv_bfloat16>, a);
   }
-  return cudaGetLastError();
+  if (smem > 48 * 1024)
+    cudaFuncSetAttribute(compress_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+  return cudaLaunchKernelEx(&cfg, compress_kernel<float>, a);
 }
 
 }  // namespace hca
