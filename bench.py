@@ -583,6 +583,8 @@ def bench_decode_1m(args, dev, rank, world, barrier, max_over_ranks, peaks, e4m3
         ops.attach_gate(d, G[s])
         descs.append(d)
     cdesc = B.make_desc(nseq, ctx0, HQ, 1, D)  # compress of the block ending at ctx0 - 1
+    O1 = torch.empty((nseq, HQ, D), dtype=torch.bfloat16, device=dev)
+    ws1 = ops.decode_workspace(descs[0], dev) if world == 1 else None
     stream = torch.cuda.current_stream()
     be = P.GpuBackend()
     group = None
@@ -590,15 +592,20 @@ def bench_decode_1m(args, dev, rank, world, barrier, max_over_ranks, peaks, e4m3
     def four_steps():
         for s in range(steps_per):
             p = ctx0 - 1 + s                 # position of the new token
-            if last:
-                # the new token into ring slot p % WIN (one launch for K and V)
-                ops.ring_append(descs[s], new_k[s], new_v[s], ctx[s], rk, rv)
-                if (p + 1) % BLOCK == 0:     # token completes block p // BLOCK
-                    B.check(B.hca_compress(cdesc, rk.data_ptr(), rv.data_ptr(), WIN,
-                                           p // BLOCK, 1, cache.c,
-                                           torch.cuda.current_stream().cuda_stream),
-                            "hca_compress")
-            P.decode_split_entries(be, group, q[s], ctx[s], cache, rk, rv, n_ent, descs[s])
+            if world == 1:
+                # the new token into ring slot p % WIN inside the decode call
+                ops.decode_append(descs[s], q[s], ctx[s], cache, new_k[s], new_v[s], rk, rv,
+                                  O=O1, workspace=ws1)
+            else:
+                if last:  # the rank holding the ring: the new token into its slot
+                    ops.ring_append(descs[s], new_k[s], new_v[s], ctx[s], rk, rv)
+                P.decode_split_entries(be, group, q[s], ctx[s], cache, rk, rv, n_ent, descs[s])
+            if last and (p + 1) % BLOCK == 0:
+                # the token completes block p // BLOCK: its entry (invisible to the token's
+                # own query) is compressed after the step
+                B.check(B.hca_compress(cdesc, rk.data_ptr(), rv.data_ptr(), WIN, p // BLOCK, 1,
+                                       cache.c, torch.cuda.current_stream().cuda_stream),
+                        "hca_compress")
 
     clocks = Clocks(dev.index)
     clocks.start()
@@ -616,8 +623,10 @@ def bench_decode_1m(args, dev, rank, world, barrier, max_over_ranks, peaks, e4m3
     byts = steps_per * byts_step + nseq * (BLOCK * D * 2 * 2 + D * 2 * eb)
     gbs = byts / (ms * 1e-3) / 1e9 / world  # per GPU
     nsplit = B.hca_decode_workspace_bytes(descs[0]) // (nseq * HQ * (D + 2) * 4)
-    # per step: ring update (the rank holding the ring), decode, merge; one compress
-    launches = (4 * 3 + 1) if world == 1 else (4 * 3 + (4 + 1 if last else 0))
+    # per step: decode (with the ring update inside), merge; one compress. N > 1: per step
+    # the ring update (the rank holding the ring), the partial decode and its merge, the
+    # merge of the gathered parts
+    launches = (4 * 2 + 1) if world == 1 else (4 * 3 + (4 + 1 if last else 0))
     return {"value": round(nseq * steps_per / (ms * 1e-3), 1), "unit": "tokens/s",
             "ms_per_step": round(ms, 4), "ms_per_decode_step": round(ms / steps_per, 4),
             "workload": "16 sequences at context 1,048,576 (8191 entries + 128 raw), 64 heads, "

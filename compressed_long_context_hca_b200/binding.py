@@ -38,7 +38,7 @@ EXPORTED = ("hca_abi_version", "hca_status_string", "hca_set_gate", "hca_compres
             "hca_attn_decode", "hca_decode_partial_bytes", "hca_attn_decode_partial",
             "hca_decode_merge", "hca_prefill_backward_workspace_bytes",
             "hca_attn_prefill_backward", "hca_gate_from_latent", "hca_vha_gate",
-            "hca_attn_decode_noalloc", "hca_ring_append")
+            "hca_attn_decode_noalloc", "hca_ring_append", "hca_attn_decode_append")
 HCA_DECODE_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
@@ -83,6 +83,10 @@ def lib() -> ctypes.CDLL:
     L.hca_compress.restype = c_int32
     L.hca_compress.argtypes = [POINTER(HcaDesc), c_void_p, c_void_p, c_int64, c_int32, c_int32,
                                POINTER(HcaCache), c_void_p]
+    L.hca_attn_decode_append.restype = c_int32
+    L.hca_attn_decode_append.argtypes = [POINTER(HcaDesc), c_void_p, c_void_p, POINTER(HcaCache),
+                                         c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                         c_void_p, c_void_p, c_size_t, c_void_p]
     L.hca_ring_append.restype = c_int32
     L.hca_ring_append.argtypes = [POINTER(HcaDesc), c_void_p, c_void_p, c_void_p, c_void_p,
                                   c_void_p, c_void_p]
@@ -161,6 +165,15 @@ def hca_compress(desc: HcaDesc, K: int, V: int, batch_stride_tokens: int, first_
                  n_blocks: int, cache: HcaCache, stream: int = 0) -> int:
     return lib().hca_compress(ctypes.byref(desc), K or None, V or None, batch_stride_tokens,
                               first_block, n_blocks, ctypes.byref(cache), stream or None)
+
+
+def hca_attn_decode_append(desc: HcaDesc, Q: int, ctx_len: int, cache: HcaCache, new_k: int,
+                           new_v: int, ring_k: int, ring_v: int, O: int, lse: int,
+                           workspace: int, workspace_bytes: int, stream: int = 0) -> int:
+    return lib().hca_attn_decode_append(ctypes.byref(desc), Q or None, ctx_len or None,
+                                        ctypes.byref(cache), new_k or None, new_v or None,
+                                        ring_k or None, ring_v or None, O or None, lse or None,
+                                        workspace or None, workspace_bytes, stream or None)
 
 
 def hca_ring_append(desc: HcaDesc, new_k: int, new_v: int, ctx_len: int, ring_k: int,

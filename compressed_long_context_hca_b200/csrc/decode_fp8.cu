@@ -120,6 +120,11 @@ struct Params8 {
   float* lse;
   const __nv_bfloat16* gate;
   int64_t gs0, gs2;
+  // the new token's rows and the raw rings, for the in-kernel ring update (nullptr = none)
+  const uint4* new_k;
+  const uint4* new_v;
+  uint4* ring_k;
+  uint4* ring_v;
   int32_t nseq, seqlen, hq, W, block, PE, max_pages, num_pages, nsplit;
   int32_t e0, e1, with_ring, partial;
   float scale_log2, k_scale, v_scale;
@@ -368,6 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
             tma_load_3d(sQ + h * (kQ16Bytes / 2), &p.tmQb, &bars->qb_full, 0, b * p.hq, 4 * h,
                         pol);
           q_issued = true;
+          if (p.new_k) append_ring_row(p, p.new_k, p.ring_k, b, sq.t);  // the new token
           for (int q = 0; q < 8 && ok; ++q) ok = load(&p.tmRk, b * p.W, q);
         }
       }
@@ -788,7 +794,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
         }
         n += (t.n + kVRows - 1) / kVRows;
       } else if (ct == 0) {
-        // the window's values, bf16, one TMA box of 16 rows x 512 values per group
+        // the window's values, bf16, one TMA box of 16 rows x 512 values per group (the new
+        // token's row written into its slot first)
+        if (p.new_v) append_ring_row(p, p.new_v, p.ring_v, b, sq.t);
         const uint64_t pol = policy_evict_first();
         uint32_t issued = 0;
         const uint32_t cv0 = cv;
@@ -876,6 +884,10 @@ cudaError_t launch_decode_fp8(const hca_desc& d, const void* Q, const int32_t* c
   p.e1 = part.e1;
   p.with_ring = part.with_ring ? 1 : 0;
   p.partial = pml ? 1 : 0;
+  p.new_k = static_cast<const uint4*>(part.new_k);
+  p.new_v = static_cast<const uint4*>(part.new_v);
+  p.ring_k = static_cast<uint4*>(const_cast<void*>(ring_k));
+  p.ring_v = static_cast<uint4*>(const_cast<void*>(ring_v));
   p.scale_log2 = d.scale * 1.4426950408889634f;
   p.k_scale = c.k_scale;
   p.v_scale = c.v_scale;

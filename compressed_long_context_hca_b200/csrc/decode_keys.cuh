@@ -85,6 +85,20 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// The new token's row (one KV head of 512 bf16 values: 64 16-byte units) into ring slot
+// t % W of sequence b, written by the calling thread, followed by a proxy fence so that the
+// bulk-tensor loads this thread issues afterwards read it. P: a parameter block with W.
+template <typename P>
+__device__ __forceinline__ void append_ring_row(const P& p, const uint4* src, uint4* ring, int b,
+                                                int t) {
+  const int64_t slot = t % p.W;
+  const uint4* s = src + (int64_t)b * 64;
+  uint4* d = ring + ((int64_t)b * p.W + slot) * 64;
+#pragma unroll 8
+  for (int i = 0; i < 64; ++i) d[i] = s[i];
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t pol;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));

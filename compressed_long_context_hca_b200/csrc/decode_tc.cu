@@ -86,6 +86,11 @@ struct Params {
   float* lse;
   const __nv_bfloat16* gate;
   int64_t gs0, gs2;
+  // the new token's rows and the raw rings, for the in-kernel ring update (nullptr = none)
+  const uint4* new_k;
+  const uint4* new_v;
+  uint4* ring_k;
+  uint4* ring_v;
   int32_t nseq, seqlen, hq, W, block, PE, max_pages, num_pages, nsplit;
   // key part of the call: visible compressed entries [e0, e1) (e0 % 128 == 0), and the raw
   // window if with_ring; partial != 0: the result is an unnormalised float32 partial
@@ -192,6 +197,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           row = page * p.PE + t.key0 % p.PE;
         } else {
           row = b * p.W;
+          // the new token into the ring (both producers write the same rows, each before
+          // its own first load of the window tile)
+          if (!is_v && p.new_k) {
+            append_ring_row(p, p.new_k, p.ring_k, b, sq.t);
+            append_ring_row(p, p.new_v, p.ring_v, b, sq.t);
+          }
         }
         const CUtensorMap* map = t.kind == kCompressed ? (is_v ? &p.tmVc : &p.tmKc)
                                                        : (is_v ? &p.tmRv : &p.tmRk);
@@ -800,6 +811,10 @@ cudaError_t launch_decode_part(const hca_desc& d, const void* Q, const int32_t* 
   p.e1 = part.e1;
   p.with_ring = part.with_ring ? 1 : 0;
   p.partial = pml ? 1 : 0;
+  p.new_k = static_cast<const uint4*>(part.new_k);
+  p.new_v = static_cast<const uint4*>(part.new_v);
+  p.ring_k = static_cast<uint4*>(const_cast<void*>(ring_k));
+  p.ring_v = static_cast<uint4*>(const_cast<void*>(ring_v));
   p.scale_log2 = d.scale * 1.4426950408889634f;
   p.O = static_cast<__nv_bfloat16*>(O);
   p.lse = lse;

@@ -374,6 +374,40 @@ int32_t hca_attn_decode(const hca_desc* d, const void* Q, const int32_t* ctx_len
       launch_decode_tc(*d, Q, ctx_len, *cache, ring_k, ring_v, O, lse, workspace, s));
 }
 
+int32_t hca_attn_decode_append(const hca_desc* d, const void* Q, const int32_t* ctx_len,
+                               const hca_cache* cache, const void* new_k, const void* new_v,
+                               void* ring_k, void* ring_v, void* O, float* lse,
+                               void* workspace, size_t workspace_bytes, hca_stream_t stream) {
+  int32_t st = check_desc(d);
+  if (st != HCA_OK) return st;
+  if ((st = check_cache(cache)) != HCA_OK) return st;
+  if (d->batch == 0) return HCA_OK;
+  if (!Q || !ctx_len || !ring_k || !ring_v || !O || !new_k || !new_v) return HCA_EINVAL;
+  if (d->seqlen < 1) return HCA_EINVAL;
+  if (!aligned16(new_k) || !aligned16(new_v)) return HCA_EINVAL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d->dtype == HCA_F32) {
+    if (d->head_dim % 32 != 0 || d->head_dim > 512 || e4m3_cache(cache))
+      return HCA_EUNSUPPORTED;
+    if ((int64_t)d->hkv * d->head_dim * 4 % 16 != 0) return HCA_EUNSUPPORTED;
+    if (!aligned16(ring_k) || !aligned16(ring_v)) return HCA_EINVAL;
+    cudaError_t e = launch_ring_append(*d, new_k, new_v, ctx_len, ring_k, ring_v, s);
+    if (e != cudaSuccess) return from_cuda(e);
+    return from_cuda(launch_decode_simt(*d, Q, ctx_len, *cache, ring_k, ring_v, O, lse, s));
+  }
+  if (!decode_tc_supported(*d, *cache)) return HCA_EUNSUPPORTED;
+  const size_t need = decode_tc_workspace_bytes(*d);
+  if (!workspace || workspace_bytes < need) return HCA_ENOSPACE;
+  if (!aligned16(Q) || !aligned16(ring_k) || !aligned16(ring_v) || !aligned16(O) ||
+      !aligned16(workspace) || !aligned16(cache->kc_pool) || !aligned16(cache->vc_pool))
+    return HCA_EINVAL;
+  DecodePart whole{0, INT32_MAX, 1, nullptr};
+  whole.new_k = new_k;
+  whole.new_v = new_v;
+  return from_cuda(
+      launch_decode_part(*d, Q, ctx_len, *cache, ring_k, ring_v, whole, O, lse, workspace, s));
+}
+
 size_t hca_decode_partial_bytes(const hca_desc* d) {
   if (check_desc(d) != HCA_OK || d->dtype != HCA_BF16) return 0;
   return decode_partial_bytes(*d);

@@ -101,9 +101,13 @@ cudaError_t launch_vha_gate(const hca_desc& d, const void* O, const float* A, co
 // The key part of a decode call: visible compressed entries [e0, e1) (e0 a multiple of 128)
 // and the raw window if with_ring. out_partial == nullptr: the call writes the final output;
 // else it writes an unnormalised float32 partial result there (decode_partial_bytes).
+// new_k / new_v (with_ring only; nullptr = none): the new token's rows [batch, 512], written
+// into ring slot t % window by the CTA that reads the window, before it reads it.
 struct DecodePart {
   int32_t e0, e1, with_ring;
   void* out_partial;
+  const void* new_k = nullptr;
+  const void* new_v = nullptr;
 };
 
 bool decode_tc_supported(const hca_desc& d, const hca_cache& c);

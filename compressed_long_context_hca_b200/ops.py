@@ -105,6 +105,29 @@ def decode(desc: B.HcaDesc, q: torch.Tensor, ctx_len: torch.Tensor, cache: B.Pag
     return O, lse
 
 
+def decode_append(desc: B.HcaDesc, q: torch.Tensor, ctx_len: torch.Tensor,
+                  cache: B.PagedCache, new_k: torch.Tensor, new_v: torch.Tensor,
+                  ring_k: torch.Tensor, ring_v: torch.Tensor, O: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None, want_lse: bool = False,
+                  stream=None):
+    """One decode step that first writes the new token's rows new_k/new_v [nseq, hkv, D]
+    into ring slot (ctx_len - 1) % W. Returns (O, lse or None)."""
+    for t in (new_k, new_v, ring_k, ring_v):
+        assert t.is_contiguous()
+    if O is None:
+        O = torch.empty_like(q)
+    if workspace is None:
+        workspace = decode_workspace(desc, q.device)
+    lse = (torch.empty(q.shape[:2], dtype=torch.float32, device=q.device) if want_lse
+           else None)
+    st = B.hca_attn_decode_append(desc, q.data_ptr(), ctx_len.data_ptr(), cache.c,
+                                  new_k.data_ptr(), new_v.data_ptr(), ring_k.data_ptr(),
+                                  ring_v.data_ptr(), O.data_ptr(), _ptr(lse), workspace.data_ptr(),
+                                  workspace.numel(), _stream(stream))
+    B.check(st, "hca_attn_decode_append")
+    return O, lse
+
+
 def prefill_range(desc: B.HcaDesc, q_pos0: int, kv_pos0: int, Q: torch.Tensor,
                   K: torch.Tensor, V: torch.Tensor, cache: B.PagedCache,
                   O: Optional[torch.Tensor] = None, want_lse: bool = False,

@@ -304,6 +304,19 @@ int32_t hca_attn_decode(const hca_desc* d, const void* Q, const int32_t* ctx_len
                         void* O, float* lse, void* workspace, size_t workspace_bytes,
                         hca_stream_t stream);
 
+/* hca_ring_append and hca_attn_decode in one call ([news 二.1]): the new token's rows
+ * new_k, new_v [batch, hkv, head_dim] go into ring slot (ctx_len[b] - 1) % window (ctx_len
+ * clamped as hca_attn_decode clamps it), then the decode step runs over the updated rings.
+ * The bf16 tensor-core kernels write the two rows from the CTA that reads the window, just
+ * before it reads it, so the step needs no separate launch; other paths run the two calls.
+ * Arguments and errors as hca_attn_decode, plus HCA_EINVAL for a NULL or not 16-byte
+ * aligned new_k / new_v. A block the new token completes is compressed after this call
+ * (its entry is not visible to the token's own query). */
+int32_t hca_attn_decode_append(const hca_desc* d, const void* Q, const int32_t* ctx_len,
+                               const hca_cache* cache, const void* new_k, const void* new_v,
+                               void* ring_k, void* ring_v, void* O, float* lse,
+                               void* workspace, size_t workspace_bytes, hca_stream_t stream);
+
 /* Bytes of one decode partial result for d (bf16 paths; 0 if d is invalid or f32). */
 size_t hca_decode_partial_bytes(const hca_desc* d);
 

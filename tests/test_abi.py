@@ -206,6 +206,11 @@ def test_ring_append_validation(L):
     assert B.hca_ring_append(odd, 16, 16, 16, 16, 16) == B.HCA_EUNSUPPORTED
     # an empty batch is a no-op
     assert B.hca_ring_append(B.make_desc(0, 1000, 64, 1, 512), 0, 0, 0, 0, 0) == B.HCA_OK
+    # the decode call with the ring update: the new rows are required and 16-byte aligned
+    c = _cache()
+    args = (16, 16, c)
+    assert B.hca_attn_decode_append(d, *args, 0, 16, 16, 16, 16, 0, 16, 1 << 30) == B.HCA_EINVAL
+    assert B.hca_attn_decode_append(d, *args, 16, 8, 16, 16, 16, 0, 16, 1 << 30) == B.HCA_EINVAL
 
 
 def test_set_gate(L):

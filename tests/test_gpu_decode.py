@@ -101,6 +101,31 @@ def test_ring_append(dtype, hkv, D):
     assert torch.equal(rk.cpu(), want_k) and torch.equal(rv.cpu(), want_v)
 
 
+@pytest.mark.parametrize("nseq,lo,hi,splits", [
+    (6, 1, 127, 0),            # window only, partly filled ring
+    (8, 8192, 40000, 0),       # several splits: only the last one reads the ring
+    (3, 20000, 30000, 1),      # one split
+])
+def test_decode_append_equals_append_then_decode(nseq, lo, hi, splits):
+    """hca_attn_decode_append (the new rows written by the CTA that reads the window)
+    gives byte-identical rings and outputs to hca_ring_append followed by hca_attn_decode."""
+    x, cache, desc = _setup(nseq, lo, hi, seed=80 + nseq, gate=True, splits=splits)
+    dev = torch.device("cuda")
+    g = torch.Generator().manual_seed(81)
+    nk = torch.randn((nseq, 1, 512), generator=g).to(torch.bfloat16).to(dev)
+    nv = torch.randn((nseq, 1, 512), generator=g).to(torch.bfloat16).to(dev)
+    q, ctx = x.q.to(dev), x.ctx_len.to(dev)
+    rk_a, rv_a = x.ring_k.to(dev), x.ring_v.to(dev)
+    rk_b, rv_b = rk_a.clone(), rv_a.clone()
+    ops.ring_append(desc, nk, nv, ctx, rk_a, rv_a)
+    O_a, l_a = ops.decode(desc, q, ctx, cache, rk_a, rv_a, want_lse=True)
+    O_b, l_b = ops.decode_append(desc, q, ctx, cache, nk, nv, rk_b, rv_b, want_lse=True)
+    torch.cuda.synchronize()
+    assert torch.equal(rk_a, rk_b) and torch.equal(rv_a, rv_b)
+    assert torch.equal(O_a, O_b) and torch.equal(l_a, l_b)
+    assert int(cache.err.item()) == 0
+
+
 # the last compressed tile holds 16 * odd entries, all visible: its last 32-column score
 # piece runs 16 columns past the tile, and those columns (stale tensor memory, scores of an
 # earlier tile) must enter neither P nor the row sum
@@ -270,17 +295,25 @@ def test_decode_1m_config_four_steps_sampled():
         q = x.q if s == 0 else tok.q[s]
         desc = B.make_desc(nseq, ctx0 + steps, 64, 1, 512)
         ctx = torch.full((nseq,), p + 1, dtype=torch.int32, device=dev)
+        ops.attach_gate(desc, tok.G[s].to(dev))
         if s > 0:
-            # the library's ring update on the device, plain indexing for the oracle's copy
-            ops.ring_append(desc, tok.k[s].to(dev).contiguous(), tok.v[s].to(dev).contiguous(),
-                            ctx, rk, rv)
+            # step 2: the library's ring update as its own launch; steps 3, 4: inside the
+            # decode call; plain indexing for the oracle's copy
+            nk, nv = tok.k[s].to(dev).contiguous(), tok.v[s].to(dev).contiguous()
+            if s == 1:
+                ops.ring_append(desc, nk, nv, ctx, rk, rv)
+                ops.decode(desc, q.to(dev), ctx, cache, rk, rv, O=O)
+            else:
+                ops.decode_append(desc, q.to(dev), ctx, cache, nk, nv, rk, rv, O=O)
             rk_h[:, p % W] = tok.k[s]
             rv_h[:, p % W] = tok.v[s]
+        else:
+            ops.decode(desc, q.to(dev), ctx, cache, rk, rv, O=O)
         if (p + 1) % blk == 0:
+            # the block the token completes: compressed after the step (its entry is not
+            # visible to the token's own query)
             B.check(B.hca_compress(cdesc, rk.data_ptr(), rv.data_ptr(), W, p // blk, 1, cache.c,
                                    torch.cuda.current_stream().cuda_stream), "hca_compress")
-        ops.attach_gate(desc, tok.G[s].to(dev))
-        ops.decode(desc, q.to(dev), ctx, cache, rk, rv, O=O)
         torch.cuda.synchronize()
         assert int(cache.err.item()) == 0
         for b in sorted(np.random.default_rng(100 + s).choice(nseq, 5, replace=False)):

@@ -196,6 +196,27 @@ def test_decode_e4m3_tile_ends_mid_piece(ctx, splits):
     assert int(cache.err.item()) == 0
 
 
+@pytest.mark.parametrize("nseq,lo,hi", [(6, 1, 127), (8, 8192, 40000)])
+def test_decode_e4m3_append_equals_append_then_decode(nseq, lo, hi):
+    """On the 8-bit cache too, the in-kernel ring update matches hca_ring_append followed by
+    hca_attn_decode byte for byte."""
+    x, cache, desc = _setup8(nseq, lo, hi, seed=90 + nseq, gate=True)
+    dev = torch.device("cuda")
+    g = torch.Generator().manual_seed(91)
+    nk = torch.randn((nseq, 1, 512), generator=g).to(torch.bfloat16).to(dev)
+    nv = torch.randn((nseq, 1, 512), generator=g).to(torch.bfloat16).to(dev)
+    q, ctx = x.q.to(dev), x.ctx_len.to(dev)
+    rk_a, rv_a = x.ring_k.to(dev), x.ring_v.to(dev)
+    rk_b, rv_b = rk_a.clone(), rv_a.clone()
+    ops.ring_append(desc, nk, nv, ctx, rk_a, rv_a)
+    O_a, l_a = ops.decode(desc, q, ctx, cache, rk_a, rv_a, want_lse=True)
+    O_b, l_b = ops.decode_append(desc, q, ctx, cache, nk, nv, rk_b, rv_b, want_lse=True)
+    torch.cuda.synchronize()
+    assert torch.equal(rk_a, rk_b) and torch.equal(rv_a, rv_b)
+    assert torch.equal(O_a, O_b) and torch.equal(l_a, l_b)
+    assert int(cache.err.item()) == 0
+
+
 def _sample_sequences(ctx_len, n, seed):
     lens = ctx_len.numpy()
     rng = np.random.default_rng(seed)
