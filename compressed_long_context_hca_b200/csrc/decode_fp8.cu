@@ -38,7 +38,9 @@
 //    the converters at the start, and again for the window tile); warp 11 loads the e4m3 V
 //    boxes into a 3-slot V ring; warp 1 issues the score UMMAs, warp 10 the P.V UMMAs;
 //    warps 2-5 run the softmax (lazy rescale, as the 16-bit kernel) and the epilogue;
-//    warps 6-9 prepare Q1/Q2 and widen V.
+//    warps 6-9 widen V; warps 2-9 together prepare Q1/Q2 at the start. With a ring update
+//    requested, warp 0 writes the new K row and the thread of warp 6 that loads the
+//    window's values the new V row, each before its own loads of the window.
 //  * TMEM: O (64 x 512 f32, M = 64 layout) in lanes 0-15 of each 32-lane subpartition;
 //    two score buffers (128 columns each) in lanes 16-31.
 //  * All mbarrier waits are bounded (HCA_ERR_TIMEOUT on give-up); on give-up every issuing
