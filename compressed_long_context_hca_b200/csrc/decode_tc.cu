@@ -21,6 +21,11 @@
 //    as two UMMAs with V N-major: the rounding of P costs ~2^-17 of the value spread instead
 //    of 2^-9. One buffer pair is enough: P(c) is written once PV(c - 1) is done, and V(c)
 //    only arrives after K(c + 1).
+//  * The softmax computes P on all 32 lanes of its warps: the score row of lane l + 16 is
+//    shared with lane l by shuffles (decode_softmax.cuh).
+//  * With a ring update requested (hca_attn_decode_append), the two producer threads of
+//    the CTA holding the window tile write the new token's K and V rows into slot t % W
+//    before their first load of that tile, then fence the async proxy.
 //  * Each CTA writes float32 partials (unnormalised O, base max m in log2 units, sum l) to
 //    the workspace; merge_kernel combines them per head, applies the gate and casts.
 //  * All mbarrier waits are bounded (HCA_ERR_TIMEOUT on give-up).
