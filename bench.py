@@ -267,12 +267,14 @@ def gpu_main(args, rank, world, local_rank):
     my_flops = prefill_flops_rows(T, t0, t1)
     achieved = my_flops / (prefill_ms * 1e-3) / 1e12
     bytes_prefill = (2 * Q.numel() + 2 * K.numel() + 2 * V.numel()) * 2  # Q,O + K,V
-    # the burst peak for a short timed region; the sustained one once the loop ran long
-    # enough for the power cap to act (the clock record shows it)
-    sustained = "sw_power_cap" in (clk or {}).get("reasons", []) or total_ms > 300.0
+    # the burst peak for a short timed loop; the sustained one (measured over a seconds-long
+    # loop under the power cap) once the timed loop itself runs for a sizeable fraction of
+    # a second
+    sustained = total_ms > 300.0
     peak_tf = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
-    peak_note = (f"{peak_kind} bf16 dense sustained (timed loop of {total_ms:.0f} ms, "
-                 f"power cap active)" if sustained else f"{peak_kind} bf16 dense burst")
+    peak_note = (f"{peak_kind} bf16 dense sustained (timed loop of {total_ms:.0f} ms)"
+                 if sustained else
+                 f"{peak_kind} bf16 dense burst (timed loop of {total_ms:.0f} ms)")
     traffic = args.traffic
     if traffic is None and T == 32768 and world == 1:
         traffic = PREFILL_TRAFFIC.get(_prefill_kernel_sha())
