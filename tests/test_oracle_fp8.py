@@ -195,3 +195,25 @@ def test_fp8_planted_mistakes_are_caught(name, monkeypatch):
         except (AssertionError, ValueError, IndexError):
             failed.append(pin.__name__)
     assert failed, f"planted mistake {name!r} passed every pin"
+
+
+def test_two_part_e4m3_query_split():
+    """The reading the 8-bit decode's scores rest on: with r_h the power of two that puts a
+    row's largest |q| in [128, 256), x = q / r_h and Q1 = e4m3(x), Q2 = e4m3(x - Q1), the
+    two parts give x exactly wherever |x| >= 1/4 (the remainder's last bit is still an e4m3
+    step) and within 2^-10 below, for bf16 rows over a wide range of magnitudes."""
+    rng = np.random.default_rng(12)
+    for trial in range(40):
+        scale = 2.0 ** rng.integers(-30, 30)
+        q = torch.tensor(rng.standard_normal(512) * scale, dtype=torch.float32)
+        q = q.to(torch.bfloat16).to(torch.float64).numpy()
+        amax = np.abs(q).max()
+        e = int(np.floor(np.log2(amax))) - 7   # r_h = 2^e: amax / r_h in [128, 256)
+        x = q / 2.0 ** e
+        assert 128.0 <= np.abs(x).max() < 256.0
+        q1 = ORC.e4m3_value(ORC.e4m3_quantize(x))
+        q2 = ORC.e4m3_value(ORC.e4m3_quantize(x - q1))
+        err = np.abs(x - (q1 + q2))
+        big = np.abs(x) >= 0.25
+        assert (err[big] == 0).all(), f"trial {trial}: inexact at |x| >= 1/4"
+        assert (err <= 2.0 ** -10).all(), f"trial {trial}: error above 2^-10"
